@@ -1,0 +1,191 @@
+/*
+ * kla_oracle.c -- plain sequential CPU oracle of the Kalman linear-attention
+ * forward pass, in fp64.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing on the product path links, loads or calls
+ * this file; only the tests, the small smoke check and the benchmark's CPU
+ * baseline leg do. It shares no code, header or constant with the CUDA path.
+ *
+ * What it computes (Kalman Linear Attention, technical summary section 1
+ * "probabilistic formulation", and the Kalman Delta Networks abstract for the
+ * isotropic variant): per sequence n and head h, an information-form Kalman
+ * filter whose state is a precision lambda and an information vector eta.
+ *
+ *   diagonal mode, per key i (one precision per key dimension):
+ *     predict (exactly discretised OU prior, decay a, process noise qn):
+ *         den      = a[t,i]^2 + qn[t,i] * lambda[i]
+ *         g        = a[t,i] / den              (forget gate, precision ratio)
+ *         lambda[i]= lambda[i] / den           (Moebius map of lambda)
+ *         eta[i,:] = g * eta[i,:]
+ *     update (token = noisy observation through k with value precision beta):
+ *         lambda[i]+= beta[t] * k[t,i]^2
+ *         eta[i,:] += beta[t] * k[t,i] * v[t,:]
+ *     readout (posterior mean through the query):
+ *         o[t,:]   = sum_i q[t,i] * eta[i,:] / lambda[i]
+ *
+ *   isotropic mode (one precision per head): a, qn per (t,h);
+ *         den = a^2 + qn*lambda ; g = a/den ; lambda = lambda/den + beta*|k|^2/dk
+ *         eta[i,:] = g*eta[i,:] + beta*k[i]*v ; o = sum_i q[i]*eta[i,:]/lambda
+ *
+ * Every step predicts and then updates, the first one included: lambda0/eta0
+ * are the posterior before the first token, so a sequence split in two calls
+ * (final state of the first handed to the second) equals one call.
+ * Varlen: each packed sequence restarts from its own lambda0/eta0.
+ *
+ * The Moebius helpers expose the 2x2 matrix form of one predict+update step,
+ *     lambda' = ((1 + b*qn) lambda + b*a^2) / (qn lambda + a^2),  b = beta*k^2,
+ * (Kalman Linear Attention, technical summary section 2, the Moebius
+ * precision recursion) for the associativity checks.
+ *
+ * Inputs are float (bf16 and fp32 values are exact in float); all arithmetic is
+ * double. Layouts are row-major with tokens flattened over the batch:
+ *   q,k [Ntok,H,dk]  v [Ntok,H,dv]  a,qn [Ntok,H,dk] (iso [Ntok,H])  beta [Ntok,H]
+ *   lambda0 [N,H,dk] (iso [N,H])  eta0 [N,H,dk,dv]   out [Ntok,H,dv]
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* One (sequence, head) unit, tokens [t0, t1). Returns 0 on success. */
+static int run_unit(int n, int h, long t0, long t1, int H, int dk, int dv, int iso,
+                    const float *q, const float *k, const float *v,
+                    const float *a, const float *qn, const float *beta,
+                    const float *lambda0, const float *eta0,
+                    double *out, double *final_lambda, double *final_eta,
+                    double *lambda_traj)
+{
+    int nl = iso ? 1 : dk;
+    double *lam = (double *)malloc(sizeof(double) * nl);
+    double *eta = (double *)malloc(sizeof(double) * (size_t)dk * dv);
+    if (!lam || !eta) { free(lam); free(eta); return 1; }
+
+    for (int i = 0; i < nl; ++i)
+        lam[i] = lambda0 ? (double)lambda0[((size_t)n * H + h) * nl + i] : 1.0;
+    for (size_t e = 0; e < (size_t)dk * dv; ++e)
+        eta[e] = eta0 ? (double)eta0[((size_t)n * H + h) * dk * dv + e] : 0.0;
+
+    for (long t = t0; t < t1; ++t) {
+        size_t th = (size_t)t * H + h;           /* token-head index */
+        const float *qt = q + th * dk, *kt = k + th * dk, *vt = v + th * dv;
+        double bt = (double)beta[th];
+        if (iso) {
+            double at = a[th], qnt = qn[th];
+            double ksq = 0.0;
+            for (int i = 0; i < dk; ++i) ksq += (double)kt[i] * (double)kt[i];
+            double den = at * at + qnt * lam[0];
+            double g = at / den;
+            lam[0] = lam[0] / den + bt * ksq / (double)dk;
+            for (int i = 0; i < dk; ++i) {
+                double w = bt * (double)kt[i];
+                double *row = eta + (size_t)i * dv;
+                for (int j = 0; j < dv; ++j) row[j] = g * row[j] + w * (double)vt[j];
+            }
+            if (lambda_traj) lambda_traj[th] = lam[0];
+        } else {
+            const float *at = a + th * dk, *qnt = qn + th * dk;
+            for (int i = 0; i < dk; ++i) {
+                double ai = at[i], ki = kt[i];
+                double den = ai * ai + (double)qnt[i] * lam[i];
+                double g = ai / den;
+                lam[i] = lam[i] / den + bt * ki * ki;
+                double w = bt * ki;
+                double *row = eta + (size_t)i * dv;
+                for (int j = 0; j < dv; ++j) row[j] = g * row[j] + w * (double)vt[j];
+                if (lambda_traj) lambda_traj[th * dk + i] = lam[i];
+            }
+        }
+        if (out) {
+            double *ot = out + th * dv;
+            for (int j = 0; j < dv; ++j) ot[j] = 0.0;
+            for (int i = 0; i < dk; ++i) {
+                double c = (double)qt[i] / lam[iso ? 0 : i];
+                const double *row = eta + (size_t)i * dv;
+                for (int j = 0; j < dv; ++j) ot[j] += c * row[j];
+            }
+        }
+    }
+    if (final_lambda)
+        for (int i = 0; i < nl; ++i) final_lambda[((size_t)n * H + h) * nl + i] = lam[i];
+    if (final_eta)
+        memcpy(final_eta + ((size_t)n * H + h) * dk * dv, eta, sizeof(double) * (size_t)dk * dv);
+    free(lam);
+    free(eta);
+    return 0;
+}
+
+/*
+ * Full forward. cu_seqlens (host int32 [num_seqs+1]) or NULL for B rows of T
+ * tokens. Any of out / final_lambda / final_eta / lambda_traj may be NULL.
+ * lambda_traj receives the posterior precision after every token
+ * ([Ntok,H,dk], iso [Ntok,H]). units_begin/units_end select a sub-range of the
+ * (sequence, head) units, unit = n*H + h (pass 0 and -1 for all); the
+ * benchmark's CPU baseline times a bounded sample this way.
+ * num_threads <= 0 uses the OpenMP default. Returns 0 on success.
+ */
+int kla_oracle_forward(int B, int T, int H, int dk, int dv, int iso,
+                       const int *cu_seqlens, int num_seqs,
+                       const float *q, const float *k, const float *v,
+                       const float *a, const float *qn, const float *beta,
+                       const float *lambda0, const float *eta0,
+                       double *out, double *final_lambda, double *final_eta,
+                       double *lambda_traj, long units_begin, long units_end,
+                       int num_threads)
+{
+    if (B < 0 || T < 0 || H <= 0 || dk <= 0 || dv <= 0) return 1;
+    int N = cu_seqlens ? num_seqs : B;
+    long units = (long)N * H;
+    if (units_end < 0 || units_end > units) units_end = units;
+    if (units_begin < 0) units_begin = 0;
+    int err = 0;
+#ifdef _OPENMP
+    if (num_threads > 0) omp_set_num_threads(num_threads);
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : err)
+#endif
+    for (long u = units_begin; u < units_end; ++u) {
+        int n = (int)(u / H), h = (int)(u % H);
+        long t0 = cu_seqlens ? cu_seqlens[n] : (long)n * T;
+        long t1 = cu_seqlens ? cu_seqlens[n + 1] : (long)(n + 1) * T;
+        err |= run_unit(n, h, t0, t1, H, dk, dv, iso, q, k, v, a, qn, beta,
+                        lambda0, eta0, out, final_lambda, final_eta, lambda_traj);
+    }
+    return err;
+}
+
+/* Threads the OpenMP runtime would use (1 without OpenMP). */
+int kla_oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* ---- Moebius form of one predict+update step ---------------------------- */
+
+/* M = [[1 + b*qn, b*a^2], [qn, a^2]] with b = beta*k^2 (or beta*|k|^2/dk in
+ * isotropic mode). lambda' = (M00 lambda + M01) / (M10 lambda + M11). */
+void kla_oracle_mobius_element(double a, double qn, double b, double *M)
+{
+    M[0] = 1.0 + b * qn;
+    M[1] = b * a * a;
+    M[2] = qn;
+    M[3] = a * a;
+}
+
+/* out = L * R (apply R first, then L). out may alias neither input. */
+void kla_oracle_mobius_compose(const double *L, const double *R, double *out)
+{
+    out[0] = L[0] * R[0] + L[1] * R[2];
+    out[1] = L[0] * R[1] + L[1] * R[3];
+    out[2] = L[2] * R[0] + L[3] * R[2];
+    out[3] = L[2] * R[1] + L[3] * R[3];
+}
+
+double kla_oracle_mobius_apply(const double *M, double lam)
+{
+    return (M[0] * lam + M[1]) / (M[2] * lam + M[3]);
+}
