@@ -1,0 +1,716 @@
+// kla_chunk_tc.cu -- the chunked form of the filter's mean path on tcgen05
+// tensor cores (sm_100a).
+//
+// Once the precision path is known, the information-vector update is affine in
+// eta with a per-key, data-dependent gate (Kalman Linear Attention, technical
+// summary sections 2-3: after the Moebius scan the mean recursion is a
+// parallelisable affine map; the forget gate g = a/(a^2 + qn*lambda) comes from
+// precision ratios). It is gated linear attention with
+//     q~ = q / lambda,  k~ = beta * k,  gate g[t,i] = a/(a^2 + qn*lambda_{t-1}).
+// Per chunk of C = 64 tokens with in-chunk cumulative log2-gate G[t,i] and a
+// per-key reference R[i] (midpoint of the chunk's G range, so that neither
+// factor leaves the fp32/bf16 exponent range):
+//     Q'[t,i] = q~[t,i] 2^(G[t,i]-R[i]),   K'[s,i] = k~[s,i] 2^(R[i]-G[s,i])
+//     U       = diag(2^R) eta_chunk_start                     (state, TMEM fp32)
+//     out     = mask_causal(Q' K'^T) V + Q' U                  (tcgen05, TMEM fp32)
+//     eta_chunk_end = diag(2^(G_last-R)) (U + K'^T V)          (tcgen05, TMEM fp32)
+// The state never leaves the SM while a CTA walks its segment: it lives in
+// TMEM as the accumulator of the K'^T V products (the pages' kernels likewise
+// avoid expanding the state in HBM).
+//
+// CTA = one segment of one (row or packed sequence, head); 320 threads:
+//   warps 0-3  gate: per key, the lambda recursion over the chunk (a, qn stream
+//              through a 4-slot TMA ring), log-gates, then Q'/K' written in
+//              place over the TMA-loaded q/k tiles (bf16, 128B-swizzled);
+//              isotropic mode runs a warp-level Moebius scan over the chunk;
+//   warps 4-7  epilogue: rescale U in TMEM and snapshot it to bf16 shared
+//              memory, mask the score tile into P, store the output rows;
+//   warp 8     TMA producer (q, k, v tiles double-buffered; a, qn ring);
+//   warp 9     TMEM owner and single-thread tcgen05.mma issuer.
+// mode 1 ("state") runs only the state recursion from eta = 0 and writes the
+// segment's transfer (eta_end, prod of gates) for the inter-segment carry.
+//
+// Every wait is bounded: after kWaitLimitNs a waiter sets the abort flag and
+// the library status bit, all roles fall through to the teardown, the
+// producer waits (bounded) for its outstanding copies, the MMA thread for its
+// outstanding MMAs, and the TMEM is released.
+#include <cstdlib>
+
+#include "kla_internal.cuh"
+#include "kla_tc_ptx.cuh"
+
+namespace kla {
+using namespace ptx;
+
+namespace {
+
+constexpr int kC = 64;             // chunk tokens
+constexpr int kSlotTok = 16;       // tokens per a/qn ring slot
+constexpr int kSlots = 4;          // ring depth (one chunk)
+constexpr int kThreads = 320;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr float kMaxSpan = 200.0f; // log2 span of G per key per chunk kept exact
+
+struct TcArgs {
+    int N, H, P, NB, seg_blocks, iso, mode;
+    long long T, Lseg;
+    const int *cu;
+    const float *a, *qn, *beta;
+    const float *lambda0, *eta0, *lam_blk;
+    float *S_io, *decay;
+    __nv_bfloat16 *out;
+    float *final_lambda, *final_eta;
+    int *status;
+};
+
+template <int DK, int DV>
+struct Layout {
+    static constexpr int QK = kC * DK * 2;
+    static constexpr int V = kC * DV * 2;
+    static constexpr int PT = kC * kC * 2;
+    static constexpr int UB = DK * DV * 2;
+    static constexpr int SLOTF = kSlotTok * DK;   // floats of one of a / qn per slot
+    static constexpr int q0 = 0;
+    static constexpr int k0 = q0 + 2 * QK;
+    static constexpr int v0 = k0 + 2 * QK;
+    static constexpr int p0 = v0 + 2 * V;
+    static constexpr int ub0 = p0 + PT;
+    static constexpr int ring0 = ub0 + UB;
+    static constexpr int fac0 = ring0 + kSlots * 2 * SLOTF * 4;
+    static constexpr int facf0 = fac0 + 2 * DK * 4;
+    static constexpr int bar0 = ((facf0 + DK * 4) + 7) & ~7;
+    static constexpr int NBAR = 22;
+    static constexpr int hold0 = bar0 + NBAR * 8;
+    static constexpr int bytes = hold0 + 16;
+    static constexpr int alloc = bytes + 1024;
+    static constexpr uint32_t NCOLS = (2 * DV + 64 <= 256) ? 256u : 512u;
+    static constexpr uint32_t colU = 0, colO = DV, colS = 2 * DV;
+};
+
+// Byte offset of element (row, col) in a 128B-swizzled bf16 tile stored as
+// 64-column atoms of `rows` rows of 128 bytes (rows 1024-byte aligned groups).
+__device__ __forceinline__ int sw_off(int row, int col, int rows) {
+    return (col >> 6) * (rows * 128) + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) + ((col & 7) << 1);
+}
+
+__device__ __forceinline__ float bf_at(const uint8_t *base, int off) {
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(base + off));
+}
+__device__ __forceinline__ void bf_put(uint8_t *base, int off, float x) {
+    *reinterpret_cast<__nv_bfloat16 *>(base + off) = __float2bfloat16_rn(x);
+}
+__device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+
+__device__ __noinline__ bool wait_slow(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int *status,
+                                       bool honour_abort) {
+    const uint64_t t0 = globaltimer();
+    for (uint32_t it = 0;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 63) == 63) {
+            if (honour_abort && *abort_flag) return false;
+            if (globaltimer() - t0 > kWaitLimitNs) {
+                *abort_flag = 1;
+                atomicOr(status, kStatusTimeout);
+                return false;
+            }
+        }
+    }
+}
+__device__ __forceinline__ bool wait1(uint64_t *bar, uint32_t parity, volatile int *ab, int *st) {
+    return mbar_try_wait(bar, parity) || wait_slow(bar, parity, ab, st, true);
+}
+// Warp-uniform wait: every lane waits, the warp proceeds only if all saw it.
+__device__ __forceinline__ bool waitw(uint64_t *bar, uint32_t parity, volatile int *ab, int *st) {
+    bool ok = wait1(bar, parity, ab, st);
+    return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ Mob shfl_up_mob(const Mob &m, int d) {
+    return Mob{__shfl_up_sync(0xffffffffu, m.m00, d), __shfl_up_sync(0xffffffffu, m.m01, d),
+               __shfl_up_sync(0xffffffffu, m.m10, d), __shfl_up_sync(0xffffffffu, m.m11, d)};
+}
+
+template <int DK>
+__device__ __forceinline__ float row_sumsq(const uint8_t *ktile, int row) {
+    float s = 0.f;
+#pragma unroll
+    for (int a = 0; a < DK / 64; ++a) {
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+            uint4 x = *reinterpret_cast<const uint4 *>(ktile + a * kC * 128 + row * 128 + ch * 16);
+            const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&x);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                float2 f = __bfloat1622float2(b[e]);
+                s = fmaf(f.x, f.x, s);
+                s = fmaf(f.y, f.y, s);
+            }
+        }
+    }
+    return s;
+}
+
+}  // namespace
+
+template <int DK, int DV>
+__global__ void __launch_bounds__(kThreads, 1)
+kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
+                    const __grid_constant__ CUtensorMap tm_qn, const TcArgs g) {
+    using L = Layout<DK, DV>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::bar0);
+    uint64_t *stage_full = bars + 0, *stage_empty = bars + 2, *qk_ready = bars + 4;
+    uint64_t *ring_full = bars + 6, *ring_empty = bars + 10;
+    uint64_t *s_full = bars + 14, *u_ready = bars + 15, *u_done = bars + 16, *p_full = bars + 17;
+    uint64_t *o_full = bars + 18, *o_empty = bars + 19, *td_bar = bars + 20, *gate_sync = bars + 21;
+    uint32_t *tmem_hold = reinterpret_cast<uint32_t *>(sm + L::hold0);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::hold0 + 4);
+    float *fac = reinterpret_cast<float *>(sm + L::fac0);
+    float *fac_final = reinterpret_cast<float *>(sm + L::facf0);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool state_mode = g.mode == 1;
+    const int P_eff = state_mode ? g.P - 1 : g.P;
+    const long long u = blockIdx.x / P_eff;
+    const int p = (int)(blockIdx.x % P_eff);
+    const int n = (int)(u / g.H), h = (int)(u % g.H);
+    long long tb, te;
+    if (g.cu) { tb = g.cu[n]; te = g.cu[n + 1]; }
+    else {
+        tb = (long long)n * g.T + (long long)p * g.Lseg;
+        te = (long long)n * g.T + min((long long)(p + 1) * g.Lseg, g.T);
+    }
+    const int nchunks = te > tb ? (int)((te - tb + kC - 1) / kC) : 0;
+    const bool last_seg = p == P_eff - 1;
+
+    if (tid == 0) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&stage_full[s], 1);
+            mbar_init(&stage_empty[s], 1);
+            mbar_init(&qk_ready[s], 128);
+        }
+        for (int j = 0; j < kSlots; ++j) {
+            mbar_init(&ring_full[j], 1);
+            mbar_init(&ring_empty[j], 128);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(u_ready, 128);
+        mbar_init(u_done, 1);
+        mbar_init(p_full, 128);
+        mbar_init(o_full, 1);
+        mbar_init(o_empty, 128);
+        mbar_init(td_bar, 1);
+        mbar_init(gate_sync, 128);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 8 && lane == 0) {
+        prefetch_map(&tm_q); prefetch_map(&tm_k); prefetch_map(&tm_v);
+        if (!g.iso) { prefetch_map(&tm_a); prefetch_map(&tm_qn); }
+    }
+    if (warp == 9) tmem_alloc(tmem_hold, L::NCOLS);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_hold;
+
+    if (warp < 4) {
+        // ================= gate warps: precision path and operand folding =====
+        const int i = tid;                       // key owned by this thread
+        const bool key = i < DK;
+        float lam = 1.0f;
+        {
+            const int il = g.iso ? 0 : i;
+            if (key || g.iso) {
+                if (p == 0) lam = g.lambda0 ? g.lambda0[u * (g.iso ? 1 : DK) + il] : 1.0f;
+                else lam = g.lam_blk[(u * g.NB + (long long)p * g.seg_blocks) * (g.iso ? 1 : DK) + il];
+            }
+        }
+        float e_prev = 0.f, log_decay = 0.f;
+        bool ok = true;
+        for (int c = 0; c < nchunks && ok; ++c) {
+            const int s = c & 1;
+            const long long tok0 = tb + (long long)c * kC;
+            uint8_t *qt = sm + L::q0 + s * L::QK;
+            uint8_t *kt = sm + L::k0 + s * L::QK;
+            if (!waitw(&stage_full[s], (c >> 1) & 1, abort_flag, g.status)) { ok = false; break; }
+            float G[kC], A[kC];
+            float gmin = 0.f, gmax = 0.f, R, Glast;
+            float bt_l0 = 0.f, bt_l1 = 0.f;   // iso: beta of this lane's two tokens
+            if (!g.iso) {
+#pragma unroll
+                for (int j = 0; j < kSlots; ++j) {
+                    if (ok) ok = waitw(&ring_full[j], c & 1, abort_flag, g.status);
+                    if (!ok) continue;
+                    const float *ra = reinterpret_cast<const float *>(sm + L::ring0) + j * 2 * L::SLOTF;
+                    const float *rq = ra + L::SLOTF;
+                    float gam = (j == 0) ? 0.f : G[16 * j - 1];
+#pragma unroll
+                    for (int r = 0; r < kSlotTok; ++r) {
+                        const int tau = kSlotTok * j + r;
+                        const long long tok = tok0 + tau;
+                        if (key && tok < te) {
+                            const float at = ra[r * DK + i], qnt = rq[r * DK + i];
+                            const float kk = bf_at(kt, sw_off(tau, i, kC));
+                            const float bt = __ldg(g.beta + tok * g.H + h);
+                            const float den = fmaf(at, at, qnt * lam);
+                            const float rr = __frcp_rn(den);
+                            lam = fmaf(bt * kk, kk, lam * rr);
+                            gam += __log2f(at * rr);
+                        }
+                        G[tau] = gam;
+                        A[tau] = gam - __log2f(lam);
+                        gmin = fminf(gmin, gam);
+                        gmax = fmaxf(gmax, gam);
+                    }
+                    mbar_arrive(&ring_empty[j]);
+                }
+                if (!ok) break;
+                R = 0.5f * (gmin + gmax);
+                Glast = G[kC - 1];
+            } else {
+                // isotropic: one precision per head; warp-level Moebius scan over
+                // the chunk (lane l owns tokens 2l, 2l+1), redundantly per warp.
+                const int t0i = 2 * lane, t1i = 2 * lane + 1;
+                const long long ta = tok0 + t0i, tb2 = tok0 + t1i;
+                const bool va = ta < te, vb = tb2 < te;
+                float a0 = 1.f, q0 = 0.f, b0 = 0.f, a1 = 1.f, q1 = 0.f, b1 = 0.f;
+                const float inv_dk = 1.0f / (float)DK;
+                if (va) {
+                    const long long th = ta * g.H + h;
+                    a0 = __ldg(g.a + th); q0 = __ldg(g.qn + th); bt_l0 = __ldg(g.beta + th);
+                    b0 = bt_l0 * row_sumsq<DK>(kt, t0i) * inv_dk;
+                }
+                if (vb) {
+                    const long long th = tb2 * g.H + h;
+                    a1 = __ldg(g.a + th); q1 = __ldg(g.qn + th); bt_l1 = __ldg(g.beta + th);
+                    b1 = bt_l1 * row_sumsq<DK>(kt, t1i) * inv_dk;
+                }
+                Mob Mp = mob_norm(mob_mul(mob_step(a1, q1, b1), mob_step(a0, q0, b0)));
+#pragma unroll
+                for (int d = 1; d < 32; d <<= 1) {
+                    Mob o = shfl_up_mob(Mp, d);
+                    if (lane >= d) Mp = mob_norm(mob_mul(Mp, o));
+                }
+                Mob E = shfl_up_mob(Mp, 1);
+                if (lane == 0) E = Mob{1.f, 0.f, 0.f, 1.f};
+                const float lamA = mob_apply(E, lam);
+                float g0 = 1.f, lamB = lamA, g1 = 1.f, lamC;
+                if (va) { float rr = __frcp_rn(fmaf(a0, a0, q0 * lamA)); g0 = a0 * rr; lamB = fmaf(lamA, rr, b0); }
+                lamC = lamB;
+                if (vb) { float rr = __frcp_rn(fmaf(a1, a1, q1 * lamB)); g1 = a1 * rr; lamC = fmaf(lamB, rr, b1); }
+                const float l0 = __log2f(g0), l1 = __log2f(g1);
+                float sum = l0 + l1;
+#pragma unroll
+                for (int d = 1; d < 32; d <<= 1) {
+                    float o = __shfl_up_sync(0xffffffffu, sum, d);
+                    if (lane >= d) sum += o;
+                }
+                const float G1 = sum, G0 = sum - l1;
+                const float A0 = G0 - __log2f(lamB), A1 = G1 - __log2f(lamC);
+                float mn = fminf(0.f, fminf(G0, G1)), mx = fmaxf(0.f, fmaxf(G0, G1));
+#pragma unroll
+                for (int d = 16; d > 0; d >>= 1) {
+                    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, d));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, d));
+                }
+                gmin = mn; gmax = mx;
+                R = 0.5f * (gmin + gmax);
+                Glast = __shfl_sync(0xffffffffu, G1, 31);
+                lam = __shfl_sync(0xffffffffu, lamC, 31);
+                // every gate warp has read the raw k rows before any overwrites them
+                mbar_arrive(gate_sync);
+                if (!waitw(gate_sync, c & 1, abort_flag, g.status)) { ok = false; break; }
+#pragma unroll
+                for (int tau = 0; tau < kC; ++tau) {
+                    const float gg0 = __shfl_sync(0xffffffffu, G0, tau >> 1);
+                    const float gg1 = __shfl_sync(0xffffffffu, G1, tau >> 1);
+                    const float aa0 = __shfl_sync(0xffffffffu, A0, tau >> 1);
+                    const float aa1 = __shfl_sync(0xffffffffu, A1, tau >> 1);
+                    G[tau] = (tau & 1) ? gg1 : gg0;
+                    A[tau] = (tau & 1) ? aa1 : aa0;
+                }
+            }
+            if (gmax - gmin > kMaxSpan && key) atomicOr(g.status, kStatusRange);
+            // ---- pass 2: fold 1/lambda, beta and the log-gates into Q', K' (in place)
+#pragma unroll
+            for (int tau = 0; tau < kC; ++tau) {
+                const long long tok = tok0 + tau;
+                float bt = 0.f;
+                if (g.iso) {
+                    const float x0 = __shfl_sync(0xffffffffu, bt_l0, tau >> 1);
+                    const float x1 = __shfl_sync(0xffffffffu, bt_l1, tau >> 1);
+                    bt = (tau & 1) ? x1 : x0;
+                }
+                if (key) {
+                    const int off = sw_off(tau, i, kC);
+                    float qv = 0.f, kv = 0.f;
+                    if (tok < te) {
+                        if (!g.iso) bt = __ldg(g.beta + tok * g.H + h);
+                        if (!state_mode) qv = bf_at(qt, off) * exp2f(A[tau] - R);
+                        kv = bt * bf_at(kt, off) * exp2f(R - G[tau]);
+                    }
+                    if (!state_mode) bf_put(qt, off, qv);
+                    bf_put(kt, off, kv);
+                }
+            }
+            if (key) {
+                fac[s * DK + i] = exp2f(R + e_prev);
+                if (c == nchunks - 1) fac_final[i] = exp2f(Glast - R);
+            }
+            e_prev = Glast - R;
+            log_decay += Glast;
+            fence_proxy_async();
+            mbar_arrive(&qk_ready[s]);
+        }
+        if (ok && !*abort_flag) {
+            if (state_mode) {
+                if (g.iso ? (tid == 0) : key) g.decay[(u * g.P + p) * (g.iso ? 1 : DK) + (g.iso ? 0 : i)] = exp2f(log_decay);
+            } else if (last_seg && g.final_lambda) {
+                if (g.iso ? (tid == 0) : key) g.final_lambda[u * (g.iso ? 1 : DK) + (g.iso ? 0 : i)] = lam;
+            }
+        }
+    } else if (warp < 8) {
+        // ================= epilogue warps ====================================
+        const int e = tid - 128, we = e >> 5, le = e & 31;
+        const uint32_t lane_base = (uint32_t)(32 * we) << 16;
+        const int row64 = 16 * we + le;
+        const bool v64 = le < 16;
+        const int rowU = (DK == 128) ? (32 * we + le) : row64;
+        const bool vU = (DK == 128) || v64;
+        uint8_t *ub = sm + L::ub0;
+        uint8_t *pt = sm + L::p0;
+        const float *sstart = nullptr;
+        if (!state_mode) {
+            if (p == 0) sstart = g.eta0 ? g.eta0 + u * DK * DV : nullptr;
+            else sstart = g.S_io + (u * g.P + p - 1) * DK * DV;
+        }
+        bool ok = true;
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c & 1;
+            const long long tok0 = tb + (long long)c * kC;
+            // ---- state U_c = diag(fac) * (eta_start or U_{c-1} + K'^T V)
+            if (!waitw(&qk_ready[s], (c >> 1) & 1, abort_flag, g.status)) { ok = false; break; }
+            if (c > 0 && !waitw(u_done, (c - 1) & 1, abort_flag, g.status)) { ok = false; break; }
+            tc_fence_after();
+            const float f = vU ? fac[s * DK + rowU] : 0.f;
+#pragma unroll
+            for (int cb = 0; cb < DV / 32; ++cb) {
+                uint32_t r[32];
+                const uint32_t ta = tbase + lane_base + L::colU + cb * 32;
+                if (c == 0) {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x)
+                        r[x] = __float_as_uint((vU && sstart) ? sstart[rowU * DV + cb * 32 + x] * f : 0.f);
+                } else {
+                    tmem_ld32(ta, r);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * f);
+                }
+                tmem_st32(ta, r);
+                if (!state_mode && vU) {
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        uint4 w;
+                        w.x = pack_bf2(__uint_as_float(r[q4 * 8 + 0]), __uint_as_float(r[q4 * 8 + 1]));
+                        w.y = pack_bf2(__uint_as_float(r[q4 * 8 + 2]), __uint_as_float(r[q4 * 8 + 3]));
+                        w.z = pack_bf2(__uint_as_float(r[q4 * 8 + 4]), __uint_as_float(r[q4 * 8 + 5]));
+                        w.w = pack_bf2(__uint_as_float(r[q4 * 8 + 6]), __uint_as_float(r[q4 * 8 + 7]));
+                        *reinterpret_cast<uint4 *>(ub + sw_off(rowU, cb * 32 + q4 * 8, DK)) = w;
+                    }
+                }
+            }
+            tmem_wait_st();
+            fence_proxy_async();
+            tc_fence_before();
+            mbar_arrive(u_ready);
+            if (state_mode) continue;
+            // ---- P = causal mask of the score tile, bf16
+            if (!waitw(s_full, c & 1, abort_flag, g.status)) { ok = false; break; }
+            tc_fence_after();
+            {
+                uint32_t r0[32], r1[32];
+                tmem_ld32(tbase + lane_base + L::colS, r0);
+                tmem_ld32(tbase + lane_base + L::colS + 32, r1);
+                tmem_wait_ld();
+                if (v64) {
+                    const int tau = row64;
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        float x[8];
+#pragma unroll
+                        for (int e2 = 0; e2 < 8; ++e2) {
+                            const int sg = ch * 8 + e2;
+                            const float sv = __uint_as_float(sg < 32 ? r0[sg] : r1[sg - 32]);
+                            x[e2] = sg <= tau ? sv : 0.f;
+                        }
+                        uint4 w;
+                        w.x = pack_bf2(x[0], x[1]); w.y = pack_bf2(x[2], x[3]);
+                        w.z = pack_bf2(x[4], x[5]); w.w = pack_bf2(x[6], x[7]);
+                        *reinterpret_cast<uint4 *>(pt + tau * 128 + ((ch ^ (tau & 7)) << 4)) = w;
+                    }
+                }
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            mbar_arrive(p_full);
+            // ---- output rows
+            if (!waitw(o_full, c & 1, abort_flag, g.status)) { ok = false; break; }
+            tc_fence_after();
+            const bool row_ok = v64 && (tok0 + row64 < te);
+            __nv_bfloat16 *orow = g.out + ((tok0 + row64) * g.H + h) * DV;
+#pragma unroll
+            for (int cb = 0; cb < DV / 32; ++cb) {
+                uint32_t r[32];
+                tmem_ld32(tbase + lane_base + L::colO + cb * 32, r);
+                tmem_wait_ld();
+                if (row_ok) {
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        uint4 w;
+                        w.x = pack_bf2(__uint_as_float(r[q4 * 8 + 0]), __uint_as_float(r[q4 * 8 + 1]));
+                        w.y = pack_bf2(__uint_as_float(r[q4 * 8 + 2]), __uint_as_float(r[q4 * 8 + 3]));
+                        w.z = pack_bf2(__uint_as_float(r[q4 * 8 + 4]), __uint_as_float(r[q4 * 8 + 5]));
+                        w.w = pack_bf2(__uint_as_float(r[q4 * 8 + 6]), __uint_as_float(r[q4 * 8 + 7]));
+                        *reinterpret_cast<uint4 *>(orow + cb * 32 + q4 * 8) = w;
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(o_empty);
+        }
+        // ---- final belief (last segment) or segment transfer (state mode)
+        float *dst = nullptr;
+        if (state_mode) dst = g.S_io + (u * g.P + p) * DK * DV;
+        else if (last_seg && g.final_eta) dst = g.final_eta + u * DK * DV;
+        if (ok && dst && !*abort_flag) {
+            if (nchunks > 0) {
+                if (waitw(u_done, (nchunks - 1) & 1, abort_flag, g.status)) {
+                    tc_fence_after();
+                    const float ff = vU ? fac_final[rowU] : 0.f;
+#pragma unroll
+                    for (int cb = 0; cb < DV / 32; ++cb) {
+                        uint32_t r[32];
+                        tmem_ld32(tbase + lane_base + L::colU + cb * 32, r);
+                        tmem_wait_ld();
+                        if (vU) {
+                            float4 *d4 = reinterpret_cast<float4 *>(dst + rowU * DV + cb * 32);
+#pragma unroll
+                            for (int x = 0; x < 8; ++x)
+                                d4[x] = make_float4(__uint_as_float(r[4 * x]) * ff, __uint_as_float(r[4 * x + 1]) * ff,
+                                                    __uint_as_float(r[4 * x + 2]) * ff, __uint_as_float(r[4 * x + 3]) * ff);
+                        }
+                    }
+                }
+            } else if (vU) {
+                for (int x = 0; x < DV; ++x) dst[rowU * DV + x] = sstart ? sstart[rowU * DV + x] : 0.f;
+            }
+        }
+    } else if (warp == 8) {
+        // ================= TMA producer =====================================
+        if (lane == 0) {
+            int last_ring = -1, last_stage[2] = {-1, -1};
+            bool ok = true;
+            for (int c = 0; c < nchunks && ok; ++c) {
+                const int tok0 = (int)(tb + (long long)c * kC);
+                if (!g.iso) {
+                    for (int j = 0; j < kSlots; ++j) {
+                        if (c > 0 && !wait1(&ring_empty[j], (c - 1) & 1, abort_flag, g.status)) { ok = false; break; }
+                        float *ra = reinterpret_cast<float *>(sm + L::ring0) + j * 2 * L::SLOTF;
+                        mbar_expect_tx(&ring_full[j], 2 * L::SLOTF * 4);
+                        tma_load_3d(ra, &tm_a, &ring_full[j], 0, h, tok0 + kSlotTok * j);
+                        tma_load_3d(ra + L::SLOTF, &tm_qn, &ring_full[j], 0, h, tok0 + kSlotTok * j);
+                    }
+                    if (!ok) break;
+                    last_ring = c;
+                }
+                const int s = c & 1;
+                if (c >= 2 && !wait1(&stage_empty[s], ((c >> 1) - 1) & 1, abort_flag, g.status)) { ok = false; break; }
+                mbar_expect_tx(&stage_full[s], (state_mode ? 0 : L::QK) + L::QK + L::V);
+#pragma unroll
+                for (int a = 0; a < DK / 64; ++a) {
+                    if (!state_mode)
+                        tma_load_3d(sm + L::q0 + s * L::QK + a * kC * 128, &tm_q, &stage_full[s], 64 * a, h, tok0);
+                    tma_load_3d(sm + L::k0 + s * L::QK + a * kC * 128, &tm_k, &stage_full[s], 64 * a, h, tok0);
+                }
+#pragma unroll
+                for (int a = 0; a < DV / 64; ++a)
+                    tma_load_3d(sm + L::v0 + s * L::V + a * kC * 128, &tm_v, &stage_full[s], 64 * a, h, tok0);
+                last_stage[s] = c;
+            }
+            if (!ok || *abort_flag) {
+                // wait (bounded) until every copy this thread issued has landed
+                if (last_ring >= 0)
+                    for (int j = 0; j < kSlots; ++j) wait_slow(&ring_full[j], last_ring & 1, abort_flag, g.status, false);
+                for (int s = 0; s < 2; ++s)
+                    if (last_stage[s] >= 0)
+                        wait_slow(&stage_full[s], (last_stage[s] >> 1) & 1, abort_flag, g.status, false);
+            }
+        }
+    } else {
+        // ================= MMA issuer =======================================
+        if (lane == 0) {
+            constexpr uint32_t iS = idesc_bf16(64, 64, false, false);
+            constexpr uint32_t iO = idesc_bf16(64, DV, false, true);
+            constexpr uint32_t iU = idesc_bf16(DK, DV, true, true);
+            const uint32_t tS = tbase + L::colS, tO = tbase + L::colO, tU = tbase + L::colU;
+            const uint32_t pa = smem_u32(sm + L::p0), uba = smem_u32(sm + L::ub0);
+            for (int c = 0; c < nchunks; ++c) {
+                const int s = c & 1;
+                if (!wait1(&qk_ready[s], (c >> 1) & 1, abort_flag, g.status)) break;
+                tc_fence_after();
+                const uint32_t qa = smem_u32(sm + L::q0 + s * L::QK);
+                const uint32_t ka = smem_u32(sm + L::k0 + s * L::QK);
+                const uint32_t va = smem_u32(sm + L::v0 + s * L::V);
+                if (!state_mode) {
+                    if (c > 0 && !wait1(o_empty, (c - 1) & 1, abort_flag, g.status)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < DK / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * (kC * 128) + (kk & 3) * 32;
+                        mma_bf16(tS, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), iS, kk > 0);
+                    }
+                    mma_commit(s_full);
+                }
+                if (!wait1(u_ready, c & 1, abort_flag, g.status)) break;
+                tc_fence_after();
+                if (!state_mode) {
+#pragma unroll
+                    for (int kk = 0; kk < DK / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * (kC * 128) + (kk & 3) * 32;
+                        mma_bf16(tO, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(uba + kk * 2048, DK * 128, 1024), iO,
+                                 kk > 0);
+                    }
+                }
+#pragma unroll
+                for (int kk = 0; kk < kC / 16; ++kk)
+                    mma_bf16(tU, sdesc_sw128(ka + kk * 2048, kC * 128, 1024), sdesc_sw128(va + kk * 2048, kC * 128, 1024),
+                             iU, 1);
+                mma_commit(u_done);
+                if (!state_mode) {
+                    if (!wait1(p_full, c & 1, abort_flag, g.status)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < kC / 16; ++kk)
+                        mma_bf16(tO, sdesc_sw128(pa + kk * 32, 16, 1024), sdesc_sw128(va + kk * 2048, kC * 128, 1024),
+                                 iO, 1);
+                    mma_commit(o_full);
+                }
+                mma_commit(&stage_empty[s]);
+            }
+            // all MMAs this thread issued have completed before TMEM is released
+            mma_commit(td_bar);
+            wait_slow(td_bar, 0, abort_flag, g.status, false);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 9) tmem_dealloc(tbase, L::NCOLS);
+}
+
+// ---- host side ---------------------------------------------------------------
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult qr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qr) == cudaSuccess &&
+            qr == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// 3-D map over [ntok][H][inner] (inner contiguous) with box (box_inner, 1, box_rows).
+bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int esize, int inner, int H, long long ntok,
+              int box_inner, int box_rows, bool swizzle) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)H, (cuuint64_t)ntok};
+    cuuint64_t strides[2] = {(cuuint64_t)inner * esize, (cuuint64_t)inner * esize * H};
+    cuuint32_t box[3] = {(cuuint32_t)box_inner, 1u, (cuuint32_t)box_rows};
+    cuuint32_t es[3] = {1u, 1u, 1u};
+    CUresult r = fn(m, dt, 3, const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int DK, int DV>
+cudaError_t launch_t(const Plan &p, const int *cu, int mode, const void *q, const void *k, const void *v,
+                     const float *a, const float *qn, const float *beta, const float *lambda0, const float *eta0,
+                     const float *lam_blk, float *S_io, float *decay, void *out, float *final_lambda,
+                     float *final_eta, int *status, cudaStream_t st) {
+    using L = Layout<DK, DV>;
+    CUtensorMap mq, mk, mv, ma, mqn;
+    const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, F32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    bool ok = make_map(&mq, q, BF, 2, DK, p.H, p.ntok, 64, kC, true) &&
+              make_map(&mk, k, BF, 2, DK, p.H, p.ntok, 64, kC, true) &&
+              make_map(&mv, v, BF, 2, DV, p.H, p.ntok, 64, kC, true);
+    if (ok && !p.iso)
+        ok = make_map(&ma, a, F32, 4, DK, p.H, p.ntok, DK, kSlotTok, false) &&
+             make_map(&mqn, qn, F32, 4, DK, p.H, p.ntok, DK, kSlotTok, false);
+    else { ma = mq; mqn = mq; }
+    if (!ok) return cudaErrorInvalidValue;
+    static bool attr[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr[dev]) {
+        cudaError_t e = cudaFuncSetAttribute(kla_chunk_tc_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             L::alloc);
+        if (e != cudaSuccess) return e;
+        attr[dev] = true;
+    }
+    TcArgs g;
+    g.N = p.N; g.H = p.H; g.P = p.P; g.NB = p.NB; g.seg_blocks = p.seg_blocks; g.iso = p.iso; g.mode = mode;
+    g.T = p.T; g.Lseg = p.Lseg; g.cu = cu;
+    g.a = a; g.qn = qn; g.beta = beta; g.lambda0 = lambda0; g.eta0 = eta0; g.lam_blk = lam_blk;
+    g.S_io = S_io; g.decay = decay; g.out = (__nv_bfloat16 *)out;
+    g.final_lambda = final_lambda; g.final_eta = final_eta; g.status = status;
+    const long long segs = mode == 1 ? p.P - 1 : p.P;
+    const unsigned grid = (unsigned)((long long)p.N * p.H * segs);
+    if (grid == 0) return cudaSuccess;
+    kla_chunk_tc_kernel<DK, DV><<<grid, kThreads, L::alloc, st>>>(mq, mk, mv, ma, mqn, g);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool chunk_tc_supported(const Plan &p) {
+    const char *env = getenv("KLA_DISABLE_TC");
+    if (env && *env && *env != '0') return false;
+    return p.bf16 && (p.dk == 64 || p.dk == 128) && (p.dv == 64 || p.dv == 128) && p.ntok < (1LL << 31);
+}
+
+cudaError_t launch_chunk_tc(const Plan &p, const int *cu, int mode, const void *q, const void *k, const void *v,
+                            const float *a, const float *qn, const float *beta, const float *lambda0,
+                            const float *eta0, const float *lam_blk, float *S_io, float *decay, void *out,
+                            float *final_lambda, float *final_eta, int *status, cudaStream_t st) {
+#define KLA_TC_CASE(DK_, DV_)                                                                                  \
+    if (p.dk == DK_ && p.dv == DV_)                                                                            \
+        return launch_t<DK_, DV_>(p, cu, mode, q, k, v, a, qn, beta, lambda0, eta0, lam_blk, S_io, decay, out, \
+                                  final_lambda, final_eta, status, st);
+    KLA_TC_CASE(64, 64)
+    KLA_TC_CASE(64, 128)
+    KLA_TC_CASE(128, 64)
+    KLA_TC_CASE(128, 128)
+#undef KLA_TC_CASE
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace kla

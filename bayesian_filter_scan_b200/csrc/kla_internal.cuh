@@ -1,0 +1,88 @@
+// kla_internal.cuh -- shared definitions of the libkla CUDA sources (sm_100a).
+//
+// Indexing conventions (all row-major, tokens flattened over the batch):
+//   token-head index  th = tok * H + h
+//   q, k  [th * dk + i]      v, out [th * dv + j]
+//   a, qn [th * dk + i]  (iso: [th])      beta [th]
+//   per-unit state: unit u = n * H + h  (n = batch row or packed sequence)
+//
+// A "segment" is a contiguous run of tokens of one (row, head) that one CTA
+// walks; a "block" is the granule of the Moebius reduction (Lb tokens). Both
+// start at row starts; segments are whole numbers of blocks.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace kla {
+
+constexpr int kBlockTokens = 256;  // Lb: tokens per Moebius-reduction block
+constexpr int kChunk = 64;         // C: tokens per chunk of the chunked form
+
+// Bits of the library's device status word (kla_check reads and clears it);
+// kernels that can detect an error receive its address and OR a bit into it.
+enum : int { kStatusRange = 1, kStatusTimeout = 2 };
+
+struct Plan {
+    int N;          // rows (or packed sequences)
+    int H, dk, dv;
+    int nl;         // precisions per (row, head): dk (diag) or 1 (iso)
+    bool iso, varlen, bf16;
+    long long T;    // tokens per row (non-varlen)
+    long long ntok; // tokens in the flattened axis (B*T)
+    int NB;         // Moebius blocks per row (non-varlen)
+    int P;          // segments per row (1 for varlen)
+    int seg_blocks; // blocks per segment
+    long long Lseg; // tokens per segment (seg_blocks * kBlockTokens)
+    // workspace layout (byte offsets; all 256-byte aligned)
+    size_t off_agg, off_lam, off_dS, off_decay, bytes;
+};
+
+__device__ __forceinline__ float ld_in(const float *p) { return __ldg(p); }
+__device__ __forceinline__ float ld_in(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+
+__device__ __forceinline__ void st_out(float *p, float x) { *p = x; }
+__device__ __forceinline__ void st_out(__nv_bfloat16 *p, float x) { *p = __float2bfloat16_rn(x); }
+
+// Four consecutive input values as float (16-byte fp32 or 8-byte bf16 loads).
+__device__ __forceinline__ float4 ld4(const float *p) { return __ldg(reinterpret_cast<const float4 *>(p)); }
+__device__ __forceinline__ float4 ld4(const __nv_bfloat16 *p) {
+    uint2 r = __ldg(reinterpret_cast<const uint2 *>(p));
+    __nv_bfloat162 lo = *reinterpret_cast<__nv_bfloat162 *>(&r.x);
+    __nv_bfloat162 hi = *reinterpret_cast<__nv_bfloat162 *>(&r.y);
+    float2 a = __bfloat1622float2(lo), b = __bfloat1622float2(hi);
+    return make_float4(a.x, a.y, b.x, b.y);
+}
+
+// 2x2 Moebius matrix (m00, m01, m10, m11) acting as x -> (m00 x + m01)/(m10 x + m11).
+struct Mob { float m00, m01, m10, m11; };
+
+// One predict+update step: lambda' = lambda/(a^2 + qn*lambda) + b
+//   = ((1 + b qn) lambda + b a^2) / (qn lambda + a^2).
+__device__ __forceinline__ Mob mob_step(float a, float qn, float b) {
+    float a2 = a * a;
+    return Mob{fmaf(b, qn, 1.0f), b * a2, qn, a2};
+}
+
+// L * R : apply R first, then L.
+__device__ __forceinline__ Mob mob_mul(const Mob &L, const Mob &R) {
+    return Mob{fmaf(L.m00, R.m00, L.m01 * R.m10), fmaf(L.m00, R.m01, L.m01 * R.m11),
+               fmaf(L.m10, R.m00, L.m11 * R.m10), fmaf(L.m10, R.m01, L.m11 * R.m11)};
+}
+
+// Rescale by an exact power of two so the largest entry is in [1, 2): the map is
+// projective, so this changes nothing but keeps the entries inside fp32 range.
+__device__ __forceinline__ Mob mob_norm(const Mob &M) {
+    float mx = fmaxf(fmaxf(M.m00, M.m01), fmaxf(M.m10, M.m11));
+    int e = ((__float_as_int(mx) >> 23) & 0xff) - 127;
+    e = max(-126, min(126, e));
+    float s = __int_as_float((127 - e) << 23);
+    return Mob{M.m00 * s, M.m01 * s, M.m10 * s, M.m11 * s};
+}
+
+__device__ __forceinline__ float mob_apply(const Mob &M, float x) {
+    return fmaf(M.m00, x, M.m01) / fmaf(M.m10, x, M.m11);
+}
+
+}  // namespace kla

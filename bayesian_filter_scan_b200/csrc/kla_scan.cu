@@ -1,0 +1,295 @@
+// kla_scan.cu -- the precision path: a parallel scan of the Moebius maps that
+// one predict+update step applies to the precision lambda (Kalman Linear
+// Attention, technical summary section 2: the posterior precision is a
+// fractional-linear function of the previous one, such maps compose
+// associatively, so lambda_1..T comes from a prefix scan).
+//
+// Three kernels, no inter-CTA waiting (reduce, then scan, then re-walk):
+//   mobius_reduce : per (row, head, block of Lb tokens, key) the composed 2x2
+//                   matrix of the block (normalised by powers of two).
+//   mobius_carry  : per (row, head, key) the exclusive prefix over blocks,
+//                   applied to lambda0: lambda at every block start.
+//   mobius_emit   : per (row/sequence, head, block, key) re-walks the block
+//                   from its start lambda and writes lambda after every token
+//                   (the kla_precision output).
+// Each thread owns 4 consecutive keys (16-byte fp32 loads of a and qn, 8-byte
+// bf16 loads of k), so one warp reads 512 contiguous bytes of a per token.
+#include "kla_internal.cuh"
+
+namespace kla {
+
+struct ScanArgs {
+    int N, H, dk;
+    long long T;      // tokens per row (non-varlen)
+    int NB;           // blocks per row
+    const int *cu;    // packed sequence offsets (emit only) or nullptr
+};
+
+// ---- reduce --------------------------------------------------------------
+
+template <typename TIn>
+__global__ void __launch_bounds__(128)
+mobius_reduce_diag(ScanArgs s, const TIn *__restrict__ k, const float *__restrict__ a,
+                   const float *__restrict__ qn, const float *__restrict__ beta,
+                   float4 *__restrict__ agg) {
+    const int nkq = s.dk / 4;
+    long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    long long pair = gid / nkq;
+    int kq = (int)(gid % nkq);
+    if (pair >= (long long)s.N * s.H * s.NB) return;
+    int blk = (int)(pair % s.NB);
+    long long u = pair / s.NB;
+    int n = (int)(u / s.H), h = (int)(u % s.H);
+    long long t0 = (long long)blk * kBlockTokens;
+    long long t1 = min(t0 + kBlockTokens, s.T);
+    Mob P[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) P[c] = Mob{1.f, 0.f, 0.f, 1.f};
+    for (long long t = t0; t < t1; t += 8) {
+        float4 av[8], qv[8], kv[8];
+        float bv[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            if (t + r < t1) {
+                long long th = ((long long)n * s.T + t + r) * s.H + h;
+                av[r] = ld4(a + th * s.dk + 4 * kq);
+                qv[r] = ld4(qn + th * s.dk + 4 * kq);
+                kv[r] = ld4(k + th * s.dk + 4 * kq);
+                bv[r] = __ldg(beta + th);
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            if (t + r < t1) {
+                const float *ap = &av[r].x, *qp = &qv[r].x, *kp = &kv[r].x;
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    P[c] = mob_mul(mob_step(ap[c], qp[c], bv[r] * kp[c] * kp[c]), P[c]);
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) P[c] = mob_norm(P[c]);
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+        agg[pair * s.dk + 4 * kq + c] = make_float4(P[c].m00, P[c].m01, P[c].m10, P[c].m11);
+}
+
+// Isotropic: one precision per head; increment beta*|k|^2/dk.
+template <typename TIn>
+__device__ __forceinline__ float ksq_row(const TIn *kr, int dk) {
+    float s = 0.f;
+    for (int i = 0; i < dk; i += 4) {
+        float4 x = ld4(kr + i);
+        s = fmaf(x.x, x.x, s); s = fmaf(x.y, x.y, s);
+        s = fmaf(x.z, x.z, s); s = fmaf(x.w, x.w, s);
+    }
+    return s;
+}
+
+template <typename TIn>
+__global__ void __launch_bounds__(128)
+mobius_reduce_iso(ScanArgs s, const TIn *__restrict__ k, const float *__restrict__ a,
+                  const float *__restrict__ qn, const float *__restrict__ beta,
+                  float4 *__restrict__ agg) {
+    long long pair = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (pair >= (long long)s.N * s.H * s.NB) return;
+    int blk = (int)(pair % s.NB);
+    long long u = pair / s.NB;
+    int n = (int)(u / s.H), h = (int)(u % s.H);
+    long long t0 = (long long)blk * kBlockTokens;
+    long long t1 = min(t0 + kBlockTokens, s.T);
+    const float inv_dk = 1.0f / (float)s.dk;
+    Mob P{1.f, 0.f, 0.f, 1.f};
+    for (long long t = t0; t < t1; ++t) {
+        long long th = ((long long)n * s.T + t) * s.H + h;
+        float b = __ldg(beta + th) * ksq_row(k + th * s.dk, s.dk) * inv_dk;
+        P = mob_mul(mob_step(__ldg(a + th), __ldg(qn + th), b), P);
+        if (((t - t0) & 7) == 7) P = mob_norm(P);
+    }
+    P = mob_norm(P);
+    agg[pair] = make_float4(P.m00, P.m01, P.m10, P.m11);
+}
+
+// ---- carry ---------------------------------------------------------------
+
+// lam_blk[(u*NB + blk)*nl + i] = (M_{blk-1} ... M_0)(lambda0): lambda at the
+// start of every block.
+__global__ void __launch_bounds__(128)
+mobius_carry(ScanArgs s, int nl, const float4 *__restrict__ agg,
+             const float *__restrict__ lambda0, float *__restrict__ lam_blk) {
+    long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gid >= (long long)s.N * s.H * nl) return;
+    long long u = gid / nl;
+    int i = (int)(gid % nl);
+    float l0 = lambda0 ? __ldg(lambda0 + gid) : 1.0f;
+    Mob P{1.f, 0.f, 0.f, 1.f};
+    const float4 *src = agg + u * s.NB * nl + i;
+    float *dst = lam_blk + u * s.NB * nl + i;
+    for (int blk = 0; blk < s.NB; blk += 8) {
+        float4 m[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+            if (blk + r < s.NB) m[r] = __ldg(src + (long long)(blk + r) * nl);
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            if (blk + r < s.NB) {
+                dst[(long long)(blk + r) * nl] = mob_apply(P, l0);
+                P = mob_norm(mob_mul(Mob{m[r].x, m[r].y, m[r].z, m[r].w}, P));
+            }
+        }
+    }
+}
+
+// ---- emit ----------------------------------------------------------------
+
+// Token range and start precision of a (pair, key) walk. Non-varlen: pair =
+// (u, blk), start from lam_blk. Varlen: pair = u (whole packed sequence), start
+// from lambda0.
+__device__ __forceinline__ void emit_range(const ScanArgs &s, long long pair, long long &u,
+                                           long long &tb, long long &te) {
+    if (s.cu) {
+        u = pair;
+        int n = (int)(u / s.H);
+        tb = s.cu[n];
+        te = s.cu[n + 1];
+    } else {
+        int blk = (int)(pair % s.NB);
+        u = pair / s.NB;
+        int n = (int)(u / s.H);
+        tb = (long long)n * s.T + (long long)blk * kBlockTokens;
+        te = (long long)n * s.T + min((long long)(blk + 1) * kBlockTokens, s.T);
+    }
+}
+
+template <typename TIn>
+__global__ void __launch_bounds__(128)
+mobius_emit_diag(ScanArgs s, const TIn *__restrict__ k, const float *__restrict__ a,
+                 const float *__restrict__ qn, const float *__restrict__ beta,
+                 const float *__restrict__ lam_start, const float *__restrict__ lambda0,
+                 float *__restrict__ lam_out) {
+    const int nkq = s.dk / 4;
+    long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    long long pair = gid / nkq;
+    int kq = (int)(gid % nkq);
+    long long npairs = s.cu ? (long long)s.N * s.H : (long long)s.N * s.H * s.NB;
+    if (pair >= npairs) return;
+    long long u, tb, te;
+    emit_range(s, pair, u, tb, te);
+    int h = (int)(u % s.H);
+    float lam[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        if (s.cu) lam[c] = lambda0 ? __ldg(lambda0 + u * s.dk + 4 * kq + c) : 1.0f;
+        else lam[c] = __ldg(lam_start + pair * s.dk + 4 * kq + c);
+    }
+    for (long long t = tb; t < te; t += 8) {
+        float4 av[8], qv[8], kv[8];
+        float bv[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            if (t + r < te) {
+                long long th = (t + r) * s.H + h;
+                av[r] = ld4(a + th * s.dk + 4 * kq);
+                qv[r] = ld4(qn + th * s.dk + 4 * kq);
+                kv[r] = ld4(k + th * s.dk + 4 * kq);
+                bv[r] = __ldg(beta + th);
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            if (t + r < te) {
+                const float *ap = &av[r].x, *qp = &qv[r].x, *kp = &kv[r].x;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    float den = fmaf(ap[c], ap[c], qp[c] * lam[c]);
+                    lam[c] = fmaf(bv[r] * kp[c], kp[c], lam[c] / den);
+                }
+                long long th = (t + r) * s.H + h;
+                *reinterpret_cast<float4 *>(lam_out + th * s.dk + 4 * kq) =
+                    make_float4(lam[0], lam[1], lam[2], lam[3]);
+            }
+        }
+    }
+}
+
+template <typename TIn>
+__global__ void __launch_bounds__(128)
+mobius_emit_iso(ScanArgs s, const TIn *__restrict__ k, const float *__restrict__ a,
+                const float *__restrict__ qn, const float *__restrict__ beta,
+                const float *__restrict__ lam_start, const float *__restrict__ lambda0,
+                float *__restrict__ lam_out) {
+    long long pair = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    long long npairs = s.cu ? (long long)s.N * s.H : (long long)s.N * s.H * s.NB;
+    if (pair >= npairs) return;
+    long long u, tb, te;
+    emit_range(s, pair, u, tb, te);
+    int h = (int)(u % s.H);
+    float lam = s.cu ? (lambda0 ? __ldg(lambda0 + u) : 1.0f) : __ldg(lam_start + pair);
+    const float inv_dk = 1.0f / (float)s.dk;
+    for (long long t = tb; t < te; ++t) {
+        long long th = t * s.H + h;
+        float at = __ldg(a + th);
+        float den = fmaf(at, at, __ldg(qn + th) * lam);
+        lam = fmaf(__ldg(beta + th) * ksq_row(k + th * s.dk, s.dk), inv_dk, lam / den);
+        lam_out[th] = lam;
+    }
+}
+
+// ---- host launchers ------------------------------------------------------
+
+static inline unsigned blocks_for(long long threads, int per) {
+    return (unsigned)((threads + per - 1) / per);
+}
+
+template <typename TIn>
+cudaError_t launch_mobius_reduce(const Plan &p, const void *k, const float *a, const float *qn,
+                                 const float *beta, float4 *agg, cudaStream_t st) {
+    ScanArgs s{p.N, p.H, p.dk, p.T, p.NB, nullptr};
+    long long pairs = (long long)p.N * p.H * p.NB;
+    if (p.iso)
+        mobius_reduce_iso<TIn><<<blocks_for(pairs, 128), 128, 0, st>>>(
+            s, (const TIn *)k, a, qn, beta, agg);
+    else
+        mobius_reduce_diag<TIn><<<blocks_for(pairs * (p.dk / 4), 128), 128, 0, st>>>(
+            s, (const TIn *)k, a, qn, beta, agg);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_mobius_carry(const Plan &p, const float4 *agg, const float *lambda0,
+                                float *lam_blk, cudaStream_t st) {
+    ScanArgs s{p.N, p.H, p.dk, p.T, p.NB, nullptr};
+    long long thr = (long long)p.N * p.H * p.nl;
+    mobius_carry<<<blocks_for(thr, 128), 128, 0, st>>>(s, p.nl, agg, lambda0, lam_blk);
+    return cudaGetLastError();
+}
+
+template <typename TIn>
+cudaError_t launch_mobius_emit(const Plan &p, const int *cu, const void *k, const float *a,
+                               const float *qn, const float *beta, const float *lam_blk,
+                               const float *lambda0, float *lam_out, cudaStream_t st) {
+    ScanArgs s{p.N, p.H, p.dk, p.T, p.NB, cu};
+    long long pairs = cu ? (long long)p.N * p.H : (long long)p.N * p.H * p.NB;
+    if (p.iso)
+        mobius_emit_iso<TIn><<<blocks_for(pairs, 128), 128, 0, st>>>(
+            s, (const TIn *)k, a, qn, beta, lam_blk, lambda0, lam_out);
+    else
+        mobius_emit_diag<TIn><<<blocks_for(pairs * (p.dk / 4), 128), 128, 0, st>>>(
+            s, (const TIn *)k, a, qn, beta, lam_blk, lambda0, lam_out);
+    return cudaGetLastError();
+}
+
+template cudaError_t launch_mobius_reduce<float>(const Plan &, const void *, const float *,
+                                                 const float *, const float *, float4 *, cudaStream_t);
+template cudaError_t launch_mobius_reduce<__nv_bfloat16>(const Plan &, const void *, const float *,
+                                                         const float *, const float *, float4 *,
+                                                         cudaStream_t);
+template cudaError_t launch_mobius_emit<float>(const Plan &, const int *, const void *, const float *,
+                                               const float *, const float *, const float *,
+                                               const float *, float *, cudaStream_t);
+template cudaError_t launch_mobius_emit<__nv_bfloat16>(const Plan &, const int *, const void *,
+                                                       const float *, const float *, const float *,
+                                                       const float *, const float *, float *,
+                                                       cudaStream_t);
+
+}  // namespace kla

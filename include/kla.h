@@ -1,0 +1,180 @@
+/*
+ * kla.h -- C ABI of libkla, the B200 (sm_100a) forward pass of a Kalman
+ * linear-attention (KLA) sequence-mixing layer.
+ *
+ * The operation (Kalman Linear Attention, technical summary section 1,
+ * "probabilistic formulation"; Kalman Delta Networks abstract for the
+ * isotropic variant). Per sequence n and head h an information-form Kalman
+ * filter keeps a precision lambda and an information matrix eta[dk][dv].
+ * For every token t, first a predict with an exactly discretised
+ * Ornstein-Uhlenbeck prior (decay a, process noise qn), then an update that
+ * treats the token as a noisy observation through the key k with value
+ * precision beta, then a readout of the posterior mean through the query q:
+ *
+ *   den = a^2 + qn*lambda ;  g = a/den                (forget gate)
+ *   lambda <- lambda/den + beta*k^2                   (a Moebius map of lambda,
+ *                                                      technical summary sec. 2)
+ *   eta[i,:] <- g*eta[i,:] + beta*k[i]*v              (affine once g is known)
+ *   out[t,:] = sum_i q[i]*eta[i,:]/lambda[i]
+ *
+ * KLA_DIAG: lambda, a, qn per key dimension i.  KLA_ISO: one lambda per head,
+ * a and qn per (token, head), increment beta*|k|^2/dk, shared gate.
+ * Every token predicts and then updates (the first one included), so
+ * lambda0/eta0 is the belief before the first token and the final state of one
+ * call is a valid lambda0/eta0 for the next: two calls over a split sequence
+ * equal one call over the whole.
+ *
+ * Layouts (row-major, tokens flattened over the batch, Ntok = B*T):
+ *   q, k        [Ntok, H, dk]        bf16 (KLA_BF16) or fp32 (KLA_FP32)
+ *   v, out      [Ntok, H, dv]        same dtype as q
+ *   a, qn       [Ntok, H, dk] fp32   (KLA_ISO: [Ntok, H])
+ *   beta        [Ntok, H]     fp32
+ *   lambda0, final_lambda  [N, H, dk] fp32 (KLA_ISO: [N, H])
+ *   eta0, final_eta        [N, H, dk, dv] fp32
+ * N = B, or num_seqs with packed variable-length sequences (cu_seqlens).
+ *
+ * Ownership: the caller owns every buffer, including the workspace; all device
+ * pointers must stay valid until the stream work completes. Calls enqueue work
+ * on `stream` and return without synchronising (except kla_check and
+ * kla_forward_host, which say so). The library never allocates device memory.
+ *
+ * Preconditions not checked on the device: a > 0, qn >= 0, beta >= 0,
+ * lambda0 > 0, finite inputs. Identical inputs give bitwise identical outputs
+ * on the same device and configuration (no atomics in any reduction).
+ */
+#ifndef KLA_H_
+#define KLA_H_
+
+#include <stddef.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KLA_OK = 0,
+    KLA_ERR_INVALID_ARG = 1,  /* bad shape, null required pointer, misaligned
+                                 pointer, workspace too small; nothing launched */
+    KLA_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement */
+    KLA_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
+    KLA_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up (kla_check) */
+    KLA_ERR_RANGE = 5         /* the in-chunk log-gate span exceeded the range
+                                 the factorised chunk form represents exactly
+                                 (kla_check); outputs of that call are unreliable */
+} kla_status;
+
+typedef enum { KLA_BF16 = 0, KLA_FP32 = 1 } kla_dtype;   /* dtype of q, k, v, out */
+typedef enum { KLA_DIAG = 0, KLA_ISO = 1 } kla_mode;      /* lambda per key / per head */
+
+typedef struct {
+    int B, T, H;          /* batch, tokens per batch row, heads (B*T = Ntok) */
+    int dk, dv;           /* key and value head dims: dk, dv in {16,32,64,128}, dv also 256 */
+    kla_dtype dtype;
+    kla_mode mode;
+    const int *cu_seqlens;  /* device int32 [num_seqs+1]: packed sequence offsets
+                               into the Ntok axis (0 = first, Ntok = last), or NULL
+                               for B independent rows of T tokens */
+    int num_seqs;           /* number of packed sequences when cu_seqlens != NULL */
+} kla_desc;
+
+/* Bytes of device workspace kla_forward needs for this descriptor on the
+ * current device (0 means the workspace pointer may be NULL). Pure host
+ * computation. Returns 0 for an invalid descriptor as well. */
+size_t kla_workspace_bytes(const kla_desc *desc);
+
+/* Bytes of device workspace kla_precision needs (0: the pointer may be NULL). */
+size_t kla_precision_workspace_bytes(const kla_desc *desc);
+
+/* The forward pass (the whole hot path: precision scan, state passing, chunked
+ * gated linear attention). q, k, v, a, qn, out: device pointers in the
+ * layouts above, 16-byte aligned; beta 4-byte aligned. lambda0 (4-byte aligned) / eta0 (16-byte
+ * aligned): device pointers, or NULL for lambda0 = 1 and eta0 = 0. final_lambda/final_eta: device pointers or NULL to
+ * skip. workspace: device, 256-byte aligned, >= kla_workspace_bytes(desc).
+ * Ntok == 0 is a no-op. Errors: KLA_ERR_INVALID_ARG / KLA_ERR_UNSUPPORTED
+ * before any launch; KLA_ERR_CUDA if a launch fails. */
+kla_status kla_forward(const kla_desc *desc,
+                       const void *q, const void *k, const void *v,
+                       const float *a, const float *qn, const float *beta,
+                       const float *lambda0, const float *eta0,
+                       void *out, float *final_lambda, float *final_eta,
+                       void *workspace, size_t workspace_bytes,
+                       cudaStream_t stream);
+
+/* kla_forward that also records six caller-created CUDA events on `stream`:
+ * events[0] before the first launch and events[1..5] after the stages
+ * 1 Moebius block reduction, 2 Moebius carry, 3 segment state pass,
+ * 4 segment state carry, 5 output pass (the chunk kernel). Stages that do
+ * not run for this descriptor record at the same point as the previous one.
+ * For measuring the stages; otherwise identical to kla_forward. */
+kla_status kla_forward_profiled(const kla_desc *desc,
+                                const void *q, const void *k, const void *v,
+                                const float *a, const float *qn, const float *beta,
+                                const float *lambda0, const float *eta0,
+                                void *out, float *final_lambda, float *final_eta,
+                                void *workspace, size_t workspace_bytes,
+                                cudaStream_t stream, cudaEvent_t *events);
+
+/* The work plan kla_forward uses for this descriptor on the current device:
+ * segments each row is split into (1: one CTA walks a whole row or packed
+ * sequence), kernel launches per call (1 or 5), and whether the chunk stages
+ * run on the tcgen05 tensor-core kernel (1) or the CUDA-core walk (0).
+ * Any output pointer may be NULL. Pure host computation. */
+kla_status kla_plan(const kla_desc *desc, int *segments_per_row, int *launches,
+                    int *tensor_core);
+
+/* The precision path alone: lambda_out[Ntok, H, dk] (KLA_ISO: [Ntok, H]) fp32
+ * receives the posterior precision after every token -- the filter's explicit
+ * uncertainty (Kalman Linear Attention, technical summary section 2: the
+ * Moebius recursion computed by a parallel prefix scan). Same argument rules
+ * as kla_forward, with a workspace of kla_precision_workspace_bytes(desc). */
+kla_status kla_precision(const kla_desc *desc, const void *k,
+                         const float *a, const float *qn, const float *beta,
+                         const float *lambda0, float *lambda_out,
+                         void *workspace, size_t workspace_bytes,
+                         cudaStream_t stream);
+
+/* One recurrent decode step per sequence (T = 1 per sequence, B = N rows):
+ * reads the belief lambda/eta in place, applies predict + update for token
+ * q,k,v,a,qn,beta ([N,H,...] with Ntok = N) and writes out[N,H,dv]; lambda and
+ * eta are overwritten with the new belief (constant-memory decoding, Kalman
+ * Delta Networks abstract). desc->T must be 1 and cu_seqlens NULL. */
+kla_status kla_decode_step(const kla_desc *desc,
+                           const void *q, const void *k, const void *v,
+                           const float *a, const float *qn, const float *beta,
+                           float *lambda, float *eta, void *out,
+                           cudaStream_t stream);
+
+/* Bytes of one device buffer kla_forward_host needs (inputs, outputs and
+ * workspace, each 256-byte aligned). */
+size_t kla_host_device_bytes(const kla_desc *desc);
+
+/* kla_forward on HOST buffers (pinned host memory gives asynchronous copies):
+ * copies the inputs into device_buffer (>= kla_host_device_bytes), runs the
+ * forward pass, copies out (and final states when the pointers are non-NULL)
+ * back, and synchronises the stream before returning. cu_seqlens in desc is a
+ * HOST pointer for this call. */
+kla_status kla_forward_host(const kla_desc *desc,
+                            const void *q, const void *k, const void *v,
+                            const float *a, const float *qn, const float *beta,
+                            const float *lambda0, const float *eta0,
+                            void *out, float *final_lambda, float *final_eta,
+                            void *device_buffer, size_t device_bytes,
+                            cudaStream_t stream);
+
+/* Synchronises `stream`, then reads and clears the library's device status
+ * word on the current device: KLA_OK, KLA_ERR_RANGE or KLA_ERR_TIMEOUT from any
+ * kernel that ran since the last check, or KLA_ERR_CUDA if the stream failed. */
+kla_status kla_check(cudaStream_t stream);
+
+/* Static description of an error code. */
+const char *kla_status_string(kla_status status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int kla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KLA_H_ */
