@@ -21,7 +21,8 @@
 // CTA = one segment of one (row or packed sequence, head); 320 threads:
 //   warps 0-3  gate: per key, the lambda recursion over the chunk (a, qn stream
 //              through a 4-slot TMA ring), log-gates, then Q'/K' written in
-//              place over the TMA-loaded q/k tiles (bf16, 128B-swizzled);
+//              place over the TMA-loaded q/k tiles (bf16, 128B-swizzled), and
+//              the bf16 remainder of K' for a two-term state update;
 //              isotropic mode runs a warp-level Moebius scan over the chunk;
 //   warps 4-7  epilogue: rescale U in TMEM and snapshot it to bf16 shared
 //              memory, mask the score tile into P, store the output rows;
@@ -75,7 +76,8 @@ struct Layout {
     static constexpr int v0 = k0 + 2 * QK;
     static constexpr int p0 = v0 + 2 * V;
     static constexpr int ub0 = p0 + PT;
-    static constexpr int ring0 = ub0 + UB;
+    static constexpr int klo0 = ub0 + UB;          // low bf16 part of K' (state update)
+    static constexpr int ring0 = klo0 + QK;
     static constexpr int fac0 = ring0 + kSlots * 2 * SLOTF * 4;
     static constexpr int facf0 = fac0 + 2 * DK * 4;
     static constexpr int bar0 = ((facf0 + DK * 4) + 7) & ~7;
@@ -337,6 +339,9 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
             }
             if (gmax - gmin > kMaxSpan && key) atomicOr(g.status, kStatusRange);
+            // the K'-low tile is single-buffered: the previous chunk's state update must be done
+            if (c > 0 && !waitw(u_done, (c - 1) & 1, abort_flag, g.status)) { ok = false; break; }
+            uint8_t *klo = sm + L::klo0;
             // ---- pass 2: fold 1/lambda, beta and the log-gates into Q', K' (in place)
 #pragma unroll
             for (int tau = 0; tau < kC; ++tau) {
@@ -356,7 +361,11 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         kv = bt * bf_at(kt, off) * exp2f(R - G[tau]);
                     }
                     if (!state_mode) bf_put(qt, off, qv);
-                    bf_put(kt, off, kv);
+                    // K' = hi + lo in two bf16 parts: the state update sums K'^T V over
+                    // whole segments, so it gets (nearly) fp32 operands; the scores use hi.
+                    const __nv_bfloat16 khi = __float2bfloat16_rn(kv);
+                    *reinterpret_cast<__nv_bfloat16 *>(kt + off) = khi;
+                    bf_put(klo, off, kv - __bfloat162float(khi));
                 }
             }
             if (key) {
@@ -560,7 +569,7 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             constexpr uint32_t iO = idesc_bf16(64, DV, false, true);
             constexpr uint32_t iU = idesc_bf16(DK, DV, true, true);
             const uint32_t tS = tbase + L::colS, tO = tbase + L::colO, tU = tbase + L::colU;
-            const uint32_t pa = smem_u32(sm + L::p0), uba = smem_u32(sm + L::ub0);
+            const uint32_t pa = smem_u32(sm + L::p0), uba = smem_u32(sm + L::ub0), kloa = smem_u32(sm + L::klo0);
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c & 1;
                 if (!wait1(&qk_ready[s], (c >> 1) & 1, abort_flag, g.status)) break;
@@ -589,9 +598,11 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     }
                 }
 #pragma unroll
-                for (int kk = 0; kk < kC / 16; ++kk)
-                    mma_bf16(tU, sdesc_sw128(ka + kk * 2048, kC * 128, 1024), sdesc_sw128(va + kk * 2048, kC * 128, 1024),
-                             iU, 1);
+                for (int kk = 0; kk < kC / 16; ++kk) {
+                    const uint64_t bv = sdesc_sw128(va + kk * 2048, kC * 128, 1024);
+                    mma_bf16(tU, sdesc_sw128(ka + kk * 2048, kC * 128, 1024), bv, iU, 1);
+                    mma_bf16(tU, sdesc_sw128(kloa + kk * 2048, kC * 128, 1024), bv, iU, 1);
+                }
                 mma_commit(u_done);
                 if (!state_mode) {
                     if (!wait1(p_full, c & 1, abort_flag, g.status)) break;
