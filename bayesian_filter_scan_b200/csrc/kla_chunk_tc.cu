@@ -223,8 +223,10 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
     if (warp < 4) {
         // ================= gate warps: precision path and operand folding =====
-        const int i = tid;                       // key owned by this thread
-        const bool key = i < DK;
+        // key owned by this thread; with dk = 64 both halves of the gate group
+        // run the recursion for the same keys and split the operand writes
+        const int i = tid & (DK - 1);
+        const bool key = true;
         float lam = 1.0f;
         {
             const int il = g.iso ? 0 : i;
@@ -233,75 +235,144 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 else lam = g.lam_blk[(u * g.NB + (long long)p * g.seg_blocks) * (g.iso ? 1 : DK) + il];
             }
         }
-        float e_prev = 0.f, log_decay = 0.f;
+        float e_prev = 1.f, log_decay = 0.f;   // e_prev = 2^(G_last - R) of the previous chunk
         bool ok = true;
+        // Per-token scalars of a chunk are loaded one chunk ahead into registers
+        // and broadcast with shuffles (no global load sits on the recursion).
+        // diag: beta of tokens (lane, lane+32); iso: a, qn, beta of (2 lane, 2 lane+1).
+        float nb0 = 0.f, nb1 = 0.f, na0 = 1.f, na1 = 1.f, nq0 = 0.f, nq1 = 0.f;
+        auto prefetch = [&](int c) {
+            const long long t0 = tb + (long long)c * kC;
+            const long long x0 = g.iso ? t0 + 2 * lane : t0 + lane;
+            const long long x1 = g.iso ? x0 + 1 : t0 + 32 + lane;
+            nb0 = x0 < te ? __ldg(g.beta + x0 * g.H + h) : 0.f;
+            nb1 = x1 < te ? __ldg(g.beta + x1 * g.H + h) : 0.f;
+            if (g.iso) {
+                na0 = x0 < te ? __ldg(g.a + x0 * g.H + h) : 1.f;
+                na1 = x1 < te ? __ldg(g.a + x1 * g.H + h) : 1.f;
+                nq0 = x0 < te ? __ldg(g.qn + x0 * g.H + h) : 0.f;
+                nq1 = x1 < te ? __ldg(g.qn + x1 * g.H + h) : 0.f;
+            }
+        };
+        if (nchunks > 0) prefetch(0);
         for (int c = 0; c < nchunks && ok; ++c) {
             const int s = c & 1;
             const long long tok0 = tb + (long long)c * kC;
             uint8_t *qt = sm + L::q0 + s * L::QK;
             uint8_t *kt = sm + L::k0 + s * L::QK;
+            const float cb0 = nb0, cb1 = nb1, ca0 = na0, ca1 = na1, cq0 = nq0, cq1 = nq1;
+            if (c + 1 < nchunks) prefetch(c + 1);
             if (!waitw(&stage_full[s], (c >> 1) & 1, abort_flag, g.status)) { ok = false; break; }
-            float G[kC], A[kC];
-            float gmin = 0.f, gmax = 0.f, R, Glast;
-            float bt_l0 = 0.f, bt_l1 = 0.f;   // iso: beta of this lane's two tokens
+            // Per token the gate warps produce two scale factors, applied in pass 2:
+            //   fq = 2^(G_t - R) / lambda_t   (query side),   fk = 2^(R - G_t)   (key side)
+            // with G_t the in-chunk cumulative log2-gate and R an integer reference at
+            // the middle of the chunk's G range (so neither factor leaves the exponent range).
+            float FQ[kC], FK[kC];
+            int gmin = 0, gmax = 0, R;
+            float glast_m;        // 2^G_last = glast_m * 2^s_last
+            int s_last;
             if (!g.iso) {
+                // Projective form of the precision: lambda = n/d with
+                //   d <- a^2 d + qn n,  n <- n + b d   (b = beta k^2),
+                // two FMAs per token on the serial chain. The gate is g = a d_prev / d,
+                // so with PA = prod a the cumulative gate telescopes (d = 1 at the chunk
+                // start): 2^G_t = PA_t / d_t and 2^G_t / lambda_t = PA_t / n_t.
+                // n, d and PA are kept as float times 2^E (n, d) and 2^F (PA); every 8
+                // tokens they are rescaled by exact powers of two.
+                float nn = lam, dd = 1.0f, pa = 1.0f;
+                int E = 0, F = 0;
+                int SG[kC / 8];
 #pragma unroll
                 for (int j = 0; j < kSlots; ++j) {
                     if (ok) ok = waitw(&ring_full[j], c & 1, abort_flag, g.status);
                     if (!ok) continue;
                     const float *ra = reinterpret_cast<const float *>(sm + L::ring0) + j * 2 * L::SLOTF;
                     const float *rq = ra + L::SLOTF;
-                    float gam = (j == 0) ? 0.f : G[16 * j - 1];
 #pragma unroll
                     for (int r = 0; r < kSlotTok; ++r) {
                         const int tau = kSlotTok * j + r;
-                        const long long tok = tok0 + tau;
-                        if (key && tok < te) {
-                            const float at = ra[r * DK + i], qnt = rq[r * DK + i];
-                            const float kk = bf_at(kt, sw_off(tau, i, kC));
-                            const float bt = __ldg(g.beta + tok * g.H + h);
-                            const float den = fmaf(at, at, qnt * lam);
-                            const float rr = __frcp_rn(den);
-                            lam = fmaf(bt * kk, kk, lam * rr);
-                            gam += __log2f(at * rr);
+                        const bool valid = tok0 + tau < te;
+                        const float bt = __shfl_sync(0xffffffffu, tau < 32 ? cb0 : cb1, tau & 31);
+                        const float kk = bf_at(kt, sw_off(tau, i, kC));
+                        const float at = valid ? ra[r * DK + i] : 1.f;
+                        const float qnt = valid ? rq[r * DK + i] : 0.f;
+                        const float b = valid ? bt * kk * kk : 0.f;
+                        dd = fmaf(at * at, dd, qnt * nn);
+                        nn = fmaf(b, dd, nn);
+                        pa *= at;
+                        const float fk = __fdividef(dd, pa);      // 2^-G_t  / 2^(E-F)
+                        FQ[tau] = __fdividef(pa, nn);             // 2^G_t/lambda_t / 2^(F-E)
+                        FK[tau] = fk;
+                        const int gi = (F - E) - (((__float_as_int(fk) >> 23) & 0xff) - 127);
+                        gmin = min(gmin, gi);
+                        gmax = max(gmax, gi);
+                        if ((tau & 7) == 7) {
+                            SG[tau >> 3] = F - E;
+                            const int e = ((__float_as_int(dd) >> 23) & 0xff) - 127;
+                            const int f = ((__float_as_int(pa) >> 23) & 0xff) - 127;
+                            const float se = __int_as_float((127 - e) << 23);
+                            nn *= se;
+                            dd *= se;
+                            pa *= __int_as_float((127 - f) << 23);
+                            E += e;
+                            F += f;
                         }
-                        G[tau] = gam;
-                        A[tau] = gam - __log2f(lam);
-                        gmin = fminf(gmin, gam);
-                        gmax = fmaxf(gmax, gam);
                     }
                     mbar_arrive(&ring_empty[j]);
                 }
                 if (!ok) break;
-                R = 0.5f * (gmin + gmax);
-                Glast = G[kC - 1];
+                lam = nn / dd;
+                R = (gmin + gmax) >> 1;
+                glast_m = 1.0f / FK[kC - 1];
+                s_last = SG[kC / 8 - 1];
+                if (gmax - gmin > (int)kMaxSpan && key) atomicOr(g.status, kStatusRange);
+                // the K'-low tile is single-buffered: the previous chunk's state update must be done
+                if (c > 0 && !waitw(u_done, (c - 1) & 1, abort_flag, g.status)) { ok = false; break; }
+                uint8_t *klo = sm + L::klo0;
+                // ---- pass 2 (dk = 64: the two halves of the gate group split the tokens)
+                const int half = (DK == 64) ? (tid >> 6) : 0;
+#pragma unroll
+                for (int grp = 0; grp < kC / 8; ++grp) {
+                    if (DK == 64 && (grp >> 2) != half) continue;
+                    const int sh = SG[grp] - R;
+                    const float mq = __int_as_float((127 + max(-126, min(127, sh))) << 23);
+                    const float mk = __int_as_float((127 + max(-126, min(127, -sh))) << 23);
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) {
+                        const int tau = grp * 8 + r;
+                        const float bt = __shfl_sync(0xffffffffu, tau < 32 ? cb0 : cb1, tau & 31);
+                        if (key) {
+                            const int off = sw_off(tau, i, kC);
+                            float qv = 0.f, kv = 0.f;
+                            if (tok0 + tau < te) {
+                                if (!state_mode) qv = bf_at(qt, off) * (FQ[tau] * mq);
+                                kv = bt * bf_at(kt, off) * (FK[tau] * mk);
+                            }
+                            if (!state_mode) bf_put(qt, off, qv);
+                            const __nv_bfloat16 khi = __float2bfloat16_rn(kv);
+                            *reinterpret_cast<__nv_bfloat16 *>(kt + off) = khi;
+                            bf_put(klo, off, kv - __bfloat162float(khi));
+                        }
+                    }
+                }
             } else {
                 // isotropic: one precision per head; warp-level Moebius scan over
                 // the chunk (lane l owns tokens 2l, 2l+1), redundantly per warp.
                 const int t0i = 2 * lane, t1i = 2 * lane + 1;
-                const long long ta = tok0 + t0i, tb2 = tok0 + t1i;
-                const bool va = ta < te, vb = tb2 < te;
-                float a0 = 1.f, q0 = 0.f, b0 = 0.f, a1 = 1.f, q1 = 0.f, b1 = 0.f;
+                const bool va = tok0 + t0i < te, vb = tok0 + t1i < te;
                 const float inv_dk = 1.0f / (float)DK;
-                if (va) {
-                    const long long th = ta * g.H + h;
-                    a0 = __ldg(g.a + th); q0 = __ldg(g.qn + th); bt_l0 = __ldg(g.beta + th);
-                    b0 = bt_l0 * row_sumsq<DK>(kt, t0i) * inv_dk;
-                }
-                if (vb) {
-                    const long long th = tb2 * g.H + h;
-                    a1 = __ldg(g.a + th); q1 = __ldg(g.qn + th); bt_l1 = __ldg(g.beta + th);
-                    b1 = bt_l1 * row_sumsq<DK>(kt, t1i) * inv_dk;
-                }
+                const float a0 = ca0, q0 = cq0, a1 = ca1, q1 = cq1;
+                const float b0 = va ? cb0 * row_sumsq<DK>(kt, t0i) * inv_dk : 0.f;
+                const float b1 = vb ? cb1 * row_sumsq<DK>(kt, t1i) * inv_dk : 0.f;
                 Mob Mp = mob_norm(mob_mul(mob_step(a1, q1, b1), mob_step(a0, q0, b0)));
 #pragma unroll
                 for (int d = 1; d < 32; d <<= 1) {
                     Mob o = shfl_up_mob(Mp, d);
                     if (lane >= d) Mp = mob_norm(mob_mul(Mp, o));
                 }
-                Mob E = shfl_up_mob(Mp, 1);
-                if (lane == 0) E = Mob{1.f, 0.f, 0.f, 1.f};
-                const float lamA = mob_apply(E, lam);
+                Mob Ex = shfl_up_mob(Mp, 1);
+                if (lane == 0) Ex = Mob{1.f, 0.f, 0.f, 1.f};
+                const float lamA = mob_apply(Ex, lam);
                 float g0 = 1.f, lamB = lamA, g1 = 1.f, lamC;
                 if (va) { float rr = __frcp_rn(fmaf(a0, a0, q0 * lamA)); g0 = a0 * rr; lamB = fmaf(lamA, rr, b0); }
                 lamC = lamB;
@@ -314,66 +385,60 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     if (lane >= d) sum += o;
                 }
                 const float G1 = sum, G0 = sum - l1;
-                const float A0 = G0 - __log2f(lamB), A1 = G1 - __log2f(lamC);
                 float mn = fminf(0.f, fminf(G0, G1)), mx = fmaxf(0.f, fmaxf(G0, G1));
 #pragma unroll
                 for (int d = 16; d > 0; d >>= 1) {
                     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, d));
                     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, d));
                 }
-                gmin = mn; gmax = mx;
-                R = 0.5f * (gmin + gmax);
-                Glast = __shfl_sync(0xffffffffu, G1, 31);
+                gmin = (int)floorf(mn); gmax = (int)ceilf(mx);
+                R = (gmin + gmax) >> 1;
+                const float Rf = (float)R;
+                const float Glast = __shfl_sync(0xffffffffu, G1, 31);
+                glast_m = exp2f(Glast);
+                s_last = 0;
                 lam = __shfl_sync(0xffffffffu, lamC, 31);
+                // per-token factors, shared by all keys of the head
+                const float fq0 = exp2f(G0 - Rf) / lamB, fq1 = exp2f(G1 - Rf) / lamC;
+                const float fk0 = exp2f(Rf - G0), fk1 = exp2f(Rf - G1);
+                if (gmax - gmin > (int)kMaxSpan && key) atomicOr(g.status, kStatusRange);
                 // every gate warp has read the raw k rows before any overwrites them
                 mbar_arrive(gate_sync);
                 if (!waitw(gate_sync, c & 1, abort_flag, g.status)) { ok = false; break; }
+                if (c > 0 && !waitw(u_done, (c - 1) & 1, abort_flag, g.status)) { ok = false; break; }
+                uint8_t *klo = sm + L::klo0;
+                const int half = (DK == 64) ? (tid >> 6) : 0;
 #pragma unroll
                 for (int tau = 0; tau < kC; ++tau) {
-                    const float gg0 = __shfl_sync(0xffffffffu, G0, tau >> 1);
-                    const float gg1 = __shfl_sync(0xffffffffu, G1, tau >> 1);
-                    const float aa0 = __shfl_sync(0xffffffffu, A0, tau >> 1);
-                    const float aa1 = __shfl_sync(0xffffffffu, A1, tau >> 1);
-                    G[tau] = (tau & 1) ? gg1 : gg0;
-                    A[tau] = (tau & 1) ? aa1 : aa0;
-                }
-            }
-            if (gmax - gmin > kMaxSpan && key) atomicOr(g.status, kStatusRange);
-            // the K'-low tile is single-buffered: the previous chunk's state update must be done
-            if (c > 0 && !waitw(u_done, (c - 1) & 1, abort_flag, g.status)) { ok = false; break; }
-            uint8_t *klo = sm + L::klo0;
-            // ---- pass 2: fold 1/lambda, beta and the log-gates into Q', K' (in place)
-#pragma unroll
-            for (int tau = 0; tau < kC; ++tau) {
-                const long long tok = tok0 + tau;
-                float bt = 0.f;
-                if (g.iso) {
-                    const float x0 = __shfl_sync(0xffffffffu, bt_l0, tau >> 1);
-                    const float x1 = __shfl_sync(0xffffffffu, bt_l1, tau >> 1);
-                    bt = (tau & 1) ? x1 : x0;
-                }
-                if (key) {
-                    const int off = sw_off(tau, i, kC);
-                    float qv = 0.f, kv = 0.f;
-                    if (tok < te) {
-                        if (!g.iso) bt = __ldg(g.beta + tok * g.H + h);
-                        if (!state_mode) qv = bf_at(qt, off) * exp2f(A[tau] - R);
-                        kv = bt * bf_at(kt, off) * exp2f(R - G[tau]);
+                    const float fq = __shfl_sync(0xffffffffu, (tau & 1) ? fq1 : fq0, tau >> 1);
+                    const float fk = __shfl_sync(0xffffffffu, (tau & 1) ? fk1 : fk0, tau >> 1);
+                    const float bt = __shfl_sync(0xffffffffu, (tau & 1) ? cb1 : cb0, tau >> 1);
+                    if (DK == 64 && (tau >> 5) != half) continue;
+                    if (key) {
+                        const int off = sw_off(tau, i, kC);
+                        float qv = 0.f, kv = 0.f;
+                        if (tok0 + tau < te) {
+                            if (!state_mode) qv = bf_at(qt, off) * fq;
+                            kv = bt * bf_at(kt, off) * fk;
+                        }
+                        if (!state_mode) bf_put(qt, off, qv);
+                        const __nv_bfloat16 khi = __float2bfloat16_rn(kv);
+                        *reinterpret_cast<__nv_bfloat16 *>(kt + off) = khi;
+                        bf_put(klo, off, kv - __bfloat162float(khi));
                     }
-                    if (!state_mode) bf_put(qt, off, qv);
-                    // K' = hi + lo in two bf16 parts: the state update sums K'^T V over
-                    // whole segments, so it gets (nearly) fp32 operands; the scores use hi.
-                    const __nv_bfloat16 khi = __float2bfloat16_rn(kv);
-                    *reinterpret_cast<__nv_bfloat16 *>(kt + off) = khi;
-                    bf_put(klo, off, kv - __bfloat162float(khi));
                 }
             }
-            if (key) {
-                fac[s * DK + i] = exp2f(R + e_prev);
-                if (c == nchunks - 1) fac_final[i] = exp2f(Glast - R);
+            // state rescale factors: U_c = diag(2^R_c) S_c, S_{c+1} = diag(2^(G_last - R_c)) (U_c + K'^T V)
+            {
+                const float glast_shift = __int_as_float((127 + max(-126, min(127, s_last - R))) << 23);
+                const float e_cur = glast_m * glast_shift;        // 2^(G_last - R)
+                if (key) {
+                    fac[s * DK + i] = e_prev * __int_as_float((127 + max(-126, min(127, R))) << 23);
+                    if (c == nchunks - 1) fac_final[i] = e_cur;
+                }
+                e_prev = e_cur;
+                log_decay += (float)s_last + __log2f(glast_m);
             }
-            e_prev = Glast - R;
-            log_decay += Glast;
             fence_proxy_async();
             mbar_arrive(&qk_ready[s]);
         }
