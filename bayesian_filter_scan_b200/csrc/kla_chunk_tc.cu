@@ -318,6 +318,9 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                             F += f;
                         }
                     }
+                    // The slot is refilled by TMA (async proxy) once every gate thread
+                    // released it: order this thread's generic reads of the slot first.
+                    fence_proxy_async();
                     mbar_arrive(&ring_empty[j]);
                 }
                 if (!ok) break;
