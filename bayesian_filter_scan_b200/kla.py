@@ -25,7 +25,7 @@ KLA_DIAG, KLA_ISO = 0, 1
 EXPORTS = ("kla_workspace_bytes", "kla_precision_workspace_bytes", "kla_forward", "kla_forward_profiled",
            "kla_plan", "kla_precision",
            "kla_decode_step", "kla_host_device_bytes", "kla_forward_host", "kla_check",
-           "kla_status_string", "kla_version")
+           "kla_status_string", "kla_version", "kla_forward_noalloc")
 
 
 class KlaError(RuntimeError):
@@ -72,6 +72,8 @@ def lib():
         L.kla_host_device_bytes.restype = ctypes.c_size_t
         L.kla_forward_host.argtypes = [D] + [_P] * 11 + [_P, ctypes.c_size_t, _P]
         L.kla_forward_host.restype = ctypes.c_int
+        L.kla_forward_noalloc.argtypes = [D] + [_P] * 11 + [_P]
+        L.kla_forward_noalloc.restype = ctypes.c_int
         L.kla_check.argtypes = [_P]
         L.kla_check.restype = ctypes.c_int
         L.kla_status_string.argtypes = [ctypes.c_int]
@@ -215,6 +217,26 @@ def forward_host(desc: KlaDesc, q, k, v, a, qn, beta, out, lambda0=None, eta0=No
                                _ptr(device_buffer), nbytes, st)
     _check(s, "kla_forward_host")
     return out
+
+
+def forward_noalloc(q, k, v, a, qn, beta, lambda0=None, eta0=None, B=None, T=None, mode="diag",
+                    final_state=False, out=None):
+    """kla_forward_noalloc: the forward pass with the library's fixed device
+    scratch area as workspace, for callers that cannot allocate device memory
+    (outputs passed in via ``out`` are used as given)."""
+    m = _mode(mode)
+    desc, N = _desc_from(q, v, B, T, m, None)
+    H, dk, dv = q.shape[1], q.shape[2], v.shape[2]
+    if out is None:
+        out = torch.empty(q.shape[0], H, dv, dtype=q.dtype, device=q.device)
+    fl = fe = None
+    if final_state:
+        fl = torch.empty((N, H) if m == KLA_ISO else (N, H, dk), dtype=torch.float32, device=q.device)
+        fe = torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device)
+    s = lib().kla_forward_noalloc(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(qn), _ptr(beta),
+                                  _ptr(lambda0), _ptr(eta0), _ptr(out), _ptr(fl), _ptr(fe), _stream())
+    _check(s, "kla_forward_noalloc")
+    return (out, fl, fe) if final_state else out
 
 
 def check(stream=None):

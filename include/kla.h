@@ -162,6 +162,33 @@ kla_status kla_forward_host(const kla_desc *desc,
                             void *device_buffer, size_t device_bytes,
                             cudaStream_t stream);
 
+/* Size of the fixed device scratch area kla_forward_noalloc uses, per GPU. */
+#define KLA_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* kla_forward for callers that cannot allocate device memory: code that runs
+ * inside an allocator or memory-pool callback, plug-ins whose host framework
+ * owns every device allocation, or processes that must keep a fixed device
+ * footprint after start-up. The pages have no counterpart of this call; it is
+ * plumbing around the same forward pass. Instead of a caller-provided
+ * workspace it uses a file-scope device array of KLA_NOALLOC_SCRATCH_BYTES,
+ * which every GPU that loads the library holds until the process exits.
+ * Arguments, layouts and errors as kla_forward. A descriptor whose
+ * kla_workspace_bytes exceeds KLA_NOALLOC_SCRATCH_BYTES (long rows with few
+ * heads, e.g. 16 heads x 128k tokens at dk = dv = 128) returns
+ * KLA_ERR_UNSUPPORTED before any launch. The first call on each device looks
+ * up the array's device address (cudaGetSymbolAddress), so make that first
+ * call before any stream capture. All calls share the one array: nothing in
+ * it needs to start at zero (each call writes every scratch value before
+ * reading it), but calls whose GPU work overlaps -- on different streams or
+ * from different host threads -- race on it and must be serialised by the
+ * caller. Never allocates, never synchronises. */
+kla_status kla_forward_noalloc(const kla_desc *desc,
+                               const void *q, const void *k, const void *v,
+                               const float *a, const float *qn, const float *beta,
+                               const float *lambda0, const float *eta0,
+                               void *out, float *final_lambda, float *final_eta,
+                               cudaStream_t stream);
+
 /* Synchronises `stream`, then reads and clears the library's device status
  * word on the current device: KLA_OK, KLA_ERR_RANGE or KLA_ERR_TIMEOUT from any
  * kernel that ran since the last check, or KLA_ERR_CUDA if the stream failed. */
