@@ -46,11 +46,12 @@ using namespace ptx;
 namespace {
 
 constexpr int kC = 64;             // chunk tokens
-constexpr int kSlotTok = 16;       // tokens per a/qn ring slot
-constexpr int kSlots = 4;          // ring depth (one chunk)
+constexpr int kSlotTok = 8;        // tokens per a/qn ring slot
+constexpr int kSlots = 6;          // ring depth (48 tokens of look-ahead)
+constexpr int kSlotsPerChunk = kC / kSlotTok;
+constexpr int kMaxOffset = 110;    // |G - R| (log2) kept inside the fp32/bf16 exponent range
 constexpr int kThreads = 320;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
-constexpr float kMaxSpan = 200.0f; // log2 span of G per key per chunk kept exact
 
 struct TcArgs {
     int N, H, P, NB, seg_blocks, iso, mode;
@@ -76,12 +77,12 @@ struct Layout {
     static constexpr int v0 = k0 + 2 * QK;
     static constexpr int p0 = v0 + 2 * V;
     static constexpr int ub0 = p0 + PT;
-    static constexpr int klo0 = ub0 + UB;          // low bf16 part of K' (state update)
-    static constexpr int ring0 = klo0 + QK;
+    static constexpr int klo0 = ub0 + UB;          // low bf16 part of K' (state update), per stage
+    static constexpr int ring0 = klo0 + 2 * QK;
     static constexpr int fac0 = ring0 + kSlots * 2 * SLOTF * 4;
     static constexpr int facf0 = fac0 + 2 * DK * 4;
     static constexpr int bar0 = ((facf0 + DK * 4) + 7) & ~7;
-    static constexpr int NBAR = 22;
+    static constexpr int NBAR = 6 + 2 * kSlots + 8;
     static constexpr int hold0 = bar0 + NBAR * 8;
     static constexpr int bytes = hold0 + 16;
     static constexpr int alloc = bytes + 1024;
@@ -167,9 +168,9 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::bar0);
     uint64_t *stage_full = bars + 0, *stage_empty = bars + 2, *qk_ready = bars + 4;
-    uint64_t *ring_full = bars + 6, *ring_empty = bars + 10;
-    uint64_t *s_full = bars + 14, *u_ready = bars + 15, *u_done = bars + 16, *p_full = bars + 17;
-    uint64_t *o_full = bars + 18, *o_empty = bars + 19, *td_bar = bars + 20, *gate_sync = bars + 21;
+    uint64_t *ring_full = bars + 6, *ring_empty = bars + 6 + kSlots;
+    uint64_t *s_full = bars + 6 + 2 * kSlots, *u_ready = s_full + 1, *u_done = s_full + 2, *p_full = s_full + 3;
+    uint64_t *o_full = s_full + 4, *o_empty = s_full + 5, *td_bar = s_full + 6, *gate_sync = s_full + 7;
     uint32_t *tmem_hold = reinterpret_cast<uint32_t *>(sm + L::hold0);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::hold0 + 4);
     float *fac = reinterpret_cast<float *>(sm + L::fac0);
@@ -177,6 +178,9 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool state_mode = g.mode == 1;
+    // gate threads that take part: one per key in diagonal mode (each thread reads
+    // and rewrites only its own key column in place), the whole group in iso mode
+    const int gate_threads = g.iso ? 128 : DK;
     const int P_eff = state_mode ? g.P - 1 : g.P;
     const long long u = blockIdx.x / P_eff;
     const int p = (int)(blockIdx.x % P_eff);
@@ -194,11 +198,11 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         for (int s = 0; s < 2; ++s) {
             mbar_init(&stage_full[s], 1);
             mbar_init(&stage_empty[s], 1);
-            mbar_init(&qk_ready[s], 128);
+            mbar_init(&qk_ready[s], gate_threads);
         }
         for (int j = 0; j < kSlots; ++j) {
             mbar_init(&ring_full[j], 1);
-            mbar_init(&ring_empty[j], 128);
+            mbar_init(&ring_empty[j], gate_threads);
         }
         mbar_init(s_full, 1);
         mbar_init(u_ready, 128);
@@ -222,9 +226,11 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const uint32_t tbase = *tmem_hold;
 
     if (warp < 4) {
+      if (tid < gate_threads) {
         // ================= gate warps: precision path and operand folding =====
-        // key owned by this thread; with dk = 64 both halves of the gate group
-        // run the recursion for the same keys and split the operand writes
+        // key owned by this thread (isotropic mode with dk = 64: both halves of the
+        // gate group own the same keys and split the tokens of the operand writes,
+        // after a group barrier that follows every read of the raw k rows)
         const int i = tid & (DK - 1);
         const bool key = true;
         float lam = 1.0f;
@@ -236,6 +242,7 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
         }
         float e_prev = 1.f, log_decay = 0.f;   // e_prev = 2^(G_last - R) of the previous chunk
+        int r_next = 0;                           // reference predicted for the next chunk
         bool ok = true;
         // Per-token scalars of a chunk are loaded one chunk ahead into registers
         // and broadcast with shuffles (no global load sits on the recursion).
@@ -263,101 +270,90 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const float cb0 = nb0, cb1 = nb1, ca0 = na0, ca1 = na1, cq0 = nq0, cq1 = nq1;
             if (c + 1 < nchunks) prefetch(c + 1);
             if (!waitw(&stage_full[s], (c >> 1) & 1, abort_flag, g.status)) { ok = false; break; }
-            // Per token the gate warps produce two scale factors, applied in pass 2:
-            //   fq = 2^(G_t - R) / lambda_t   (query side),   fk = 2^(R - G_t)   (key side)
-            // with G_t the in-chunk cumulative log2-gate and R an integer reference at
-            // the middle of the chunk's G range (so neither factor leaves the exponent range).
-            float FQ[kC], FK[kC];
-            int gmin = 0, gmax = 0, R;
-            float glast_m;        // 2^G_last = glast_m * 2^s_last
-            int s_last;
+            int R;                 // integer log2 reference of this chunk (per key)
+            float e_cur;           // 2^(G_last - R)
+            float glast_log2;      // G_last
+            uint8_t *klo = sm + L::klo0 + s * L::QK;
             if (!g.iso) {
-                // Projective form of the precision: lambda = n/d with
+                // One pass per chunk. Projective form of the precision: lambda = n/d with
                 //   d <- a^2 d + qn n,  n <- n + b d   (b = beta k^2),
                 // two FMAs per token on the serial chain. The gate is g = a d_prev / d,
                 // so with PA = prod a the cumulative gate telescopes (d = 1 at the chunk
-                // start): 2^G_t = PA_t / d_t and 2^G_t / lambda_t = PA_t / n_t.
-                // n, d and PA are kept as float times 2^E (n, d) and 2^F (PA); every 8
-                // tokens they are rescaled by exact powers of two.
+                // start): 2^G = PA/d and 2^G/lambda = PA/n. n, d and PA are floats times
+                // 2^E (n, d) and 2^F (PA), rescaled by exact powers of two every 8 tokens.
+                // The operands are written at once against the reference R predicted
+                // from the previous chunk's decay; the chunk's actual G range is checked.
+                R = r_next;
                 float nn = lam, dd = 1.0f, pa = 1.0f;
-                int E = 0, F = 0;
-                int SG[kC / 8];
-#pragma unroll
-                for (int j = 0; j < kSlots; ++j) {
-                    if (ok) ok = waitw(&ring_full[j], c & 1, abort_flag, g.status);
-                    if (!ok) continue;
-                    const float *ra = reinterpret_cast<const float *>(sm + L::ring0) + j * 2 * L::SLOTF;
+                int E = 0, F = 0, gmin = 0, gmax = 0;
+                float mq = __int_as_float((127 - R) << 23), mk = __int_as_float((127 + R) << 23);
+#pragma unroll 1
+                for (int j = 0; j < kSlotsPerChunk; ++j) {
+                    const int n = c * kSlotsPerChunk + j, slot = n % kSlots;
+                    if (!waitw(&ring_full[slot], (n / kSlots) & 1, abort_flag, g.status)) { ok = false; break; }
+                    const float *ra = reinterpret_cast<const float *>(sm + L::ring0) + slot * 2 * L::SLOTF;
                     const float *rq = ra + L::SLOTF;
+                    const float bsrc = (j < 4) ? cb0 : cb1;
 #pragma unroll
                     for (int r = 0; r < kSlotTok; ++r) {
                         const int tau = kSlotTok * j + r;
                         const bool valid = tok0 + tau < te;
-                        const float bt = __shfl_sync(0xffffffffu, tau < 32 ? cb0 : cb1, tau & 31);
-                        const float kk = bf_at(kt, sw_off(tau, i, kC));
+                        const float bt = __shfl_sync(0xffffffffu, bsrc, tau & 31);
+                        const int off = sw_off(tau, i, kC);
+                        const float kk = bf_at(kt, off);
                         const float at = valid ? ra[r * DK + i] : 1.f;
                         const float qnt = valid ? rq[r * DK + i] : 0.f;
                         const float b = valid ? bt * kk * kk : 0.f;
                         dd = fmaf(at * at, dd, qnt * nn);
                         nn = fmaf(b, dd, nn);
                         pa *= at;
-                        const float fk = __fdividef(dd, pa);      // 2^-G_t  / 2^(E-F)
-                        FQ[tau] = __fdividef(pa, nn);             // 2^G_t/lambda_t / 2^(F-E)
-                        FK[tau] = fk;
-                        const int gi = (F - E) - (((__float_as_int(fk) >> 23) & 0xff) - 127);
-                        gmin = min(gmin, gi);
-                        gmax = max(gmax, gi);
-                        if ((tau & 7) == 7) {
-                            SG[tau >> 3] = F - E;
-                            const int e = ((__float_as_int(dd) >> 23) & 0xff) - 127;
-                            const int f = ((__float_as_int(pa) >> 23) & 0xff) - 127;
-                            const float se = __int_as_float((127 - e) << 23);
-                            nn *= se;
-                            dd *= se;
-                            pa *= __int_as_float((127 - f) << 23);
-                            E += e;
-                            F += f;
-                        }
-                    }
-                    // The slot is refilled by TMA (async proxy) once every gate thread
-                    // released it: order this thread's generic reads of the slot first.
-                    fence_proxy_async();
-                    mbar_arrive(&ring_empty[j]);
-                }
-                if (!ok) break;
-                lam = nn / dd;
-                R = (gmin + gmax) >> 1;
-                glast_m = 1.0f / FK[kC - 1];
-                s_last = SG[kC / 8 - 1];
-                if (gmax - gmin > (int)kMaxSpan && key) atomicOr(g.status, kStatusRange);
-                // the K'-low tile is single-buffered: the previous chunk's state update must be done
-                if (c > 0 && !waitw(u_done, (c - 1) & 1, abort_flag, g.status)) { ok = false; break; }
-                uint8_t *klo = sm + L::klo0;
-                // ---- pass 2 (dk = 64: the two halves of the gate group split the tokens)
-                const int half = (DK == 64) ? (tid >> 6) : 0;
-#pragma unroll
-                for (int grp = 0; grp < kC / 8; ++grp) {
-                    if (DK == 64 && (grp >> 2) != half) continue;
-                    const int sh = SG[grp] - R;
-                    const float mq = __int_as_float((127 + max(-126, min(127, sh))) << 23);
-                    const float mk = __int_as_float((127 + max(-126, min(127, -sh))) << 23);
-#pragma unroll
-                    for (int r = 0; r < 8; ++r) {
-                        const int tau = grp * 8 + r;
-                        const float bt = __shfl_sync(0xffffffffu, tau < 32 ? cb0 : cb1, tau & 31);
-                        if (key) {
-                            const int off = sw_off(tau, i, kC);
+                        {
+                            const float rk = __fdividef(dd, pa);            // 2^-G * 2^(F-E)
+                            const int gi = (F - E) - (((__float_as_int(rk) >> 23) & 0xff) - 127);
+                            gmin = min(gmin, gi);
+                            gmax = max(gmax, gi);
                             float qv = 0.f, kv = 0.f;
-                            if (tok0 + tau < te) {
-                                if (!state_mode) qv = bf_at(qt, off) * (FQ[tau] * mq);
-                                kv = bt * bf_at(kt, off) * (FK[tau] * mk);
+                            if (valid) {
+                                if (!state_mode) qv = bf_at(qt, off) * (__fdividef(pa, nn) * mq);
+                                kv = bt * kk * (rk * mk);
                             }
                             if (!state_mode) bf_put(qt, off, qv);
+                            // K' = hi + lo in two bf16 parts: the state update sums K'^T V
+                            // over whole segments, so it gets (nearly) fp32 operands.
                             const __nv_bfloat16 khi = __float2bfloat16_rn(kv);
                             *reinterpret_cast<__nv_bfloat16 *>(kt + off) = khi;
                             bf_put(klo, off, kv - __bfloat162float(khi));
                         }
                     }
+                    // exact power-of-two rescale of (n, d) and PA
+                    {
+                        const int e = ((__float_as_int(dd) >> 23) & 0xff) - 127;
+                        const int f = ((__float_as_int(pa) >> 23) & 0xff) - 127;
+                        const float se = __int_as_float((127 - e) << 23);
+                        nn *= se;
+                        dd *= se;
+                        pa *= __int_as_float((127 - f) << 23);
+                        E += e;
+                        F += f;
+                        const int sh = max(-126, min(127, (F - E) - R));
+                        mq = __int_as_float((127 + sh) << 23);
+                        mk = __int_as_float((127 - sh) << 23);
+                    }
+                    // the slot is refilled by TMA (async proxy) once every gate thread
+                    // released it: order this thread's generic reads of the slot first
+                    fence_proxy_async();
+                    mbar_arrive(&ring_empty[slot]);
                 }
+                if (!ok) break;
+                lam = nn / dd;
+                const float gm = pa / dd;                 // 2^G_last = gm * 2^(F-E)
+                const int sl = F - E;
+                e_cur = gm * __int_as_float((127 + max(-126, min(127, sl - R))) << 23);
+                glast_log2 = (float)sl + __log2f(gm);
+                if (gmax - R > kMaxOffset || R - gmin > kMaxOffset) atomicOr(g.status, kStatusRange);
+                // predicted middle of the next chunk's G range (same decay rate)
+                const int gl = sl + (((__float_as_int(gm) >> 23) & 0xff) - 127);
+                r_next = max(-kMaxOffset, min(kMaxOffset, gl / 2));
             } else {
                 // isotropic: one precision per head; warp-level Moebius scan over
                 // the chunk (lane l owns tokens 2l, 2l+1), redundantly per warp.
@@ -394,22 +390,20 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, d));
                     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, d));
                 }
-                gmin = (int)floorf(mn); gmax = (int)ceilf(mx);
+                const int gmin = (int)floorf(mn), gmax = (int)ceilf(mx);
                 R = (gmin + gmax) >> 1;
                 const float Rf = (float)R;
                 const float Glast = __shfl_sync(0xffffffffu, G1, 31);
-                glast_m = exp2f(Glast);
-                s_last = 0;
+                e_cur = exp2f(Glast - Rf);
+                glast_log2 = Glast;
                 lam = __shfl_sync(0xffffffffu, lamC, 31);
                 // per-token factors, shared by all keys of the head
                 const float fq0 = exp2f(G0 - Rf) / lamB, fq1 = exp2f(G1 - Rf) / lamC;
                 const float fk0 = exp2f(Rf - G0), fk1 = exp2f(Rf - G1);
-                if (gmax - gmin > (int)kMaxSpan && key) atomicOr(g.status, kStatusRange);
+                if (gmax - gmin > 2 * kMaxOffset) atomicOr(g.status, kStatusRange);
                 // every gate warp has read the raw k rows before any overwrites them
                 mbar_arrive(gate_sync);
                 if (!waitw(gate_sync, c & 1, abort_flag, g.status)) { ok = false; break; }
-                if (c > 0 && !waitw(u_done, (c - 1) & 1, abort_flag, g.status)) { ok = false; break; }
-                uint8_t *klo = sm + L::klo0;
                 const int half = (DK == 64) ? (tid >> 6) : 0;
 #pragma unroll
                 for (int tau = 0; tau < kC; ++tau) {
@@ -417,31 +411,23 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const float fk = __shfl_sync(0xffffffffu, (tau & 1) ? fk1 : fk0, tau >> 1);
                     const float bt = __shfl_sync(0xffffffffu, (tau & 1) ? cb1 : cb0, tau >> 1);
                     if (DK == 64 && (tau >> 5) != half) continue;
-                    if (key) {
-                        const int off = sw_off(tau, i, kC);
-                        float qv = 0.f, kv = 0.f;
-                        if (tok0 + tau < te) {
-                            if (!state_mode) qv = bf_at(qt, off) * fq;
-                            kv = bt * bf_at(kt, off) * fk;
-                        }
-                        if (!state_mode) bf_put(qt, off, qv);
-                        const __nv_bfloat16 khi = __float2bfloat16_rn(kv);
-                        *reinterpret_cast<__nv_bfloat16 *>(kt + off) = khi;
-                        bf_put(klo, off, kv - __bfloat162float(khi));
+                    const int off = sw_off(tau, i, kC);
+                    float qv = 0.f, kv = 0.f;
+                    if (tok0 + tau < te) {
+                        if (!state_mode) qv = bf_at(qt, off) * fq;
+                        kv = bt * bf_at(kt, off) * fk;
                     }
+                    if (!state_mode) bf_put(qt, off, qv);
+                    const __nv_bfloat16 khi = __float2bfloat16_rn(kv);
+                    *reinterpret_cast<__nv_bfloat16 *>(kt + off) = khi;
+                    bf_put(klo, off, kv - __bfloat162float(khi));
                 }
             }
             // state rescale factors: U_c = diag(2^R_c) S_c, S_{c+1} = diag(2^(G_last - R_c)) (U_c + K'^T V)
-            {
-                const float glast_shift = __int_as_float((127 + max(-126, min(127, s_last - R))) << 23);
-                const float e_cur = glast_m * glast_shift;        // 2^(G_last - R)
-                if (key) {
-                    fac[s * DK + i] = e_prev * __int_as_float((127 + max(-126, min(127, R))) << 23);
-                    if (c == nchunks - 1) fac_final[i] = e_cur;
-                }
-                e_prev = e_cur;
-                log_decay += (float)s_last + __log2f(glast_m);
-            }
+            fac[s * DK + i] = e_prev * __int_as_float((127 + max(-126, min(127, R))) << 23);
+            if (c == nchunks - 1) fac_final[i] = e_cur;
+            e_prev = e_cur;
+            log_decay += glast_log2;
             fence_proxy_async();
             mbar_arrive(&qk_ready[s]);
         }
@@ -452,6 +438,7 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (g.iso ? (tid == 0) : key) g.final_lambda[u * (g.iso ? 1 : DK) + (g.iso ? 0 : i)] = lam;
             }
         }
+      }
     } else if (warp < 8) {
         // ================= epilogue warps ====================================
         const int e = tid - 128, we = e >> 5, le = e & 31;
@@ -592,21 +579,11 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     } else if (warp == 8) {
         // ================= TMA producer =====================================
         if (lane == 0) {
-            int last_ring = -1, last_stage[2] = {-1, -1};
+            int last_ring[kSlots], last_stage[2] = {-1, -1};
+            for (int j = 0; j < kSlots; ++j) last_ring[j] = -1;
             bool ok = true;
             for (int c = 0; c < nchunks && ok; ++c) {
                 const int tok0 = (int)(tb + (long long)c * kC);
-                if (!g.iso) {
-                    for (int j = 0; j < kSlots; ++j) {
-                        if (c > 0 && !wait1(&ring_empty[j], (c - 1) & 1, abort_flag, g.status)) { ok = false; break; }
-                        float *ra = reinterpret_cast<float *>(sm + L::ring0) + j * 2 * L::SLOTF;
-                        mbar_expect_tx(&ring_full[j], 2 * L::SLOTF * 4);
-                        tma_load_3d(ra, &tm_a, &ring_full[j], 0, h, tok0 + kSlotTok * j);
-                        tma_load_3d(ra + L::SLOTF, &tm_qn, &ring_full[j], 0, h, tok0 + kSlotTok * j);
-                    }
-                    if (!ok) break;
-                    last_ring = c;
-                }
                 const int s = c & 1;
                 if (c >= 2 && !wait1(&stage_empty[s], ((c >> 1) - 1) & 1, abort_flag, g.status)) { ok = false; break; }
                 mbar_expect_tx(&stage_full[s], (state_mode ? 0 : L::QK) + L::QK + L::V);
@@ -620,11 +597,26 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 for (int a = 0; a < DV / 64; ++a)
                     tma_load_3d(sm + L::v0 + s * L::V + a * kC * 128, &tm_v, &stage_full[s], 64 * a, h, tok0);
                 last_stage[s] = c;
+                if (!g.iso) {
+                    for (int j = 0; j < kSlotsPerChunk; ++j) {
+                        const int n = c * kSlotsPerChunk + j, slot = n % kSlots;
+                        if (n >= kSlots && !wait1(&ring_empty[slot], ((n / kSlots) - 1) & 1, abort_flag, g.status)) {
+                            ok = false;
+                            break;
+                        }
+                        float *ra = reinterpret_cast<float *>(sm + L::ring0) + slot * 2 * L::SLOTF;
+                        mbar_expect_tx(&ring_full[slot], 2 * L::SLOTF * 4);
+                        tma_load_3d(ra, &tm_a, &ring_full[slot], 0, h, tok0 + kSlotTok * j);
+                        tma_load_3d(ra + L::SLOTF, &tm_qn, &ring_full[slot], 0, h, tok0 + kSlotTok * j);
+                        last_ring[slot] = n;
+                    }
+                }
             }
             if (!ok || *abort_flag) {
                 // wait (bounded) until every copy this thread issued has landed
-                if (last_ring >= 0)
-                    for (int j = 0; j < kSlots; ++j) wait_slow(&ring_full[j], last_ring & 1, abort_flag, g.status, false);
+                for (int j = 0; j < kSlots; ++j)
+                    if (last_ring[j] >= 0)
+                        wait_slow(&ring_full[j], (last_ring[j] / kSlots) & 1, abort_flag, g.status, false);
                 for (int s = 0; s < 2; ++s)
                     if (last_stage[s] >= 0)
                         wait_slow(&stage_full[s], (last_stage[s] >> 1) & 1, abort_flag, g.status, false);
@@ -637,7 +629,7 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             constexpr uint32_t iO = idesc_bf16(64, DV, false, true);
             constexpr uint32_t iU = idesc_bf16(DK, DV, true, true);
             const uint32_t tS = tbase + L::colS, tO = tbase + L::colO, tU = tbase + L::colU;
-            const uint32_t pa = smem_u32(sm + L::p0), uba = smem_u32(sm + L::ub0), kloa = smem_u32(sm + L::klo0);
+            const uint32_t pa = smem_u32(sm + L::p0), uba = smem_u32(sm + L::ub0);
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c & 1;
                 if (!wait1(&qk_ready[s], (c >> 1) & 1, abort_flag, g.status)) break;
@@ -645,6 +637,7 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const uint32_t qa = smem_u32(sm + L::q0 + s * L::QK);
                 const uint32_t ka = smem_u32(sm + L::k0 + s * L::QK);
                 const uint32_t va = smem_u32(sm + L::v0 + s * L::V);
+                const uint32_t kloa = smem_u32(sm + L::klo0 + s * L::QK);
                 if (!state_mode) {
                     if (c > 0 && !wait1(o_empty, (c - 1) & 1, abort_flag, g.status)) break;
                     tc_fence_after();
