@@ -50,7 +50,17 @@ constexpr int kSlotTok = 8;        // tokens per a/qn ring slot
 constexpr int kSlots = 6;          // ring depth (48 tokens of look-ahead)
 constexpr int kSlotsPerChunk = kC / kSlotTok;
 constexpr int kMaxOffset = 110;    // |G - R| (log2) kept inside the fp32/bf16 exponent range
-constexpr int kThreads = 320;
+// Warp roles. dk = 128: gate warps 0-3, epilogue 4-7, TMA producer 8, MMA 9.
+// dk = 64: gate warps 0 and 2, producer 1, MMA 3, epilogue 4-7 (8 warps, so
+// two CTAs fit on one SM when dv = 64 as well).
+template <int DK, int DV>
+struct Roles {
+    static constexpr int NGW = (DK == 64) ? 2 : 4;
+    static constexpr int THREADS = (NGW + 6) * 32;
+    static constexpr int MIN_BLOCKS = (DK == 64 && DV == 64) ? 2 : 1;
+    static constexpr int PRODW = (NGW == 2) ? 1 : 8;
+    static constexpr int MMAW = (NGW == 2) ? 3 : 9;
+};
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 struct TcArgs {
@@ -110,15 +120,14 @@ __device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
 __device__ __noinline__ bool wait_slow(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int *status,
                                        bool honour_abort) {
     const uint64_t t0 = globaltimer();
-    for (uint32_t it = 0;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63) == 63) {
-            if (honour_abort && *abort_flag) return false;
-            if (globaltimer() - t0 > kWaitLimitNs) {
-                *abort_flag = 1;
-                atomicOr(status, kStatusTimeout);
-                return false;
-            }
+    for (;;) {
+        // sleeps until the phase completes (or 0.1 ms), then re-checks the limits
+        if (mbar_try_wait_sleep(bar, parity, 100000u)) return true;
+        if (honour_abort && *abort_flag) return false;
+        if (globaltimer() - t0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            atomicOr(status, kStatusTimeout);
+            return false;
         }
     }
 }
@@ -159,11 +168,12 @@ __device__ __forceinline__ float row_sumsq(const uint8_t *ktile, int row) {
 }  // namespace
 
 template <int DK, int DV>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Roles<DK, DV>::THREADS, Roles<DK, DV>::MIN_BLOCKS)
 kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
                     const __grid_constant__ CUtensorMap tm_qn, const TcArgs g) {
     using L = Layout<DK, DV>;
+    using RL = Roles<DK, DV>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::bar0);
@@ -178,9 +188,10 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool state_mode = g.mode == 1;
-    // gate threads that take part: one per key in diagonal mode (each thread reads
-    // and rewrites only its own key column in place), the whole group in iso mode
-    const int gate_threads = g.iso ? 128 : DK;
+    // one gate thread per key: each reads and rewrites only its own key column
+    const int gate_threads = DK;
+    const bool is_gate = (RL::NGW == 4) ? (warp < 4) : (warp == 0 || warp == 2);
+    const int gt = (RL::NGW == 4) ? tid : ((warp >> 1) * 32 + lane);   // gate rank
     const int P_eff = state_mode ? g.P - 1 : g.P;
     const long long u = blockIdx.x / P_eff;
     const int p = (int)(blockIdx.x % P_eff);
@@ -211,27 +222,24 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mbar_init(o_full, 1);
         mbar_init(o_empty, 128);
         mbar_init(td_bar, 1);
-        mbar_init(gate_sync, 128);
+        mbar_init(gate_sync, gate_threads);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == 8 && lane == 0) {
+    if (warp == RL::PRODW && lane == 0) {
         prefetch_map(&tm_q); prefetch_map(&tm_k); prefetch_map(&tm_v);
         if (!g.iso) { prefetch_map(&tm_a); prefetch_map(&tm_qn); }
     }
-    if (warp == 9) tmem_alloc(tmem_hold, L::NCOLS);
+    if (warp == RL::MMAW) tmem_alloc(tmem_hold, L::NCOLS);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_hold;
 
-    if (warp < 4) {
-      if (tid < gate_threads) {
+    if (is_gate) {
+      {
         // ================= gate warps: precision path and operand folding =====
-        // key owned by this thread (isotropic mode with dk = 64: both halves of the
-        // gate group own the same keys and split the tokens of the operand writes,
-        // after a group barrier that follows every read of the raw k rows)
-        const int i = tid & (DK - 1);
+        const int i = gt;                    // key owned by this thread
         const bool key = true;
         float lam = 1.0f;
         {
@@ -284,6 +292,7 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 // The operands are written at once against the reference R predicted
                 // from the previous chunk's decay; the chunk's actual G range is checked.
                 R = r_next;
+                const int nvalid = (int)min((long long)kC, te - tok0);
                 float nn = lam, dd = 1.0f, pa = 1.0f;
                 int E = 0, F = 0, gmin = 0, gmax = 0;
                 float mq = __int_as_float((127 - R) << 23), mk = __int_as_float((127 + R) << 23);
@@ -294,36 +303,68 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const float *ra = reinterpret_cast<const float *>(sm + L::ring0) + slot * 2 * L::SLOTF;
                     const float *rq = ra + L::SLOTF;
                     const float bsrc = (j < 4) ? cb0 : cb1;
+                    // Load the slot's inputs first (the tile is rewritten in place below,
+                    // so loads and stores are kept in separate phases), then release
+                    // the ring slot, then run the recursion, then write the operands.
+                    float kr[kSlotTok], qr[kSlotTok], ar[kSlotTok], qnr[kSlotTok], br[kSlotTok];
 #pragma unroll
                     for (int r = 0; r < kSlotTok; ++r) {
                         const int tau = kSlotTok * j + r;
-                        const bool valid = tok0 + tau < te;
-                        const float bt = __shfl_sync(0xffffffffu, bsrc, tau & 31);
                         const int off = sw_off(tau, i, kC);
-                        const float kk = bf_at(kt, off);
-                        const float at = valid ? ra[r * DK + i] : 1.f;
-                        const float qnt = valid ? rq[r * DK + i] : 0.f;
-                        const float b = valid ? bt * kk * kk : 0.f;
-                        dd = fmaf(at * at, dd, qnt * nn);
-                        nn = fmaf(b, dd, nn);
-                        pa *= at;
-                        {
-                            const float rk = __fdividef(dd, pa);            // 2^-G * 2^(F-E)
-                            const int gi = (F - E) - (((__float_as_int(rk) >> 23) & 0xff) - 127);
-                            gmin = min(gmin, gi);
-                            gmax = max(gmax, gi);
-                            float qv = 0.f, kv = 0.f;
-                            if (valid) {
-                                if (!state_mode) qv = bf_at(qt, off) * (__fdividef(pa, nn) * mq);
-                                kv = bt * kk * (rk * mk);
-                            }
-                            if (!state_mode) bf_put(qt, off, qv);
-                            // K' = hi + lo in two bf16 parts: the state update sums K'^T V
-                            // over whole segments, so it gets (nearly) fp32 operands.
-                            const __nv_bfloat16 khi = __float2bfloat16_rn(kv);
-                            *reinterpret_cast<__nv_bfloat16 *>(kt + off) = khi;
-                            bf_put(klo, off, kv - __bfloat162float(khi));
+                        kr[r] = bf_at(kt, off);
+                        qr[r] = state_mode ? 0.f : bf_at(qt, off);
+                        ar[r] = ra[r * DK + i];
+                        qnr[r] = rq[r * DK + i];
+                        br[r] = __shfl_sync(0xffffffffu, bsrc, tau & 31);
+                    }
+                    // the slot is refilled by TMA (async proxy) once every gate thread
+                    // released it: order this thread's generic reads of the slot first
+                    fence_proxy_async();
+                    mbar_arrive(&ring_empty[slot]);
+                    float qo[kSlotTok], ko[kSlotTok];
+                    float rkmin = 3.0e38f, rkmax = 0.f;
+                    if (nvalid >= kSlotTok * (j + 1)) {
+                        // every token of the slot is inside the segment
+#pragma unroll
+                        for (int r = 0; r < kSlotTok; ++r) {
+                            const float at = ar[r], bk = br[r] * kr[r];
+                            dd = fmaf(at * at, dd, qnr[r] * nn);
+                            nn = fmaf(bk * kr[r], dd, nn);
+                            pa *= at;
+                            const float rk = __fdividef(dd, pa);        // 2^-G * 2^(F-E)
+                            rkmin = fminf(rkmin, rk);
+                            rkmax = fmaxf(rkmax, rk);
+                            qo[r] = qr[r] * (__fdividef(pa, nn) * mq);
+                            ko[r] = bk * (rk * mk);
                         }
+                    } else {
+#pragma unroll
+                        for (int r = 0; r < kSlotTok; ++r) {
+                            const bool valid = kSlotTok * j + r < nvalid;
+                            const float at = valid ? ar[r] : 1.f;
+                            const float bk = valid ? br[r] * kr[r] : 0.f;
+                            dd = fmaf(at * at, dd, valid ? qnr[r] * nn : 0.f);
+                            nn = fmaf(bk * kr[r], dd, nn);
+                            pa *= at;
+                            const float rk = __fdividef(dd, pa);
+                            rkmin = fminf(rkmin, rk);
+                            rkmax = fmaxf(rkmax, rk);
+                            qo[r] = valid ? qr[r] * (__fdividef(pa, nn) * mq) : 0.f;
+                            ko[r] = bk * (rk * mk);
+                        }
+                    }
+                    // G = (F - E) - log2(rk); integer bounds of this slot's G range
+                    gmin = min(gmin, (F - E) - (((__float_as_int(rkmax) >> 23) & 0xff) - 126));
+                    gmax = max(gmax, (F - E) - (((__float_as_int(rkmin) >> 23) & 0xff) - 127));
+#pragma unroll
+                    for (int r = 0; r < kSlotTok; ++r) {
+                        const int off = sw_off(kSlotTok * j + r, i, kC);
+                        if (!state_mode) bf_put(qt, off, qo[r]);
+                        // K' = hi + lo in two bf16 parts: the state update sums K'^T V
+                        // over whole segments, so it gets (nearly) fp32 operands.
+                        const __nv_bfloat16 khi = __float2bfloat16_rn(ko[r]);
+                        *reinterpret_cast<__nv_bfloat16 *>(kt + off) = khi;
+                        bf_put(klo, off, ko[r] - __bfloat162float(khi));
                     }
                     // exact power-of-two rescale of (n, d) and PA
                     {
@@ -339,10 +380,6 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         mq = __int_as_float((127 + sh) << 23);
                         mk = __int_as_float((127 - sh) << 23);
                     }
-                    // the slot is refilled by TMA (async proxy) once every gate thread
-                    // released it: order this thread's generic reads of the slot first
-                    fence_proxy_async();
-                    mbar_arrive(&ring_empty[slot]);
                 }
                 if (!ok) break;
                 lam = nn / dd;
@@ -404,23 +441,34 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 // every gate warp has read the raw k rows before any overwrites them
                 mbar_arrive(gate_sync);
                 if (!waitw(gate_sync, c & 1, abort_flag, g.status)) { ok = false; break; }
-                const int half = (DK == 64) ? (tid >> 6) : 0;
 #pragma unroll
-                for (int tau = 0; tau < kC; ++tau) {
-                    const float fq = __shfl_sync(0xffffffffu, (tau & 1) ? fq1 : fq0, tau >> 1);
-                    const float fk = __shfl_sync(0xffffffffu, (tau & 1) ? fk1 : fk0, tau >> 1);
-                    const float bt = __shfl_sync(0xffffffffu, (tau & 1) ? cb1 : cb0, tau >> 1);
-                    if (DK == 64 && (tau >> 5) != half) continue;
-                    const int off = sw_off(tau, i, kC);
-                    float qv = 0.f, kv = 0.f;
-                    if (tok0 + tau < te) {
-                        if (!state_mode) qv = bf_at(qt, off) * fq;
-                        kv = bt * bf_at(kt, off) * fk;
+                for (int grp = 0; grp < kC / 8; ++grp) {
+                    float fqv[8], fkv[8], btv[8], qr[8], kr[8];
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) {
+                        const int tau = grp * 8 + r;
+                        fqv[r] = __shfl_sync(0xffffffffu, (tau & 1) ? fq1 : fq0, tau >> 1);
+                        fkv[r] = __shfl_sync(0xffffffffu, (tau & 1) ? fk1 : fk0, tau >> 1);
+                        btv[r] = __shfl_sync(0xffffffffu, (tau & 1) ? cb1 : cb0, tau >> 1);
                     }
-                    if (!state_mode) bf_put(qt, off, qv);
-                    const __nv_bfloat16 khi = __float2bfloat16_rn(kv);
-                    *reinterpret_cast<__nv_bfloat16 *>(kt + off) = khi;
-                    bf_put(klo, off, kv - __bfloat162float(khi));
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) {
+                        const int off = sw_off(grp * 8 + r, i, kC);
+                        qr[r] = state_mode ? 0.f : bf_at(qt, off);
+                        kr[r] = bf_at(kt, off);
+                    }
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) {
+                        const int tau = grp * 8 + r;
+                        const int off = sw_off(tau, i, kC);
+                        const bool valid = tok0 + tau < te;
+                        const float qv = valid ? qr[r] * fqv[r] : 0.f;
+                        const float kv = valid ? btv[r] * kr[r] * fkv[r] : 0.f;
+                        if (!state_mode) bf_put(qt, off, qv);
+                        const __nv_bfloat16 khi = __float2bfloat16_rn(kv);
+                        *reinterpret_cast<__nv_bfloat16 *>(kt + off) = khi;
+                        bf_put(klo, off, kv - __bfloat162float(khi));
+                    }
                 }
             }
             // state rescale factors: U_c = diag(2^R_c) S_c, S_{c+1} = diag(2^(G_last - R_c)) (U_c + K'^T V)
@@ -433,13 +481,13 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         if (ok && !*abort_flag) {
             if (state_mode) {
-                if (g.iso ? (tid == 0) : key) g.decay[(u * g.P + p) * (g.iso ? 1 : DK) + (g.iso ? 0 : i)] = exp2f(log_decay);
+                if (g.iso ? (gt == 0) : key) g.decay[(u * g.P + p) * (g.iso ? 1 : DK) + (g.iso ? 0 : i)] = exp2f(log_decay);
             } else if (last_seg && g.final_lambda) {
-                if (g.iso ? (tid == 0) : key) g.final_lambda[u * (g.iso ? 1 : DK) + (g.iso ? 0 : i)] = lam;
+                if (g.iso ? (gt == 0) : key) g.final_lambda[u * (g.iso ? 1 : DK) + (g.iso ? 0 : i)] = lam;
             }
         }
       }
-    } else if (warp < 8) {
+    } else if (warp >= 4 && warp < 8) {
         // ================= epilogue warps ====================================
         const int e = tid - 128, we = e >> 5, le = e & 31;
         const uint32_t lane_base = (uint32_t)(32 * we) << 16;
@@ -576,7 +624,7 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 for (int x = 0; x < DV; ++x) dst[rowU * DV + x] = sstart ? sstart[rowU * DV + x] : 0.f;
             }
         }
-    } else if (warp == 8) {
+    } else if (warp == RL::PRODW) {
         // ================= TMA producer =====================================
         if (lane == 0) {
             int last_ring[kSlots], last_stage[2] = {-1, -1};
@@ -622,7 +670,7 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         wait_slow(&stage_full[s], (last_stage[s] >> 1) & 1, abort_flag, g.status, false);
             }
         }
-    } else {
+    } else if (warp == RL::MMAW) {
         // ================= MMA issuer =======================================
         if (lane == 0) {
             constexpr uint32_t iS = idesc_bf16(64, 64, false, false);
@@ -685,7 +733,7 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 9) tmem_dealloc(tbase, L::NCOLS);
+    if (warp == RL::MMAW) tmem_dealloc(tbase, L::NCOLS);
 }
 
 // ---- host side ---------------------------------------------------------------
@@ -757,7 +805,7 @@ cudaError_t launch_t(const Plan &p, const int *cu, int mode, const void *q, cons
     const long long segs = mode == 1 ? p.P - 1 : p.P;
     const unsigned grid = (unsigned)((long long)p.N * p.H * segs);
     if (grid == 0) return cudaSuccess;
-    kla_chunk_tc_kernel<DK, DV><<<grid, kThreads, L::alloc, st>>>(mq, mk, mv, ma, mqn, g);
+    kla_chunk_tc_kernel<DK, DV><<<grid, Roles<DK, DV>::THREADS, L::alloc, st>>>(mq, mk, mv, ma, mqn, g);
     return cudaGetLastError();
 }
 
