@@ -3,7 +3,7 @@
 //
 // Launch sequence of kla_forward for B rows of T tokens split into P segments
 // per row (P = 1 when rows x heads already fill the GPU):
-//   P > 1:  mobius_reduce -> mobius_carry        (lambda at every block start)
+//   P > 1:  mobius_reduce -> mobius_carry        (lambda at every segment start)
 //           walk(state) on segments 0..P-2      (each segment's eta transfer)
 //           state_carry                          (eta at every segment start)
 //   always: walk(output) on every segment        (chunk kernel or SIMT walk)
@@ -69,8 +69,10 @@ static bool pow2_in(int x, int lo, int hi) {
 }
 
 // Segments per row: enough (row, head, segment) units to fill the SMs twice,
-// unless rows x heads already fill them. KLA_SEGMENTS overrides (tuning only;
-// the result does not depend on it beyond rounding).
+// unless rows x heads already occupy at least half of them (splitting then
+// costs more in the extra precision and state passes than it gains).
+// KLA_SEGMENTS overrides (tuning only; the result does not depend on it beyond
+// rounding).
 static int choose_segments(long long units, int NB) {
     const char *env = getenv("KLA_SEGMENTS");
     if (env && *env) {
@@ -78,7 +80,7 @@ static int choose_segments(long long units, int NB) {
         return P < 1 ? 1 : (P > NB ? NB : P);
     }
     int sms = sm_count();
-    if (units >= sms) return 1;
+    if (2 * units >= sms) return 1;
     long long P = (2LL * sms + units - 1) / units;
     return (int)(P > NB ? NB : P);
 }

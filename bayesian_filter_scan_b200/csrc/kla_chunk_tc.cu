@@ -241,6 +241,11 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // ================= gate warps: precision path and operand folding =====
         const int i = gt;                    // key owned by this thread
         const bool key = true;
+        // byte offset of (row r of an 8-row group, key i) in a 64-row 128B-swizzled
+        // tile; row 8j + r of the chunk is at j * 1024 + offr[r]
+        int offr[kSlotTok];
+#pragma unroll
+        for (int r = 0; r < kSlotTok; ++r) offr[r] = sw_off(r, i, kC);
         float lam = 1.0f;
         {
             const int il = g.iso ? 0 : i;
@@ -293,51 +298,153 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 // from the previous chunk's decay; the chunk's actual G range is checked.
                 R = r_next;
                 const int nvalid = (int)min((long long)kC, te - tok0);
-                float nn = lam, dd = 1.0f, pa = 1.0f;
-                int E = 0, F = 0, gmin = 0, gmax = 0;
-                float mq = __int_as_float((127 - R) << 23), mk = __int_as_float((127 + R) << 23);
-#pragma unroll 1
-                for (int j = 0; j < kSlotsPerChunk; ++j) {
-                    const int n = c * kSlotsPerChunk + j, slot = n % kSlots;
-                    if (!waitw(&ring_full[slot], (n / kSlots) & 1, abort_flag, g.status)) { ok = false; break; }
-                    const float *ra = reinterpret_cast<const float *>(sm + L::ring0) + slot * 2 * L::SLOTF;
-                    const float *rq = ra + L::SLOTF;
-                    const float bsrc = (j < 4) ? cb0 : cb1;
-                    // Load the slot's inputs first (the tile is rewritten in place below,
-                    // so loads and stores are kept in separate phases), then release
-                    // the ring slot, then run the recursion, then write the operands.
-                    float kr[kSlotTok], qr[kSlotTok], ar[kSlotTok], qnr[kSlotTok], br[kSlotTok];
-#pragma unroll
-                    for (int r = 0; r < kSlotTok; ++r) {
-                        const int tau = kSlotTok * j + r;
-                        const int off = sw_off(tau, i, kC);
-                        kr[r] = bf_at(kt, off);
-                        qr[r] = state_mode ? 0.f : bf_at(qt, off);
-                        ar[r] = ra[r * DK + i];
-                        qnr[r] = rq[r * DK + i];
-                        br[r] = __shfl_sync(0xffffffffu, bsrc, tau & 31);
-                    }
-                    // the slot is refilled by TMA (async proxy) once every gate thread
-                    // released it: order this thread's generic reads of the slot first
-                    fence_proxy_async();
-                    mbar_arrive(&ring_empty[slot]);
-                    float qo[kSlotTok], ko[kSlotTok];
+                float nn = lam, dd = 1.0f, pa = 1.0f, mq, mk;
+                int E = 0, F = 0;
+                bool range_bad = false;
+                {
+                    const int sh0 = max(-126, min(127, -R));
+                    mq = __int_as_float((127 + sh0) << 23);
+                    mk = __int_as_float((127 - sh0) << 23);
+                }
+                if (nvalid == kC) {
+                    // Full chunk, software-pipelined over 8-token slots: the serial
+                    // chain of slot j+1 (two FMAs per token on (n, d), one on PA) is
+                    // interleaved with the independent per-token work of slot j:
+                    //   rk = (d/PA) * mk = 2^(R - G)      K' = beta k rk (bf16 hi + lo)
+                    //   Q' = q * (PA/n) * mq = q / lambda * 2^(G - R)
+                    // bf16 packing by integer rounding (no conversion-unit work).
+                    // per slot buffer: beta k, d/PA and PA/n of each token
+                    float bkv[2][kSlotTok], rkv[2][kSlotTok], qfv[2][kSlotTok];
+                    float msq[2], msk[2];
+                    float xa[kSlotTok], xn[kSlotTok], xk[kSlotTok];
                     float rkmin = 3.0e38f, rkmax = 0.f;
-                    if (nvalid >= kSlotTok * (j + 1)) {
-                        // every token of the slot is inside the segment
+                    const int n0 = c * kSlotsPerChunk;
+                    // The three steps of a slot; between the wait/release barriers no
+                    // memory fence separates the chain of slot j+1 from the operand
+                    // work of slot j, so the two interleave.
+                    auto load_slot = [&](int j) {
+                        const int n = n0 + j, slot = n % kSlots;
+                        if (!waitw(&ring_full[slot], (n / kSlots) & 1, abort_flag, g.status)) return false;
+                        const float *ra = reinterpret_cast<const float *>(sm + L::ring0) + slot * 2 * L::SLOTF + i;
 #pragma unroll
                         for (int r = 0; r < kSlotTok; ++r) {
-                            const float at = ar[r], bk = br[r] * kr[r];
-                            dd = fmaf(at * at, dd, qnr[r] * nn);
-                            nn = fmaf(bk * kr[r], dd, nn);
-                            pa *= at;
-                            const float rk = __fdividef(dd, pa);        // 2^-G * 2^(F-E)
-                            rkmin = fminf(rkmin, rk);
-                            rkmax = fmaxf(rkmax, rk);
-                            qo[r] = qr[r] * (__fdividef(pa, nn) * mq);
-                            ko[r] = bk * (rk * mk);
+                            xa[r] = ra[r * DK];
+                            xn[r] = ra[L::SLOTF + r * DK];
+                            xk[r] = bf_at(kt, j * 1024 + offr[r]);
                         }
-                    } else {
+                        return true;
+                    };
+                    auto chain_slot = [&](int j, int b) {
+                        const float bsrc = (j < 4) ? cb0 : cb1;
+#pragma unroll
+                        for (int r = 0; r < kSlotTok; ++r)
+                            bkv[b][r] = __shfl_sync(0xffffffffu, bsrc, (kSlotTok * j + r) & 31) * xk[r];
+                        float nnt[kSlotTok], pat[kSlotTok];
+#pragma unroll
+                        for (int r = 0; r < kSlotTok; ++r) {
+                            const float at = xa[r];
+                            dd = fmaf(at * at, dd, xn[r] * nn);
+                            nn = fmaf(bkv[b][r] * xk[r], dd, nn);
+                            pa *= at;
+                            nnt[r] = nn;
+                            pat[r] = pa;
+                            rkv[b][r] = dd;
+                        }
+#pragma unroll
+                        for (int r = 0; r < kSlotTok; ++r) {
+                            rkv[b][r] *= rcp_approx(pat[r]);
+                            qfv[b][r] = pat[r] * rcp_approx(nnt[r]);
+                        }
+                        msq[b] = mq;
+                        msk[b] = mk;
+                        // exact power-of-two rescale of (n, d) and PA
+                        const int e = ((__float_as_int(dd) >> 23) & 0xff) - 127;
+                        const int f = ((__float_as_int(pa) >> 23) & 0xff) - 127;
+                        const float se = __int_as_float((127 - e) << 23);
+                        nn *= se;
+                        dd *= se;
+                        pa *= __int_as_float((127 - f) << 23);
+                        E += e;
+                        F += f;
+                        const int sh = max(-126, min(127, (F - E) - R));
+                        mq = __int_as_float((127 + sh) << 23);
+                        mk = __int_as_float((127 - sh) << 23);
+                    };
+                    // operands of slot j from its chain values, written over the tiles
+                    auto fold_slot = [&](int j, int b) {
+                        float xq[kSlotTok];
+                        if (!state_mode) {
+#pragma unroll
+                            for (int r = 0; r < kSlotTok; ++r) xq[r] = bf_at(qt, j * 1024 + offr[r]);
+                        }
+#pragma unroll
+                        for (int r = 0; r < kSlotTok; ++r) {
+                            const float rkm = rkv[b][r] * msk[b];
+                            rkmin = fminf(rkmin, rkm);
+                            rkmax = fmaxf(rkmax, rkm);
+                            const float ko = bkv[b][r] * rkm;
+                            const uint32_t t = __float_as_uint(ko) + 0x8000u;     // K' hi, rounded
+                            const int off = j * 1024 + offr[r];
+                            *reinterpret_cast<uint16_t *>(kt + off) = (uint16_t)(t >> 16);
+                            *reinterpret_cast<uint16_t *>(klo + off) =
+                                (uint16_t)(__float_as_uint(ko - __uint_as_float(t & 0xffff0000u)) >> 16);
+                        }
+                        if (!state_mode) {
+#pragma unroll
+                            for (int r = 0; r < kSlotTok; ++r) {
+                                const float qo = xq[r] * (qfv[b][r] * msq[b]);
+                                *reinterpret_cast<uint16_t *>(qt + j * 1024 + offr[r]) =
+                                    (uint16_t)((__float_as_uint(qo) + 0x8000u) >> 16);
+                            }
+                        }
+                    };
+                    // a ring slot read into registers is released after its chain
+                    // (generic reads ordered before the TMA refill)
+                    auto release_slot = [&](int j) {
+                        fence_proxy_async();
+                        mbar_arrive(&ring_empty[(n0 + j) % kSlots]);
+                    };
+                    if (!load_slot(0)) { ok = false; break; }
+                    chain_slot(0, 0);
+                    release_slot(0);
+#pragma unroll
+                    for (int j = 0; j < kSlotsPerChunk; ++j) {
+                        if (j + 1 < kSlotsPerChunk) {
+                            if (!load_slot(j + 1)) { ok = false; break; }
+                            chain_slot(j + 1, (j + 1) & 1);
+                        }
+                        fold_slot(j, j & 1);
+                        if (j + 1 < kSlotsPerChunk) release_slot(j + 1);
+                    }
+                    if (!ok) break;
+                    // rk = 2^(R - G): |G - R| beyond the kept range leaves the exponent window
+                    range_bad = (((__float_as_int(rkmax) >> 23) & 0xff) - 127 >= kMaxOffset) ||
+                                (((__float_as_int(rkmin) >> 23) & 0xff) - 127 < -kMaxOffset);
+                } else {
+                    // Partial chunk (end of a segment or sequence): same recursion, one
+                    // slot at a time, with per-token validity.
+                    int gmin = 0, gmax = 0;
+#pragma unroll 1
+                    for (int j = 0; j < kSlotsPerChunk; ++j) {
+                        const int n = c * kSlotsPerChunk + j, slot = n % kSlots;
+                        if (!waitw(&ring_full[slot], (n / kSlots) & 1, abort_flag, g.status)) { ok = false; break; }
+                        const float *ra = reinterpret_cast<const float *>(sm + L::ring0) + slot * 2 * L::SLOTF;
+                        const float *rq = ra + L::SLOTF;
+                        const float bsrc = (j < 4) ? cb0 : cb1;
+                        float kr[kSlotTok], qr[kSlotTok], ar[kSlotTok], qnr[kSlotTok], br[kSlotTok];
+#pragma unroll
+                        for (int r = 0; r < kSlotTok; ++r) {
+                            const int off = j * 1024 + offr[r];
+                            kr[r] = bf_at(kt, off);
+                            qr[r] = state_mode ? 0.f : bf_at(qt, off);
+                            ar[r] = ra[r * DK + i];
+                            qnr[r] = rq[r * DK + i];
+                            br[r] = __shfl_sync(0xffffffffu, bsrc, (kSlotTok * j + r) & 31);
+                        }
+                        fence_proxy_async();
+                        mbar_arrive(&ring_empty[slot]);
+                        float qo[kSlotTok], ko[kSlotTok];
+                        float rkmin = 3.0e38f, rkmax = 0.f;
 #pragma unroll
                         for (int r = 0; r < kSlotTok; ++r) {
                             const bool valid = kSlotTok * j + r < nvalid;
@@ -352,22 +459,17 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                             qo[r] = valid ? qr[r] * (__fdividef(pa, nn) * mq) : 0.f;
                             ko[r] = bk * (rk * mk);
                         }
-                    }
-                    // G = (F - E) - log2(rk); integer bounds of this slot's G range
-                    gmin = min(gmin, (F - E) - (((__float_as_int(rkmax) >> 23) & 0xff) - 126));
-                    gmax = max(gmax, (F - E) - (((__float_as_int(rkmin) >> 23) & 0xff) - 127));
+                        // G = (F - E) - log2(rk); integer bounds of this slot's G range
+                        gmin = min(gmin, (F - E) - (((__float_as_int(rkmax) >> 23) & 0xff) - 126));
+                        gmax = max(gmax, (F - E) - (((__float_as_int(rkmin) >> 23) & 0xff) - 127));
 #pragma unroll
-                    for (int r = 0; r < kSlotTok; ++r) {
-                        const int off = sw_off(kSlotTok * j + r, i, kC);
-                        if (!state_mode) bf_put(qt, off, qo[r]);
-                        // K' = hi + lo in two bf16 parts: the state update sums K'^T V
-                        // over whole segments, so it gets (nearly) fp32 operands.
-                        const __nv_bfloat16 khi = __float2bfloat16_rn(ko[r]);
-                        *reinterpret_cast<__nv_bfloat16 *>(kt + off) = khi;
-                        bf_put(klo, off, ko[r] - __bfloat162float(khi));
-                    }
-                    // exact power-of-two rescale of (n, d) and PA
-                    {
+                        for (int r = 0; r < kSlotTok; ++r) {
+                            const int off = j * 1024 + offr[r];
+                            if (!state_mode) bf_put(qt, off, qo[r]);
+                            const __nv_bfloat16 khi = __float2bfloat16_rn(ko[r]);
+                            *reinterpret_cast<__nv_bfloat16 *>(kt + off) = khi;
+                            bf_put(klo, off, ko[r] - __bfloat162float(khi));
+                        }
                         const int e = ((__float_as_int(dd) >> 23) & 0xff) - 127;
                         const int f = ((__float_as_int(pa) >> 23) & 0xff) - 127;
                         const float se = __int_as_float((127 - e) << 23);
@@ -380,14 +482,15 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         mq = __int_as_float((127 + sh) << 23);
                         mk = __int_as_float((127 - sh) << 23);
                     }
+                    if (!ok) break;
+                    range_bad = gmax - R > kMaxOffset || R - gmin > kMaxOffset;
                 }
-                if (!ok) break;
                 lam = nn / dd;
                 const float gm = pa / dd;                 // 2^G_last = gm * 2^(F-E)
                 const int sl = F - E;
                 e_cur = gm * __int_as_float((127 + max(-126, min(127, sl - R))) << 23);
                 glast_log2 = (float)sl + __log2f(gm);
-                if (gmax - R > kMaxOffset || R - gmin > kMaxOffset) atomicOr(g.status, kStatusRange);
+                if (range_bad) atomicOr(g.status, kStatusRange);
                 // predicted middle of the next chunk's G range (same decay rate)
                 const int gl = sl + (((__float_as_int(gm) >> 23) & 0xff) - 127);
                 r_next = max(-kMaxOffset, min(kMaxOffset, gl / 2));
@@ -645,6 +748,23 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 for (int a = 0; a < DV / 64; ++a)
                     tma_load_3d(sm + L::v0 + s * L::V + a * kC * 128, &tm_v, &stage_full[s], 64 * a, h, tok0);
                 last_stage[s] = c;
+                // L2 prefetch of the chunk two ahead, so that the TMA copies above
+                // and the ring refills below are served from L2
+                if (c + 2 < nchunks) {
+                    const int tp = tok0 + 2 * kC;
+#pragma unroll
+                    for (int a = 0; a < DK / 64; ++a) {
+                        if (!state_mode) tma_prefetch_3d(&tm_q, 64 * a, h, tp);
+                        tma_prefetch_3d(&tm_k, 64 * a, h, tp);
+                    }
+#pragma unroll
+                    for (int a = 0; a < DV / 64; ++a) tma_prefetch_3d(&tm_v, 64 * a, h, tp);
+                    if (!g.iso)
+                        for (int j = 0; j < kSlotsPerChunk; ++j) {
+                            tma_prefetch_3d(&tm_a, 0, h, tp + kSlotTok * j);
+                            tma_prefetch_3d(&tm_qn, 0, h, tp + kSlotTok * j);
+                        }
+                }
                 if (!g.iso) {
                     for (int j = 0; j < kSlotsPerChunk; ++j) {
                         const int n = c * kSlotsPerChunk + j, slot = n % kSlots;

@@ -17,7 +17,7 @@
 
 namespace kla {
 
-constexpr int kBlockTokens = 256;  // Lb: tokens per Moebius-reduction block
+constexpr int kBlockTokens = 64;   // Lb: tokens per Moebius-reduction block (one chunk)
 constexpr int kChunk = 64;         // C: tokens per chunk of the chunked form
 
 // Bits of the library's device status word (kla_check reads and clears it);

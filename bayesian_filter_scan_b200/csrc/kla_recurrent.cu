@@ -262,10 +262,26 @@ kla_state_carry(int N, int H, int dk, int dv, int nl, int P, const float *__rest
     long long u = gid / per, e = gid % per;
     int il = (nl == 1) ? 0 : (int)(e / dv);
     float S = eta0 ? eta0[gid] : 0.0f;
-    for (int p = 1; p < P; ++p) {
-        long long slot = (u * P + p - 1) * per + e;
-        S = fmaf(decay[(u * P + p - 1) * nl + il], S, S_io[slot]);
-        S_io[slot] = S;
+    // segments in batches of 8: every transfer of a batch is read before any
+    // carried state is written back, so the loads overlap
+    for (int p0 = 1; p0 < P; p0 += 8) {
+        float x[8], dc[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const int p = p0 + r;
+            if (p < P) {
+                x[r] = S_io[(u * P + p - 1) * per + e];
+                dc[r] = decay[(u * P + p - 1) * nl + il];
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const int p = p0 + r;
+            if (p < P) {
+                S = fmaf(dc[r], S, x[r]);
+                S_io[(u * P + p - 1) * per + e] = S;
+            }
+        }
     }
 }
 

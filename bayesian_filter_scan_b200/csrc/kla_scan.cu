@@ -6,14 +6,15 @@
 //
 // Three kernels, no inter-CTA waiting (reduce, then scan, then re-walk):
 //   mobius_reduce : per (row, head, block of Lb tokens, key) the composed 2x2
-//                   matrix of the block (normalised by powers of two).
-//   mobius_carry  : per (row, head, key) the exclusive prefix over blocks,
-//                   applied to lambda0: lambda at every block start.
+//                   matrix of the block (normalised by powers of two); one CTA
+//                   per block, sub-blocks of dk tokens per thread, composed in
+//                   shared memory.
+//   mobius_carry  : per (row, head, key) one warp: the product of each
+//                   segment's blocks, a shuffle scan over segments, applied to
+//                   lambda0: lambda at every segment start.
 //   mobius_emit   : per (row/sequence, head, block, key) re-walks the block
 //                   from its start lambda and writes lambda after every token
-//                   (the kla_precision output).
-// Each thread owns 4 consecutive keys (16-byte fp32 loads of a and qn, 8-byte
-// bf16 loads of k), so one warp reads 512 contiguous bytes of a per token.
+//                   (the kla_precision output; there segments are blocks).
 #include "kla_internal.cuh"
 
 namespace kla {
@@ -27,52 +28,54 @@ struct ScanArgs {
 
 // ---- reduce --------------------------------------------------------------
 
+// CTA = one (row, head, block of Lb tokens), 256 threads = (sub-block, key):
+// the block is cut into 256/dk sub-blocks of Lb*dk/256 tokens, each walked by
+// one thread per key (coalesced fp32 loads of a and qn across the keys of a
+// token), and the sub-block products are composed in shared memory.
 template <typename TIn>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(256)
 mobius_reduce_diag(ScanArgs s, const TIn *__restrict__ k, const float *__restrict__ a,
                    const float *__restrict__ qn, const float *__restrict__ beta,
                    float4 *__restrict__ agg) {
-    const int nkq = s.dk / 4;
-    long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    long long pair = gid / nkq;
-    int kq = (int)(gid % nkq);
-    if (pair >= (long long)s.N * s.H * s.NB) return;
-    int blk = (int)(pair % s.NB);
-    long long u = pair / s.NB;
-    int n = (int)(u / s.H), h = (int)(u % s.H);
-    long long t0 = (long long)blk * kBlockTokens;
-    long long t1 = min(t0 + kBlockTokens, s.T);
-    Mob P[4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) P[c] = Mob{1.f, 0.f, 0.f, 1.f};
+    __shared__ float4 part[256];
+    const int dk = s.dk;
+    const int nsub = 256 / dk;
+    const int i = threadIdx.x % dk, sub = threadIdx.x / dk;
+    const long long pair = blockIdx.x;
+    const int blk = (int)(pair % s.NB);
+    const long long u = pair / s.NB;
+    const int n = (int)(u / s.H), h = (int)(u % s.H);
+    const int len = kBlockTokens * dk / 256;
+    const long long t0 = (long long)blk * kBlockTokens + (long long)sub * len;
+    const long long t1 = min(t0 + len, s.T);
+    Mob P{1.f, 0.f, 0.f, 1.f};
     for (long long t = t0; t < t1; t += 8) {
-        float4 av[8], qv[8], kv[8];
-        float bv[8];
+        float av[8], qv[8], kv[8], bv[8];
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
+            av[r] = 1.f; qv[r] = 0.f; kv[r] = 0.f; bv[r] = 0.f;
             if (t + r < t1) {
-                long long th = ((long long)n * s.T + t + r) * s.H + h;
-                av[r] = ld4(a + th * s.dk + 4 * kq);
-                qv[r] = ld4(qn + th * s.dk + 4 * kq);
-                kv[r] = ld4(k + th * s.dk + 4 * kq);
+                const long long th = ((long long)n * s.T + t + r) * s.H + h;
+                av[r] = __ldg(a + th * dk + i);
+                qv[r] = __ldg(qn + th * dk + i);
+                kv[r] = ld_in(k + th * dk + i);
                 bv[r] = __ldg(beta + th);
             }
         }
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            if (t + r < t1) {
-                const float *ap = &av[r].x, *qp = &qv[r].x, *kp = &kv[r].x;
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    P[c] = mob_mul(mob_step(ap[c], qp[c], bv[r] * kp[c] * kp[c]), P[c]);
-            }
-        }
-#pragma unroll
-        for (int c = 0; c < 4; ++c) P[c] = mob_norm(P[c]);
+        for (int r = 0; r < 8; ++r) P = mob_mul(mob_step(av[r], qv[r], bv[r] * kv[r] * kv[r]), P);
+        P = mob_norm(P);
     }
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-        agg[pair * s.dk + 4 * kq + c] = make_float4(P[c].m00, P[c].m01, P[c].m10, P[c].m11);
+    part[threadIdx.x] = make_float4(P.m00, P.m01, P.m10, P.m11);
+    __syncthreads();
+    if (sub == 0) {
+        Mob acc = P;
+        for (int b = 1; b < nsub; ++b) {
+            const float4 m = part[b * dk + i];
+            acc = mob_norm(mob_mul(Mob{m.x, m.y, m.z, m.w}, acc));
+        }
+        agg[pair * dk + i] = make_float4(acc.m00, acc.m01, acc.m10, acc.m11);
+    }
 }
 
 // Isotropic: one precision per head; increment beta*|k|^2/dk.
@@ -113,31 +116,56 @@ mobius_reduce_iso(ScanArgs s, const TIn *__restrict__ k, const float *__restrict
 
 // ---- carry ---------------------------------------------------------------
 
-// lam_blk[(u*NB + blk)*nl + i] = (M_{blk-1} ... M_0)(lambda0): lambda at the
-// start of every block.
+// lam_blk[(u*NB + p*seg_blocks)*nl + i] = (all blocks before segment p)(lambda0):
+// lambda at every segment start (every block start when segments are blocks).
+// One warp per (row, head, key): lane l composes the blocks of segments l,
+// l+32, ..., then a warp-shuffle scan of the 2x2 maps gives the exclusive
+// prefixes, carried across groups of 32 segments.
+__device__ __forceinline__ Mob shfl_up_m(const Mob &m, int d) {
+    return Mob{__shfl_up_sync(0xffffffffu, m.m00, d), __shfl_up_sync(0xffffffffu, m.m01, d),
+               __shfl_up_sync(0xffffffffu, m.m10, d), __shfl_up_sync(0xffffffffu, m.m11, d)};
+}
+__device__ __forceinline__ Mob shfl_m(const Mob &m, int src) {
+    return Mob{__shfl_sync(0xffffffffu, m.m00, src), __shfl_sync(0xffffffffu, m.m01, src),
+               __shfl_sync(0xffffffffu, m.m10, src), __shfl_sync(0xffffffffu, m.m11, src)};
+}
+
 __global__ void __launch_bounds__(128)
-mobius_carry(ScanArgs s, int nl, const float4 *__restrict__ agg,
+mobius_carry(ScanArgs s, int nl, int P, int seg_blocks, const float4 *__restrict__ agg,
              const float *__restrict__ lambda0, float *__restrict__ lam_blk) {
-    long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (gid >= (long long)s.N * s.H * nl) return;
-    long long u = gid / nl;
-    int i = (int)(gid % nl);
-    float l0 = lambda0 ? __ldg(lambda0 + gid) : 1.0f;
-    Mob P{1.f, 0.f, 0.f, 1.f};
+    const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (gw >= (long long)s.N * s.H * nl) return;
+    const long long u = gw / nl;
+    const int i = (int)(gw % nl);
+    const float l0 = lambda0 ? __ldg(lambda0 + gw) : 1.0f;
     const float4 *src = agg + u * s.NB * nl + i;
-    float *dst = lam_blk + u * s.NB * nl + i;
-    for (int blk = 0; blk < s.NB; blk += 8) {
-        float4 m[8];
+    Mob carry{1.f, 0.f, 0.f, 1.f};
+    for (int base = 0; base < P; base += 32) {
+        const int p = base + lane;
+        Mob S{1.f, 0.f, 0.f, 1.f};
+        if (p < P) {
+            const int b0 = p * seg_blocks, b1 = min(b0 + seg_blocks, s.NB);
+            for (int b = b0; b < b1; b += 8) {
+                float4 m[8];
 #pragma unroll
-        for (int r = 0; r < 8; ++r)
-            if (blk + r < s.NB) m[r] = __ldg(src + (long long)(blk + r) * nl);
+                for (int r = 0; r < 8; ++r)
+                    if (b + r < b1) m[r] = __ldg(src + (long long)(b + r) * nl);
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            if (blk + r < s.NB) {
-                dst[(long long)(blk + r) * nl] = mob_apply(P, l0);
-                P = mob_norm(mob_mul(Mob{m[r].x, m[r].y, m[r].z, m[r].w}, P));
+                for (int r = 0; r < 8; ++r)
+                    if (b + r < b1) S = mob_norm(mob_mul(Mob{m[r].x, m[r].y, m[r].z, m[r].w}, S));
             }
         }
+        Mob incl = S;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const Mob o = shfl_up_m(incl, d);
+            if (lane >= d) incl = mob_norm(mob_mul(incl, o));
+        }
+        Mob excl = shfl_up_m(incl, 1);
+        if (lane == 0) excl = Mob{1.f, 0.f, 0.f, 1.f};
+        if (p < P) lam_blk[(u * s.NB + (long long)p * seg_blocks) * nl + i] = mob_apply(mob_mul(excl, carry), l0);
+        carry = mob_norm(mob_mul(shfl_m(incl, 31), carry));
     }
 }
 
@@ -251,16 +279,15 @@ cudaError_t launch_mobius_reduce(const Plan &p, const void *k, const float *a, c
         mobius_reduce_iso<TIn><<<blocks_for(pairs, 128), 128, 0, st>>>(
             s, (const TIn *)k, a, qn, beta, agg);
     else
-        mobius_reduce_diag<TIn><<<blocks_for(pairs * (p.dk / 4), 128), 128, 0, st>>>(
-            s, (const TIn *)k, a, qn, beta, agg);
+        mobius_reduce_diag<TIn><<<(unsigned)pairs, 256, 0, st>>>(s, (const TIn *)k, a, qn, beta, agg);
     return cudaGetLastError();
 }
 
 cudaError_t launch_mobius_carry(const Plan &p, const float4 *agg, const float *lambda0,
                                 float *lam_blk, cudaStream_t st) {
     ScanArgs s{p.N, p.H, p.dk, p.T, p.NB, nullptr};
-    long long thr = (long long)p.N * p.H * p.nl;
-    mobius_carry<<<blocks_for(thr, 128), 128, 0, st>>>(s, p.nl, agg, lambda0, lam_blk);
+    long long thr = (long long)p.N * p.H * p.nl * 32;
+    mobius_carry<<<blocks_for(thr, 128), 128, 0, st>>>(s, p.nl, p.P, p.seg_blocks, agg, lambda0, lam_blk);
     return cudaGetLastError();
 }
 

@@ -60,6 +60,21 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *b, uint32_t parity
     return ok != 0;
 }
 
+// Hardware reciprocal (one special-function-unit op, about 1 ulp); inputs here
+// are positive normal floats.
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+// L2 prefetch of one TMA box (no shared-memory destination, no barrier).
+__device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap *map, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"((uint64_t)map),
+                 "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+
 // ---- fences ------------------------------------------------------------
 __device__ __forceinline__ void fence_proxy_async() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

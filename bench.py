@@ -47,6 +47,7 @@ from bayesian_filter_scan_b200.inputs import WORKLOADS, make_inputs  # noqa: E40
 METRIC = "KLA forward tokens/s per layer (B*T/s) on 1 B200; % of HBM / bf16 TC roofline"
 UNIT = "tokens/s"
 FLUSH_BYTES = 512 << 20
+SWEEP_BYTES = 256 << 20
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -261,6 +262,13 @@ def main():
     nws = kla.workspace_bytes(desc)
     ws = torch.empty(max(nws, 256), dtype=torch.uint8, device="cuda")
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    sweep = torch.ones(SWEEP_BYTES // 4, dtype=torch.float32, device="cuda")
+
+    def flush_l2():
+        # write 512 MiB (evicts every line of ours), then read 256 MiB so that the
+        # flush's own dirty lines are written back here, not inside the timed step
+        flush.fill_(1)
+        sweep.sum()
     stream = torch.cuda.current_stream()
     L = kla.lib()
     P = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())  # noqa: E731
@@ -278,7 +286,7 @@ def main():
     ev_ptrs = [(ctypes.c_void_p * 6)(*[ctypes.c_void_p(e.cuda_event) for e in row]) for row in evs]
 
     def step(i=None):
-        flush.fill_(1)
+        flush_l2()
         if i is None:
             s = L.kla_forward(*args_fwd)
         else:
@@ -306,6 +314,9 @@ def main():
     tot = [r[0].elapsed_time(r[5]) for r in evs]              # ms, whole forward
     chunk = [r[4].elapsed_time(r[5]) for r in evs]            # ms, output pass (chunk kernel)
     pre = [r[0].elapsed_time(r[4]) for r in evs]
+    # per launch of the sequence: reduce, carry, state pass, state carry, output pass
+    stage_names = ("mobius_reduce", "mobius_carry", "state_pass", "state_carry", "output_pass")
+    per_stage = {n: statistics.mean(r[i].elapsed_time(r[i + 1]) for r in evs) for i, n in enumerate(stage_names)}
     ms_per_step, value = aggregate(world, w.tokens, sum(tot), steps, dist)
 
     # ---- e2e through the host-buffer entry point
@@ -323,11 +334,11 @@ def main():
              P(pin["beta"]), None, None, P(hout), None, None, P(dbuf), nb, ctypes.c_void_p(stream.cuda_stream)]
     e2e_steps = max(3, min(args.e2e_steps, steps))
     for _ in range(3):
-        flush.fill_(1)
+        flush_l2()
         kla._check(L.kla_forward_host(*hargs), "kla_forward_host")
     e_t = 0.0
     for _ in range(e2e_steps):
-        flush.fill_(1)
+        flush_l2()
         a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a0.record(stream)
         kla._check(L.kla_forward_host(*hargs), "kla_forward_host")
@@ -354,14 +365,14 @@ def main():
         "config": {"workload": workload_label(w), "B": w.B, "H": H, "T": w.T, "dk": dk, "dv": dv,
                    "mode": w.mode, "varlen": w.varlen, "tokens_per_step_per_gpu": w.tokens,
                    "segments_per_row": plan["segments"], "tensor_core_chunk_kernel": plan["tensor_core"],
-                   "l2": "flushed between timed steps (512 MiB device write)", "parallelism": "dp%d" % world},
+                   "l2": "flushed between timed steps (512 MiB device write, then 256 MiB read)", "parallelism": "dp%d" % world},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "kernel": "kla_chunk_tc_kernel (output pass)" if plan["tensor_core"] else "kla_walk_simt",
                      "alg_bytes_per_launch": alg_bytes, "launch_ms": chunk_ms,
                      "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_src},
         "stages_ms": {"pre_passes": statistics.mean(pre), "output_pass": chunk_ms,
-                      "total": statistics.mean(tot)},
+                      "total": statistics.mean(tot), "launches": per_stage},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h_in, "d2h_bytes_per_step": h_out},
         "gpu_launches": steps * plan["launches"],
         "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"],
