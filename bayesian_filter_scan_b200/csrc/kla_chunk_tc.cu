@@ -50,6 +50,7 @@ constexpr int kSlotTok = 8;        // tokens per a/qn ring slot
 constexpr int kSlots = 6;          // ring depth (48 tokens of look-ahead)
 constexpr int kSlotsPerChunk = kC / kSlotTok;
 constexpr int kMaxOffset = 110;    // |G - R| (log2) kept inside the fp32/bf16 exponent range
+constexpr int kRebase = 64;        // diagonal mode: predicted |G - rho| that moves the reference
 // Warp roles. dk = 128: gate warps 0-3, epilogue 4-7, TMA producer 8, MMA 9.
 // dk = 64: gate warps 0 and 2, producer 1, MMA 3, epilogue 4-7 (8 warps, so
 // two CTAs fit on one SM when dv = 64 as well).
@@ -255,8 +256,15 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
         }
         float e_prev = 1.f, log_decay = 0.f;   // e_prev = 2^(G_last - R) of the previous chunk
-        int r_next = 0;                           // reference predicted for the next chunk
         bool ok = true;
+        // Diagonal mode keeps the precision chain and the log-gate reference across
+        // chunks: G is the cumulative log2 gate since the segment start, rho a
+        // per-key integer reference that moves only when the next chunk's predicted
+        // G range would leave [rho - kRebase, rho + kRebase]. The state in TMEM is
+        // U = diag(2^(rho - G)) eta, so it needs no rescale while rho stays put.
+        float nn = lam, dd = 1.0f, pa = 1.0f;
+        int E = 0, F = 0, rho = 0, dpred = 0;
+        float gprev = 0.f;
         // Per-token scalars of a chunk are loaded one chunk ahead into registers
         // and broadcast with shuffles (no global load sits on the recursion).
         // diag: beta of tokens (lane, lane+32); iso: a, qn, beta of (2 lane, 2 lane+1).
@@ -284,6 +292,7 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (c + 1 < nchunks) prefetch(c + 1);
             if (!waitw(&stage_full[s], (c >> 1) & 1, abort_flag, g.status)) { ok = false; break; }
             int R;                 // integer log2 reference of this chunk (per key)
+            float fac_c = 1.f;     // diagonal mode: rescale of U at this chunk's start
             float e_cur;           // 2^(G_last - R)
             float glast_log2;      // G_last
             uint8_t *klo = sm + L::klo0 + s * L::QK;
@@ -296,16 +305,24 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 // 2^E (n, d) and 2^F (PA), rescaled by exact powers of two every 8 tokens.
                 // The operands are written at once against the reference R predicted
                 // from the previous chunk's decay; the chunk's actual G range is checked.
-                R = r_next;
                 const int nvalid = (int)min((long long)kC, te - tok0);
-                float nn = lam, dd = 1.0f, pa = 1.0f, mq, mk;
-                int E = 0, F = 0;
+                float mq, mk;
                 bool range_bad = false;
                 {
-                    const int sh0 = max(-126, min(127, -R));
+                    // G at the chunk start is F - E to within one (n, d, PA are kept
+                    // in [1, 2) by the per-slot rescale); dpred = the last chunk's drift
+                    const int gs = F - E;
+                    const int lo = gs + min(0, dpred) - 2, hi = gs + max(0, dpred) + 2;
+                    int rnew = rho;
+                    if (hi - rho > kRebase || rho - lo > kRebase) rnew = gs + dpred / 2;
+                    fac_c = __int_as_float((127 + max(-126, min(127, rnew - rho))) << 23);
+                    rho = rnew;
+                    R = rho;
+                    const int sh0 = max(-126, min(127, gs - R));
                     mq = __int_as_float((127 + sh0) << 23);
                     mk = __int_as_float((127 - sh0) << 23);
                 }
+                const int gs_chunk = F - E;
                 if (nvalid == kC) {
                     // Full chunk, software-pipelined over 8-token slots: the serial
                     // chain of slot j+1 (two FMAs per token on (n, d), one on PA) is
@@ -423,7 +440,7 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 } else {
                     // Partial chunk (end of a segment or sequence): same recursion, one
                     // slot at a time, with per-token validity.
-                    int gmin = 0, gmax = 0;
+                    int gmin = F - E, gmax = F - E;     // G at the chunk start (absolute)
 #pragma unroll 1
                     for (int j = 0; j < kSlotsPerChunk; ++j) {
                         const int n = c * kSlotsPerChunk + j, slot = n % kSlots;
@@ -486,14 +503,14 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     range_bad = gmax - R > kMaxOffset || R - gmin > kMaxOffset;
                 }
                 lam = nn / dd;
-                const float gm = pa / dd;                 // 2^G_last = gm * 2^(F-E)
+                const float gm = pa / dd;                 // 2^G = gm * 2^(F-E)
                 const int sl = F - E;
-                e_cur = gm * __int_as_float((127 + max(-126, min(127, sl - R))) << 23);
-                glast_log2 = (float)sl + __log2f(gm);
+                e_cur = gm * __int_as_float((127 + max(-126, min(127, sl - R))) << 23);   // 2^(G - rho)
+                const float gnow = (float)sl + __log2f(gm);
+                glast_log2 = gnow - gprev;                 // this chunk's log2 decay
+                gprev = gnow;
+                dpred = sl - gs_chunk;
                 if (range_bad) atomicOr(g.status, kStatusRange);
-                // predicted middle of the next chunk's G range (same decay rate)
-                const int gl = sl + (((__float_as_int(gm) >> 23) & 0xff) - 127);
-                r_next = max(-kMaxOffset, min(kMaxOffset, gl / 2));
             } else {
                 // isotropic: one precision per head; warp-level Moebius scan over
                 // the chunk (lane l owns tokens 2l, 2l+1), redundantly per warp.
@@ -575,7 +592,7 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
             }
             // state rescale factors: U_c = diag(2^R_c) S_c, S_{c+1} = diag(2^(G_last - R_c)) (U_c + K'^T V)
-            fac[s * DK + i] = e_prev * __int_as_float((127 + max(-126, min(127, R))) << 23);
+            fac[s * DK + i] = g.iso ? e_prev * __int_as_float((127 + max(-126, min(127, R))) << 23) : fac_c;
             if (c == nchunks - 1) fac_final[i] = e_cur;
             e_prev = e_cur;
             log_decay += glast_log2;
@@ -613,22 +630,11 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (!waitw(&qk_ready[s], (c >> 1) & 1, abort_flag, g.status)) { ok = false; break; }
             if (c > 0 && !waitw(u_done, (c - 1) & 1, abort_flag, g.status)) { ok = false; break; }
             tc_fence_after();
-            const float f = vU ? fac[s * DK + rowU] : 0.f;
-#pragma unroll
-            for (int cb = 0; cb < DV / 32; ++cb) {
-                uint32_t r[32];
-                const uint32_t ta = tbase + lane_base + L::colU + cb * 32;
-                if (c == 0) {
-#pragma unroll
-                    for (int x = 0; x < 32; ++x)
-                        r[x] = __float_as_uint((vU && sstart) ? sstart[rowU * DV + cb * 32 + x] * f : 0.f);
-                } else {
-                    tmem_ld32(ta, r);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * f);
-                }
-                tmem_st32(ta, r);
+            // diag: f = 1 unless the gate moved this key's reference; the warp then
+            // only snapshots U (bf16, for the readout MMA) without rewriting TMEM
+            const float f = vU ? fac[s * DK + rowU] : 1.f;
+            const bool rmw = (c == 0) || __any_sync(0xffffffffu, f != 1.0f);
+            auto snap = [&](const uint32_t (&r)[32], int cb) {
                 if (!state_mode && vU) {
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) {
@@ -639,6 +645,37 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         w.w = pack_bf2(__uint_as_float(r[q4 * 8 + 6]), __uint_as_float(r[q4 * 8 + 7]));
                         *reinterpret_cast<uint4 *>(ub + sw_off(rowU, cb * 32 + q4 * 8, DK)) = w;
                     }
+                }
+            };
+            if (c == 0) {
+#pragma unroll
+                for (int cb = 0; cb < DV / 32; ++cb) {
+                    uint32_t r[32];
+#pragma unroll
+                    for (int x = 0; x < 32; ++x)
+                        r[x] = __float_as_uint((vU && sstart) ? sstart[rowU * DV + cb * 32 + x] * f : 0.f);
+                    tmem_st32(tbase + lane_base + L::colU + cb * 32, r);
+                    snap(r, cb);
+                }
+            } else if (rmw || !state_mode) {
+#pragma unroll
+                for (int cb = 0; cb < DV / 32; cb += 2) {
+                    uint32_t r0[32], r1[32];
+                    const uint32_t ta = tbase + lane_base + L::colU + cb * 32;
+                    tmem_ld32(ta, r0);
+                    tmem_ld32(ta + 32, r1);
+                    tmem_wait_ld();
+                    if (rmw) {
+#pragma unroll
+                        for (int x = 0; x < 32; ++x) {
+                            r0[x] = __float_as_uint(__uint_as_float(r0[x]) * f);
+                            r1[x] = __float_as_uint(__uint_as_float(r1[x]) * f);
+                        }
+                        tmem_st32(ta, r0);
+                        tmem_st32(ta + 32, r1);
+                    }
+                    snap(r0, cb);
+                    snap(r1, cb + 1);
                 }
             }
             tmem_wait_st();
@@ -681,19 +718,24 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             const bool row_ok = v64 && (tok0 + row64 < te);
             __nv_bfloat16 *orow = g.out + ((tok0 + row64) * g.H + h) * DV;
 #pragma unroll
-            for (int cb = 0; cb < DV / 32; ++cb) {
-                uint32_t r[32];
-                tmem_ld32(tbase + lane_base + L::colO + cb * 32, r);
+            for (int cb = 0; cb < DV / 32; cb += 2) {
+                uint32_t rr[2][32];
+                tmem_ld32(tbase + lane_base + L::colO + cb * 32, rr[0]);
+                tmem_ld32(tbase + lane_base + L::colO + cb * 32 + 32, rr[1]);
                 tmem_wait_ld();
                 if (row_ok) {
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        uint4 w;
-                        w.x = pack_bf2(__uint_as_float(r[q4 * 8 + 0]), __uint_as_float(r[q4 * 8 + 1]));
-                        w.y = pack_bf2(__uint_as_float(r[q4 * 8 + 2]), __uint_as_float(r[q4 * 8 + 3]));
-                        w.z = pack_bf2(__uint_as_float(r[q4 * 8 + 4]), __uint_as_float(r[q4 * 8 + 5]));
-                        w.w = pack_bf2(__uint_as_float(r[q4 * 8 + 6]), __uint_as_float(r[q4 * 8 + 7]));
-                        *reinterpret_cast<uint4 *>(orow + cb * 32 + q4 * 8) = w;
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const uint32_t *r = rr[hh];
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            uint4 w;
+                            w.x = pack_bf2(__uint_as_float(r[q4 * 8 + 0]), __uint_as_float(r[q4 * 8 + 1]));
+                            w.y = pack_bf2(__uint_as_float(r[q4 * 8 + 2]), __uint_as_float(r[q4 * 8 + 3]));
+                            w.z = pack_bf2(__uint_as_float(r[q4 * 8 + 4]), __uint_as_float(r[q4 * 8 + 5]));
+                            w.w = pack_bf2(__uint_as_float(r[q4 * 8 + 6]), __uint_as_float(r[q4 * 8 + 7]));
+                            *reinterpret_cast<uint4 *>(orow + (cb + hh) * 32 + q4 * 8) = w;
+                        }
                     }
                 }
             }
