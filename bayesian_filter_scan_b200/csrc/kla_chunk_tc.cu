@@ -263,8 +263,10 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const __grid_constant__ CUtensorMap tm_qn, const TcArgs g) {
     using L = Layout<DK, DV>;
     using RL = Roles<DK, DV>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    // 1024-byte aligned base (128B-swizzle atoms), derived by pointer arithmetic
+    // on the shared array so that every tile access stays a shared-space access
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::bar0);
     uint64_t *stage_full = bars + 0, *stage_empty = bars + 2, *qk_ready = bars + 4;
     uint64_t *ring_full = bars + 6, *ring_empty = bars + 6 + kSlots;
