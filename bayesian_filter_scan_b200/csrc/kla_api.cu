@@ -68,20 +68,22 @@ static bool pow2_in(int x, int lo, int hi) {
     return x >= lo && x <= hi && (x & (x - 1)) == 0;
 }
 
-// Segments per row: enough (row, head, segment) units to fill the SMs twice,
-// unless rows x heads already occupy at least half of them (splitting then
-// costs more in the extra precision and state passes than it gains).
-// KLA_SEGMENTS overrides (tuning only; the result does not depend on it beyond
-// rounding).
-static int choose_segments(long long units, int NB) {
+// Segments per row. The walk kernel keeps one segment per CTA and
+// `per_sm` CTAs fit on an SM, so the segment count is the largest that keeps
+// every (row, head, segment) unit in one wave: more units would add a partial
+// wave, fewer would leave SMs idle. Rows x heads that already occupy half the
+// SMs are not split (the extra precision and state passes would cost more than
+// they gain). KLA_SEGMENTS overrides (tuning only; the result does not depend
+// on it beyond rounding).
+static int choose_segments(long long units, int NB, int per_sm) {
     const char *env = getenv("KLA_SEGMENTS");
     if (env && *env) {
         int P = atoi(env);
         return P < 1 ? 1 : (P > NB ? NB : P);
     }
-    int sms = sm_count();
-    if (2 * units >= sms) return 1;
-    long long P = (2LL * sms + units - 1) / units;
+    const long long cap = (long long)sm_count() * per_sm;
+    if (2 * units >= cap) return 1;
+    const long long P = cap / units;
     return (int)(P > NB ? NB : P);
 }
 
@@ -107,7 +109,9 @@ static kla_status make_plan(const kla_desc *d, Plan &p, bool precision_only) {
     } else {
         p.NB = (int)((p.T + kBlockTokens - 1) / kBlockTokens);
         if (p.NB < 1) p.NB = 1;
-        int P = precision_only ? p.NB : choose_segments((long long)p.N * p.H, p.NB);
+        // resident walk CTAs per SM: two for the dk = dv = 64 tensor-core kernel
+        const int per_sm = (p.bf16 && p.dk == 64 && p.dv == 64) ? 2 : 1;
+        int P = precision_only ? p.NB : choose_segments((long long)p.N * p.H, p.NB, per_sm);
         p.seg_blocks = (p.NB + P - 1) / P;
         p.P = (p.NB + p.seg_blocks - 1) / p.seg_blocks;
         p.Lseg = (long long)p.seg_blocks * kBlockTokens;

@@ -28,53 +28,84 @@ struct ScanArgs {
 
 // ---- reduce --------------------------------------------------------------
 
-// CTA = one (row, head, block of Lb tokens), 256 threads = (sub-block, key):
-// the block is cut into 256/dk sub-blocks of Lb*dk/256 tokens, each walked by
-// one thread per key (coalesced fp32 loads of a and qn across the keys of a
-// token), and the sub-block products are composed in shared memory.
+// CTA = one (row, head, block of Lb tokens); dk threads = 4 sub-blocks of
+// Lb/4 tokens x dk/4 quads of keys. A thread walks its sub-block for 4
+// consecutive keys (16-byte loads of a and qn, 8-byte loads of bf16 k). The
+// block matrix is carried as its two columns, the images of (1, 0) and (0, 1):
+// each step is the projective chain d <- a^2 d + qn n, n <- n + b d on both
+// columns (b = beta k^2), three fp32 operations per column. The four sub-block
+// products are composed in shared memory. CTAs run head-fastest, so that the
+// heads of one token range (adjacent in memory) are read together.
 template <typename TIn>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(128)
 mobius_reduce_diag(ScanArgs s, const TIn *__restrict__ k, const float *__restrict__ a,
                    const float *__restrict__ qn, const float *__restrict__ beta,
                    float4 *__restrict__ agg) {
-    __shared__ float4 part[256];
-    const int dk = s.dk;
-    const int nsub = 256 / dk;
-    const int i = threadIdx.x % dk, sub = threadIdx.x / dk;
-    const long long pair = blockIdx.x;
-    const int blk = (int)(pair % s.NB);
-    const long long u = pair / s.NB;
+    constexpr int kSub = 4, kLen = kBlockTokens / kSub;
+    __shared__ float4 part[kSub][128];
+    const int dk = s.dk, nq = dk / 4;
+    const int quad = threadIdx.x % nq, sub = threadIdx.x / nq;
+    const long long units = (long long)s.N * s.H;
+    const long long u = blockIdx.x % units;
+    const int blk = (int)(blockIdx.x / units);
     const int n = (int)(u / s.H), h = (int)(u % s.H);
-    const int len = kBlockTokens * dk / 256;
-    const long long t0 = (long long)blk * kBlockTokens + (long long)sub * len;
-    const long long t1 = min(t0 + len, s.T);
-    Mob P{1.f, 0.f, 0.f, 1.f};
-    for (long long t = t0; t < t1; t += 8) {
-        float av[8], qv[8], kv[8], bv[8];
+    const long long t0 = (long long)blk * kBlockTokens + (long long)sub * kLen;
+    const int len = (int)max(0LL, min((long long)kLen, s.T - t0));
+    float n1[4], d1[4], n2[4], d2[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) { n1[c] = 1.f; d1[c] = 0.f; n2[c] = 0.f; d2[c] = 1.f; }
+#pragma unroll
+    for (int half = 0; half < kLen; half += 8) {
+        float4 av[8], qv[8], kv[8];
+        float bv[8];
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
-            av[r] = 1.f; qv[r] = 0.f; kv[r] = 0.f; bv[r] = 0.f;
-            if (t + r < t1) {
-                const long long th = ((long long)n * s.T + t + r) * s.H + h;
-                av[r] = __ldg(a + th * dk + i);
-                qv[r] = __ldg(qn + th * dk + i);
-                kv[r] = ld_in(k + th * dk + i);
+            av[r] = make_float4(1.f, 1.f, 1.f, 1.f);
+            qv[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+            kv[r] = qv[r];
+            bv[r] = 0.f;
+            if (half + r < len) {
+                const long long th = ((long long)n * s.T + t0 + half + r) * s.H + h;
+                av[r] = ld4(a + th * dk + 4 * quad);
+                qv[r] = ld4(qn + th * dk + 4 * quad);
+                kv[r] = ld4(k + th * dk + 4 * quad);
                 bv[r] = __ldg(beta + th);
             }
         }
 #pragma unroll
-        for (int r = 0; r < 8; ++r) P = mob_mul(mob_step(av[r], qv[r], bv[r] * kv[r] * kv[r]), P);
-        P = mob_norm(P);
+        for (int r = 0; r < 8; ++r) {
+            const float *ap = &av[r].x, *qp = &qv[r].x, *kp = &kv[r].x;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const float a2 = ap[c] * ap[c], b = bv[r] * kp[c] * kp[c];
+                d1[c] = fmaf(a2, d1[c], qp[c] * n1[c]);
+                n1[c] = fmaf(b, d1[c], n1[c]);
+                d2[c] = fmaf(a2, d2[c], qp[c] * n2[c]);
+                n2[c] = fmaf(b, d2[c], n2[c]);
+            }
+        }
+        // exact power-of-two rescale of each key's matrix (entries are >= 0)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const Mob m = mob_norm(Mob{n1[c], n2[c], d1[c], d2[c]});
+            n1[c] = m.m00; n2[c] = m.m01; d1[c] = m.m10; d2[c] = m.m11;
+        }
     }
-    part[threadIdx.x] = make_float4(P.m00, P.m01, P.m10, P.m11);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) part[sub][4 * quad + c] = make_float4(n1[c], n2[c], d1[c], d2[c]);
     __syncthreads();
     if (sub == 0) {
-        Mob acc = P;
-        for (int b = 1; b < nsub; ++b) {
-            const float4 m = part[b * dk + i];
-            acc = mob_norm(mob_mul(Mob{m.x, m.y, m.z, m.w}, acc));
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            const int i = 4 * quad + c;
+            Mob acc{n1[c], n2[c], d1[c], d2[c]};
+#pragma unroll
+            for (int b = 1; b < kSub; ++b) {
+                const float4 m = part[b][i];
+                acc = mob_norm(mob_mul(Mob{m.x, m.y, m.z, m.w}, acc));
+            }
+            agg[(u * s.NB + blk) * dk + i] = make_float4(acc.m00, acc.m01, acc.m10, acc.m11);
         }
-        agg[pair * dk + i] = make_float4(acc.m00, acc.m01, acc.m10, acc.m11);
     }
 }
 
@@ -279,7 +310,7 @@ cudaError_t launch_mobius_reduce(const Plan &p, const void *k, const float *a, c
         mobius_reduce_iso<TIn><<<blocks_for(pairs, 128), 128, 0, st>>>(
             s, (const TIn *)k, a, qn, beta, agg);
     else
-        mobius_reduce_diag<TIn><<<(unsigned)pairs, 256, 0, st>>>(s, (const TIn *)k, a, qn, beta, agg);
+        mobius_reduce_diag<TIn><<<(unsigned)pairs, p.dk, 0, st>>>(s, (const TIn *)k, a, qn, beta, agg);
     return cudaGetLastError();
 }
 
