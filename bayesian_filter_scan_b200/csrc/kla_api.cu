@@ -22,7 +22,7 @@ __device__ int g_status = 0;
 
 template <typename TIn>
 cudaError_t launch_mobius_reduce(const Plan &, const void *, const float *, const float *,
-                                 const float *, float4 *, cudaStream_t);
+                                 const float *, float4 *, int *, cudaStream_t);
 cudaError_t launch_mobius_carry(const Plan &, const float4 *, const float *, float *, cudaStream_t);
 template <typename TIn>
 cudaError_t launch_mobius_emit(const Plan &, const int *, const void *, const float *, const float *,
@@ -104,6 +104,7 @@ static kla_status make_plan(const kla_desc *d, Plan &p, bool precision_only) {
     p.bf16 = d->dtype == KLA_BF16;
     p.T = d->T;
     p.ntok = (long long)d->B * d->T;
+    p.sms = sm_count();
     if (p.varlen) {
         p.NB = 1; p.P = 1; p.seg_blocks = 1; p.Lseg = 0;
     } else {
@@ -204,8 +205,8 @@ static kla_status forward_impl(const kla_desc *d, const void *q, const void *k, 
     };
     mark(0);
     if (p.P > 1) {
-        e = p.bf16 ? launch_mobius_reduce<__nv_bfloat16>(p, k, a, qn, beta, agg, st)
-                   : launch_mobius_reduce<float>(p, k, a, qn, beta, agg, st);
+        e = p.bf16 ? launch_mobius_reduce<__nv_bfloat16>(p, k, a, qn, beta, agg, status, st)
+                   : launch_mobius_reduce<float>(p, k, a, qn, beta, agg, status, st);
         mark(1);
         if (e == cudaSuccess) e = launch_mobius_carry(p, agg, lambda0, lam_blk, st);
         mark(2);
@@ -276,10 +277,12 @@ kla_status kla_precision(const kla_desc *d, const void *k, const float *a, const
     char *w = (char *)ws;
     float4 *agg = (float4 *)(w + p.off_agg);
     float *lam_blk = (float *)(w + p.off_lam);
+    int *status = status_ptr();
+    if (!status) return KLA_ERR_CUDA;
     cudaError_t e = cudaSuccess;
     if (!p.varlen) {
-        e = p.bf16 ? launch_mobius_reduce<__nv_bfloat16>(p, k, a, qn, beta, agg, st)
-                   : launch_mobius_reduce<float>(p, k, a, qn, beta, agg, st);
+        e = p.bf16 ? launch_mobius_reduce<__nv_bfloat16>(p, k, a, qn, beta, agg, status, st)
+                   : launch_mobius_reduce<float>(p, k, a, qn, beta, agg, status, st);
         if (e == cudaSuccess) e = launch_mobius_carry(p, agg, lambda0, lam_blk, st);
     }
     if (e == cudaSuccess)

@@ -1008,9 +1008,11 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
+}  // namespace
+
 // 3-D map over [ntok][H][inner] (inner contiguous) with box (box_inner, 1, box_rows).
-bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int esize, int inner, int H, long long ntok,
-              int box_inner, int box_rows, bool swizzle) {
+bool make_tma_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int esize, int inner, int H,
+                  long long ntok, int box_inner, int box_rows, bool swizzle) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)H, (cuuint64_t)ntok};
@@ -1023,6 +1025,8 @@ bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int esiz
     return r == CUDA_SUCCESS;
 }
 
+namespace {
+
 template <int DK, int DV>
 cudaError_t launch_t(const Plan &p, const int *cu, int mode, const void *q, const void *k, const void *v,
                      const float *a, const float *qn, const float *beta, const float *lambda0, const float *eta0,
@@ -1031,12 +1035,12 @@ cudaError_t launch_t(const Plan &p, const int *cu, int mode, const void *q, cons
     using L = Layout<DK, DV>;
     CUtensorMap mq, mk, mv, ma, mqn;
     const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, F32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
-    bool ok = make_map(&mq, q, BF, 2, DK, p.H, p.ntok, 64, kC, true) &&
-              make_map(&mk, k, BF, 2, DK, p.H, p.ntok, 64, kC, true) &&
-              make_map(&mv, v, BF, 2, DV, p.H, p.ntok, 64, kC, true);
+    bool ok = make_tma_map(&mq, q, BF, 2, DK, p.H, p.ntok, 64, kC, true) &&
+              make_tma_map(&mk, k, BF, 2, DK, p.H, p.ntok, 64, kC, true) &&
+              make_tma_map(&mv, v, BF, 2, DV, p.H, p.ntok, 64, kC, true);
     if (ok && !p.iso)
-        ok = make_map(&ma, a, F32, 4, DK, p.H, p.ntok, DK, kSlotTok, false) &&
-             make_map(&mqn, qn, F32, 4, DK, p.H, p.ntok, DK, kSlotTok, false);
+        ok = make_tma_map(&ma, a, F32, 4, DK, p.H, p.ntok, DK, kSlotTok, false) &&
+             make_tma_map(&mqn, qn, F32, 4, DK, p.H, p.ntok, DK, kSlotTok, false);
     else { ma = mq; mqn = mq; }
     if (!ok) return cudaErrorInvalidValue;
     static bool attr[64] = {};

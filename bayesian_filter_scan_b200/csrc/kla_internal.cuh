@@ -11,6 +11,7 @@
 // start at row starts; segments are whole numbers of blocks.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -34,6 +35,7 @@ struct Plan {
     int NB;         // Moebius blocks per row (non-varlen)
     int P;          // segments per row (1 for varlen)
     int seg_blocks; // blocks per segment
+    int sms;        // SMs of the current device
     long long Lseg; // tokens per segment (seg_blocks * kBlockTokens)
     // workspace layout (byte offsets; all 256-byte aligned)
     size_t off_agg, off_lam, off_dS, off_decay, bytes;
@@ -54,6 +56,11 @@ __device__ __forceinline__ float4 ld4(const __nv_bfloat16 *p) {
     float2 a = __bfloat1622float2(lo), b = __bfloat1622float2(hi);
     return make_float4(a.x, a.y, b.x, b.y);
 }
+
+// 3-D TMA tensor map over [ntok][H][inner] (inner contiguous) with box
+// (box_inner, 1, box_rows); false if the driver entry point or the encoding fails.
+bool make_tma_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int esize, int inner, int H,
+                  long long ntok, int box_inner, int box_rows, bool swizzle);
 
 // 2x2 Moebius matrix (m00, m01, m10, m11) acting as x -> (m00 x + m01)/(m10 x + m11).
 struct Mob { float m00, m01, m10, m11; };

@@ -6,16 +6,20 @@
 //
 // Three kernels, no inter-CTA waiting (reduce, then scan, then re-walk):
 //   mobius_reduce : per (row, head, block of Lb tokens, key) the composed 2x2
-//                   matrix of the block (normalised by powers of two); one CTA
-//                   per block, sub-blocks of dk tokens per thread, composed in
-//                   shared memory.
+//                   matrix of the block (normalised by powers of two); diagonal
+//                   mode streams a, qn, k through a TMA-fed shared-memory ring
+//                   in persistent CTAs, eight 8-token sub-blocks per block
+//                   composed by a tree in shared memory.
 //   mobius_carry  : per (row, head, key) one warp: the product of each
 //                   segment's blocks, a shuffle scan over segments, applied to
 //                   lambda0: lambda at every segment start.
 //   mobius_emit   : per (row/sequence, head, block, key) re-walks the block
 //                   from its start lambda and writes lambda after every token
 //                   (the kla_precision output; there segments are blocks).
+#include <algorithm>
+
 #include "kla_internal.cuh"
+#include "kla_tc_ptx.cuh"
 
 namespace kla {
 
@@ -28,85 +32,165 @@ struct ScanArgs {
 
 // ---- reduce --------------------------------------------------------------
 
-// CTA = one (row, head, block of Lb tokens); dk threads = 4 sub-blocks of
-// Lb/4 tokens x dk/4 quads of keys. A thread walks its sub-block for 4
-// consecutive keys (16-byte loads of a and qn, 8-byte loads of bf16 k). The
-// block matrix is carried as its two columns, the images of (1, 0) and (0, 1):
-// each step is the projective chain d <- a^2 d + qn n, n <- n + b d on both
-// columns (b = beta k^2), three fp32 operations per column. The four sub-block
-// products are composed in shared memory. CTAs run head-fastest, so that the
-// heads of one token range (adjacent in memory) are read together.
+// Diagonal: per (row, head, block of Lb tokens, key) the composed block
+// matrix, carried as its two columns, the images of (1, 0) and (0, 1): each
+// step is the projective chain d <- a^2 d + qn n, n <- n + b d on both columns
+// (b = beta k^2), three fp32 operations per column. Persistent and TMA-fed:
+// work item = (block of Lb
+// tokens, row x head, half of the keys: min(dk, 64) keys), head-fastest. A CTA
+// of 8 sub-blocks x (keys/4) quads streams its items through a 2-stage
+// shared-memory ring filled by TMA (a, qn fp32 and k tiles of Lb rows), so the
+// loads in flight do not occupy registers; beta of the next item is loaded
+// into registers while the current one is composed. Thread 0 issues the
+// copies; every wait is bounded (on timeout the status bit is set and the CTA
+// stops after its copies in flight have landed).
+constexpr int kRedStages = 2;
+constexpr int kRedSub = 8, kRedLen = kBlockTokens / kRedSub;
+
+__host__ __device__ constexpr int red_stage_bytes(int dki, int kes) { return kBlockTokens * dki * (8 + kes); }
+
 template <typename TIn>
-__global__ void __launch_bounds__(128)
-mobius_reduce_diag(ScanArgs s, const TIn *__restrict__ k, const float *__restrict__ a,
-                   const float *__restrict__ qn, const float *__restrict__ beta,
-                   float4 *__restrict__ agg) {
-    constexpr int kSub = 4, kLen = kBlockTokens / kSub;
-    __shared__ float4 part[kSub][128];
-    const int dk = s.dk, nq = dk / 4;
+__global__ void __launch_bounds__(128, 2)
+mobius_reduce_tma(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_qn,
+                  const __grid_constant__ CUtensorMap tm_k, ScanArgs s, const float *__restrict__ beta,
+                  float4 *__restrict__ agg, long long nitems, int *status) {
+    using namespace ptx;
+    const int dki = min(s.dk, 64), nq = dki / 4, nhalf = s.dk / dki;
+    const int stA = kBlockTokens * dki * 4, stK = kBlockTokens * dki * (int)sizeof(TIn);
+    const int stB = 2 * stA + stK;
+    extern __shared__ __align__(128) uint8_t smraw[];
+    float4 *part = reinterpret_cast<float4 *>(smraw + kRedStages * stB);    // [kRedSub][64]
+    uint64_t *full = reinterpret_cast<uint64_t *>(part + kRedSub * 64), *empty = full + kRedStages;
     const int quad = threadIdx.x % nq, sub = threadIdx.x / nq;
     const long long units = (long long)s.N * s.H;
-    const long long u = blockIdx.x % units;
-    const int blk = (int)(blockIdx.x / units);
-    const int n = (int)(u / s.H), h = (int)(u % s.H);
-    const long long t0 = (long long)blk * kBlockTokens + (long long)sub * kLen;
-    const int len = (int)max(0LL, min((long long)kLen, s.T - t0));
-    float n1[4], d1[4], n2[4], d2[4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) { n1[c] = 1.f; d1[c] = 0.f; n2[c] = 0.f; d2[c] = 1.f; }
-#pragma unroll
-    for (int half = 0; half < kLen; half += 8) {
-        float4 av[8], qv[8], kv[8];
-        float bv[8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            av[r] = make_float4(1.f, 1.f, 1.f, 1.f);
-            qv[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-            kv[r] = qv[r];
-            bv[r] = 0.f;
-            if (half + r < len) {
-                const long long th = ((long long)n * s.T + t0 + half + r) * s.H + h;
-                av[r] = ld4(a + th * dk + 4 * quad);
-                qv[r] = ld4(qn + th * dk + 4 * quad);
-                kv[r] = ld4(k + th * dk + 4 * quad);
-                bv[r] = __ldg(beta + th);
-            }
+    const long long step = gridDim.x;
+    if (threadIdx.x == 0) {
+        for (int j = 0; j < kRedStages; ++j) {
+            mbar_init(&full[j], 1);
+            mbar_init(&empty[j], blockDim.x);
         }
-#pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            const float *ap = &av[r].x, *qp = &qv[r].x, *kp = &kv[r].x;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const float a2 = ap[c] * ap[c], b = bv[r] * kp[c] * kp[c];
-                d1[c] = fmaf(a2, d1[c], qp[c] * n1[c]);
-                n1[c] = fmaf(b, d1[c], n1[c]);
-                d2[c] = fmaf(a2, d2[c], qp[c] * n2[c]);
-                n2[c] = fmaf(b, d2[c], n2[c]);
-            }
-        }
-        // exact power-of-two rescale of each key's matrix (entries are >= 0)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const Mob m = mob_norm(Mob{n1[c], n2[c], d1[c], d2[c]});
-            n1[c] = m.m00; n2[c] = m.m01; d1[c] = m.m10; d2[c] = m.m11;
-        }
+        fence_mbar_init();
     }
-#pragma unroll
-    for (int c = 0; c < 4; ++c) part[sub][4 * quad + c] = make_float4(n1[c], n2[c], d1[c], d2[c]);
     __syncthreads();
-    if (sub == 0) {
+    auto decode = [&](long long w, long long &u, int &blk, int &half) {
+        half = (int)(w % nhalf);
+        const long long r = w / nhalf;
+        u = r % units;
+        blk = (int)(r / units);
+    };
+    auto issue = [&](long long w, int st) {
+        long long u; int blk, half;
+        decode(w, u, blk, half);
+        const int n = (int)(u / s.H), h = (int)(u % s.H);
+        const int tok = (int)((long long)n * s.T + (long long)blk * kBlockTokens);
+        uint8_t *d = smraw + st * stB;
+        mbar_expect_tx(&full[st], stB);
+        tma_load_3d(d, &tm_a, &full[st], half * dki, h, tok);
+        tma_load_3d(d + stA, &tm_qn, &full[st], half * dki, h, tok);
+        tma_load_3d(d + 2 * stA, &tm_k, &full[st], half * dki, h, tok);
+    };
+    auto wait = [&](uint64_t *bar, uint32_t par) -> bool {
+        if (mbar_try_wait(bar, par)) return true;
+        const uint64_t t0 = globaltimer();
+        while (!mbar_try_wait_sleep(bar, par, 20000u))
+            if (globaltimer() - t0 > 2000000000ull) { atomicOr(status, kStatusTimeout); return false; }
+        return true;
+    };
+    long long nmine = 0;
+    if ((long long)blockIdx.x < nitems) nmine = (nitems - 1 - blockIdx.x) / step + 1;
+    if (threadIdx.x == 0)
+        for (int j = 0; j < kRedStages && j < nmine; ++j) issue(blockIdx.x + j * step, j);
+    float bv[kRedLen];
+    auto load_beta = [&](long long w) {
+        long long u; int blk, half;
+        decode(w, u, blk, half);
+        const int n = (int)(u / s.H), h = (int)(u % s.H);
+        const long long t0 = (long long)blk * kBlockTokens + sub * kRedLen;
+#pragma unroll
+        for (int r = 0; r < kRedLen; ++r)
+            bv[r] = t0 + r < s.T ? __ldg(beta + ((long long)n * s.T + t0 + r) * s.H + h) : 0.f;
+    };
+    if (nmine > 0) load_beta(blockIdx.x);
+    bool ok = true;
+    long long issued = min((long long)kRedStages, nmine), consumed = 0;
+    for (long long j = 0; j < nmine; ++j) {
+        const int st = (int)(j % kRedStages);
+        const long long w = blockIdx.x + j * step;
+        long long u; int blk, half;
+        decode(w, u, blk, half);
+        const long long t0 = (long long)blk * kBlockTokens + sub * kRedLen;
+        const int len = (int)max(0LL, min((long long)kRedLen, s.T - t0));
+        float cb[kRedLen];
+#pragma unroll
+        for (int r = 0; r < kRedLen; ++r) cb[r] = bv[r];
+        if (j + 1 < nmine) load_beta(w + step);
+        // every thread waits; the CTA goes on only if all saw the copy land
+        if (!__syncthreads_and(wait(&full[st], (uint32_t)((j / kRedStages) & 1)))) { ok = false; consumed = j; break; }
+        const uint8_t *d = smraw + st * stB;
+        const float *sa = reinterpret_cast<const float *>(d) + (sub * kRedLen) * dki + 4 * quad;
+        const float *sq = reinterpret_cast<const float *>(d + stA) + (sub * kRedLen) * dki + 4 * quad;
+        const TIn *sk = reinterpret_cast<const TIn *>(d + 2 * stA) + (sub * kRedLen) * dki + 4 * quad;
+        float4 av[kRedLen], qv[kRedLen], kv[kRedLen];
+#pragma unroll
+        for (int r = 0; r < kRedLen; ++r) {
+            av[r] = *reinterpret_cast<const float4 *>(sa + r * dki);
+            qv[r] = *reinterpret_cast<const float4 *>(sq + r * dki);
+            if constexpr (sizeof(TIn) == 2) {
+                const uint2 x = *reinterpret_cast<const uint2 *>(sk + r * dki);
+                kv[r] = make_float4(__uint_as_float(x.x << 16), __uint_as_float(x.x & 0xffff0000u),
+                                    __uint_as_float(x.y << 16), __uint_as_float(x.y & 0xffff0000u));
+            } else {
+                kv[r] = *reinterpret_cast<const float4 *>(sk + r * dki);
+            }
+        }
+        // stage read into registers: release it, and refill it with the item kRedStages ahead
+        mbar_arrive(&empty[st]);
+        if (threadIdx.x == 0 && issued < nmine) {
+            if (!wait(&empty[st], (uint32_t)((j / kRedStages) & 1))) { ok = false; }
+            else { issue(blockIdx.x + issued * step, st); ++issued; }
+        }
+        Mob m[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-            const int i = 4 * quad + c;
-            Mob acc{n1[c], n2[c], d1[c], d2[c]};
+            float n1 = 1.f, d1 = 0.f, n2 = 0.f, d2 = 1.f;
 #pragma unroll
-            for (int b = 1; b < kSub; ++b) {
-                const float4 m = part[b][i];
-                acc = mob_norm(mob_mul(Mob{m.x, m.y, m.z, m.w}, acc));
+            for (int r = 0; r < kRedLen; ++r) {
+                if (r < len) {
+                    const float ac = (&av[r].x)[c], qc = (&qv[r].x)[c], kc = (&kv[r].x)[c];
+                    const float a2 = ac * ac, b = cb[r] * kc * kc;
+                    d1 = fmaf(a2, d1, qc * n1);
+                    n1 = fmaf(b, d1, n1);
+                    d2 = fmaf(a2, d2, qc * n2);
+                    n2 = fmaf(b, d2, n2);
+                }
             }
-            agg[(u * s.NB + blk) * dk + i] = make_float4(acc.m00, acc.m01, acc.m10, acc.m11);
+            m[c] = mob_norm(Mob{n1, n2, d1, d2});
+            part[sub * 64 + 4 * quad + c] = make_float4(m[c].m00, m[c].m01, m[c].m10, m[c].m11);
         }
+#pragma unroll
+        for (int wd = 1; wd < kRedSub; wd <<= 1) {
+            __syncthreads();
+            if ((sub & (2 * wd - 1)) == 0) {
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const float4 x = part[(sub + wd) * 64 + 4 * quad + c];
+                    m[c] = mob_norm(mob_mul(Mob{x.x, x.y, x.z, x.w}, m[c]));
+                    if (2 * wd < kRedSub) part[sub * 64 + 4 * quad + c] = make_float4(m[c].m00, m[c].m01, m[c].m10, m[c].m11);
+                }
+            }
+        }
+        if (sub == 0) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                agg[(u * s.NB + blk) * s.dk + half * dki + 4 * quad + c] =
+                    make_float4(m[c].m00, m[c].m01, m[c].m10, m[c].m11);
+        }
+        // part is rewritten by the next item; a failed refill stops every thread
+        if (!__syncthreads_and(ok)) { ok = false; consumed = j + 1; break; }
     }
+    // on a timeout, the copies issued but not consumed land before the CTA exits
+    if (threadIdx.x == 0 && !ok)
+        for (long long j = consumed; j < issued; ++j) wait(&full[j % kRedStages], (uint32_t)((j / kRedStages) & 1));
 }
 
 // Isotropic: one precision per head; increment beta*|k|^2/dk.
@@ -303,14 +387,36 @@ static inline unsigned blocks_for(long long threads, int per) {
 
 template <typename TIn>
 cudaError_t launch_mobius_reduce(const Plan &p, const void *k, const float *a, const float *qn,
-                                 const float *beta, float4 *agg, cudaStream_t st) {
+                                 const float *beta, float4 *agg, int *status, cudaStream_t st) {
     ScanArgs s{p.N, p.H, p.dk, p.T, p.NB, nullptr};
     long long pairs = (long long)p.N * p.H * p.NB;
-    if (p.iso)
-        mobius_reduce_iso<TIn><<<blocks_for(pairs, 128), 128, 0, st>>>(
-            s, (const TIn *)k, a, qn, beta, agg);
-    else
-        mobius_reduce_diag<TIn><<<(unsigned)pairs, p.dk, 0, st>>>(s, (const TIn *)k, a, qn, beta, agg);
+    if (p.iso) {
+        mobius_reduce_iso<TIn><<<blocks_for(pairs, 128), 128, 0, st>>>(s, (const TIn *)k, a, qn, beta, agg);
+        return cudaGetLastError();
+    }
+    const int dki = p.dk < 64 ? p.dk : 64, nhalf = p.dk / dki;
+    const int kes = (int)sizeof(TIn);
+    const CUtensorMapDataType F32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const CUtensorMapDataType KT = kes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : F32;
+    CUtensorMap ma, mq, mk;
+    if (!make_tma_map(&ma, a, F32, 4, p.dk, p.H, p.ntok, dki, kBlockTokens, false) ||
+        !make_tma_map(&mq, qn, F32, 4, p.dk, p.H, p.ntok, dki, kBlockTokens, false) ||
+        !make_tma_map(&mk, k, KT, kes, p.dk, p.H, p.ntok, dki, kBlockTokens, false))
+        return cudaErrorInvalidValue;
+    const int smem = kRedStages * red_stage_bytes(dki, kes) + kRedSub * 64 * 16 + 2 * kRedStages * 8;
+    static bool attr[2][64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 64 && !attr[kes == 2][dev]) {
+        // the largest request (64-key items) once per device and input type
+        const int smax = kRedStages * red_stage_bytes(64, kes) + kRedSub * 64 * 16 + 2 * kRedStages * 8;
+        cudaError_t e = cudaFuncSetAttribute(mobius_reduce_tma<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, smax);
+        if (e != cudaSuccess) return e;
+        attr[kes == 2][dev] = true;
+    }
+    const long long nitems = pairs * nhalf;
+    const long long grid = std::min(nitems, 2LL * p.sms);
+    mobius_reduce_tma<TIn><<<(unsigned)grid, kRedSub * dki / 4, smem, st>>>(ma, mq, mk, s, beta, agg, nitems, status);
     return cudaGetLastError();
 }
 
@@ -338,9 +444,9 @@ cudaError_t launch_mobius_emit(const Plan &p, const int *cu, const void *k, cons
 }
 
 template cudaError_t launch_mobius_reduce<float>(const Plan &, const void *, const float *,
-                                                 const float *, const float *, float4 *, cudaStream_t);
+                                                 const float *, const float *, float4 *, int *, cudaStream_t);
 template cudaError_t launch_mobius_reduce<__nv_bfloat16>(const Plan &, const void *, const float *,
-                                                         const float *, const float *, float4 *,
+                                                         const float *, const float *, float4 *, int *,
                                                          cudaStream_t);
 template cudaError_t launch_mobius_emit<float>(const Plan &, const int *, const void *, const float *,
                                                const float *, const float *, const float *,
