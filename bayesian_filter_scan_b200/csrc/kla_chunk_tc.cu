@@ -20,9 +20,10 @@
 //
 // CTA = one segment of one (row or packed sequence, head); 320 threads:
 //   warps 0-3  gate: per key, the lambda recursion over the chunk (a, qn stream
-//              through a 4-slot TMA ring), log-gates, then Q'/K' written in
+//              through a 5-slot TMA ring), log-gates, then Q'/K' written in
 //              place over the TMA-loaded q/k tiles (bf16, 128B-swizzled), and
-//              the bf16 remainder of K' for a two-term state update;
+//              the bf16 remainder of K' for a two-term state update, slot by
+//              slot (the gate warps fold every slot themselves);
 //              isotropic mode runs a warp-level Moebius scan over the chunk;
 //   warps 4-7  epilogue: rescale U in TMEM and snapshot it to bf16 shared
 //              memory, mask the score tile into P, store the output rows;
@@ -62,11 +63,6 @@ struct Roles {
     static constexpr int PRODW = (NGW == 2) ? 1 : 8;
     static constexpr int MMAW = (NGW == 2) ? 3 : 9;
 };
-// The last kSlotsPerChunk - kSplit slots of every full chunk are folded by the
-// epilogue warps (idle while the gate works), from the chain state the gate
-// warps publish at each of those slots.
-constexpr int kSplit = 6;
-constexpr int kBSlots = 8 - kSplit;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 struct TcArgs {
@@ -97,14 +93,12 @@ struct Layout {
     static constexpr int ring0 = klo0 + 2 * QK;
     static constexpr int fac0 = ring0 + kSlots * 2 * SLOTF * 4;
     static constexpr int facf0 = fac0 + 2 * DK * 4;
-    // chain state at each epilogue-folded slot, per stage: [stage][slot][n, d, PA, E, F][DK], then R[DK]
-    static constexpr int BSTW = kBSlots * 5 + 1;  // words per key and stage
-    static constexpr int bst0 = facf0 + DK * 4;
-    static constexpr int bar0 = ((bst0 + 2 * BSTW * DK * 4) + 7) & ~7;
-    static constexpr int NBAR = 6 + 2 * kSlots + 8 + 2 * kBSlots;
+    static constexpr int bar0 = ((facf0 + DK * 4) + 7) & ~7;
+    static constexpr int NBAR = 6 + 2 * kSlots + 8;
     static constexpr int hold0 = bar0 + NBAR * 8;
     static constexpr int bytes = hold0 + 16;
     static constexpr int alloc = bytes + 1024;
+    static_assert(alloc <= 232448, "shared memory per CTA");
     static constexpr uint32_t NCOLS = (2 * DV + 64 <= 256) ? 256u : 512u;
     static constexpr uint32_t colU = 0, colO = DV, colS = 2 * DV;
 };
@@ -178,31 +172,27 @@ __device__ __forceinline__ float row_sumsq(const uint8_t *ktile, int row) {
 // key i of this thread. The precision runs in projective form, lambda = n/d:
 //   d <- a^2 d + qn n,   n <- n + b d   (b = beta k^2),   PA <- PA a,
 // two FMAs per token on the serial chain; with G the cumulative log2 gate,
-// 2^G = PA/d and 2^G / lambda = PA/n (n, d, PA carry exponents E, E, F). With
-// FOLD the slot's operands are written over the q/k tiles:
+// 2^G = PA/d and 2^G / lambda = PA/n (n, d, PA carry exponents E, E, F). The
+// slot's operands are then written over the q/k tiles:
 //   K' = beta k 2^(R - G) = beta k (d/PA) mk   (bf16 hi + bf16 remainder)
 //   Q' = q / lambda 2^(G - R) = q (PA/n) mq    (bf16)
 // (mk = 2^(R - (F - E)), mq = 1/mk), packed to bf16 by integer rounding. The
 // chain runs first, then every token's reciprocals and stores, which are
 // independent of one another. Ends with the exact power-of-two rescale.
-// a and qn come from the ring slot ra (RING) or from registers ga, gq.
-// wbar (if not null): wait for it (parity wpar) before the in-place stores.
-// Returns false if that wait gave up.
-template <int DK, bool FOLD, bool RING = true>
-__device__ __forceinline__ bool gate_slot(int j, const float *ra, const float (&ga)[kSlotTok],
-                                          const float (&gq)[kSlotTok], uint8_t *qt, uint8_t *kt, uint8_t *klo,
+// a and qn come from the ring slot ra.
+template <int DK>
+__device__ __forceinline__ void gate_slot(int j, const float *ra, uint8_t *qt, uint8_t *kt, uint8_t *klo,
                                           const int (&offr)[kSlotTok], float bsrc, bool state_mode, int R,
-                                          float &nn, float &dd, float &pa, int &E, int &F, float &mq,
-                                          float &mk, float &rkmin, float &rkmax, uint64_t *wbar, uint32_t wpar,
-                                          volatile int *abort_flag, int *status) {
+                                          float &nn, float &dd, float &pa, int &E, int &F, float &mq, float &mk,
+                                          float &rkmin, float &rkmax) {
     constexpr int SLOTF = kSlotTok * DK;
     float xa[kSlotTok], xn[kSlotTok], xk[kSlotTok], xq[kSlotTok];
 #pragma unroll
     for (int r = 0; r < kSlotTok; ++r) {
-        xa[r] = RING ? ra[r * DK] : ga[r];
-        xn[r] = RING ? ra[SLOTF + r * DK] : gq[r];
+        xa[r] = ra[r * DK];
+        xn[r] = ra[SLOTF + r * DK];
         xk[r] = bf_at(kt, j * 1024 + offr[r]);
-        if (FOLD) xq[r] = state_mode ? 0.f : bf_at(qt, j * 1024 + offr[r]);
+        xq[r] = state_mode ? 0.f : bf_at(qt, j * 1024 + offr[r]);
     }
     float bk[kSlotTok], nt[kSlotTok], pt[kSlotTok], dt[kSlotTok];
 #pragma unroll
@@ -217,27 +207,23 @@ __device__ __forceinline__ bool gate_slot(int j, const float *ra, const float (&
         pt[r] = pa;
         dt[r] = dd;
     }
-    if (FOLD) {
-        if (wbar && !waitw(wbar, wpar, abort_flag, status)) return false;
+#pragma unroll
+    for (int r = 0; r < kSlotTok; ++r) {
+        const float rkm = (dt[r] * mk) * rcp_approx(pt[r]);      // 2^(R - G)
+        rkmin = fminf(rkmin, rkm);
+        rkmax = fmaxf(rkmax, rkm);
+        const float ko = bk[r] * rkm;
+        const uint32_t t = __float_as_uint(ko) + 0x8000u;         // K' hi, rounded
+        const int off = j * 1024 + offr[r];
+        *reinterpret_cast<uint16_t *>(kt + off) = (uint16_t)(t >> 16);
+        *reinterpret_cast<uint16_t *>(klo + off) =
+            (uint16_t)(__float_as_uint(ko - __uint_as_float(t & 0xffff0000u)) >> 16);
+    }
+    if (!state_mode) {
 #pragma unroll
         for (int r = 0; r < kSlotTok; ++r) {
-            const float rkm = (dt[r] * mk) * rcp_approx(pt[r]);      // 2^(R - G)
-            rkmin = fminf(rkmin, rkm);
-            rkmax = fmaxf(rkmax, rkm);
-            const float ko = bk[r] * rkm;
-            const uint32_t t = __float_as_uint(ko) + 0x8000u;         // K' hi, rounded
-            const int off = j * 1024 + offr[r];
-            *reinterpret_cast<uint16_t *>(kt + off) = (uint16_t)(t >> 16);
-            *reinterpret_cast<uint16_t *>(klo + off) =
-                (uint16_t)(__float_as_uint(ko - __uint_as_float(t & 0xffff0000u)) >> 16);
-        }
-        if (!state_mode) {
-#pragma unroll
-            for (int r = 0; r < kSlotTok; ++r) {
-                const float qo = xq[r] * ((pt[r] * mq) * rcp_approx(nt[r]));
-                *reinterpret_cast<uint16_t *>(qt + j * 1024 + offr[r]) =
-                    (uint16_t)((__float_as_uint(qo) + 0x8000u) >> 16);
-            }
+            const float qo = xq[r] * ((pt[r] * mq) * rcp_approx(nt[r]));
+            *reinterpret_cast<uint16_t *>(qt + j * 1024 + offr[r]) = (uint16_t)((__float_as_uint(qo) + 0x8000u) >> 16);
         }
     }
     const int e = ((__float_as_int(dd) >> 23) & 0xff) - 127;
@@ -251,7 +237,6 @@ __device__ __forceinline__ bool gate_slot(int j, const float *ra, const float (&
     const int sh = max(-126, min(127, (F - E) - R));
     mq = __int_as_float((127 + sh) << 23);
     mk = __int_as_float((127 - sh) << 23);
-    return true;
 }
 
 }  // namespace
@@ -272,10 +257,6 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     uint64_t *ring_full = bars + 6, *ring_empty = bars + 6 + kSlots;
     uint64_t *s_full = bars + 6 + 2 * kSlots, *u_ready = s_full + 1, *u_done = s_full + 2, *p_full = s_full + 3;
     uint64_t *o_full = s_full + 4, *o_empty = s_full + 5, *td_bar = s_full + 6, *gate_sync = s_full + 7;
-    // bslot_ready[s * kBSlots + b]: the gate warps published the chain state at
-    // slot kSplit + b and have read that slot's raw k rows
-    uint64_t *bslot_ready = s_full + 8;
-    float *bst = reinterpret_cast<float *>(sm + L::bst0);
     uint32_t *tmem_hold = reinterpret_cast<uint32_t *>(sm + L::hold0);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::hold0 + 4);
     float *fac = reinterpret_cast<float *>(sm + L::fac0);
@@ -304,8 +285,7 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         for (int s = 0; s < 2; ++s) {
             mbar_init(&stage_full[s], 1);
             mbar_init(&stage_empty[s], 1);
-            mbar_init(&qk_ready[s], gate_threads + 128);
-            for (int b = 0; b < kBSlots; ++b) mbar_init(&bslot_ready[s * kBSlots + b], gate_threads);
+            mbar_init(&qk_ready[s], gate_threads);
         }
         for (int j = 0; j < kSlots; ++j) {
             mbar_init(&ring_full[j], 1);
@@ -419,13 +399,9 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
                 const int gs_chunk = F - E;
                 if (nvalid == kC) {
-                    // Full chunk: the chain over every slot, the operands of the first
-                    // kSplit slots; for each later slot the chain state at its start
-                    // is published for the epilogue warps, which fold it.
+                    // Full chunk: the chain and the operands of every slot.
                     float rkmin = 3.0e38f, rkmax = 0.f;
                     const int n0 = c * kSlotsPerChunk;
-                    const float no_regs[kSlotTok] = {};
-                    float *bs = bst + s * L::BSTW * DK;
                     // not unrolled: one slot's code stays resident in the instruction cache
 #pragma unroll 1
                     for (int j = 0; j < kSlotsPerChunk; ++j) {
@@ -433,22 +409,8 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         if (!waitw(&ring_full[slot], (n / kSlots) & 1, abort_flag, g.status)) { ok = false; break; }
                         const float *ra = reinterpret_cast<const float *>(sm + L::ring0) + slot * 2 * L::SLOTF + i;
                         const float bsrc = (j < 4) ? cb0 : cb1;
-                        if (j < kSplit) {
-                            gate_slot<DK, true>(j, ra, no_regs, no_regs, qt, kt, klo, offr, bsrc, state_mode, R, nn, dd,
-                                                pa, E, F, mq, mk, rkmin, rkmax, nullptr, 0, abort_flag, g.status);
-                        } else {
-                            float *b = bs + (j - kSplit) * 5 * DK;
-                            b[i] = nn;
-                            b[DK + i] = dd;
-                            b[2 * DK + i] = pa;
-                            reinterpret_cast<int *>(b)[3 * DK + i] = E;
-                            reinterpret_cast<int *>(b)[4 * DK + i] = F;
-                            if (j == kSplit) reinterpret_cast<int *>(bs)[kBSlots * 5 * DK + i] = R;
-                            gate_slot<DK, false>(j, ra, no_regs, no_regs, qt, kt, klo, offr, bsrc, state_mode, R, nn,
-                                                 dd, pa, E, F, mq, mk, rkmin, rkmax, nullptr, 0, abort_flag, g.status);
-                            // state published and raw k rows read: the epilogue warps may fold
-                            mbar_arrive(&bslot_ready[s * kBSlots + (j - kSplit)]);
-                        }
+                        gate_slot<DK>(j, ra, qt, kt, klo, offr, bsrc, state_mode, R, nn, dd, pa, E, F, mq, mk, rkmin,
+                                      rkmax);
                         // ring slot read into registers: release it (generic reads
                         // ordered before the TMA refill)
                         fence_proxy_async();
@@ -644,36 +606,6 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             else sstart = g.S_io + (u * g.P + p - 1) * DK * DV;
         }
         bool ok = true;
-        // Fold role: the last kBSlots slots of every full diagonal chunk, from the
-        // chain state the gate warps publish. dk = 128: key e, every such slot;
-        // dk = 64: key e % 64, slot kSplit + e / 64. a and qn come straight from
-        // global memory (L2: the producer prefetches two chunks ahead), loaded one
-        // chunk ahead; beta of tokens 32 + lane likewise.
-        constexpr int FPER = (DK == 128) ? kBSlots : 1;
-        static_assert(DK == 128 || kBSlots == 2, "dk = 64 folds one slot per thread");
-        const int fk = e & (DK - 1), fb0 = (DK == 128) ? 0 : (e >> 6);
-        int foffr[kSlotTok];
-#pragma unroll
-        for (int r = 0; r < kSlotTok; ++r) foffr[r] = sw_off(r, fk, kC);
-        float fbeta = 0.f, fa[FPER][kSlotTok], fq[FPER][kSlotTok];
-        auto f_full = [&](int cc) { return !g.iso && tb + (long long)(cc + 1) * kC <= te; };
-        auto f_prefetch = [&](int cc) {
-            const long long t0 = tb + (long long)cc * kC;
-            const long long x1 = t0 + 32 + lane;
-            fbeta = x1 < te ? __ldg(g.beta + x1 * g.H + h) : 0.f;
-            if (f_full(cc)) {
-#pragma unroll
-                for (int sl = 0; sl < FPER; ++sl) {
-                    const long long t = t0 + kSlotTok * (kSplit + fb0 + sl);
-#pragma unroll
-                    for (int r = 0; r < kSlotTok; ++r) {
-                        const long long o = ((t + r) * g.H + h) * DK + fk;
-                        fa[sl][r] = __ldg(g.a + o);
-                        fq[sl][r] = __ldg(g.qn + o);
-                    }
-                }
-            }
-        };
         // output rows of chunk cc (TMEM O -> bf16 -> global)
         auto emit_out = [&](int cc) -> bool {
             if (!waitw(o_full, cc & 1, abort_flag, g.status)) return false;
@@ -707,40 +639,8 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             mbar_arrive(o_empty);
             return true;
         };
-        if (nchunks > 0) f_prefetch(0);
         for (int c = 0; c < nchunks; ++c) {
             const int s = c & 1;
-            // ---- fold: the epilogue-folded slots of chunk c
-            if (f_full(c)) {
-                uint8_t *qt = sm + L::q0 + s * L::QK;
-                uint8_t *kt = sm + L::k0 + s * L::QK;
-                uint8_t *klo = sm + L::klo0 + s * L::QK;
-                if (!waitw(&stage_full[s], (c >> 1) & 1, abort_flag, g.status)) { ok = false; break; }
-                const float *bs = bst + s * L::BSTW * DK;
-                float rkmin = 3.0e38f, rkmax = 0.f;
-#pragma unroll
-                for (int sl = 0; sl < FPER; ++sl) {
-                    const int b = fb0 + sl, j = kSplit + b;
-                    if (!waitw(&bslot_ready[s * kBSlots + b], (c >> 1) & 1, abort_flag, g.status)) { ok = false; break; }
-                    // published before the barrier: state at slot j and the chunk's reference
-                    const float *st = bs + b * 5 * DK;
-                    const int *sti = reinterpret_cast<const int *>(st);
-                    const int R = reinterpret_cast<const int *>(bs)[kBSlots * 5 * DK + fk];
-                    float nn = st[fk], dd = st[DK + fk], pa = st[2 * DK + fk];
-                    int E = sti[3 * DK + fk], F = sti[4 * DK + fk];
-                    const int sh = max(-126, min(127, (F - E) - R));
-                    float mq = __int_as_float((127 + sh) << 23), mk = __int_as_float((127 - sh) << 23);
-                    gate_slot<DK, true, false>(j, nullptr, fa[sl], fq[sl], qt, kt, klo, foffr, fbeta, state_mode, R, nn,
-                                               dd, pa, E, F, mq, mk, rkmin, rkmax, nullptr, 0, abort_flag, g.status);
-                }
-                if (!ok) break;
-                if ((((__float_as_int(rkmax) >> 23) & 0xff) - 127 >= kMaxOffset) ||
-                    (((__float_as_int(rkmin) >> 23) & 0xff) - 127 < -kMaxOffset))
-                    atomicOr(g.status, kStatusRange);
-            }
-            fence_proxy_async();
-            mbar_arrive(&qk_ready[s]);
-            if (c + 1 < nchunks) f_prefetch(c + 1);
             // ---- output rows of the previous chunk (its MMAs finished meanwhile)
             if (!state_mode && c > 0 && !emit_out(c - 1)) { ok = false; break; }
             // ---- state U_c = diag(fac) * (eta_start or U_{c-1} + K'^T V)
