@@ -31,6 +31,7 @@ cudaError_t launch_walk(const Plan &, const int *, int, const void *, const void
                         const float *, const float *, const float *, const float *, const float *,
                         const float *, float *, float *, void *, float *, float *, cudaStream_t);
 cudaError_t launch_state_carry(const Plan &, const float *, const float *, float *, cudaStream_t);
+cudaError_t launch_seq_order(const Plan &, const int *, int *, cudaStream_t);
 bool chunk_tc_supported(const Plan &);
 cudaError_t launch_chunk_tc(const Plan &, const int *, int, const void *, const void *, const void *,
                             const float *, const float *, const float *, const float *, const float *,
@@ -131,6 +132,12 @@ static kla_status make_plan(const kla_desc *d, Plan &p, bool precision_only) {
         p.off_decay = off;
         off += align256(units * p.P * p.nl * sizeof(float));
     }
+    // longest-first launch order of packed sequences (list scheduling of the
+    // walks: the long ones start first, the short ones fill in behind them)
+    p.order = !precision_only && p.varlen && p.N >= 2 && p.N <= kMaxOrderSeqs;
+    p.off_perm = off;
+    if (p.order) off += align256((size_t)p.N * sizeof(int));
+    p.perm = nullptr;
     p.bytes = off;
     return KLA_OK;
 }
@@ -204,7 +211,12 @@ static kla_status forward_impl(const kla_desc *d, const void *q, const void *k, 
         if (ev && e == cudaSuccess) e = cudaEventRecord(ev[i], st);
     };
     mark(0);
-    if (p.P > 1) {
+    if (p.order) {
+        int *perm = (int *)(w + p.off_perm);
+        e = launch_seq_order(p, cu, perm, st);
+        p.perm = perm;
+    }
+    if (e == cudaSuccess && p.P > 1) {
         e = p.bf16 ? launch_mobius_reduce<__nv_bfloat16>(p, k, a, qn, beta, agg, status, st)
                    : launch_mobius_reduce<float>(p, k, a, qn, beta, agg, status, st);
         mark(1);
@@ -256,7 +268,7 @@ kla_status kla_plan(const kla_desc *d, int *segments_per_row, int *launches, int
     kla_status s = make_plan(d, p, false);
     if (s != KLA_OK) return s;
     if (segments_per_row) *segments_per_row = p.P;
-    if (launches) *launches = p.P > 1 ? 5 : 1;
+    if (launches) *launches = (p.P > 1 ? 5 : 1) + (p.order ? 1 : 0);
     if (tensor_core) *tensor_core = chunk_tc_supported(p) ? 1 : 0;
     return KLA_OK;
 }

@@ -68,7 +68,7 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;
 struct TcArgs {
     int N, H, P, NB, seg_blocks, iso, mode;
     long long T, Lseg;
-    const int *cu;
+    const int *cu, *perm;
     const float *a, *qn, *beta;
     const float *lambda0, *eta0, *lam_blk;
     float *S_io, *decay;
@@ -269,9 +269,13 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const bool is_gate = (RL::NGW == 4) ? (warp < 4) : (warp == 0 || warp == 2);
     const int gt = (RL::NGW == 4) ? tid : ((warp >> 1) * 32 + lane);   // gate rank
     const int P_eff = state_mode ? g.P - 1 : g.P;
-    const long long u = blockIdx.x / P_eff;
+    // unit u = (row or packed sequence n, head h); packed sequences in the
+    // longest-first order when one is given
+    const long long ur = blockIdx.x / P_eff;
     const int p = (int)(blockIdx.x % P_eff);
-    const int n = (int)(u / g.H), h = (int)(u % g.H);
+    const int h = (int)(ur % g.H);
+    const int n = g.perm ? g.perm[ur / g.H] : (int)(ur / g.H);
+    const long long u = (long long)n * g.H + h;
     long long tb, te;
     if (g.cu) { tb = g.cu[n]; te = g.cu[n + 1]; }
     else {
@@ -954,7 +958,7 @@ cudaError_t launch_t(const Plan &p, const int *cu, int mode, const void *q, cons
     }
     TcArgs g;
     g.N = p.N; g.H = p.H; g.P = p.P; g.NB = p.NB; g.seg_blocks = p.seg_blocks; g.iso = p.iso; g.mode = mode;
-    g.T = p.T; g.Lseg = p.Lseg; g.cu = cu;
+    g.T = p.T; g.Lseg = p.Lseg; g.cu = cu; g.perm = cu ? p.perm : nullptr;
     g.a = a; g.qn = qn; g.beta = beta; g.lambda0 = lambda0; g.eta0 = eta0; g.lam_blk = lam_blk;
     g.S_io = S_io; g.decay = decay; g.out = (__nv_bfloat16 *)out;
     g.final_lambda = final_lambda; g.final_eta = final_eta; g.status = status;

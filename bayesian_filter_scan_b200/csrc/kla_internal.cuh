@@ -20,6 +20,7 @@ namespace kla {
 
 constexpr int kBlockTokens = 64;   // Lb: tokens per Moebius-reduction block (one chunk)
 constexpr int kChunk = 64;         // C: tokens per chunk of the chunked form
+constexpr int kMaxOrderSeqs = 1024; // packed sequences ranked by length for the launch order
 
 // Bits of the library's device status word (kla_check reads and clears it);
 // kernels that can detect an error receive its address and OR a bit into it.
@@ -39,6 +40,12 @@ struct Plan {
     long long Lseg; // tokens per segment (seg_blocks * kBlockTokens)
     // workspace layout (byte offsets; all 256-byte aligned)
     size_t off_agg, off_lam, off_dS, off_decay, bytes;
+    // packed sequences: longest-first launch order (int per sequence, in the
+    // workspace at off_perm) when `order`; perm is its device address once the
+    // workspace is known, else nullptr (launch in sequence order)
+    bool order;
+    size_t off_perm;
+    const int *perm;
 };
 
 __device__ __forceinline__ float ld_in(const float *p) { return __ldg(p); }

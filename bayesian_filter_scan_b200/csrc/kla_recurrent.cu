@@ -39,6 +39,7 @@ struct WalkArgs {
     float *decay;              // [u][P][nl] product of gates over a segment
     void *out;
     float *final_lambda, *final_eta;
+    const int *perm;           // longest-first order of packed sequences or nullptr
 };
 
 constexpr int kWalkThreads = 256;
@@ -66,9 +67,11 @@ kla_walk_simt(WalkArgs w) {
     const int tid = threadIdx.x;
     const int j = tid % dv, kg = tid / dv;
     const int P_eff = (w.mode == kState) ? (w.P - 1) : w.P;
-    const long long u = blockIdx.x / P_eff;
+    const long long ur = blockIdx.x / P_eff;
     const int p = (int)(blockIdx.x % P_eff);
-    const int n = (int)(u / w.H), h = (int)(u % w.H);
+    const int h = (int)(ur % w.H);
+    const int n = w.perm ? w.perm[ur / w.H] : (int)(ur / w.H);
+    const long long u = (long long)n * w.H + h;
     long long tb, te;
     if (w.cu) { tb = w.cu[n]; te = w.cu[n + 1]; }
     else {
@@ -243,7 +246,8 @@ cudaError_t launch_walk(const Plan &p, const int *cu, int mode, const void *q, c
                         float *decay, void *out, float *final_lambda, float *final_eta,
                         cudaStream_t st) {
     WalkArgs w{p.N, p.H, p.dk, p.dv, p.nl, p.T, p.Lseg, p.P, p.NB, p.seg_blocks, cu, p.iso, mode,
-               q, k, v, a, qn, beta, lambda0, eta0, lam_blk, S_io, decay, out, final_lambda, final_eta};
+               q, k, v, a, qn, beta, lambda0, eta0, lam_blk, S_io, decay, out, final_lambda, final_eta,
+               cu ? p.perm : nullptr};
     long long segs = (mode == kState) ? (p.P - 1) : p.P;
     unsigned grid = (unsigned)((long long)p.N * p.H * segs);
     if (grid == 0) return cudaSuccess;

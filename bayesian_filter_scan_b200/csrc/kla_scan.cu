@@ -379,6 +379,27 @@ mobius_emit_iso(ScanArgs s, const TIn *__restrict__ k, const float *__restrict__
     }
 }
 
+// ---- launch order of packed sequences -------------------------------------
+
+// perm[r] = the packed sequence of rank r by length, longest first (ties by
+// index). The walk kernels map their block index through it, so the longest
+// walks start first and the short ones fill in behind (list scheduling).
+__global__ void __launch_bounds__(256)
+kla_seq_order(const int *__restrict__ cu, int N, int *__restrict__ perm) {
+    __shared__ int len[kMaxOrderSeqs];
+    for (int i = threadIdx.x; i < N; i += blockDim.x) len[i] = cu[i + 1] - cu[i];
+    __syncthreads();
+    for (int i = threadIdx.x; i < N; i += blockDim.x) {
+        const int li = len[i];
+        int r = 0;
+        for (int j = 0; j < N; ++j) {
+            const int lj = len[j];
+            r += (lj > li) || (lj == li && j < i);
+        }
+        perm[r] = i;
+    }
+}
+
 // ---- host launchers ------------------------------------------------------
 
 static inline unsigned blocks_for(long long threads, int per) {
@@ -417,6 +438,12 @@ cudaError_t launch_mobius_reduce(const Plan &p, const void *k, const float *a, c
     const long long nitems = pairs * nhalf;
     const long long grid = std::min(nitems, 2LL * p.sms);
     mobius_reduce_tma<TIn><<<(unsigned)grid, kRedSub * dki / 4, smem, st>>>(ma, mq, mk, s, beta, agg, nitems, status);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_seq_order(const Plan &p, const int *cu, int *perm, cudaStream_t st) {
+    if (p.N > kMaxOrderSeqs) return cudaErrorInvalidValue;
+    kla_seq_order<<<1, 256, 0, st>>>(cu, p.N, perm);
     return cudaGetLastError();
 }
 

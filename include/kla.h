@@ -79,8 +79,11 @@ typedef struct {
 } kla_desc;
 
 /* Bytes of device workspace kla_forward needs for this descriptor on the
- * current device (0 means the workspace pointer may be NULL). Pure host
- * computation. Returns 0 for an invalid descriptor as well. */
+ * current device (0 means the workspace pointer may be NULL): the Moebius
+ * block aggregates and segment states when rows are split into segments, and
+ * one int per packed sequence (up to 1024 sequences) for the longest-first
+ * launch order. Pure host computation. Returns 0 for an invalid descriptor as
+ * well. */
 size_t kla_workspace_bytes(const kla_desc *desc);
 
 /* Bytes of device workspace kla_precision needs (0: the pointer may be NULL). */
@@ -117,7 +120,8 @@ kla_status kla_forward_profiled(const kla_desc *desc,
 
 /* The work plan kla_forward uses for this descriptor on the current device:
  * segments each row is split into (1: one CTA walks a whole row or packed
- * sequence), kernel launches per call (1 or 5), and whether the chunk stages
+ * sequence), kernel launches per call (1 or 5, plus 1 for the launch order of
+ * packed sequences), and whether the chunk stages
  * run on the tcgen05 tensor-core kernel (1) or the CUDA-core walk (0).
  * Any output pointer may be NULL. Pure host computation. */
 kla_status kla_plan(const kla_desc *desc, int *segments_per_row, int *launches,
