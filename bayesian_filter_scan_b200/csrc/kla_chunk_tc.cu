@@ -93,8 +93,9 @@ struct Layout {
     static constexpr int ring0 = klo0 + 2 * QK;
     static constexpr int fac0 = ring0 + kSlots * 2 * SLOTF * 4;
     static constexpr int facf0 = fac0 + 2 * DK * 4;
-    static constexpr int bar0 = ((facf0 + DK * 4) + 7) & ~7;
-    static constexpr int NBAR = 6 + 2 * kSlots + 8;
+    static constexpr int isof0 = facf0 + DK * 4;   // iso: per-token factors (q, beta k) of a chunk
+    static constexpr int bar0 = ((isof0 + kC * 8) + 7) & ~7;
+    static constexpr int NBAR = 6 + 2 * kSlots + 9;
     static constexpr int hold0 = bar0 + NBAR * 8;
     static constexpr int bytes = hold0 + 16;
     static constexpr int alloc = bytes + 1024;
@@ -257,10 +258,12 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     uint64_t *ring_full = bars + 6, *ring_empty = bars + 6 + kSlots;
     uint64_t *s_full = bars + 6 + 2 * kSlots, *u_ready = s_full + 1, *u_done = s_full + 2, *p_full = s_full + 3;
     uint64_t *o_full = s_full + 4, *o_empty = s_full + 5, *td_bar = s_full + 6, *gate_sync = s_full + 7;
+    uint64_t *gate_sync2 = s_full + 8;   // iso: the chunk's per-token factors are in shared memory
     uint32_t *tmem_hold = reinterpret_cast<uint32_t *>(sm + L::hold0);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::hold0 + 4);
     float *fac = reinterpret_cast<float *>(sm + L::fac0);
     float *fac_final = reinterpret_cast<float *>(sm + L::facf0);
+    float2 *isof = reinterpret_cast<float2 *>(sm + L::isof0);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool state_mode = g.mode == 1;
@@ -303,6 +306,7 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mbar_init(o_empty, 128);
         mbar_init(td_bar, 1);
         mbar_init(gate_sync, gate_threads);
+        mbar_init(gate_sync2, gate_threads);
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -542,39 +546,41 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 glast_log2 = Glast;
                 lam = __shfl_sync(0xffffffffu, lamC, 31);
                 // per-token factors, shared by all keys of the head
-                const float fq0 = exp2f(G0 - Rf) / lamB, fq1 = exp2f(G1 - Rf) / lamC;
-                const float fk0 = exp2f(Rf - G0), fk1 = exp2f(Rf - G1);
                 if (gmax - gmin > 2 * kMaxOffset) atomicOr(g.status, kStatusRange);
-                // every gate warp has read the raw k rows before any overwrites them
+                // every gate warp has read the raw k rows, and the previous chunk's
+                // factors, before any of them is overwritten
                 mbar_arrive(gate_sync);
                 if (!waitw(gate_sync, c & 1, abort_flag, g.status)) { ok = false; break; }
+                // per-token factors, shared by all keys of the head: q / lambda 2^(G-R)
+                // and beta 2^(R-G), zero past the end of the sequence
+                if (warp == 0) {
+                    isof[t0i] = va ? make_float2(exp2f(G0 - Rf) / lamB, cb0 * exp2f(Rf - G0)) : make_float2(0.f, 0.f);
+                    isof[t1i] = vb ? make_float2(exp2f(G1 - Rf) / lamC, cb1 * exp2f(Rf - G1)) : make_float2(0.f, 0.f);
+                }
+                mbar_arrive(gate_sync2);
+                if (!waitw(gate_sync2, c & 1, abort_flag, g.status)) { ok = false; break; }
+#pragma unroll 1
+                for (int j = 0; j < kSlotsPerChunk; ++j) {
+                    float qr[kSlotTok], kr[kSlotTok];
+                    float2 fv[kSlotTok];
 #pragma unroll
-                for (int grp = 0; grp < kC / 8; ++grp) {
-                    float fqv[8], fkv[8], btv[8], qr[8], kr[8];
-#pragma unroll
-                    for (int r = 0; r < 8; ++r) {
-                        const int tau = grp * 8 + r;
-                        fqv[r] = __shfl_sync(0xffffffffu, (tau & 1) ? fq1 : fq0, tau >> 1);
-                        fkv[r] = __shfl_sync(0xffffffffu, (tau & 1) ? fk1 : fk0, tau >> 1);
-                        btv[r] = __shfl_sync(0xffffffffu, (tau & 1) ? cb1 : cb0, tau >> 1);
-                    }
-#pragma unroll
-                    for (int r = 0; r < 8; ++r) {
-                        const int off = sw_off(grp * 8 + r, i, kC);
+                    for (int r = 0; r < kSlotTok; ++r) {
+                        const int off = j * 1024 + offr[r];
                         qr[r] = state_mode ? 0.f : bf_at(qt, off);
                         kr[r] = bf_at(kt, off);
+                        fv[r] = isof[kSlotTok * j + r];
                     }
 #pragma unroll
-                    for (int r = 0; r < 8; ++r) {
-                        const int tau = grp * 8 + r;
-                        const int off = sw_off(tau, i, kC);
-                        const bool valid = tok0 + tau < te;
-                        const float qv = valid ? qr[r] * fqv[r] : 0.f;
-                        const float kv = valid ? btv[r] * kr[r] * fkv[r] : 0.f;
-                        if (!state_mode) bf_put(qt, off, qv);
-                        const __nv_bfloat16 khi = __float2bfloat16_rn(kv);
-                        *reinterpret_cast<__nv_bfloat16 *>(kt + off) = khi;
-                        bf_put(klo, off, kv - __bfloat162float(khi));
+                    for (int r = 0; r < kSlotTok; ++r) {
+                        const int off = j * 1024 + offr[r];
+                        const float ko = kr[r] * fv[r].y;
+                        const uint32_t t = __float_as_uint(ko) + 0x8000u;         // K' hi, rounded
+                        *reinterpret_cast<uint16_t *>(kt + off) = (uint16_t)(t >> 16);
+                        *reinterpret_cast<uint16_t *>(klo + off) =
+                            (uint16_t)(__float_as_uint(ko - __uint_as_float(t & 0xffff0000u)) >> 16);
+                        if (!state_mode)
+                            *reinterpret_cast<uint16_t *>(qt + off) =
+                                (uint16_t)((__float_as_uint(qr[r] * fv[r].x) + 0x8000u) >> 16);
                     }
                 }
             }
