@@ -228,7 +228,8 @@ static kla_status forward_impl(const kla_desc *d, const void *q, const void *k, 
                    : launch_walk(p, cu, 1, q, k, v, a, qn, beta, lambda0, eta0, lam_blk, S_io, decay,
                                  out, final_lambda, final_eta, st);
         mark(3);
-        if (e == cudaSuccess) e = launch_state_carry(p, eta0, decay, S_io, st);
+        // the tensor-core output pass carries the segment states itself
+        if (e == cudaSuccess && !tc) e = launch_state_carry(p, eta0, decay, S_io, st);
         mark(4);
     } else {
         mark(1); mark(2); mark(3); mark(4);
@@ -268,7 +269,7 @@ kla_status kla_plan(const kla_desc *d, int *segments_per_row, int *launches, int
     kla_status s = make_plan(d, p, false);
     if (s != KLA_OK) return s;
     if (segments_per_row) *segments_per_row = p.P;
-    if (launches) *launches = (p.P > 1 ? 5 : 1) + (p.order ? 1 : 0);
+    if (launches) *launches = (p.P > 1 ? (chunk_tc_supported(p) ? 4 : 5) : 1) + (p.order ? 1 : 0);
     if (tensor_core) *tensor_core = chunk_tc_supported(p) ? 1 : 0;
     return KLA_OK;
 }

@@ -610,12 +610,43 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const bool vU = (DK == 128) || v64;
         uint8_t *ub = sm + L::ub0;
         uint8_t *pt = sm + L::p0;
-        const float *sstart = nullptr;
-        if (!state_mode) {
-            if (p == 0) sstart = g.eta0 ? g.eta0 + u * DK * DV : nullptr;
-            else sstart = g.S_io + (u * g.P + p - 1) * DK * DV;
-        }
+        const float *eta0 = (!state_mode && g.eta0) ? g.eta0 + u * DK * DV : nullptr;
         bool ok = true;
+        // Belief at the segment start, written into the U columns of TMEM before
+        // the first chunk (while the gate works on it): eta0 carried through the
+        // transfers of the row's earlier segments, S <- D_q S + dS_q for q < p
+        // (D_q: the segment's gate product per key, dS_q: its state transfer).
+        if (!state_mode && nchunks > 0) {
+            const int nl = g.iso ? 1 : DK;
+#pragma unroll
+            for (int cb = 0; cb < DV / 32; ++cb) {
+                float acc[32];
+#pragma unroll
+                for (int x = 0; x < 32; x += 4) {
+                    const float4 e4 = (vU && eta0) ? *reinterpret_cast<const float4 *>(eta0 + rowU * DV + cb * 32 + x)
+                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+                    acc[x] = e4.x; acc[x + 1] = e4.y; acc[x + 2] = e4.z; acc[x + 3] = e4.w;
+                }
+#pragma unroll 4
+                for (int q = 0; q < p; ++q) {
+                    const float dq = vU ? g.decay[(u * g.P + q) * nl + (g.iso ? 0 : rowU)] : 0.f;
+                    const float *src = g.S_io + ((u * g.P + q) * DK + rowU) * DV + cb * 32;
+#pragma unroll
+                    for (int x = 0; x < 32; x += 4) {
+                        const float4 d4 = vU ? *reinterpret_cast<const float4 *>(src + x) : make_float4(0.f, 0.f, 0.f, 0.f);
+                        acc[x] = fmaf(dq, acc[x], d4.x);
+                        acc[x + 1] = fmaf(dq, acc[x + 1], d4.y);
+                        acc[x + 2] = fmaf(dq, acc[x + 2], d4.z);
+                        acc[x + 3] = fmaf(dq, acc[x + 3], d4.w);
+                    }
+                }
+                uint32_t r[32];
+#pragma unroll
+                for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(acc[x]);
+                tmem_st32(tbase + lane_base + L::colU + cb * 32, r);
+            }
+            tmem_wait_st();
+        }
         // output rows of chunk cc (TMEM O -> bf16 -> global)
         auto emit_out = [&](int cc) -> bool {
             if (!waitw(o_full, cc & 1, abort_flag, g.status)) return false;
@@ -674,15 +705,13 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     }
                 }
             };
-            if (c == 0) {
+            if (c == 0 && state_mode) {
 #pragma unroll
                 for (int cb = 0; cb < DV / 32; ++cb) {
                     uint32_t r[32];
 #pragma unroll
-                    for (int x = 0; x < 32; ++x)
-                        r[x] = __float_as_uint((vU && sstart) ? sstart[rowU * DV + cb * 32 + x] * f : 0.f);
+                    for (int x = 0; x < 32; ++x) r[x] = 0u;
                     tmem_st32(tbase + lane_base + L::colU + cb * 32, r);
-                    snap(r, cb);
                 }
             } else if (rmw || !state_mode) {
 #pragma unroll
@@ -765,7 +794,8 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     }
                 }
             } else if (vU) {
-                for (int x = 0; x < DV; ++x) dst[rowU * DV + x] = sstart ? sstart[rowU * DV + x] : 0.f;
+                // no tokens (an empty packed sequence, a single segment): the belief is eta0
+                for (int x = 0; x < DV; ++x) dst[rowU * DV + x] = eta0 ? eta0[rowU * DV + x] : 0.f;
             }
         }
     } else if (warp == RL::PRODW) {
