@@ -138,6 +138,8 @@ static kla_status make_plan(const kla_desc *d, Plan &p, bool precision_only) {
     p.off_perm = off;
     if (p.order) off += align256((size_t)p.N * sizeof(int));
     p.perm = nullptr;
+    p.inline_carry = false;
+    p.agg = nullptr;
     p.bytes = off;
     return KLA_OK;
 }
@@ -220,7 +222,10 @@ static kla_status forward_impl(const kla_desc *d, const void *q, const void *k, 
         e = p.bf16 ? launch_mobius_reduce<__nv_bfloat16>(p, k, a, qn, beta, agg, status, st)
                    : launch_mobius_reduce<float>(p, k, a, qn, beta, agg, status, st);
         mark(1);
-        if (e == cudaSuccess) e = launch_mobius_carry(p, agg, lambda0, lam_blk, st);
+        // short segments: the tensor-core kernel composes the block aggregates itself
+        p.inline_carry = tc && (long long)(p.P - 1) * p.seg_blocks <= kInlineCarryBlocks;
+        p.agg = agg;
+        if (e == cudaSuccess && !p.inline_carry) e = launch_mobius_carry(p, agg, lambda0, lam_blk, st);
         mark(2);
         if (e == cudaSuccess)
             e = tc ? launch_chunk_tc(p, cu, 1, q, k, v, a, qn, beta, lambda0, eta0, lam_blk, S_io, decay,
@@ -269,7 +274,12 @@ kla_status kla_plan(const kla_desc *d, int *segments_per_row, int *launches, int
     kla_status s = make_plan(d, p, false);
     if (s != KLA_OK) return s;
     if (segments_per_row) *segments_per_row = p.P;
-    if (launches) *launches = (p.P > 1 ? (chunk_tc_supported(p) ? 4 : 5) : 1) + (p.order ? 1 : 0);
+    int n = 1;
+    if (p.P > 1) {
+        const bool tc = chunk_tc_supported(p);
+        n = tc ? ((long long)(p.P - 1) * p.seg_blocks <= kInlineCarryBlocks ? 3 : 4) : 5;
+    }
+    if (launches) *launches = n + (p.order ? 1 : 0);
     if (tensor_core) *tensor_core = chunk_tc_supported(p) ? 1 : 0;
     return KLA_OK;
 }

@@ -71,6 +71,7 @@ struct TcArgs {
     const int *cu, *perm;
     const float *a, *qn, *beta;
     const float *lambda0, *eta0, *lam_blk;
+    const float4 *agg;   // block aggregates when the segment-start precision is composed here
     float *S_io, *decay;
     __nv_bfloat16 *out;
     float *final_lambda, *final_eta;
@@ -334,8 +335,27 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         {
             const int il = g.iso ? 0 : i;
             if (key || g.iso) {
-                if (p == 0) lam = g.lambda0 ? g.lambda0[u * (g.iso ? 1 : DK) + il] : 1.0f;
-                else lam = g.lam_blk[(u * g.NB + (long long)p * g.seg_blocks) * (g.iso ? 1 : DK) + il];
+                const int nl = g.iso ? 1 : DK;
+                lam = g.lambda0 ? g.lambda0[u * nl + il] : 1.0f;
+                if (p > 0 && g.agg) {
+                    // compose the Moebius aggregates of the blocks before this segment
+                    // (in order) and apply them to lambda0
+                    const float4 *src = g.agg + u * g.NB * nl + il;
+                    const int nb = p * g.seg_blocks;
+                    Mob M{1.f, 0.f, 0.f, 1.f};
+                    for (int b0 = 0; b0 < nb; b0 += 16) {
+                        float4 m[16];
+#pragma unroll
+                        for (int r = 0; r < 16; ++r)
+                            if (b0 + r < nb) m[r] = __ldg(src + (long long)(b0 + r) * nl);
+#pragma unroll
+                        for (int r = 0; r < 16; ++r)
+                            if (b0 + r < nb) M = mob_norm(mob_mul(Mob{m[r].x, m[r].y, m[r].z, m[r].w}, M));
+                    }
+                    lam = mob_apply(M, lam);
+                } else if (p > 0) {
+                    lam = g.lam_blk[(u * g.NB + (long long)p * g.seg_blocks) * nl + il];
+                }
             }
         }
         float e_prev = 1.f, log_decay = 0.f;   // e_prev = 2^(G_last - R) of the previous chunk
@@ -996,6 +1016,7 @@ cudaError_t launch_t(const Plan &p, const int *cu, int mode, const void *q, cons
     g.N = p.N; g.H = p.H; g.P = p.P; g.NB = p.NB; g.seg_blocks = p.seg_blocks; g.iso = p.iso; g.mode = mode;
     g.T = p.T; g.Lseg = p.Lseg; g.cu = cu; g.perm = cu ? p.perm : nullptr;
     g.a = a; g.qn = qn; g.beta = beta; g.lambda0 = lambda0; g.eta0 = eta0; g.lam_blk = lam_blk;
+    g.agg = p.inline_carry ? p.agg : nullptr;
     g.S_io = S_io; g.decay = decay; g.out = (__nv_bfloat16 *)out;
     g.final_lambda = final_lambda; g.final_eta = final_eta; g.status = status;
     const long long segs = mode == 1 ? p.P - 1 : p.P;

@@ -21,6 +21,7 @@ namespace kla {
 constexpr int kBlockTokens = 64;   // Lb: tokens per Moebius-reduction block (one chunk)
 constexpr int kChunk = 64;         // C: tokens per chunk of the chunked form
 constexpr int kMaxOrderSeqs = 1024; // packed sequences ranked by length for the launch order
+constexpr int kInlineCarryBlocks = 64; // at most this many blocks before a segment: carry in the walk kernel
 
 // Bits of the library's device status word (kla_check reads and clears it);
 // kernels that can detect an error receive its address and OR a bit into it.
@@ -46,6 +47,10 @@ struct Plan {
     bool order;
     size_t off_perm;
     const int *perm;
+    // segment-start precision composed inside the walk kernel from the block
+    // aggregates at agg (short segments), instead of a separate carry launch
+    bool inline_carry;
+    const float4 *agg;
 };
 
 __device__ __forceinline__ float ld_in(const float *p) { return __ldg(p); }
