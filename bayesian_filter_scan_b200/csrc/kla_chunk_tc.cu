@@ -20,7 +20,7 @@
 //
 // CTA = one segment of one (row or packed sequence, head); 320 threads:
 //   warps 0-3  gate: per key, the lambda recursion over the chunk (a, qn stream
-//              through a 5-slot TMA ring), log-gates, then Q'/K' written in
+//              through a TMA ring of three 16-token slots), log-gates, then Q'/K' written in
 //              place over the TMA-loaded q/k tiles (bf16, 128B-swizzled), and
 //              the bf16 remainder of K' for a two-term state update, slot by
 //              slot (the gate warps fold every slot themselves);
@@ -47,9 +47,11 @@ using namespace ptx;
 namespace {
 
 constexpr int kC = 64;             // chunk tokens
-constexpr int kSlotTok = 8;        // tokens per a/qn ring slot
-constexpr int kSlots = 5;          // ring depth (40 tokens of look-ahead)
+constexpr int kSlotTok = 8;        // tokens per gate slot (one pass of the chain and fold)
 constexpr int kSlotsPerChunk = kC / kSlotTok;
+constexpr int kRingTok = 16;       // tokens per a/qn ring slot (two gate slots per wait)
+constexpr int kRings = 3;          // ring depth (48 tokens of look-ahead)
+constexpr int kRingsPerChunk = kC / kRingTok;
 constexpr int kMaxOffset = 110;    // |G - R| (log2) kept inside the fp32/bf16 exponent range
 constexpr int kRebase = 64;        // diagonal mode: predicted |G - rho| that moves the reference
 // Warp roles. dk = 128: gate warps 0-3, epilogue 4-7, TMA producer 8, MMA 9.
@@ -84,7 +86,7 @@ struct Layout {
     static constexpr int V = kC * DV * 2;
     static constexpr int PT = kC * kC * 2;
     static constexpr int UB = DK * DV * 2;
-    static constexpr int SLOTF = kSlotTok * DK;   // floats of one of a / qn per slot
+    static constexpr int RINGF = kRingTok * DK;   // floats of one of a / qn per ring slot
     static constexpr int q0 = 0;
     static constexpr int k0 = q0 + 2 * QK;
     static constexpr int v0 = k0 + 2 * QK;
@@ -92,11 +94,11 @@ struct Layout {
     static constexpr int ub0 = p0 + PT;
     static constexpr int klo0 = ub0 + UB;          // low bf16 part of K' (state update), per stage
     static constexpr int ring0 = klo0 + 2 * QK;
-    static constexpr int fac0 = ring0 + kSlots * 2 * SLOTF * 4;
+    static constexpr int fac0 = ring0 + kRings * 2 * RINGF * 4;
     static constexpr int facf0 = fac0 + 2 * DK * 4;
     static constexpr int isof0 = facf0 + DK * 4;   // iso: per-token factors (q, beta k) of a chunk
     static constexpr int bar0 = ((isof0 + kC * 8) + 7) & ~7;
-    static constexpr int NBAR = 6 + 2 * kSlots + 9;
+    static constexpr int NBAR = 6 + 2 * kRings + 9;
     static constexpr int hold0 = bar0 + NBAR * 8;
     static constexpr int bytes = hold0 + 16;
     static constexpr int alloc = bytes + 1024;
@@ -187,12 +189,12 @@ __device__ __forceinline__ void gate_slot(int j, const float *ra, uint8_t *qt, u
                                           const int (&offr)[kSlotTok], float bsrc, bool state_mode, int R,
                                           float &nn, float &dd, float &pa, int &E, int &F, float &mq, float &mk,
                                           float &rkmin, float &rkmax) {
-    constexpr int SLOTF = kSlotTok * DK;
+    constexpr int RINGF = kRingTok * DK;    // qn follows a in the ring slot
     float xa[kSlotTok], xn[kSlotTok], xk[kSlotTok], xq[kSlotTok];
 #pragma unroll
     for (int r = 0; r < kSlotTok; ++r) {
         xa[r] = ra[r * DK];
-        xn[r] = ra[SLOTF + r * DK];
+        xn[r] = ra[RINGF + r * DK];
         xk[r] = bf_at(kt, j * 1024 + offr[r]);
         xq[r] = state_mode ? 0.f : bf_at(qt, j * 1024 + offr[r]);
     }
@@ -256,8 +258,8 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::bar0);
     uint64_t *stage_full = bars + 0, *stage_empty = bars + 2, *qk_ready = bars + 4;
-    uint64_t *ring_full = bars + 6, *ring_empty = bars + 6 + kSlots;
-    uint64_t *s_full = bars + 6 + 2 * kSlots, *u_ready = s_full + 1, *u_done = s_full + 2, *p_full = s_full + 3;
+    uint64_t *ring_full = bars + 6, *ring_empty = bars + 6 + kRings;
+    uint64_t *s_full = bars + 6 + 2 * kRings, *u_ready = s_full + 1, *u_done = s_full + 2, *p_full = s_full + 3;
     uint64_t *o_full = s_full + 4, *o_empty = s_full + 5, *td_bar = s_full + 6, *gate_sync = s_full + 7;
     uint64_t *gate_sync2 = s_full + 8;   // iso: the chunk's per-token factors are in shared memory
     uint32_t *tmem_hold = reinterpret_cast<uint32_t *>(sm + L::hold0);
@@ -295,7 +297,7 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             mbar_init(&stage_empty[s], 1);
             mbar_init(&qk_ready[s], gate_threads);
         }
-        for (int j = 0; j < kSlots; ++j) {
+        for (int j = 0; j < kRings; ++j) {
             mbar_init(&ring_full[j], 1);
             mbar_init(&ring_empty[j], gate_threads);
         }
@@ -429,20 +431,26 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (nvalid == kC) {
                     // Full chunk: the chain and the operands of every slot.
                     float rkmin = 3.0e38f, rkmax = 0.f;
-                    const int n0 = c * kSlotsPerChunk;
                     // not unrolled: one slot's code stays resident in the instruction cache
 #pragma unroll 1
                     for (int j = 0; j < kSlotsPerChunk; ++j) {
-                        const int n = n0 + j, slot = n % kSlots;
-                        if (!waitw(&ring_full[slot], (n / kSlots) & 1, abort_flag, g.status)) { ok = false; break; }
-                        const float *ra = reinterpret_cast<const float *>(sm + L::ring0) + slot * 2 * L::SLOTF + i;
+                        const int n = c * kRingsPerChunk + (j >> 1), slot = n % kRings;
+                        // one wait per ring slot of two gate slots
+                        if (!(j & 1) && !waitw(&ring_full[slot], (n / kRings) & 1, abort_flag, g.status)) {
+                            ok = false;
+                            break;
+                        }
+                        const float *ra = reinterpret_cast<const float *>(sm + L::ring0) + slot * 2 * L::RINGF +
+                                          (j & 1) * kSlotTok * DK + i;
                         const float bsrc = (j < 4) ? cb0 : cb1;
                         gate_slot<DK>(j, ra, qt, kt, klo, offr, bsrc, state_mode, R, nn, dd, pa, E, F, mq, mk, rkmin,
                                       rkmax);
-                        // ring slot read into registers: release it (generic reads
-                        // ordered before the TMA refill)
-                        fence_proxy_async();
-                        mbar_arrive(&ring_empty[slot]);
+                        if (j & 1) {
+                            // ring slot read into registers: release it (generic reads
+                            // ordered before the TMA refill)
+                            fence_proxy_async();
+                            mbar_arrive(&ring_empty[slot]);
+                        }
                     }
                     if (!ok) break;
                     // rk = 2^(R - G): |G - R| beyond the kept range leaves the exponent window
@@ -454,10 +462,14 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     int gmin = F - E, gmax = F - E;     // G at the chunk start (absolute)
 #pragma unroll 1
                     for (int j = 0; j < kSlotsPerChunk; ++j) {
-                        const int n = c * kSlotsPerChunk + j, slot = n % kSlots;
-                        if (!waitw(&ring_full[slot], (n / kSlots) & 1, abort_flag, g.status)) { ok = false; break; }
-                        const float *ra = reinterpret_cast<const float *>(sm + L::ring0) + slot * 2 * L::SLOTF;
-                        const float *rq = ra + L::SLOTF;
+                        const int n = c * kRingsPerChunk + (j >> 1), slot = n % kRings;
+                        if (!(j & 1) && !waitw(&ring_full[slot], (n / kRings) & 1, abort_flag, g.status)) {
+                            ok = false;
+                            break;
+                        }
+                        const float *ra = reinterpret_cast<const float *>(sm + L::ring0) + slot * 2 * L::RINGF +
+                                          (j & 1) * kSlotTok * DK;
+                        const float *rq = ra + L::RINGF;
                         const float bsrc = (j < 4) ? cb0 : cb1;
                         float kr[kSlotTok], qr[kSlotTok], ar[kSlotTok], qnr[kSlotTok], br[kSlotTok];
 #pragma unroll
@@ -469,8 +481,10 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                             qnr[r] = rq[r * DK + i];
                             br[r] = __shfl_sync(0xffffffffu, bsrc, (kSlotTok * j + r) & 31);
                         }
-                        fence_proxy_async();
-                        mbar_arrive(&ring_empty[slot]);
+                        if (j & 1) {
+                            fence_proxy_async();
+                            mbar_arrive(&ring_empty[slot]);
+                        }
                         float qo[kSlotTok], ko[kSlotTok];
                         float rkmin = 3.0e38f, rkmax = 0.f;
 #pragma unroll
@@ -821,8 +835,8 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     } else if (warp == RL::PRODW) {
         // ================= TMA producer =====================================
         if (lane == 0) {
-            int last_ring[kSlots], last_stage[2] = {-1, -1};
-            for (int j = 0; j < kSlots; ++j) last_ring[j] = -1;
+            int last_ring[kRings], last_stage[2] = {-1, -1};
+            for (int j = 0; j < kRings; ++j) last_ring[j] = -1;
             bool ok = true;
             for (int c = 0; c < nchunks && ok; ++c) {
                 const int tok0 = (int)(tb + (long long)c * kC);
@@ -851,31 +865,31 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
                     for (int a = 0; a < DV / 64; ++a) tma_prefetch_3d(&tm_v, 64 * a, h, tp);
                     if (!g.iso)
-                        for (int j = 0; j < kSlotsPerChunk; ++j) {
-                            tma_prefetch_3d(&tm_a, 0, h, tp + kSlotTok * j);
-                            tma_prefetch_3d(&tm_qn, 0, h, tp + kSlotTok * j);
+                        for (int j = 0; j < kRingsPerChunk; ++j) {
+                            tma_prefetch_3d(&tm_a, 0, h, tp + kRingTok * j);
+                            tma_prefetch_3d(&tm_qn, 0, h, tp + kRingTok * j);
                         }
                 }
                 if (!g.iso) {
-                    for (int j = 0; j < kSlotsPerChunk; ++j) {
-                        const int n = c * kSlotsPerChunk + j, slot = n % kSlots;
-                        if (n >= kSlots && !wait1(&ring_empty[slot], ((n / kSlots) - 1) & 1, abort_flag, g.status)) {
+                    for (int j = 0; j < kRingsPerChunk; ++j) {
+                        const int n = c * kRingsPerChunk + j, slot = n % kRings;
+                        if (n >= kRings && !wait1(&ring_empty[slot], ((n / kRings) - 1) & 1, abort_flag, g.status)) {
                             ok = false;
                             break;
                         }
-                        float *ra = reinterpret_cast<float *>(sm + L::ring0) + slot * 2 * L::SLOTF;
-                        mbar_expect_tx(&ring_full[slot], 2 * L::SLOTF * 4);
-                        tma_load_3d(ra, &tm_a, &ring_full[slot], 0, h, tok0 + kSlotTok * j);
-                        tma_load_3d(ra + L::SLOTF, &tm_qn, &ring_full[slot], 0, h, tok0 + kSlotTok * j);
+                        float *ra = reinterpret_cast<float *>(sm + L::ring0) + slot * 2 * L::RINGF;
+                        mbar_expect_tx(&ring_full[slot], 2 * L::RINGF * 4);
+                        tma_load_3d(ra, &tm_a, &ring_full[slot], 0, h, tok0 + kRingTok * j);
+                        tma_load_3d(ra + L::RINGF, &tm_qn, &ring_full[slot], 0, h, tok0 + kRingTok * j);
                         last_ring[slot] = n;
                     }
                 }
             }
             if (!ok || *abort_flag) {
                 // wait (bounded) until every copy this thread issued has landed
-                for (int j = 0; j < kSlots; ++j)
+                for (int j = 0; j < kRings; ++j)
                     if (last_ring[j] >= 0)
-                        wait_slow(&ring_full[j], (last_ring[j] / kSlots) & 1, abort_flag, g.status, false);
+                        wait_slow(&ring_full[j], (last_ring[j] / kRings) & 1, abort_flag, g.status, false);
                 for (int s = 0; s < 2; ++s)
                     if (last_stage[s] >= 0)
                         wait_slow(&stage_full[s], (last_stage[s] >> 1) & 1, abort_flag, g.status, false);
@@ -999,8 +1013,8 @@ cudaError_t launch_t(const Plan &p, const int *cu, int mode, const void *q, cons
               make_tma_map(&mk, k, BF, 2, DK, p.H, p.ntok, 64, kC, true) &&
               make_tma_map(&mv, v, BF, 2, DV, p.H, p.ntok, 64, kC, true);
     if (ok && !p.iso)
-        ok = make_tma_map(&ma, a, F32, 4, DK, p.H, p.ntok, DK, kSlotTok, false) &&
-             make_tma_map(&mqn, qn, F32, 4, DK, p.H, p.ntok, DK, kSlotTok, false);
+        ok = make_tma_map(&ma, a, F32, 4, DK, p.H, p.ntok, DK, kRingTok, false) &&
+             make_tma_map(&mqn, qn, F32, 4, DK, p.H, p.ntok, DK, kRingTok, false);
     else { ma = mq; mqn = mq; }
     if (!ok) return cudaErrorInvalidValue;
     static bool attr[64] = {};
