@@ -222,10 +222,15 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--T", type=int, default=None,
+                    help="tokens per row instead of the workload's (smaller cases of the same "
+                         "workload for profiler captures; not a bench line)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = WORKLOADS[args.workload]
+    if args.T is not None:
+        w = w.with_(T=args.T)
     if args.impl == "reference":
         run_reference(args, w)
         return
