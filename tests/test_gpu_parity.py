@@ -113,6 +113,18 @@ def test_diagonal_varlen_small():
     compare(w, make_inputs(w))
 
 
+@pytest.mark.parametrize("len_hi", [9, 30])
+def test_many_packed_sequences(len_hi):
+    # ~1700 sequences (beyond the 1024 the device ranks by length: launched in
+    # input order) and ~600 (ranked, longest first); lengths 1..len_hi
+    w = WORKLOADS[1].with_(B=1, H=2, T=9000, varlen=True, len_lo=1, len_hi=len_hi)
+    inp = make_inputs(w)
+    N = inp["cu_seqlens"].numel() - 1
+    assert (N > 1024) == (len_hi == 9)
+    lam0, eta0 = random_state(w, N, seed=5)
+    compare(w, inp, lam0, eta0)
+
+
 def test_isotropic_unpacked_segmented(monkeypatch):
     monkeypatch.setenv("KLA_SEGMENTS", "4")
     w = WORKLOADS[4].with_(B=1, H=2, T=3000, varlen=False)
