@@ -32,6 +32,7 @@ cudaError_t launch_walk(const Plan &, const int *, int, const void *, const void
                         const float *, float *, float *, void *, float *, float *, cudaStream_t);
 cudaError_t launch_state_carry(const Plan &, const float *, const float *, float *, cudaStream_t);
 cudaError_t launch_seq_order(const Plan &, const int *, int *, cudaStream_t);
+cudaError_t launch_correct(const Plan &, const float *, const float *, void *, float *, int *, cudaStream_t);
 bool chunk_tc_supported(const Plan &);
 cudaError_t launch_chunk_tc(const Plan &, const int *, int, const void *, const void *, const void *,
                             const float *, const float *, const float *, const float *, const float *,
@@ -132,6 +133,15 @@ static kla_status make_plan(const kla_desc *d, Plan &p, bool precision_only) {
         p.off_decay = off;
         off += align256(units * p.P * p.nl * sizeof(float));
     }
+    // split rows on the tensor-core path: the walk's folded q tiles and the
+    // per-chunk factors for the correction pass
+    p.local = !precision_only && p.P > 1 && chunk_tc_supported(p);
+    p.off_qbuf = off;
+    if (p.local) off += align256((size_t)p.ntok * p.H * p.dk * 2);
+    p.off_rlog = off;
+    if (p.local) off += align256(units * p.NB * p.dk * sizeof(float));
+    p.qbuf = nullptr;
+    p.rlog = nullptr;
     // longest-first launch order of packed sequences (list scheduling of the
     // walks: the long ones start first, the short ones fill in behind them)
     p.order = !precision_only && p.varlen && p.N >= 2 && p.N <= kMaxOrderSeqs;
@@ -227,14 +237,27 @@ static kla_status forward_impl(const kla_desc *d, const void *q, const void *k, 
         p.agg = agg;
         if (e == cudaSuccess && !p.inline_carry) e = launch_mobius_carry(p, agg, lambda0, lam_blk, st);
         mark(2);
+        if (p.local) {
+            // tensor-core path: every segment walks from a zero state (segment 0
+            // from eta0) and exports its transfer, gate product, folded q tiles
+            // and chunk factors; the correction pass then adds the carried state
+            p.qbuf = w + p.off_qbuf;
+            p.rlog = (float *)(w + p.off_rlog);
+            mark(3);
+            mark(4);
+            if (e == cudaSuccess)
+                e = launch_chunk_tc(p, cu, 2, q, k, v, a, qn, beta, lambda0, eta0, lam_blk, S_io, decay, out,
+                                    final_lambda, final_eta, status, st);
+            mark(5);
+            if (e == cudaSuccess) e = launch_correct(p, S_io, decay, out, final_eta, status, st);
+            mark(6);
+            return cuda_status(e);
+        }
         if (e == cudaSuccess)
-            e = tc ? launch_chunk_tc(p, cu, 1, q, k, v, a, qn, beta, lambda0, eta0, lam_blk, S_io, decay,
-                                     out, final_lambda, final_eta, status, st)
-                   : launch_walk(p, cu, 1, q, k, v, a, qn, beta, lambda0, eta0, lam_blk, S_io, decay,
-                                 out, final_lambda, final_eta, st);
+            e = launch_walk(p, cu, 1, q, k, v, a, qn, beta, lambda0, eta0, lam_blk, S_io, decay, out, final_lambda,
+                            final_eta, st);
         mark(3);
-        // the tensor-core output pass carries the segment states itself
-        if (e == cudaSuccess && !tc) e = launch_state_carry(p, eta0, decay, S_io, st);
+        if (e == cudaSuccess) e = launch_state_carry(p, eta0, decay, S_io, st);
         mark(4);
     } else {
         mark(1); mark(2); mark(3); mark(4);
@@ -245,6 +268,7 @@ static kla_status forward_impl(const kla_desc *d, const void *q, const void *k, 
                : launch_walk(p, cu, 0, q, k, v, a, qn, beta, lambda0, eta0, lam_blk, S_io, decay,
                              out, final_lambda, final_eta, st);
     mark(5);
+    mark(6);
     return cuda_status(e);
 }
 
@@ -263,7 +287,7 @@ kla_status kla_forward_profiled(const kla_desc *d, const void *q, const void *k,
                                 float *final_lambda, float *final_eta, void *ws, size_t ws_bytes,
                                 cudaStream_t st, cudaEvent_t *events) {
     if (!events) return KLA_ERR_INVALID_ARG;
-    for (int i = 0; i < 6; ++i)
+    for (int i = 0; i < 7; ++i)
         if (!events[i]) return KLA_ERR_INVALID_ARG;
     return forward_impl(d, q, k, v, a, qn, beta, lambda0, eta0, out, final_lambda, final_eta, ws,
                         ws_bytes, st, events);

@@ -78,6 +78,12 @@ struct TcArgs {
     __nv_bfloat16 *out;
     float *final_lambda, *final_eta;
     int *status;
+    // mode 2 (segments from a zero state): per chunk and key, the log2 factor
+    // that takes the folded q' of the chunk to the segment-start frame,
+    // rlog[(u * NC + chunk of the row) * DK + key]; the folded q tiles go to
+    // the tensor map of the q' buffer
+    float *rlog;
+    int NC;
 };
 
 template <int DK, int DV>
@@ -249,7 +255,8 @@ template <int DK, int DV>
 __global__ void __launch_bounds__(Roles<DK, DV>::THREADS, Roles<DK, DV>::MIN_BLOCKS)
 kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
-                    const __grid_constant__ CUtensorMap tm_qn, const TcArgs g) {
+                    const __grid_constant__ CUtensorMap tm_qn, const __grid_constant__ CUtensorMap tm_qs,
+                    const TcArgs g) {
     using L = Layout<DK, DV>;
     using RL = Roles<DK, DV>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -270,6 +277,10 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool state_mode = g.mode == 1;
+    // mode 2: every segment walks from a zero state (segment 0 from eta0), writes
+    // its transfer and decay, and segments p > 0 export their folded q tiles and
+    // chunk references for the correction pass that adds the carried state
+    const bool local_mode = g.mode == 2;
     // one gate thread per key: each reads and rewrites only its own key column
     const int gate_threads = DK;
     const bool is_gate = (RL::NGW == 4) ? (warp < 4) : (warp == 0 || warp == 2);
@@ -423,6 +434,8 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     fac_c = __int_as_float((127 + max(-126, min(127, rnew - rho))) << 23);
                     rho = rnew;
                     R = rho;
+                    if (local_mode && p > 0)
+                        g.rlog[(u * g.NC + (tok0 - tb) / kC + (long long)p * g.seg_blocks) * DK + i] = (float)R;
                     const int sh0 = max(-126, min(127, gs - R));
                     mq = __int_as_float((127 + sh0) << 23);
                     mk = __int_as_float((127 - sh0) << 23);
@@ -575,6 +588,10 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const int gmin = (int)floorf(mn), gmax = (int)ceilf(mx);
                 R = (gmin + gmax) >> 1;
                 const float Rf = (float)R;
+                // G here runs from the chunk start: the segment-start frame adds the
+                // log2 decay of the segment's earlier chunks
+                if (local_mode && p > 0)
+                    g.rlog[(u * g.NC + (tok0 - tb) / kC + (long long)p * g.seg_blocks) * DK + i] = Rf + log_decay;
                 const float Glast = __shfl_sync(0xffffffffu, G1, 31);
                 e_cur = exp2f(Glast - Rf);
                 glast_log2 = Glast;
@@ -627,9 +644,10 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             mbar_arrive(&qk_ready[s]);
         }
         if (ok && !*abort_flag) {
-            if (state_mode) {
+            if (state_mode || local_mode) {
                 if (g.iso ? (gt == 0) : key) g.decay[(u * g.P + p) * (g.iso ? 1 : DK) + (g.iso ? 0 : i)] = exp2f(log_decay);
-            } else if (last_seg && g.final_lambda) {
+            }
+            if (!state_mode && last_seg && g.final_lambda) {
                 if (g.iso ? (gt == 0) : key) g.final_lambda[u * (g.iso ? 1 : DK) + (g.iso ? 0 : i)] = lam;
             }
         }
@@ -644,7 +662,7 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const bool vU = (DK == 128) || v64;
         uint8_t *ub = sm + L::ub0;
         uint8_t *pt = sm + L::p0;
-        const float *eta0 = (!state_mode && g.eta0) ? g.eta0 + u * DK * DV : nullptr;
+        const float *eta0 = (!state_mode && (!local_mode || p == 0) && g.eta0) ? g.eta0 + u * DK * DV : nullptr;
         bool ok = true;
         // Belief at the segment start, written into the U columns of TMEM before
         // the first chunk (while the gate works on it): eta0 carried through the
@@ -661,8 +679,9 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
                     acc[x] = e4.x; acc[x + 1] = e4.y; acc[x + 2] = e4.z; acc[x + 3] = e4.w;
                 }
+                const int nprev = local_mode ? 0 : p;   // mode 2: segments from a zero state
 #pragma unroll 4
-                for (int q = 0; q < p; ++q) {
+                for (int q = 0; q < nprev; ++q) {
                     const float dq = vU ? g.decay[(u * g.P + q) * nl + (g.iso ? 0 : rowU)] : 0.f;
                     const float *src = g.S_io + ((u * g.P + q) * DK + rowU) * DV + cb * 32;
 #pragma unroll
@@ -806,7 +825,7 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (ok && !state_mode && nchunks > 0 && !emit_out(nchunks - 1)) ok = false;
         // ---- final belief (last segment) or segment transfer (state mode)
         float *dst = nullptr;
-        if (state_mode) dst = g.S_io + (u * g.P + p) * DK * DV;
+        if (state_mode || local_mode) dst = g.S_io + (u * g.P + p) * DK * DV;
         else if (last_seg && g.final_eta) dst = g.final_eta + u * DK * DV;
         if (ok && dst && !*abort_flag) {
             if (nchunks > 0) {
@@ -911,6 +930,15 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const uint32_t ka = smem_u32(sm + L::k0 + s * L::QK);
                 const uint32_t va = smem_u32(sm + L::v0 + s * L::V);
                 const uint32_t kloa = smem_u32(sm + L::klo0 + s * L::QK);
+                if (local_mode && p > 0) {
+                    // export the folded q tile (the correction pass multiplies it by the
+                    // carried segment-start state)
+                    const int tok0 = (int)(tb + (long long)c * kC);
+#pragma unroll
+                    for (int a = 0; a < DK / 64; ++a)
+                        tma_store_3d(&tm_qs, sm + L::q0 + s * L::QK + a * kC * 128, 64 * a, h, tok0);
+                    tma_store_commit();
+                }
                 if (!state_mode) {
 #pragma unroll
                     for (int kk = 0; kk < DK / 16; ++kk) {
@@ -948,8 +976,11 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                                  iO, 1);
                     mma_commit(o_full);
                 }
+                // the stage is refilled only after the q' export read it
+                if (local_mode && p > 0) tma_store_wait_read();
                 mma_commit(&stage_empty[s]);
             }
+            if (local_mode && p > 0) tma_store_wait_all();
             // all MMAs this thread issued have completed before TMEM is released
             mma_commit(td_bar);
             wait_slow(td_bar, 0, abort_flag, g.status, false);
@@ -1007,7 +1038,7 @@ cudaError_t launch_t(const Plan &p, const int *cu, int mode, const void *q, cons
                      const float *lam_blk, float *S_io, float *decay, void *out, float *final_lambda,
                      float *final_eta, int *status, cudaStream_t st) {
     using L = Layout<DK, DV>;
-    CUtensorMap mq, mk, mv, ma, mqn;
+    CUtensorMap mq, mk, mv, ma, mqn, mqs;
     const CUtensorMapDataType BF = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, F32 = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     bool ok = make_tma_map(&mq, q, BF, 2, DK, p.H, p.ntok, 64, kC, true) &&
               make_tma_map(&mk, k, BF, 2, DK, p.H, p.ntok, 64, kC, true) &&
@@ -1016,6 +1047,8 @@ cudaError_t launch_t(const Plan &p, const int *cu, int mode, const void *q, cons
         ok = make_tma_map(&ma, a, F32, 4, DK, p.H, p.ntok, DK, kRingTok, false) &&
              make_tma_map(&mqn, qn, F32, 4, DK, p.H, p.ntok, DK, kRingTok, false);
     else { ma = mq; mqn = mq; }
+    if (ok && mode == 2) ok = make_tma_map(&mqs, p.qbuf, BF, 2, DK, p.H, p.ntok, 64, kC, true);
+    else mqs = mq;
     if (!ok) return cudaErrorInvalidValue;
     static bool attr[64] = {};
     int dev = 0;
@@ -1031,12 +1064,13 @@ cudaError_t launch_t(const Plan &p, const int *cu, int mode, const void *q, cons
     g.T = p.T; g.Lseg = p.Lseg; g.cu = cu; g.perm = cu ? p.perm : nullptr;
     g.a = a; g.qn = qn; g.beta = beta; g.lambda0 = lambda0; g.eta0 = eta0; g.lam_blk = lam_blk;
     g.agg = p.inline_carry ? p.agg : nullptr;
+    g.rlog = p.rlog; g.NC = p.NB;
     g.S_io = S_io; g.decay = decay; g.out = (__nv_bfloat16 *)out;
     g.final_lambda = final_lambda; g.final_eta = final_eta; g.status = status;
     const long long segs = mode == 1 ? p.P - 1 : p.P;
     const unsigned grid = (unsigned)((long long)p.N * p.H * segs);
     if (grid == 0) return cudaSuccess;
-    kla_chunk_tc_kernel<DK, DV><<<grid, Roles<DK, DV>::THREADS, L::alloc, st>>>(mq, mk, mv, ma, mqn, g);
+    kla_chunk_tc_kernel<DK, DV><<<grid, Roles<DK, DV>::THREADS, L::alloc, st>>>(mq, mk, mv, ma, mqn, mqs, g);
     return cudaGetLastError();
 }
 

@@ -51,6 +51,14 @@ struct Plan {
     // aggregates at agg (short segments), instead of a separate carry launch
     bool inline_carry;
     const float4 *agg;
+    // split rows on the tensor-core path: segments walk from a zero state and a
+    // correction pass adds the carried state; the walk exports its folded q
+    // tiles (qbuf [Ntok, H, dk] bf16) and per-chunk log2 factors (rlog
+    // [N*H][NB][dk] fp32), in the workspace at off_qbuf / off_rlog
+    bool local;
+    size_t off_qbuf, off_rlog;
+    void *qbuf;
+    float *rlog;
 };
 
 __device__ __forceinline__ float ld_in(const float *p) { return __ldg(p); }

@@ -282,13 +282,13 @@ def main():
                 ctypes.c_void_p(stream.cuda_stream)]
 
     steps = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(steps)]
-    ev_ptrs = [(ctypes.c_void_p * 6)(*[ctypes.c_void_p(e.cuda_event) for e in row]) for row in evs]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(steps)]
+    ev_ptrs = [(ctypes.c_void_p * 7)(*[ctypes.c_void_p(e.cuda_event) for e in row]) for row in evs]
     for row in evs:
         for e in row:
             e.record(stream)   # materialise the events
     torch.cuda.synchronize()
-    ev_ptrs = [(ctypes.c_void_p * 6)(*[ctypes.c_void_p(e.cuda_event) for e in row]) for row in evs]
+    ev_ptrs = [(ctypes.c_void_p * 7)(*[ctypes.c_void_p(e.cuda_event) for e in row]) for row in evs]
 
     # timed steps: one kla_forward between two events (the headline); the
     # per-launch breakdown comes from a separate run with an event between
@@ -333,7 +333,7 @@ def main():
     chunk = [r[4].elapsed_time(r[5]) for r in evs]            # ms, output pass (chunk kernel)
     pre = [r[0].elapsed_time(r[4]) for r in evs]
     # per launch of the sequence: reduce, carry, state pass, state carry, output pass
-    stage_names = ("mobius_reduce", "mobius_carry", "state_pass", "state_carry", "output_pass")
+    stage_names = ("mobius_reduce", "mobius_carry", "state_pass", "state_carry", "output_pass", "correction")
     per_stage = {n: statistics.mean(r[i].elapsed_time(r[i + 1]) for r in evs) for i, n in enumerate(stage_names)}
     ms_per_step, value = aggregate(world, w.tokens, sum(tot), steps, dist)
 
@@ -391,7 +391,7 @@ def main():
                      "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_src},
         "stages_ms": {"note": "separate run with an event between every launch",
                       "pre_passes": statistics.mean(pre), "output_pass": chunk_ms,
-                      "total": statistics.mean(r[0].elapsed_time(r[5]) for r in evs), "launches": per_stage},
+                      "total": statistics.mean(r[0].elapsed_time(r[6]) for r in evs), "launches": per_stage},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h_in, "d2h_bytes_per_step": h_out},
         "gpu_launches": steps * plan["launches"],
         "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"],
