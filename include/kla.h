@@ -79,11 +79,12 @@ typedef struct {
 } kla_desc;
 
 /* Bytes of device workspace kla_forward needs for this descriptor on the
- * current device (0 means the workspace pointer may be NULL): the Moebius
- * block aggregates and segment states when rows are split into segments, and
- * one int per packed sequence (up to 1024 sequences) for the longest-first
- * launch order. Pure host computation. Returns 0 for an invalid descriptor as
- * well. */
+ * current device (0 means the workspace pointer may be NULL): when rows are
+ * split into segments, the Moebius block aggregates and the segment states,
+ * and on the tensor-core path also the segments' folded queries (2*dk bytes
+ * per token and head) and per-chunk factors for the correction pass; one int
+ * per packed sequence (up to 1024 sequences) for the longest-first launch
+ * order. Pure host computation. Returns 0 for an invalid descriptor as well. */
 size_t kla_workspace_bytes(const kla_desc *desc);
 
 /* Bytes of device workspace kla_precision needs (0: the pointer may be NULL). */
