@@ -152,19 +152,18 @@ mobius_reduce_tma(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         Mob m[4];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-            float n1 = 1.f, d1 = 0.f, n2 = 0.f, d2 = 1.f;
+            // the two columns (n1, n2), (d1, d2) share a^2, qn and b: paired fp32
+            float2 nn = make_float2(1.f, 0.f), dd = make_float2(0.f, 1.f);
 #pragma unroll
             for (int r = 0; r < kRedLen; ++r) {
                 if (r < len) {
                     const float ac = (&av[r].x)[c], qc = (&qv[r].x)[c], kc = (&kv[r].x)[c];
                     const float a2 = ac * ac, b = cb[r] * kc * kc;
-                    d1 = fmaf(a2, d1, qc * n1);
-                    n1 = fmaf(b, d1, n1);
-                    d2 = fmaf(a2, d2, qc * n2);
-                    n2 = fmaf(b, d2, n2);
+                    dd = __ffma2_rn(make_float2(a2, a2), dd, __fmul2_rn(make_float2(qc, qc), nn));
+                    nn = __ffma2_rn(make_float2(b, b), dd, nn);
                 }
             }
-            m[c] = mob_norm(Mob{n1, n2, d1, d2});
+            m[c] = mob_norm(Mob{nn.x, nn.y, dd.x, dd.y});
             part[sub * 64 + 4 * quad + c] = make_float4(m[c].m00, m[c].m01, m[c].m10, m[c].m11);
         }
 #pragma unroll
