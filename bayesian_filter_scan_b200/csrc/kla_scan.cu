@@ -10,9 +10,10 @@
 //                   mode streams a, qn, k through a TMA-fed shared-memory ring
 //                   in persistent CTAs, eight 8-token sub-blocks per block
 //                   composed by a tree in shared memory.
-//   mobius_carry  : per (row, head, key) one warp: the product of each
-//                   segment's blocks, a shuffle scan over segments, applied to
-//                   lambda0: lambda at every segment start.
+//   mobius_carry  : per (row, head, key) one warp: each segment's product
+//                   (lanes compose slices, a shuffle tree joins them), carried
+//                   in order and applied to lambda0: lambda at every segment
+//                   start.
 //   mobius_emit   : per (row/sequence, head, block, key) re-walks the block
 //                   from its start lambda and writes lambda after every token
 //                   (the kla_precision output; there segments are blocks).
@@ -232,9 +233,58 @@ mobius_reduce_iso(ScanArgs s, const TIn *__restrict__ k, const float *__restrict
 
 // lam_blk[(u*NB + p*seg_blocks)*nl + i] = (all blocks before segment p)(lambda0):
 // lambda at every segment start (every block start when segments are blocks).
-// One warp per (row, head, key): lane l composes the blocks of segments l,
-// l+32, ..., then a warp-shuffle scan of the 2x2 maps gives the exclusive
-// prefixes, carried across groups of 32 segments.
+// One warp per (row, head, key), segments in order: the warp's lanes compose
+// consecutive slices of the segment's blocks, a shuffle tree combines the
+// slices in order into the segment's product, and lane 0 carries the prefix.
+__device__ __forceinline__ Mob shfl_down_m(const Mob &m, int d) {
+    return Mob{__shfl_down_sync(0xffffffffu, m.m00, d), __shfl_down_sync(0xffffffffu, m.m01, d),
+               __shfl_down_sync(0xffffffffu, m.m10, d), __shfl_down_sync(0xffffffffu, m.m11, d)};
+}
+
+__global__ void __launch_bounds__(128)
+mobius_carry(ScanArgs s, int nl, int P, int seg_blocks, const float4 *__restrict__ agg,
+             const float *__restrict__ lambda0, float *__restrict__ lam_blk) {
+    const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (gw >= (long long)s.N * s.H * nl) return;
+    const long long u = gw / nl;
+    const int i = (int)(gw % nl);
+    const float l0 = lambda0 ? __ldg(lambda0 + gw) : 1.0f;
+    const float4 *src = agg + u * s.NB * nl + i;
+    Mob carry{1.f, 0.f, 0.f, 1.f};
+    for (int p = 0; p < P; ++p) {
+        if (lane == 0) lam_blk[(u * s.NB + (long long)p * seg_blocks) * nl + i] = mob_apply(carry, l0);
+        if (p == P - 1) break;
+        const int b0 = p * seg_blocks, b1 = min(b0 + seg_blocks, s.NB);
+        const int per = (b1 - b0 + 31) / 32;
+        // this lane's slice [b0 + lane * per, ...), composed in order
+        Mob M{1.f, 0.f, 0.f, 1.f};
+        for (int q0 = 0; q0 < per; q0 += 8) {
+            float4 m[8];
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const int b = b0 + lane * per + q0 + r;
+                if (q0 + r < per && b < b1) m[r] = __ldg(src + (long long)b * nl);
+            }
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const int b = b0 + lane * per + q0 + r;
+                if (q0 + r < per && b < b1) M = mob_norm(mob_mul(Mob{m[r].x, m[r].y, m[r].z, m[r].w}, M));
+            }
+        }
+        // slices in order: lane l takes the product of lanes l .. l + 2d - 1
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const Mob o = shfl_down_m(M, d);
+            if ((lane & (2 * d - 1)) == 0) M = mob_norm(mob_mul(o, M));
+        }
+        carry = mob_norm(mob_mul(M, carry));
+    }
+}
+
+// Short segments (fewer than 32 blocks each, e.g. every block a segment):
+// lane l composes the blocks of segments l, l+32, ..., a warp-shuffle scan of
+// the 2x2 maps gives the exclusive prefixes, carried across groups of 32.
 __device__ __forceinline__ Mob shfl_up_m(const Mob &m, int d) {
     return Mob{__shfl_up_sync(0xffffffffu, m.m00, d), __shfl_up_sync(0xffffffffu, m.m01, d),
                __shfl_up_sync(0xffffffffu, m.m10, d), __shfl_up_sync(0xffffffffu, m.m11, d)};
@@ -245,7 +295,7 @@ __device__ __forceinline__ Mob shfl_m(const Mob &m, int src) {
 }
 
 __global__ void __launch_bounds__(128)
-mobius_carry(ScanArgs s, int nl, int P, int seg_blocks, const float4 *__restrict__ agg,
+mobius_carry_lanes(ScanArgs s, int nl, int P, int seg_blocks, const float4 *__restrict__ agg,
              const float *__restrict__ lambda0, float *__restrict__ lam_blk) {
     const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
@@ -450,7 +500,10 @@ cudaError_t launch_mobius_carry(const Plan &p, const float4 *agg, const float *l
                                 float *lam_blk, cudaStream_t st) {
     ScanArgs s{p.N, p.H, p.dk, p.T, p.NB, nullptr};
     long long thr = (long long)p.N * p.H * p.nl * 32;
-    mobius_carry<<<blocks_for(thr, 128), 128, 0, st>>>(s, p.nl, p.P, p.seg_blocks, agg, lambda0, lam_blk);
+    if (p.seg_blocks >= 32)
+        mobius_carry<<<blocks_for(thr, 128), 128, 0, st>>>(s, p.nl, p.P, p.seg_blocks, agg, lambda0, lam_blk);
+    else
+        mobius_carry_lanes<<<blocks_for(thr, 128), 128, 0, st>>>(s, p.nl, p.P, p.seg_blocks, agg, lambda0, lam_blk);
     return cudaGetLastError();
 }
 
