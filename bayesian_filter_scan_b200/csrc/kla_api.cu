@@ -301,7 +301,9 @@ kla_status kla_plan(const kla_desc *d, int *segments_per_row, int *launches, int
     int n = 1;
     if (p.P > 1) {
         const bool tc = chunk_tc_supported(p);
-        n = tc ? ((long long)(p.P - 1) * p.seg_blocks <= kInlineCarryBlocks ? 3 : 4) : 5;
+        // tensor cores: reduce, [carry], chunk kernel, segment starts, correction;
+        // CUDA cores: reduce, carry, state walk, state carry, output walk
+        n = tc ? ((long long)(p.P - 1) * p.seg_blocks <= kInlineCarryBlocks ? 4 : 5) : 5;
     }
     if (launches) *launches = n + (p.order ? 1 : 0);
     if (tensor_core) *tensor_core = chunk_tc_supported(p) ? 1 : 0;

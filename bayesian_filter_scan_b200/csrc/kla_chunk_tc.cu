@@ -285,22 +285,6 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const int gate_threads = DK;
     const bool is_gate = (RL::NGW == 4) ? (warp < 4) : (warp == 0 || warp == 2);
     const int gt = (RL::NGW == 4) ? tid : ((warp >> 1) * 32 + lane);   // gate rank
-    const int P_eff = state_mode ? g.P - 1 : g.P;
-    // unit u = (row or packed sequence n, head h); packed sequences in the
-    // longest-first order when one is given
-    const long long ur = blockIdx.x / P_eff;
-    const int p = (int)(blockIdx.x % P_eff);
-    const int h = (int)(ur % g.H);
-    const int n = g.perm ? g.perm[ur / g.H] : (int)(ur / g.H);
-    const long long u = (long long)n * g.H + h;
-    long long tb, te;
-    if (g.cu) { tb = g.cu[n]; te = g.cu[n + 1]; }
-    else {
-        tb = (long long)n * g.T + (long long)p * g.Lseg;
-        te = (long long)n * g.T + min((long long)(p + 1) * g.Lseg, g.T);
-    }
-    const int nchunks = te > tb ? (int)((te - tb + kC - 1) / kC) : 0;
-    const bool last_seg = p == P_eff - 1;
 
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
@@ -333,6 +317,24 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_hold;
+    pdl_release();
+    pdl_wait();
+    const int P_eff = state_mode ? g.P - 1 : g.P;
+    // unit u = (row or packed sequence n, head h); packed sequences in the
+    // longest-first order when one is given
+    const long long ur = blockIdx.x / P_eff;
+    const int p = (int)(blockIdx.x % P_eff);
+    const int h = (int)(ur % g.H);
+    const int n = g.perm ? g.perm[ur / g.H] : (int)(ur / g.H);
+    const long long u = (long long)n * g.H + h;
+    long long tb, te;
+    if (g.cu) { tb = g.cu[n]; te = g.cu[n + 1]; }
+    else {
+        tb = (long long)n * g.T + (long long)p * g.Lseg;
+        te = (long long)n * g.T + min((long long)(p + 1) * g.Lseg, g.T);
+    }
+    const int nchunks = te > tb ? (int)((te - tb + kC - 1) / kC) : 0;
+    const bool last_seg = p == P_eff - 1;
 
     if (is_gate) {
       {
@@ -1070,8 +1072,8 @@ cudaError_t launch_t(const Plan &p, const int *cu, int mode, const void *q, cons
     const long long segs = mode == 1 ? p.P - 1 : p.P;
     const unsigned grid = (unsigned)((long long)p.N * p.H * segs);
     if (grid == 0) return cudaSuccess;
-    kla_chunk_tc_kernel<DK, DV><<<grid, Roles<DK, DV>::THREADS, L::alloc, st>>>(mq, mk, mv, ma, mqn, mqs, g);
-    return cudaGetLastError();
+    return launch_pdl(kla_chunk_tc_kernel<DK, DV>, grid, Roles<DK, DV>::THREADS, L::alloc, st, mq, mk, mv, ma, mqn,
+                      mqs, g);
 }
 
 }  // namespace

@@ -94,6 +94,8 @@ __device__ __noinline__ bool cwait(uint64_t *bar, uint32_t parity, int *status) 
 __global__ void __launch_bounds__(256)
 kla_segment_starts(long long units, int DKV, int dv, int nl, int P, const float *__restrict__ decay,
                    float *__restrict__ S_io, float *__restrict__ final_eta) {
+    pdl_release();
+    pdl_wait();
     const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (gid >= units * DKV) return;
     const long long u = gid / DKV;
@@ -165,6 +167,8 @@ kla_correct_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_hold;
+    pdl_release();
+    pdl_wait();
 
     float *lmax = reinterpret_cast<float *>(sm + L::m0);
     int *list = reinterpret_cast<int *>(sm + L::l0);
@@ -359,8 +363,7 @@ cudaError_t launch_correct_t(const Plan &p, const float *S_io, void *out, int *s
     ranges = std::max(ranges, (p.seg_blocks + kMaxRange - 1) / kMaxRange);
     g.cpr = (p.seg_blocks + ranges - 1) / ranges;
     ranges = (p.seg_blocks + g.cpr - 1) / g.cpr;
-    kla_correct_kernel<DK, DV><<<(unsigned)(segs * ranges), 128, L::alloc, st>>>(mqs, mo, g);
-    return cudaGetLastError();
+    return launch_pdl(kla_correct_kernel<DK, DV>, (unsigned)(segs * ranges), 128, L::alloc, st, mqs, mo, g);
 }
 
 }  // namespace
@@ -370,9 +373,8 @@ cudaError_t launch_correct(const Plan &p, const float *S_io, const float *decay,
     // segment-start beliefs (and the final belief) first
     const long long units = (long long)p.N * p.H;
     const long long thr = units * p.dk * p.dv;
-    kla_segment_starts<<<(unsigned)((thr + 255) / 256), 256, 0, st>>>(units, p.dk * p.dv, p.dv, p.nl, p.P, decay,
-                                                                      (float *)S_io, final_eta);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(kla_segment_starts, (unsigned)((thr + 255) / 256), 256, 0, st, units, p.dk * p.dv,
+                               p.dv, p.nl, p.P, decay, (float *)S_io, final_eta);
     if (e != cudaSuccess) return e;
 #define KLA_CORR_CASE(DK_, DV_) \
     if (p.dk == DK_ && p.dv == DV_) return launch_correct_t<DK_, DV_>(p, S_io, out, status, st);

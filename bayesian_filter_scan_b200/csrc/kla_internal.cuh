@@ -16,6 +16,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <utility>
+
 namespace kla {
 
 constexpr int kBlockTokens = 64;   // Lb: tokens per Moebius-reduction block (one chunk)
@@ -110,6 +112,38 @@ __device__ __forceinline__ Mob mob_norm(const Mob &M) {
 
 __device__ __forceinline__ float mob_apply(const Mob &M, float x) {
     return fmaf(M.m00, x, M.m01) / fmaf(M.m10, x, M.m11);
+}
+
+// Programmatic dependent launch. Every kernel of the library is launched with
+// programmatic stream serialization, so it may start while the kernel before
+// it in the stream is still running. Each kernel therefore
+//  * calls pdl_wait() before its first global-memory access (read or write):
+//    it returns once the preceding grid has completed and its writes are
+//    visible, so the data dependences are those of plain stream order;
+//  * calls pdl_release() once it holds every on-chip resource it will take
+//    (after its tensor-memory allocation): the next kernel's CTAs may become
+//    resident from then on and run their prologue (barrier setup, tensor-map
+//    prefetch, tensor-memory allocation) under this kernel's tail. Releasing
+//    only after the allocation means a waiting dependent can never hold
+//    tensor memory that a CTA of this grid still needs.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Launches `kern` on `st` with programmatic stream serialization (see above).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args &&...args) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 }  // namespace kla

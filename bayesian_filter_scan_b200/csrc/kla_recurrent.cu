@@ -53,6 +53,8 @@ __host__ __device__ inline size_t walk_smem_bytes(int dk, int dv) {
 template <typename TIn, int KPG>
 __global__ void __launch_bounds__(kWalkThreads)
 kla_walk_simt(WalkArgs w) {
+    pdl_release();
+    pdl_wait();
     extern __shared__ float sm[];
     const int dk = w.dk, dv = w.dv;
     const int nkg = kWalkThreads / dv;
@@ -220,8 +222,7 @@ static cudaError_t launch_walk_t(const WalkArgs &w, unsigned grid, cudaStream_t 
         if (e != cudaSuccess) return e;
         attr_set[dev] = true;
     }
-    kla_walk_simt<TIn, KPG><<<grid, kWalkThreads, smem, st>>>(w);
-    return cudaGetLastError();
+    return launch_pdl(kla_walk_simt<TIn, KPG>, grid, kWalkThreads, smem, st, w);
 }
 
 template <typename TIn>
@@ -260,6 +261,8 @@ cudaError_t launch_walk(const Plan &p, const int *cu, int mode, const void *q, c
 __global__ void __launch_bounds__(256)
 kla_state_carry(int N, int H, int dk, int dv, int nl, int P, const float *__restrict__ eta0,
                 const float *__restrict__ decay, float *__restrict__ S_io) {
+    pdl_release();
+    pdl_wait();
     long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     long long per = (long long)dk * dv;
     if (gid >= (long long)N * H * per) return;
@@ -292,9 +295,8 @@ kla_state_carry(int N, int H, int dk, int dv, int nl, int P, const float *__rest
 cudaError_t launch_state_carry(const Plan &p, const float *eta0, const float *decay, float *S_io,
                                cudaStream_t st) {
     long long thr = (long long)p.N * p.H * p.dk * p.dv;
-    kla_state_carry<<<(unsigned)((thr + 255) / 256), 256, 0, st>>>(p.N, p.H, p.dk, p.dv, p.nl, p.P,
-                                                                    eta0, decay, S_io);
-    return cudaGetLastError();
+    return launch_pdl(kla_state_carry, (unsigned)((thr + 255) / 256), 256, 0, st, p.N, p.H, p.dk, p.dv, p.nl,
+                      p.P, eta0, decay, S_io);
 }
 
 }  // namespace kla

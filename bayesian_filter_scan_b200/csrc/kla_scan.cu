@@ -73,6 +73,8 @@ mobius_reduce_tma(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         fence_mbar_init();
     }
     __syncthreads();
+    pdl_release();
+    pdl_wait();
     auto decode = [&](long long w, long long &u, int &blk, int &half) {
         half = (int)(w % nhalf);
         const long long r = w / nhalf;
@@ -210,6 +212,8 @@ __global__ void __launch_bounds__(128)
 mobius_reduce_iso(ScanArgs s, const TIn *__restrict__ k, const float *__restrict__ a,
                   const float *__restrict__ qn, const float *__restrict__ beta,
                   float4 *__restrict__ agg) {
+    pdl_release();
+    pdl_wait();
     long long pair = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (pair >= (long long)s.N * s.H * s.NB) return;
     int blk = (int)(pair % s.NB);
@@ -244,6 +248,8 @@ __device__ __forceinline__ Mob shfl_down_m(const Mob &m, int d) {
 __global__ void __launch_bounds__(128)
 mobius_carry(ScanArgs s, int nl, int P, int seg_blocks, const float4 *__restrict__ agg,
              const float *__restrict__ lambda0, float *__restrict__ lam_blk) {
+    pdl_release();
+    pdl_wait();
     const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (gw >= (long long)s.N * s.H * nl) return;
@@ -297,6 +303,8 @@ __device__ __forceinline__ Mob shfl_m(const Mob &m, int src) {
 __global__ void __launch_bounds__(128)
 mobius_carry_lanes(ScanArgs s, int nl, int P, int seg_blocks, const float4 *__restrict__ agg,
              const float *__restrict__ lambda0, float *__restrict__ lam_blk) {
+    pdl_release();
+    pdl_wait();
     const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (gw >= (long long)s.N * s.H * nl) return;
@@ -360,6 +368,8 @@ mobius_emit_diag(ScanArgs s, const TIn *__restrict__ k, const float *__restrict_
                  const float *__restrict__ qn, const float *__restrict__ beta,
                  const float *__restrict__ lam_start, const float *__restrict__ lambda0,
                  float *__restrict__ lam_out) {
+    pdl_release();
+    pdl_wait();
     const int nkq = s.dk / 4;
     long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     long long pair = gid / nkq;
@@ -411,6 +421,8 @@ mobius_emit_iso(ScanArgs s, const TIn *__restrict__ k, const float *__restrict__
                 const float *__restrict__ qn, const float *__restrict__ beta,
                 const float *__restrict__ lam_start, const float *__restrict__ lambda0,
                 float *__restrict__ lam_out) {
+    pdl_release();
+    pdl_wait();
     long long pair = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     long long npairs = s.cu ? (long long)s.N * s.H : (long long)s.N * s.H * s.NB;
     if (pair >= npairs) return;
@@ -435,6 +447,8 @@ mobius_emit_iso(ScanArgs s, const TIn *__restrict__ k, const float *__restrict__
 // walks start first and the short ones fill in behind (list scheduling).
 __global__ void __launch_bounds__(256)
 kla_seq_order(const int *__restrict__ cu, int N, int *__restrict__ perm) {
+    pdl_release();
+    pdl_wait();
     __shared__ int len[kMaxOrderSeqs];
     for (int i = threadIdx.x; i < N; i += blockDim.x) len[i] = cu[i + 1] - cu[i];
     __syncthreads();
@@ -461,8 +475,8 @@ cudaError_t launch_mobius_reduce(const Plan &p, const void *k, const float *a, c
     ScanArgs s{p.N, p.H, p.dk, p.T, p.NB, nullptr};
     long long pairs = (long long)p.N * p.H * p.NB;
     if (p.iso) {
-        mobius_reduce_iso<TIn><<<blocks_for(pairs, 128), 128, 0, st>>>(s, (const TIn *)k, a, qn, beta, agg);
-        return cudaGetLastError();
+        return launch_pdl(mobius_reduce_iso<TIn>, blocks_for(pairs, 128), 128, 0, st, s, (const TIn *)k, a, qn,
+                          beta, agg);
     }
     const int dki = p.dk < 64 ? p.dk : 64, nhalf = p.dk / dki;
     const int kes = (int)sizeof(TIn);
@@ -486,25 +500,21 @@ cudaError_t launch_mobius_reduce(const Plan &p, const void *k, const float *a, c
     }
     const long long nitems = pairs * nhalf;
     const long long grid = std::min(nitems, 2LL * p.sms);
-    mobius_reduce_tma<TIn><<<(unsigned)grid, kRedSub * dki / 4, smem, st>>>(ma, mq, mk, s, beta, agg, nitems, status);
-    return cudaGetLastError();
+    return launch_pdl(mobius_reduce_tma<TIn>, (unsigned)grid, kRedSub * dki / 4, smem, st, ma, mq, mk, s, beta, agg,
+                      nitems, status);
 }
 
 cudaError_t launch_seq_order(const Plan &p, const int *cu, int *perm, cudaStream_t st) {
     if (p.N > kMaxOrderSeqs) return cudaErrorInvalidValue;
-    kla_seq_order<<<1, 256, 0, st>>>(cu, p.N, perm);
-    return cudaGetLastError();
+    return launch_pdl(kla_seq_order, 1, 256, 0, st, cu, p.N, perm);
 }
 
 cudaError_t launch_mobius_carry(const Plan &p, const float4 *agg, const float *lambda0,
                                 float *lam_blk, cudaStream_t st) {
     ScanArgs s{p.N, p.H, p.dk, p.T, p.NB, nullptr};
     long long thr = (long long)p.N * p.H * p.nl * 32;
-    if (p.seg_blocks >= 32)
-        mobius_carry<<<blocks_for(thr, 128), 128, 0, st>>>(s, p.nl, p.P, p.seg_blocks, agg, lambda0, lam_blk);
-    else
-        mobius_carry_lanes<<<blocks_for(thr, 128), 128, 0, st>>>(s, p.nl, p.P, p.seg_blocks, agg, lambda0, lam_blk);
-    return cudaGetLastError();
+    return launch_pdl(p.seg_blocks >= 32 ? mobius_carry : mobius_carry_lanes, blocks_for(thr, 128), 128, 0, st,
+                      s, p.nl, p.P, p.seg_blocks, agg, lambda0, lam_blk);
 }
 
 template <typename TIn>
@@ -514,12 +524,10 @@ cudaError_t launch_mobius_emit(const Plan &p, const int *cu, const void *k, cons
     ScanArgs s{p.N, p.H, p.dk, p.T, p.NB, cu};
     long long pairs = cu ? (long long)p.N * p.H : (long long)p.N * p.H * p.NB;
     if (p.iso)
-        mobius_emit_iso<TIn><<<blocks_for(pairs, 128), 128, 0, st>>>(
-            s, (const TIn *)k, a, qn, beta, lam_blk, lambda0, lam_out);
-    else
-        mobius_emit_diag<TIn><<<blocks_for(pairs * (p.dk / 4), 128), 128, 0, st>>>(
-            s, (const TIn *)k, a, qn, beta, lam_blk, lambda0, lam_out);
-    return cudaGetLastError();
+        return launch_pdl(mobius_emit_iso<TIn>, blocks_for(pairs, 128), 128, 0, st, s, (const TIn *)k, a, qn,
+                          beta, lam_blk, lambda0, lam_out);
+    return launch_pdl(mobius_emit_diag<TIn>, blocks_for(pairs * (p.dk / 4), 128), 128, 0, st, s,
+                      (const TIn *)k, a, qn, beta, lam_blk, lambda0, lam_out);
 }
 
 template cudaError_t launch_mobius_reduce<float>(const Plan &, const void *, const float *,

@@ -124,9 +124,11 @@ kla_status kla_forward_profiled(const kla_desc *desc,
 
 /* The work plan kla_forward uses for this descriptor on the current device:
  * segments each row is split into (1: one CTA walks a whole row or packed
- * sequence), kernel launches per call (1 unsplit; split rows: 4 on the
- * tensor-core path, whose output pass carries the segment states itself, 5 on
- * the CUDA-core walk; plus 1 for the launch order of packed sequences), and
+ * sequence), kernel launches per call (1 unsplit; split rows on the
+ * tensor-core path: Moebius reduce, Moebius carry unless the chunk kernel
+ * composes the short segments' aggregates itself, chunk kernel, segment starts
+ * and correction, so 4 or 5; 5 on the CUDA-core walk; plus 1 for the launch
+ * order of packed sequences), and
  * whether the chunk stages
  * run on the tcgen05 tensor-core kernel (1) or the CUDA-core walk (0).
  * Any output pointer may be NULL. Pure host computation. */
