@@ -54,7 +54,7 @@ template <typename TIn>
 __global__ void __launch_bounds__(128, 2)
 mobius_reduce_tma(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_qn,
                   const __grid_constant__ CUtensorMap tm_k, ScanArgs s, const float *__restrict__ beta,
-                  float4 *__restrict__ agg, long long nitems, int *status) {
+                  float4 *__restrict__ agg, int nitems, int *status) {
     using namespace ptx;
     const int dki = min(s.dk, 64), nq = dki / 4, nhalf = s.dk / dki;
     const int stA = kBlockTokens * dki * 4, stK = kBlockTokens * dki * (int)sizeof(TIn);
@@ -63,8 +63,10 @@ mobius_reduce_tma(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     float4 *part = reinterpret_cast<float4 *>(smraw + kRedStages * stB);    // [kRedSub][64]
     uint64_t *full = reinterpret_cast<uint64_t *>(part + kRedSub * 64), *empty = full + kRedStages;
     const int quad = threadIdx.x % nq, sub = threadIdx.x / nq;
-    const long long units = (long long)s.N * s.H;
-    const long long step = gridDim.x;
+    // 32-bit index arithmetic (the host checks the item count and the token
+    // axis fit): one unsigned division per decode
+    const unsigned units = (unsigned)(s.N * s.H), H = (unsigned)s.H;
+    const int step = gridDim.x;
     if (threadIdx.x == 0) {
         for (int j = 0; j < kRedStages; ++j) {
             mbar_init(&full[j], 1);
@@ -75,17 +77,21 @@ mobius_reduce_tma(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     __syncthreads();
     pdl_release();
     pdl_wait();
-    auto decode = [&](long long w, long long &u, int &blk, int &half) {
-        half = (int)(w % nhalf);
-        const long long r = w / nhalf;
-        u = r % units;
-        blk = (int)(r / units);
+    struct Item { unsigned u, n, h; int blk, half; };
+    auto decode = [&](int w) {
+        Item it;
+        const unsigned r = nhalf == 2 ? (unsigned)w >> 1 : (unsigned)w;   // nhalf is 1 or 2
+        it.half = nhalf == 2 ? (w & 1) : 0;
+        it.blk = (int)(r / units);
+        it.u = r - (unsigned)it.blk * units;
+        it.n = it.u / H;
+        it.h = it.u - it.n * H;
+        return it;
     };
-    auto issue = [&](long long w, int st) {
-        long long u; int blk, half;
-        decode(w, u, blk, half);
-        const int n = (int)(u / s.H), h = (int)(u % s.H);
-        const int tok = (int)((long long)n * s.T + (long long)blk * kBlockTokens);
+    auto issue = [&](int w, int st) {
+        const Item it = decode(w);
+        const int blk = it.blk, half = it.half, h = (int)it.h;
+        const int tok = (int)it.n * (int)s.T + blk * kBlockTokens;
         uint8_t *d = smraw + st * stB;
         mbar_expect_tx(&full[st], stB);
         tma_load_3d(d, &tm_a, &full[st], half * dki, h, tok);
@@ -99,34 +105,36 @@ mobius_reduce_tma(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
             if (globaltimer() - t0 > 2000000000ull) { atomicOr(status, kStatusTimeout); return false; }
         return true;
     };
-    long long nmine = 0;
-    if ((long long)blockIdx.x < nitems) nmine = (nitems - 1 - blockIdx.x) / step + 1;
+    int nmine = 0;
+    if ((int)blockIdx.x < nitems) nmine = (nitems - 1 - (int)blockIdx.x) / step + 1;
     if (threadIdx.x == 0)
-        for (int j = 0; j < kRedStages && j < nmine; ++j) issue(blockIdx.x + j * step, j);
+        for (int j = 0; j < kRedStages && j < nmine; ++j) issue((int)blockIdx.x + j * step, j);
     float bv[kRedLen];
-    auto load_beta = [&](long long w) {
-        long long u; int blk, half;
-        decode(w, u, blk, half);
-        const int n = (int)(u / s.H), h = (int)(u % s.H);
-        const long long t0 = (long long)blk * kBlockTokens + sub * kRedLen;
+    const int T = (int)s.T;
+    auto load_beta = [&](const Item &it) {
+        const int t0 = it.blk * kBlockTokens + sub * kRedLen;
+        const float *bp = beta + ((long long)it.n * T + t0) * H + it.h;
 #pragma unroll
-        for (int r = 0; r < kRedLen; ++r)
-            bv[r] = t0 + r < s.T ? __ldg(beta + ((long long)n * s.T + t0 + r) * s.H + h) : 0.f;
+        for (int r = 0; r < kRedLen; ++r) bv[r] = t0 + r < T ? __ldg(bp + r * H) : 0.f;
     };
-    if (nmine > 0) load_beta(blockIdx.x);
+    Item nxt = decode((int)blockIdx.x);
+    if (nmine > 0) load_beta(nxt);
     bool ok = true;
-    long long issued = min((long long)kRedStages, nmine), consumed = 0;
-    for (long long j = 0; j < nmine; ++j) {
-        const int st = (int)(j % kRedStages);
-        const long long w = blockIdx.x + j * step;
-        long long u; int blk, half;
-        decode(w, u, blk, half);
-        const long long t0 = (long long)blk * kBlockTokens + sub * kRedLen;
-        const int len = (int)max(0LL, min((long long)kRedLen, s.T - t0));
+    int issued = min(kRedStages, nmine), consumed = 0;
+    for (int j = 0; j < nmine; ++j) {
+        const int st = j % kRedStages;
+        const int w = (int)blockIdx.x + j * step;
+        const Item cur = nxt;
+        const int blk = cur.blk, half = cur.half;
+        const int t0 = blk * kBlockTokens + sub * kRedLen;
+        const int len = max(0, min(kRedLen, T - t0));
         float cb[kRedLen];
 #pragma unroll
         for (int r = 0; r < kRedLen; ++r) cb[r] = bv[r];
-        if (j + 1 < nmine) load_beta(w + step);
+        if (j + 1 < nmine) {
+            nxt = decode(w + step);
+            load_beta(nxt);
+        }
         // every thread waits; the CTA goes on only if all saw the copy land
         if (!__syncthreads_and(wait(&full[st], (uint32_t)((j / kRedStages) & 1)))) { ok = false; consumed = j; break; }
         const uint8_t *d = smraw + st * stB;
@@ -184,7 +192,7 @@ mobius_reduce_tma(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
         if (sub == 0) {
 #pragma unroll
             for (int c = 0; c < 4; ++c)
-                agg[(u * s.NB + blk) * s.dk + half * dki + 4 * quad + c] =
+                agg[((long long)cur.u * s.NB + blk) * s.dk + half * dki + 4 * quad + c] =
                     make_float4(m[c].m00, m[c].m01, m[c].m10, m[c].m11);
         }
         // part is rewritten by the next item; a failed refill stops every thread
@@ -192,7 +200,7 @@ mobius_reduce_tma(const __grid_constant__ CUtensorMap tm_a, const __grid_constan
     }
     // on a timeout, the copies issued but not consumed land before the CTA exits
     if (threadIdx.x == 0 && !ok)
-        for (long long j = consumed; j < issued; ++j) wait(&full[j % kRedStages], (uint32_t)((j / kRedStages) & 1));
+        for (int j = consumed; j < issued; ++j) wait(&full[j % kRedStages], (uint32_t)((j / kRedStages) & 1));
 }
 
 // Isotropic: one precision per head; increment beta*|k|^2/dk.
@@ -499,9 +507,11 @@ cudaError_t launch_mobius_reduce(const Plan &p, const void *k, const float *a, c
         attr[kes == 2][dev] = true;
     }
     const long long nitems = pairs * nhalf;
+    // the kernel indexes items and tokens in 32 bits (TMA coordinates are 32-bit too)
+    if (nitems >= (1LL << 31) || p.ntok >= (1LL << 31)) return cudaErrorInvalidValue;
     const long long grid = std::min(nitems, 2LL * p.sms);
     return launch_pdl(mobius_reduce_tma<TIn>, (unsigned)grid, kRedSub * dki / 4, smem, st, ma, mq, mk, s, beta, agg,
-                      nitems, status);
+                      (int)nitems, status);
 }
 
 cudaError_t launch_seq_order(const Plan &p, const int *cu, int *perm, cudaStream_t st) {
