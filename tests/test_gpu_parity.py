@@ -83,6 +83,18 @@ def test_segmented_path_matches(monkeypatch, segments):
     compare(w, inp, lam0, eta0)
 
 
+@pytest.mark.parametrize("segments", ["2", "24"])
+def test_long_and_many_segments(monkeypatch, segments):
+    # two long segments (24 blocks each: the correction pass runs its zero test
+    # and several chunks per CTA) and 24 short ones (one or two blocks each:
+    # the Moebius carry runs as its own launch, not inside the walk kernel)
+    monkeypatch.setenv("KLA_SEGMENTS", segments)
+    w = WORKLOADS[1].with_(B=1, H=2, T=3000)
+    inp = make_inputs(w)
+    lam0, eta0 = random_state(w, w.B, seed=23)
+    compare(w, inp, lam0, eta0)
+
+
 @pytest.mark.parametrize("T", [1, 5, 63, 64, 65, 127, 257, 1000])
 def test_ragged_lengths(T):
     w = WORKLOADS[1].with_(B=2, H=2, T=T)
