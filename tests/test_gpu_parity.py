@@ -86,8 +86,8 @@ def test_segmented_path_matches(monkeypatch, segments):
 @pytest.mark.parametrize("segments", ["2", "24"])
 def test_long_and_many_segments(monkeypatch, segments):
     # two long segments (24 blocks each: the correction pass runs its zero test
-    # and several chunks per CTA) and 24 short ones (one or two blocks each:
-    # the Moebius carry runs as its own launch, not inside the walk kernel)
+    # over several chunks per CTA) and 24 short ones (two blocks each: 23
+    # segment-start beliefs chained before the last segment)
     monkeypatch.setenv("KLA_SEGMENTS", segments)
     w = WORKLOADS[1].with_(B=1, H=2, T=3000)
     inp = make_inputs(w)
