@@ -29,8 +29,11 @@
 //              memory, mask the score tile into P, store the output rows;
 //   warp 8     TMA producer (q, k, v tiles double-buffered; a, qn ring);
 //   warp 9     TMEM owner and single-thread tcgen05.mma issuer.
-// mode 1 ("state") runs only the state recursion from eta = 0 and writes the
-// segment's transfer (eta_end, prod of gates) for the inter-segment carry.
+// mode 0 walks whole rows or packed sequences (from lambda0, eta0); mode 2
+// walks every segment of split rows from a zero state (segment 0 from eta0)
+// and exports what the correction pass needs. The kernel is instantiated per
+// (dk, dv, isotropic or diagonal precision), each variant with only its own
+// gate code.
 //
 // Every wait is bounded: after kWaitLimitNs a waiter sets the abort flag and
 // the library status bit, all roles fall through to the teardown, the
@@ -251,7 +254,7 @@ __device__ __forceinline__ void gate_slot(int j, const float *ra, uint8_t *qt, u
 
 }  // namespace
 
-template <int DK, int DV>
+template <int DK, int DV, bool ISO>
 __global__ void __launch_bounds__(Roles<DK, DV>::THREADS, Roles<DK, DV>::MIN_BLOCKS)
 kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
@@ -276,7 +279,10 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     float2 *isof = reinterpret_cast<float2 *>(sm + L::isof0);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const bool state_mode = g.mode == 1;
+    // the transfer-only pass (mode 1) runs on the CUDA-core walk; this kernel
+    // takes modes 0 and 2, and is instantiated per precision mode (ISO), so that
+    // each variant holds only its own gate code
+    constexpr bool state_mode = false;
     // mode 2: every segment walks from a zero state (segment 0 from eta0), writes
     // its transfer and decay, and segments p > 0 export their folded q tiles and
     // chunk references for the correction pass that adds the carried state
@@ -310,7 +316,7 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     }
     if (warp == RL::PRODW && lane == 0) {
         prefetch_map(&tm_q); prefetch_map(&tm_k); prefetch_map(&tm_v);
-        if (!g.iso) { prefetch_map(&tm_a); prefetch_map(&tm_qn); }
+        if (!ISO) { prefetch_map(&tm_a); prefetch_map(&tm_qn); }
     }
     if (warp == RL::MMAW) tmem_alloc(tmem_hold, L::NCOLS);
     tc_fence_before();
@@ -348,9 +354,9 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         for (int r = 0; r < kSlotTok; ++r) offr[r] = sw_off(r, i, kC);
         float lam = 1.0f;
         {
-            const int il = g.iso ? 0 : i;
-            if (key || g.iso) {
-                const int nl = g.iso ? 1 : DK;
+            const int il = ISO ? 0 : i;
+            if (key || ISO) {
+                const int nl = ISO ? 1 : DK;
                 lam = g.lambda0 ? g.lambda0[u * nl + il] : 1.0f;
                 if (p > 0 && g.agg) {
                     // compose the Moebius aggregates of the blocks before this segment
@@ -389,11 +395,11 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         float nb0 = 0.f, nb1 = 0.f, na0 = 1.f, na1 = 1.f, nq0 = 0.f, nq1 = 0.f;
         auto prefetch = [&](int c) {
             const long long t0 = tb + (long long)c * kC;
-            const long long x0 = g.iso ? t0 + 2 * lane : t0 + lane;
-            const long long x1 = g.iso ? x0 + 1 : t0 + 32 + lane;
+            const long long x0 = ISO ? t0 + 2 * lane : t0 + lane;
+            const long long x1 = ISO ? x0 + 1 : t0 + 32 + lane;
             nb0 = x0 < te ? __ldg(g.beta + x0 * g.H + h) : 0.f;
             nb1 = x1 < te ? __ldg(g.beta + x1 * g.H + h) : 0.f;
-            if (g.iso) {
+            if (ISO) {
                 na0 = x0 < te ? __ldg(g.a + x0 * g.H + h) : 1.f;
                 na1 = x1 < te ? __ldg(g.a + x1 * g.H + h) : 1.f;
                 nq0 = x0 < te ? __ldg(g.qn + x0 * g.H + h) : 0.f;
@@ -414,7 +420,7 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             float e_cur;           // 2^(G_last - R)
             float glast_log2;      // G_last
             uint8_t *klo = sm + L::klo0 + s * L::QK;
-            if (!g.iso) {
+            if (!ISO) {
                 // One pass per chunk. Projective form of the precision: lambda = n/d with
                 //   d <- a^2 d + qn n,  n <- n + b d   (b = beta k^2),
                 // two FMAs per token on the serial chain. The gate is g = a d_prev / d,
@@ -638,7 +644,7 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
             }
             // state rescale factors: U_c = diag(2^R_c) S_c, S_{c+1} = diag(2^(G_last - R_c)) (U_c + K'^T V)
-            fac[s * DK + i] = g.iso ? e_prev * __int_as_float((127 + max(-126, min(127, R))) << 23) : fac_c;
+            fac[s * DK + i] = ISO ? e_prev * __int_as_float((127 + max(-126, min(127, R))) << 23) : fac_c;
             if (c == nchunks - 1) fac_final[i] = e_cur;
             e_prev = e_cur;
             log_decay += glast_log2;
@@ -647,10 +653,10 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         if (ok && !*abort_flag) {
             if (state_mode || local_mode) {
-                if (g.iso ? (gt == 0) : key) g.decay[(u * g.P + p) * (g.iso ? 1 : DK) + (g.iso ? 0 : i)] = exp2f(log_decay);
+                if (ISO ? (gt == 0) : key) g.decay[(u * g.P + p) * (ISO ? 1 : DK) + (ISO ? 0 : i)] = exp2f(log_decay);
             }
             if (!state_mode && last_seg && g.final_lambda) {
-                if (g.iso ? (gt == 0) : key) g.final_lambda[u * (g.iso ? 1 : DK) + (g.iso ? 0 : i)] = lam;
+                if (ISO ? (gt == 0) : key) g.final_lambda[u * (ISO ? 1 : DK) + (ISO ? 0 : i)] = lam;
             }
         }
       }
@@ -671,7 +677,7 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // transfers of the row's earlier segments, S <- D_q S + dS_q for q < p
         // (D_q: the segment's gate product per key, dS_q: its state transfer).
         if (!state_mode && nchunks > 0) {
-            const int nl = g.iso ? 1 : DK;
+            const int nl = ISO ? 1 : DK;
 #pragma unroll
             for (int cb = 0; cb < DV / 32; ++cb) {
                 float acc[32];
@@ -684,7 +690,7 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const int nprev = local_mode ? 0 : p;   // mode 2: segments from a zero state
 #pragma unroll 4
                 for (int q = 0; q < nprev; ++q) {
-                    const float dq = vU ? g.decay[(u * g.P + q) * nl + (g.iso ? 0 : rowU)] : 0.f;
+                    const float dq = vU ? g.decay[(u * g.P + q) * nl + (ISO ? 0 : rowU)] : 0.f;
                     const float *src = g.S_io + ((u * g.P + q) * DK + rowU) * DV + cb * 32;
 #pragma unroll
                     for (int x = 0; x < 32; x += 4) {
@@ -885,13 +891,13 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     }
 #pragma unroll
                     for (int a = 0; a < DV / 64; ++a) tma_prefetch_3d(&tm_v, 64 * a, h, tp);
-                    if (!g.iso)
+                    if (!ISO)
                         for (int j = 0; j < kRingsPerChunk; ++j) {
                             tma_prefetch_3d(&tm_a, 0, h, tp + kRingTok * j);
                             tma_prefetch_3d(&tm_qn, 0, h, tp + kRingTok * j);
                         }
                 }
-                if (!g.iso) {
+                if (!ISO) {
                     for (int j = 0; j < kRingsPerChunk; ++j) {
                         const int n = c * kRingsPerChunk + j, slot = n % kRings;
                         if (n >= kRings && !wait1(&ring_empty[slot], ((n / kRings) - 1) & 1, abort_flag, g.status)) {
@@ -1052,12 +1058,16 @@ cudaError_t launch_t(const Plan &p, const int *cu, int mode, const void *q, cons
     if (ok && mode == 2) ok = make_tma_map(&mqs, p.qbuf, BF, 2, DK, p.H, p.ntok, 64, kC, true);
     else mqs = mq;
     if (!ok) return cudaErrorInvalidValue;
+    if (mode != 0 && mode != 2) return cudaErrorInvalidValue;
     static bool attr[64] = {};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(kla_chunk_tc_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             L::alloc);
+        cudaError_t e = cudaFuncSetAttribute(kla_chunk_tc_kernel<DK, DV, false>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, L::alloc);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(kla_chunk_tc_kernel<DK, DV, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     L::alloc);
         if (e != cudaSuccess) return e;
         attr[dev] = true;
     }
@@ -1069,10 +1079,10 @@ cudaError_t launch_t(const Plan &p, const int *cu, int mode, const void *q, cons
     g.rlog = p.rlog; g.NC = p.NB;
     g.S_io = S_io; g.decay = decay; g.out = (__nv_bfloat16 *)out;
     g.final_lambda = final_lambda; g.final_eta = final_eta; g.status = status;
-    const long long segs = mode == 1 ? p.P - 1 : p.P;
+    const long long segs = p.P;
     const unsigned grid = (unsigned)((long long)p.N * p.H * segs);
     if (grid == 0) return cudaSuccess;
-    return launch_pdl(kla_chunk_tc_kernel<DK, DV>, grid, Roles<DK, DV>::THREADS, L::alloc, st, mq, mk, mv, ma, mqn,
+    return launch_pdl(p.iso ? kla_chunk_tc_kernel<DK, DV, true> : kla_chunk_tc_kernel<DK, DV, false>, grid, Roles<DK, DV>::THREADS, L::alloc, st, mq, mk, mv, ma, mqn,
                       mqs, g);
 }
 
