@@ -254,7 +254,7 @@ __device__ __forceinline__ void gate_slot(int j, const float *ra, uint8_t *qt, u
 
 }  // namespace
 
-template <int DK, int DV, bool ISO>
+template <int DK, int DV, bool ISO, bool LOCAL>
 __global__ void __launch_bounds__(Roles<DK, DV>::THREADS, Roles<DK, DV>::MIN_BLOCKS)
 kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
@@ -280,13 +280,13 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     // the transfer-only pass (mode 1) runs on the CUDA-core walk; this kernel
-    // takes modes 0 and 2, and is instantiated per precision mode (ISO), so that
-    // each variant holds only its own gate code
+    // takes modes 0 and 2 and is instantiated per precision mode (ISO) and walk
+    // mode (LOCAL), so that each variant holds only its own code
     constexpr bool state_mode = false;
     // mode 2: every segment walks from a zero state (segment 0 from eta0), writes
     // its transfer and decay, and segments p > 0 export their folded q tiles and
     // chunk references for the correction pass that adds the carried state
-    const bool local_mode = g.mode == 2;
+    constexpr bool local_mode = LOCAL;
     // one gate thread per key: each reads and rewrites only its own key column
     const int gate_threads = DK;
     const bool is_gate = (RL::NGW == 4) ? (warp < 4) : (warp == 0 || warp == 2);
@@ -673,11 +673,10 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const float *eta0 = (!state_mode && (!local_mode || p == 0) && g.eta0) ? g.eta0 + u * DK * DV : nullptr;
         bool ok = true;
         // Belief at the segment start, written into the U columns of TMEM before
-        // the first chunk (while the gate works on it): eta0 carried through the
-        // transfers of the row's earlier segments, S <- D_q S + dS_q for q < p
-        // (D_q: the segment's gate product per key, dS_q: its state transfer).
+        // the first chunk (while the gate works on it): eta0 for whole rows and
+        // first segments, zero for the later segments of split rows (their
+        // carried state is added by the correction pass)
         if (!state_mode && nchunks > 0) {
-            const int nl = ISO ? 1 : DK;
 #pragma unroll
             for (int cb = 0; cb < DV / 32; ++cb) {
                 float acc[32];
@@ -686,20 +685,6 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     const float4 e4 = (vU && eta0) ? *reinterpret_cast<const float4 *>(eta0 + rowU * DV + cb * 32 + x)
                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
                     acc[x] = e4.x; acc[x + 1] = e4.y; acc[x + 2] = e4.z; acc[x + 3] = e4.w;
-                }
-                const int nprev = local_mode ? 0 : p;   // mode 2: segments from a zero state
-#pragma unroll 4
-                for (int q = 0; q < nprev; ++q) {
-                    const float dq = vU ? g.decay[(u * g.P + q) * nl + (ISO ? 0 : rowU)] : 0.f;
-                    const float *src = g.S_io + ((u * g.P + q) * DK + rowU) * DV + cb * 32;
-#pragma unroll
-                    for (int x = 0; x < 32; x += 4) {
-                        const float4 d4 = vU ? *reinterpret_cast<const float4 *>(src + x) : make_float4(0.f, 0.f, 0.f, 0.f);
-                        acc[x] = fmaf(dq, acc[x], d4.x);
-                        acc[x + 1] = fmaf(dq, acc[x + 1], d4.y);
-                        acc[x + 2] = fmaf(dq, acc[x + 2], d4.z);
-                        acc[x + 3] = fmaf(dq, acc[x + 3], d4.w);
-                    }
                 }
                 uint32_t r[32];
 #pragma unroll
@@ -1063,12 +1048,15 @@ cudaError_t launch_t(const Plan &p, const int *cu, int mode, const void *q, cons
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 64 && !attr[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(kla_chunk_tc_kernel<DK, DV, false>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, L::alloc);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(kla_chunk_tc_kernel<DK, DV, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     L::alloc);
-        if (e != cudaSuccess) return e;
+        void (*const kerns[4])(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap,
+                               TcArgs) = {kla_chunk_tc_kernel<DK, DV, false, false>,
+                                          kla_chunk_tc_kernel<DK, DV, false, true>,
+                                          kla_chunk_tc_kernel<DK, DV, true, false>,
+                                          kla_chunk_tc_kernel<DK, DV, true, true>};
+        for (auto kern : kerns) {
+            const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::alloc);
+            if (e != cudaSuccess) return e;
+        }
         attr[dev] = true;
     }
     TcArgs g;
@@ -1082,7 +1070,10 @@ cudaError_t launch_t(const Plan &p, const int *cu, int mode, const void *q, cons
     const long long segs = p.P;
     const unsigned grid = (unsigned)((long long)p.N * p.H * segs);
     if (grid == 0) return cudaSuccess;
-    return launch_pdl(p.iso ? kla_chunk_tc_kernel<DK, DV, true> : kla_chunk_tc_kernel<DK, DV, false>, grid, Roles<DK, DV>::THREADS, L::alloc, st, mq, mk, mv, ma, mqn,
+    auto kern = p.iso ? (mode == 2 ? kla_chunk_tc_kernel<DK, DV, true, true> : kla_chunk_tc_kernel<DK, DV, true, false>)
+                      : (mode == 2 ? kla_chunk_tc_kernel<DK, DV, false, true>
+                                   : kla_chunk_tc_kernel<DK, DV, false, false>);
+    return launch_pdl(kern, grid, Roles<DK, DV>::THREADS, L::alloc, st, mq, mk, mv, ma, mqn,
                       mqs, g);
 }
 
