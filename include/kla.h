@@ -96,7 +96,10 @@ size_t kla_precision_workspace_bytes(const kla_desc *desc);
  * aligned): device pointers, or NULL for lambda0 = 1 and eta0 = 0. final_lambda/final_eta: device pointers or NULL to
  * skip. workspace: device, 256-byte aligned, >= kla_workspace_bytes(desc).
  * Ntok == 0 is a no-op. Errors: KLA_ERR_INVALID_ARG / KLA_ERR_UNSUPPORTED
- * before any launch; KLA_ERR_CUDA if a launch fails. */
+ * before any launch; KLA_ERR_CUDA if a launch fails. Stream order holds as
+ * for any launch: the library's kernels use programmatic dependent launch
+ * among themselves, and each waits for the work before it in the stream to
+ * complete before it touches global memory. */
 kla_status kla_forward(const kla_desc *desc,
                        const void *q, const void *k, const void *v,
                        const float *a, const float *qn, const float *beta,
