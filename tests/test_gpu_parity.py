@@ -95,6 +95,16 @@ def test_long_and_many_segments(monkeypatch, segments):
     compare(w, inp, lam0, eta0)
 
 
+def test_correction_zero_test(monkeypatch):
+    # 64 rows x heads in two segments of 32 blocks: correction CTAs of four
+    # chunks, so the zero test over the chunks runs
+    monkeypatch.setenv("KLA_SEGMENTS", "2")
+    w = WORKLOADS[1].with_(B=4, H=16, T=4096)
+    inp = make_inputs(w)
+    lam0, eta0 = random_state(w, w.B, seed=29)
+    compare(w, inp, lam0, eta0)
+
+
 @pytest.mark.parametrize("T", [1, 5, 63, 64, 65, 127, 257, 1000])
 def test_ragged_lengths(T):
     w = WORKLOADS[1].with_(B=2, H=2, T=T)
