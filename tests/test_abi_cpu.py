@@ -102,3 +102,27 @@ def test_host_buffer_size_covers_inputs_outputs_and_workspace(L):
     ntok = 2000
     io = ntok * 4 * (64 * 2 * 2 + 128 * 2 * 2 + 64 * 4 * 2 + 4)
     assert n >= io + L.kla_workspace_bytes(ctypes.byref(desc))
+
+
+class _FakePtr:
+    """A stand-in for a device tensor: the plan reads only the descriptor's
+    shapes, never the packed-sequence offsets themselves."""
+
+    def data_ptr(self):
+        return 256
+
+
+@pytest.mark.parametrize("shape,expect", [
+    # (B, T, H, dk, dv, dtype, mode, packed sequences) -> (segments per row, launches, tensor cores)
+    ((4, 2048, 8, 64, 64, kla.KLA_BF16, kla.KLA_DIAG, 0), (8, 4, True)),      # small layer: 256 CTAs, one wave
+    ((8, 4096, 16, 128, 128, kla.KLA_BF16, kla.KLA_DIAG, 0), (1, 1, True)),   # 1.3B layer: rows fill the SMs
+    ((1, 131072, 16, 128, 128, kla.KLA_BF16, kla.KLA_DIAG, 0), (9, 5, True)),  # long context: separate carry
+    ((2, 16384, 32, 64, 128, kla.KLA_BF16, kla.KLA_ISO, 8), (1, 2, True)),   # packed: length ranking + walk
+    ((1, 256, 2, 16, 16, kla.KLA_FP32, kla.KLA_DIAG, 0), (4, 5, False)),      # fp32: CUDA-core walk passes
+])
+def test_launch_plan_of_the_workloads(L, shape, expect):
+    # on a host without a GPU the plan assumes the 148 SMs of a B200
+    B, T, H, dk, dv, dt, mode, nseq = shape
+    d = kla.make_desc(B, T, H, dk, dv, dt, mode, _FakePtr() if nseq else None, nseq)
+    p = kla.plan(d)
+    assert (p["segments"], p["launches"], p["tensor_core"]) == expect
