@@ -10,9 +10,10 @@ inputs resident in HBM. Prints ONE JSON line (rank 0):
               (512 MiB write) between timed steps, max over ranks;
   e2e         the same metric through kla_forward_host: pinned host inputs
               copied in, forward, output copied back, inside the timed region;
-  roofline    the dominant kernel (the chunk kernel's output pass) against the
-              measured HBM copy bandwidth: algorithmic bytes (inputs read once,
-              output written once) / its event-timed duration;
+  roofline    the dominant kernel (the chunk kernel walking whole rows, or the
+              segments of split rows) against the measured HBM copy bandwidth:
+              algorithmic bytes (inputs read once, output written once) / its
+              event-timed duration;
   cpu_baseline the CPU oracle (plain fp64 C, OpenMP) on a bounded sample of
               the same workload, on this host's cores.
 
@@ -330,11 +331,21 @@ def main():
         step(i, profiled=True)
     torch.cuda.synchronize()
     kla.check()
-    chunk = [r[4].elapsed_time(r[5]) for r in evs]            # ms, output pass (chunk kernel)
+    chunk = [r[4].elapsed_time(r[5]) for r in evs]            # ms, the walk kernel
     pre = [r[0].elapsed_time(r[4]) for r in evs]
-    # per launch of the sequence: reduce, carry, state pass, state carry, output pass
-    stage_names = ("mobius_reduce", "mobius_carry", "state_pass", "state_carry", "output_pass", "correction")
-    per_stage = {n: statistics.mean(r[i].elapsed_time(r[i + 1]) for r in evs) for i, n in enumerate(stage_names)}
+    # the launches of this plan, by the event pair that brackets each (an event
+    # between every launch; stages without a launch of this plan are left out)
+    if plan["tensor_core"] and plan["segments"] > 1:
+        named = [(0, "mobius_reduce")] + ([(1, "mobius_carry")] if plan["launches"] == 5 else []) + \
+                [(4, "segment_walk"), (5, "segment_starts_and_correction")]
+        walk_label = "kla_chunk_tc_kernel (segment walk)"
+    elif plan["segments"] > 1:
+        named = [(0, "mobius_reduce"), (1, "mobius_carry"), (2, "state_pass"), (3, "state_carry"), (4, "output_pass")]
+        walk_label = "kla_walk_simt (output pass)"
+    else:
+        named = ([(0, "sequence_order")] if plan["launches"] == 2 else []) + [(4, "walk")]
+        walk_label = "kla_chunk_tc_kernel (whole rows)" if plan["tensor_core"] else "kla_walk_simt"
+    per_stage = {n: statistics.mean(r[i].elapsed_time(r[i + 1]) for r in evs) for i, n in named}
     ms_per_step, value = aggregate(world, w.tokens, sum(tot), steps, dist)
 
     # ---- e2e through the host-buffer entry point
@@ -386,11 +397,11 @@ def main():
                    "l2": "flushed between timed steps (512 MiB device write, then 256 MiB read)", "parallelism": "dp%d" % world},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "kla_chunk_tc_kernel (output pass)" if plan["tensor_core"] else "kla_walk_simt",
+                     "kernel": walk_label,
                      "alg_bytes_per_launch": alg_bytes, "launch_ms": chunk_ms,
                      "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_src},
-        "stages_ms": {"note": "separate run with an event between every launch",
-                      "pre_passes": statistics.mean(pre), "output_pass": chunk_ms,
+        "stages_ms": {"note": "separate run with an event between every launch (each adds about 2.6 us)",
+                      "before_walk": statistics.mean(pre), "walk_kernel": chunk_ms,
                       "total": statistics.mean(r[0].elapsed_time(r[6]) for r in evs), "launches": per_stage},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h_in, "d2h_bytes_per_step": h_out},
         "gpu_launches": steps * plan["launches"],
