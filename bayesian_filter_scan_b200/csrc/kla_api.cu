@@ -74,8 +74,8 @@ static bool pow2_in(int x, int lo, int hi) {
 // `per_sm` CTAs fit on an SM, so the segment count is the largest that keeps
 // every (row, head, segment) unit in one wave: more units would add a partial
 // wave, fewer would leave SMs idle. Rows x heads that already occupy half the
-// SMs are not split (the extra precision and state passes would cost more than
-// they gain). KLA_SEGMENTS overrides (tuning only; the result does not depend
+// SMs are not split (the Moebius reduce and the correction pass would cost more
+// than they gain). KLA_SEGMENTS overrides (tuning only; the result does not depend
 // on it beyond rounding).
 static int choose_segments(long long units, int NB, int per_sm) {
     const char *env = getenv("KLA_SEGMENTS");

@@ -109,14 +109,15 @@ kla_status kla_forward(const kla_desc *desc,
                        cudaStream_t stream);
 
 /* kla_forward that also records seven caller-created CUDA events on `stream`:
- * events[0] before the first launch and events[1..6] after the stages
- * 1 Moebius block reduction, 2 Moebius carry, 3 segment state pass,
- * 4 segment state carry, 5 output pass (the chunk walk), 6 correction pass
+ * events[0] before the first launch (the length ranking of packed sequences
+ * falls between events[0] and events[1]) and events[1..6] after the stages
+ * 1 Moebius block reduction, 2 Moebius carry, 3 segment state pass and
+ * 4 segment state carry (CUDA-core walk only), 5 the walk (whole rows, or
+ * every segment of split rows), 6 segment-start beliefs and correction pass
  * (split rows on the tensor-core path: the carried segment-start states added
- * to the outputs of segments walked from a zero state; there stages 3 and 4 do
- * not run). Stages that do not run for this descriptor record at the same
- * point as the previous one. For measuring the stages; otherwise identical to
- * kla_forward. */
+ * to the outputs of segments walked from a zero state). Stages that do not run
+ * for this descriptor record at the same point as the previous one. For
+ * measuring the stages; otherwise identical to kla_forward. */
 kla_status kla_forward_profiled(const kla_desc *desc,
                                 const void *q, const void *k, const void *v,
                                 const float *a, const float *qn, const float *beta,
