@@ -118,6 +118,10 @@ class _FakePtr:
     ((8, 4096, 16, 128, 128, kla.KLA_BF16, kla.KLA_DIAG, 0), (1, 1, True)),   # 1.3B layer: rows fill the SMs
     ((1, 131072, 16, 128, 128, kla.KLA_BF16, kla.KLA_DIAG, 0), (9, 5, True)),  # long context: separate carry
     ((2, 16384, 32, 64, 128, kla.KLA_BF16, kla.KLA_ISO, 8), (1, 2, True)),   # packed: length ranking + walk
+    ((1, 9000, 2, 64, 64, kla.KLA_BF16, kla.KLA_DIAG, 1700), (1, 1, True)),  # > 1024 sequences: input order
+    # 128 blocks, room for 74 CTAs per row x head: 64 segments of 2 blocks; 126
+    # blocks before the last segment, so the Moebius carry is its own launch
+    ((1, 8192, 2, 64, 128, kla.KLA_BF16, kla.KLA_DIAG, 0), (64, 5, True)),
     ((1, 256, 2, 16, 16, kla.KLA_FP32, kla.KLA_DIAG, 0), (4, 5, False)),      # fp32: CUDA-core walk passes
 ])
 def test_launch_plan_of_the_workloads(L, shape, expect):
