@@ -56,7 +56,7 @@ typedef enum {
     KLA_OK = 0,
     KLA_ERR_INVALID_ARG = 1,  /* bad shape, null required pointer, misaligned
                                  pointer, workspace too small; nothing launched */
-    KLA_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement */
+    KLA_ERR_UNSUPPORTED = 2,  /* valid request the library does not implement */
     KLA_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
     KLA_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up (kla_check) */
     KLA_ERR_RANGE = 5         /* the in-chunk log-gate span exceeded the range
