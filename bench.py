@@ -184,6 +184,31 @@ def cpu_baseline(w, inp, target_s=12.0):
                 n_units, units_total, t, reps)}
 
 
+def arm_config(w, plan, world):
+    """The workload's `config` object, the same on both arms."""
+    return {"workload": workload_label(w), "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv,
+            "mode": w.mode, "varlen": w.varlen, "tokens_per_step_per_gpu": w.tokens,
+            "segments_per_row": plan["segments"], "tensor_core_chunk_kernel": plan["tensor_core"],
+            "l2": "flushed between timed steps (512 MiB device write, then 256 MiB read)",
+            "parallelism": "dp%d" % world}
+
+
+class _HostOffsets:
+    """Stands in for the packed-sequence offsets when only the plan is asked
+    for: the plan reads the descriptor's shapes, never the offsets."""
+
+    def data_ptr(self):
+        return 256
+
+
+def host_plan(w, num_seqs):
+    mode = kla.KLA_ISO if w.mode == "iso" else kla.KLA_DIAG
+    dt = kla.KLA_BF16 if w.dtype == "bf16" else kla.KLA_FP32
+    desc = kla.make_desc(w.B, w.T, w.H, w.dk, w.dv, dt, mode, _HostOffsets() if w.varlen else None,
+                         num_seqs if w.varlen else 0)
+    return kla.plan(desc)
+
+
 def run_reference(args, w):
     """Reference arm: the CPU oracle timed on this host's cores."""
     rank = int(os.environ.get("RANK", "0"))
@@ -207,7 +232,7 @@ def run_reference(args, w):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": workload_label(w)},
+        "config": arm_config(w, host_plan(w, units_total // w.H), args.gpus),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -391,10 +416,7 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-        "config": {"workload": workload_label(w), "B": w.B, "H": H, "T": w.T, "dk": dk, "dv": dv,
-                   "mode": w.mode, "varlen": w.varlen, "tokens_per_step_per_gpu": w.tokens,
-                   "segments_per_row": plan["segments"], "tensor_core_chunk_kernel": plan["tensor_core"],
-                   "l2": "flushed between timed steps (512 MiB device write, then 256 MiB read)", "parallelism": "dp%d" % world},
+        "config": arm_config(w, plan, world),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "kernel": walk_label,
