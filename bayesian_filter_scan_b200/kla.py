@@ -20,6 +20,8 @@ LIB_PATH = os.path.join(_HERE, "libkla.so")
 KLA_OK, KLA_ERR_INVALID_ARG, KLA_ERR_UNSUPPORTED, KLA_ERR_CUDA, KLA_ERR_TIMEOUT, KLA_ERR_RANGE = range(6)
 KLA_BF16, KLA_FP32 = 0, 1
 KLA_DIAG, KLA_ISO = 0, 1
+# KLA_NOALLOC_SCRATCH_BYTES of include/kla.h: the fixed scratch area of kla_forward_noalloc
+NOALLOC_SCRATCH_BYTES = 32 << 20
 
 # Every symbol include/kla.h declares.
 EXPORTS = ("kla_workspace_bytes", "kla_precision_workspace_bytes", "kla_forward", "kla_forward_profiled",

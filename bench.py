@@ -3,21 +3,27 @@
 
 One step = one kla_forward call over one batch of the workload (the whole hot
 path: Moebius precision scan, state passing, chunked tensor-core pass) with
-inputs resident in HBM. Prints ONE JSON line (rank 0):
+inputs resident in HBM. The default workload is the largest single-GPU one,
+the 128k-token long context (B=1, H=16, T=131072, dk=dv=128, final state
+returned). Prints ONE JSON line (rank 0):
 
-  value       tokens/s (B*T per second, all ranks together), device-timed with
-              CUDA events on the launching stream around each call, L2 flushed
-              (512 MiB write) between timed steps, max over ranks;
-  e2e         the same metric through kla_forward_host: pinned host inputs
-              copied in, forward, output copied back, inside the timed region;
-  roofline    the dominant kernel (the chunk kernel walking whole rows, or the
-              segments of split rows) against the measured HBM copy bandwidth:
-              algorithmic bytes (inputs read once, output written once) / its
-              event-timed duration;
+  value        tokens/s (B*T per second, all ranks together), device-timed with
+               CUDA events on the launching stream around each call, L2 flushed
+               (512 MiB write) between timed steps, max over ranks;
+  e2e          the same metric through kla_forward_host: pinned host inputs
+               copied in, forward, output copied back, inside the timed region;
+  roofline     the dominant kernel (the chunk kernel walking whole rows, or the
+               segments of split rows) against the measured HBM copy bandwidth:
+               algorithmic bytes (inputs read once, output written once) / its
+               event-timed duration;
+  roofline_scan the Moebius precision scan's block reduction (rows split into
+               segments) against the same peak;
+  max_err      the largest scaled error |gpu - oracle| / (1 + |oracle|) of the
+               timed output on the units the CPU baseline computed;
   cpu_baseline the CPU oracle (plain fp64 C, OpenMP) on a bounded sample of
-              the same workload, on this host's cores.
+               the same workload, on this host's cores.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 1] [--impl reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 3] [--impl reference]
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own batch of
 the workload (independent sequences; no collective on the data path), so the
@@ -31,25 +37,26 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
+import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
+import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from bayesian_filter_scan_b200 import kla  # noqa: E402
 from bayesian_filter_scan_b200.inputs import WORKLOADS, make_inputs  # noqa: E402
 
 METRIC = "KLA forward tokens/s per layer (B*T/s) on 1 B200; % of HBM / bf16 TC roofline"
 UNIT = "tokens/s"
+DEFAULT_WORKLOAD = 3
 FLUSH_BYTES = 512 << 20
 SWEEP_BYTES = 256 << 20
 FALLBACK_HBM_GBS = 6650.0
+TOL = {"bf16": 2e-2, "fp32": 1e-4}
 
 
 def log(*a):
@@ -69,6 +76,14 @@ def bytes_per_token_head(w) -> int:
     return es * (2 * w.dk + 2 * w.dv) + 4 * 2 * nl + 4
 
 
+def scan_bytes_per_token_head(w) -> int:
+    """Algorithmic bytes of the Moebius block reduction per (token, head): the
+    key, the decay and process noise, and the value precision, read once."""
+    es = 2 if w.dtype == "bf16" else 4
+    nl = 1 if w.mode == "iso" else w.dk
+    return es * w.dk + 4 * 2 * nl + 4
+
+
 def flops_per_token_head(w) -> int:
     """The recurrence's own arithmetic: rank-1 state update and readout."""
     return 4 * w.dk * w.dv
@@ -82,70 +97,91 @@ def measured_peaks():
         return {"hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
 
 
-def chunk_kernel_hash() -> str:
-    with open(os.path.join(ROOT, "bayesian_filter_scan_b200", "csrc", "kla_chunk_tc.cu"), "rb") as f:
+def source_hash(name: str) -> str:
+    with open(os.path.join(ROOT, "bayesian_filter_scan_b200", "csrc", name), "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def traffic_record(wid):
-    """DRAM bytes per launch of the chunk kernel from a committed ncu summary,
-    if it was taken on the current kernel source."""
+def traffic_record(wid, kernel_file="kla_chunk_tc.cu"):
+    """DRAM bytes per launch of the dominant kernel from a committed ncu
+    summary, if it was taken on the current kernel source."""
     path = os.path.join(ROOT, "profiles", "chunk_kernel_traffic.json")
     try:
         rec = json.load(open(path)).get(str(wid))
     except Exception:
         return None
-    if not rec or rec.get("kernel_sha") != chunk_kernel_hash():
+    if not rec or rec.get("kernel_sha") != source_hash(kernel_file):
         return None
     return rec.get("dram_bytes_per_launch")
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    """SM clock and clock-event reasons of this process's GPU, read through
+    NVML every 5 ms on a background thread while the timed region runs (read
+    only: no clock or other setting is changed)."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+             ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+             ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+             ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = None
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.samples = []
+        self.err = None
+        self._stop = threading.Event()
+        self._thr = None
+        self.nv = None
+        self.handle = None
+        self.max_mhz = None
+
+    def _open(self):
+        import pynvml as nv
+        nv.nvmlInit()
+        props = torch.cuda.get_device_properties(self.dev)
+        h = None
+        try:
+            bus = "%08X:%02X:%02X.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+            h = nv.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            h = nv.nvmlDeviceGetHandleByIndex(self.dev)
+        self.nv, self.handle = nv, h
+        self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+
+    def _run(self):
+        nv, h = self.nv, self.handle
+        while not self._stop.is_set():
+            try:
+                mhz = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                rs = int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
+                self.samples.append((mhz, rs))
+            except Exception as e:  # noqa: BLE001
+                self.err = str(e)
+                return
+            time.sleep(0.005)
 
     def start(self):
-        fd, self.path = tempfile.mkstemp(prefix="kla_clocks_", suffix=".csv")
-        os.close(fd)
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.Q, "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+            self._open()
+        except Exception as e:  # noqa: BLE001
+            self.err = "NVML unavailable: %s" % e
+            return
+        self._thr = threading.Thread(target=self._run, daemon=True)
+        self._thr.start()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        rows = []
-        for line in open(self.path):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
-            except ValueError:
-                continue
-        os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for _, _, r in rows for i in range(4) if r[i].lower() == "active"})
-        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": reasons, "samples": len(rows)}
+        if self._thr is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.err or "no sampler"], "samples": 0}
+        self._stop.set()
+        self._thr.join(timeout=5)
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [self.err or "no samples"],
+                    "samples": 0}
+        reasons = sorted({name for _, rs in self.samples for name, attr in self.NAMES
+                          if rs & int(getattr(self.nv, attr, 0))})
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "sm_mhz_min": min(m for m, _ in self.samples), "reasons": reasons,
+                "samples": len(self.samples), "source": "NVML, every 5 ms during the timed region"}
 
 
 def rank_seed(w, rank: int) -> int:
@@ -162,77 +198,113 @@ def aggregate(world: int, tokens_per_rank: int, local_ms_total: float, steps: in
     return ms_per_step, world * tokens_per_rank / (ms_per_step * 1e-3)
 
 
-def cpu_baseline(w, inp, target_s=12.0):
-    """The oracle, as it stands, on a bounded sample of (row, head) units."""
+def _units_total(w, inp):
+    return (inp["cu_seqlens"].numel() - 1 if inp["cu_seqlens"] is not None else w.B) * w.H
+
+
+def _unit_tokens(w, inp, n_units):
+    """Tokens (summed over heads, / H) of the first n_units (sequence, head) units."""
+    if inp["cu_seqlens"] is None:
+        return n_units * w.T / w.H
+    cu = inp["cu_seqlens"].tolist()
+    return sum(cu[u // w.H + 1] - cu[u // w.H] for u in range(n_units)) / w.H
+
+
+def sample_units(w, inp, target_s):
+    """How many (sequence, head) units of the workload the oracle computes in
+    about target_s seconds on this host's cores (at least one)."""
     import oracle
-    units_total = (inp["cu_seqlens"].numel() - 1 if inp["cu_seqlens"] is not None else w.B) * w.H
-    t1 = oracle.time_forward(inp, w, (0, 1))
-    per_unit = max(t1, 1e-4)
-    n_units = int(max(1, min(units_total, target_s / per_unit * oracle.max_threads())))
-    reps, t = 0, 0.0
+    t1 = time.perf_counter()
+    oracle.forward_inputs(inp, w, units=(0, 1), want_final=False)
+    per_unit = max(time.perf_counter() - t1, 1e-4)
+    return int(max(1, min(_units_total(w, inp), target_s / per_unit * oracle.max_threads())))
+
+
+def cpu_baseline(w, inp, target_s=12.0):
+    """The oracle, as it stands, on a bounded sample of (row, head) units.
+    Returns the baseline record and the oracle's result on those units."""
+    import oracle
+    n_units = sample_units(w, inp, target_s)
+    reps, t, ref = 0, 0.0, None
     while reps == 0 or t < 2.0:       # repeat a small sample for a stable time
-        t += oracle.time_forward(inp, w, (0, n_units))
+        t0 = time.perf_counter()
+        ref = oracle.forward_inputs(inp, w, units=(0, n_units), want_final=True)
+        t += time.perf_counter() - t0
         reps += 1
     t /= reps
-    if inp["cu_seqlens"] is not None:
-        cu = inp["cu_seqlens"].tolist()
-        tok = sum(cu[u // w.H + 1] - cu[u // w.H] for u in range(n_units)) / w.H
-    else:
-        tok = n_units * w.T / w.H
-    return {"value": tok / t, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
-            "sample": "%d of %d (row, head) units of the workload, fp64 C oracle, %.3f s per pass, %d passes" % (
-                n_units, units_total, t, reps)}
+    rec = {"value": _unit_tokens(w, inp, n_units) / t, "unit": UNIT, "cores": oracle.max_threads(),
+           "kind": "oracle",
+           "sample": "%d of %d (row, head) units of the workload, fp64 C oracle, %.3f s per pass, %d passes" % (
+               n_units, _units_total(w, inp), t, reps)}
+    return rec, ref, n_units
 
 
-def arm_config(w, plan, world):
-    """The workload's `config` object, the same on both arms."""
+def scaled_err(got: torch.Tensor, want: np.ndarray) -> float:
+    """max |got - want| / (1 + |want|), computed in slices to bound host memory."""
+    g = got.reshape(got.shape[0], -1)
+    r = want.reshape(want.shape[0], -1)
+    worst = 0.0
+    step = max(1, (1 << 24) // max(1, g.shape[1]))
+    for s in range(0, g.shape[0], step):
+        gs = g[s:s + step].float().cpu().numpy().astype(np.float64)
+        rs = r[s:s + step]
+        worst = max(worst, float(np.max(np.abs(gs - rs) / (1.0 + np.abs(rs)))) if gs.size else 0.0)
+    return worst
+
+
+def max_err(w, inp, ref, n_units, out, fl, fe):
+    """Scaled error of the GPU results against the oracle on its sampled units."""
+    H = w.H
+    cu = inp["cu_seqlens"].tolist() if inp["cu_seqlens"] is not None else None
+    e_out = e_fl = e_fe = 0.0
+    for u in range(n_units):
+        n, h = divmod(u, H)
+        s, e = (cu[n], cu[n + 1]) if cu else (n * w.T, (n + 1) * w.T)
+        e_out = max(e_out, scaled_err(out[s:e, h], ref["out"][s:e, h]))
+        if fl is not None:
+            e_fl = max(e_fl, scaled_err(fl[n:n + 1, h], ref["final_lambda"][n:n + 1, h]))
+            e_fe = max(e_fe, scaled_err(fe[n:n + 1, h], ref["final_eta"][n:n + 1, h]))
+    res = {"out": e_out, "units": n_units, "tol": TOL[w.dtype],
+           "definition": "max |gpu - oracle| / (1 + |oracle|) over the sampled units"}
+    if fl is not None:
+        res["final_lambda"], res["final_eta"] = e_fl, e_fe
+    return res
+
+
+def arm_config(w, world):
+    """The workload's `config` object, identical on both arms."""
     return {"workload": workload_label(w), "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv,
-            "mode": w.mode, "varlen": w.varlen, "tokens_per_step_per_gpu": w.tokens,
-            "segments_per_row": plan["segments"], "tensor_core_chunk_kernel": plan["tensor_core"],
+            "mode": w.mode, "varlen": w.varlen, "final_state": w.final_state,
+            "tokens_per_step_per_gpu": w.tokens,
             "l2": "flushed between timed steps (512 MiB device write, then 256 MiB read)",
             "parallelism": "dp%d" % world}
 
 
-class _HostOffsets:
-    """Stands in for the packed-sequence offsets when only the plan is asked
-    for: the plan reads the descriptor's shapes, never the offsets."""
-
-    def data_ptr(self):
-        return 256
-
-
-def host_plan(w, num_seqs):
-    mode = kla.KLA_ISO if w.mode == "iso" else kla.KLA_DIAG
-    dt = kla.KLA_BF16 if w.dtype == "bf16" else kla.KLA_FP32
-    desc = kla.make_desc(w.B, w.T, w.H, w.dk, w.dv, dt, mode, _HostOffsets() if w.varlen else None,
-                         num_seqs if w.varlen else 0)
-    return kla.plan(desc)
-
-
 def run_reference(args, w):
-    """Reference arm: the CPU oracle timed on this host's cores."""
+    """Reference arm: the CPU oracle timed on this host's cores. It loads only
+    the oracle, never the CUDA library."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
     import oracle
     inp = make_inputs(w)
-    units_total = (inp["cu_seqlens"].numel() - 1 if inp["cu_seqlens"] is not None else w.B) * w.H
-    per_unit = max(oracle.time_forward(inp, w, (0, 1)), 1e-4)
     budget = 120.0 / max(1, args.steps + args.warmup)
-    n_units = int(max(1, min(units_total, budget / per_unit * oracle.max_threads())))
+    n_units = sample_units(w, inp, budget)
     for _ in range(args.warmup):
-        oracle.time_forward(inp, w, (0, n_units))
-    ts = [oracle.time_forward(inp, w, (0, n_units)) for _ in range(args.steps)]
-    tok = n_units * w.T / w.H if inp["cu_seqlens"] is None else sum(
-        inp["cu_seqlens"][u // w.H + 1].item() - inp["cu_seqlens"][u // w.H].item() for u in range(n_units)) / w.H
+        oracle.forward_inputs(inp, w, units=(0, n_units), want_final=False)
+    ts = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.forward_inputs(inp, w, units=(0, n_units), want_final=False)
+        ts.append(time.perf_counter() - t0)
     t = sum(ts) / len(ts)
-    value = tok / t
-    sample = "%d of %d (row, head) units per step, fp64 C oracle" % (n_units, units_total)
+    value = _unit_tokens(w, inp, n_units) / t
+    sample = "%d of %d (row, head) units per step, fp64 C oracle" % (n_units, _units_total(w, inp))
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": arm_config(w, host_plan(w, units_total // w.H), args.gpus),
+        "config": arm_config(w, args.gpus),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -242,11 +314,11 @@ def run_reference(args, w):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", type=int, default=1, choices=sorted(WORKLOADS))
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--T", type=int, default=None,
                     help="tokens per row instead of the workload's (smaller cases of the same "
@@ -260,6 +332,8 @@ def main():
     if args.impl == "reference":
         run_reference(args, w)
         return
+
+    from bayesian_filter_scan_b200 import kla
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -309,7 +383,6 @@ def main():
 
     steps = args.steps
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(steps)]
-    ev_ptrs = [(ctypes.c_void_p * 7)(*[ctypes.c_void_p(e.cuda_event) for e in row]) for row in evs]
     for row in evs:
         for e in row:
             e.record(stream)   # materialise the events
@@ -340,24 +413,24 @@ def main():
     kla.check()
     barrier()
     torch.cuda.synchronize()
-    clocks = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
+    clocks = ClockSampler(local)
     clocks.start()
-    time.sleep(0.3)
     t_wall = time.perf_counter()
     for i in range(steps):
         step(i)
     torch.cuda.synchronize()
     t_wall = time.perf_counter() - t_wall
-    barrier()
     clk = clocks.stop()
+    barrier()
     kla.check()
     tot = [e0.elapsed_time(e1) for e0, e1 in fwd_ev]         # ms, whole forward
     for i in range(steps):
         step(i, profiled=True)
     torch.cuda.synchronize()
     kla.check()
-    chunk = [r[4].elapsed_time(r[5]) for r in evs]            # ms, the walk kernel
+    walk = [r[4].elapsed_time(r[5]) for r in evs]             # ms, the walk kernel
     pre = [r[0].elapsed_time(r[4]) for r in evs]
+    reduce_ms = statistics.mean(r[0].elapsed_time(r[1]) for r in evs)
     # the launches of this plan, by the event pair that brackets each (an event
     # between every launch; stages without a launch of this plan are left out)
     if plan["tensor_core"] and plan["segments"] > 1:
@@ -400,6 +473,7 @@ def main():
         a1.synchronize()
         e_t += a0.elapsed_time(a1)
     _, e2e_value = aggregate(world, w.tokens, e_t, e2e_steps, dist)
+    del pin, hout, dbuf
     if dist is not None:
         dist.destroy_process_group()
 
@@ -408,8 +482,8 @@ def main():
     peaks, peak_src = measured_peaks()
     units = w.tokens * H
     alg_bytes = bytes_per_token_head(w) * units
-    chunk_ms = statistics.mean(chunk)
-    achieved = alg_bytes / (chunk_ms * 1e-3) / 1e9
+    walk_ms = statistics.mean(walk)
+    achieved = alg_bytes / (walk_ms * 1e-3) / 1e9
     peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
     # the committed DRAM record is of the workload's own size
     traffic = traffic_record(args.workload) if not args.T else None
@@ -417,23 +491,34 @@ def main():
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-        "config": arm_config(w, plan, world),
+        "config": arm_config(w, world),
+        "plan": {"segments_per_row": plan["segments"], "launches_per_step": plan["launches"],
+                 "tensor_core_chunk_kernel": plan["tensor_core"]},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "kernel": walk_label,
-                     "alg_bytes_per_launch": alg_bytes, "launch_ms": chunk_ms,
+                     "alg_bytes_per_launch": alg_bytes, "launch_ms": walk_ms,
+                     "alg_bytes_per_token_head": bytes_per_token_head(w),
                      "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_src},
         "stages_ms": {"note": "separate run with an event between every launch (each adds about 2.6 us)",
-                      "before_walk": statistics.mean(pre), "walk_kernel": chunk_ms,
+                      "before_walk": statistics.mean(pre), "walk_kernel": walk_ms,
                       "total": statistics.mean(r[0].elapsed_time(r[6]) for r in evs), "launches": per_stage},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h_in, "d2h_bytes_per_step": h_out},
         "gpu_launches": steps * plan["launches"],
-        "clocks": {"sm_mhz": clk["sm_mhz"], "sm_max_mhz": clk["sm_max_mhz"], "reasons": clk["reasons"],
-                   "samples": clk.get("samples", 0)},
+        "clocks": clk,
         "timed_region_wall_s": t_wall,
     }
+    if plan["segments"] > 1 and plan["tensor_core"]:
+        sbytes = scan_bytes_per_token_head(w) * units
+        sach = sbytes / (reduce_ms * 1e-3) / 1e9
+        res["roofline_scan"] = {"bound": "hbm", "kernel": "mobius_reduce_tma (precision scan)",
+                                "achieved": sach, "peak": peak, "unit": "GB/s", "frac": sach / peak,
+                                "alg_bytes_per_launch": sbytes, "launch_ms": reduce_ms,
+                                "alg_bytes_per_token_head": scan_bytes_per_token_head(w)}
     if world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(w, inp)
+        rec, ref, n_units = cpu_baseline(w, inp)
+        res["cpu_baseline"] = rec
+        res["max_err"] = max_err(w, inp, ref, n_units, out, fl, fe)
     print(json.dumps(res), flush=True)
 
 
