@@ -3,11 +3,17 @@
 //
 // Launch sequence of kla_forward for B rows of T tokens split into P segments
 // per row (P = 1 when rows x heads already fill the GPU):
-//   P > 1:  mobius_reduce -> mobius_carry        (lambda at every segment start)
-//           walk(state) on segments 0..P-2      (each segment's eta transfer)
-//           state_carry                          (eta at every segment start)
-//   always: walk(output) on every segment        (chunk kernel or SIMT walk)
-// Packed variable-length sequences (cu_seqlens) use P = 1 per sequence.
+//   tensor-core path (bf16, dk and dv in {64, 128}):
+//     P = 1:  chunk kernel walking whole rows                       (1 launch)
+//     P > 1:  mobius_reduce [-> mobius_carry for long segments]      (lambda at
+//             every segment start) -> chunk kernel walking every segment from a
+//             zero state -> segment-start beliefs -> correction pass (4 or 5)
+//   CUDA-core walk (fp32 inputs, other head dims):
+//     P > 1:  mobius_reduce -> mobius_carry -> state walk of segments 0..P-2 ->
+//             state carry -> output walk of every segment               (5)
+//     P = 1:  output walk                                                (1)
+// Packed variable-length sequences (cu_seqlens) are walked whole, longest
+// first (one more launch ranks them by length).
 // Nothing allocates, nothing synchronises; all work goes on the caller's stream.
 #include <cstdlib>
 #include <cstring>
@@ -39,29 +45,31 @@ cudaError_t launch_chunk_tc(const Plan &, const int *, int, const void *, const 
                             const float *, float *, float *, void *, float *, float *, int *,
                             cudaStream_t);
 
+// Device address of the status word, looked up once per device.
 static int *status_ptr() {
-    static int *ptrs[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return nullptr;
-    if (!ptrs[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
-        ptrs[dev] = (int *)p;
+    static PerDevice<int *> ptrs;
+    const int dev = current_device();
+    if (dev < 0) return nullptr;
+    int *p = ptrs.v[dev].load(std::memory_order_acquire);
+    if (!p) {
+        void *a = nullptr;
+        if (cudaGetSymbolAddress(&a, g_status) != cudaSuccess) return nullptr;
+        p = (int *)a;
+        ptrs.v[dev].store(p, std::memory_order_release);
     }
-    return ptrs[dev];
+    return p;
 }
 
 static int sm_count() {
-    static int counts[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return 148;
-    if (!counts[dev]) {
-        int c = 0;
-        if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0)
-            c = 148;
-        counts[dev] = c;
+    static PerDevice<int> counts;
+    const int dev = current_device();
+    if (dev < 0) return 148;
+    int c = counts.v[dev].load(std::memory_order_acquire);
+    if (!c) {
+        if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c <= 0) c = 148;
+        counts.v[dev].store(c, std::memory_order_release);
     }
-    return counts[dev];
+    return c;
 }
 
 static inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -112,8 +120,8 @@ static kla_status make_plan(const kla_desc *d, Plan &p, bool precision_only) {
     } else {
         p.NB = (int)((p.T + kBlockTokens - 1) / kBlockTokens);
         if (p.NB < 1) p.NB = 1;
-        // resident walk CTAs per SM: two for the dk = dv = 64 tensor-core kernel
-        const int per_sm = (p.bf16 && p.dk == 64 && p.dv == 64) ? 2 : 1;
+        // resident walk CTAs per SM (one for every walk kernel)
+        const int per_sm = 1;
         int P = precision_only ? p.NB : choose_segments((long long)p.N * p.H, p.NB, per_sm);
         p.seg_blocks = (p.NB + P - 1) / P;
         p.P = (p.NB + p.seg_blocks - 1) / p.seg_blocks;
@@ -139,7 +147,7 @@ static kla_status make_plan(const kla_desc *d, Plan &p, bool precision_only) {
     p.off_qbuf = off;
     if (p.local) off += align256((size_t)p.ntok * p.H * p.dk * 2);
     p.off_rlog = off;
-    if (p.local) off += align256(units * p.NB * p.dk * sizeof(float));
+    if (p.local) off += align256(units * p.NB * kQuarters * p.dk * sizeof(float));
     p.qbuf = nullptr;
     p.rlog = nullptr;
     // longest-first launch order of packed sequences (list scheduling of the

@@ -7,33 +7,47 @@
 // parallelisable affine map; the forget gate g = a/(a^2 + qn*lambda) comes from
 // precision ratios). It is gated linear attention with
 //     q~ = q / lambda,  k~ = beta * k,  gate g[t,i] = a/(a^2 + qn*lambda_{t-1}).
-// Per chunk of C = 64 tokens with in-chunk cumulative log2-gate G[t,i] and a
-// per-key reference R[i] (midpoint of the chunk's G range, so that neither
-// factor leaves the fp32/bf16 exponent range):
-//     Q'[t,i] = q~[t,i] 2^(G[t,i]-R[i]),   K'[s,i] = k~[s,i] 2^(R[i]-G[s,i])
-//     U       = diag(2^R) eta_chunk_start                     (state, TMEM fp32)
-//     out     = mask_causal(Q' K'^T) V + Q' U                  (tcgen05, TMEM fp32)
-//     eta_chunk_end = diag(2^(G_last-R)) (U + K'^T V)          (tcgen05, TMEM fp32)
+// With G[t,i] the cumulative log2 gate since the segment start and a per-key
+// integer reference rho[i] (the frame of the state):
+//     Q'[t,i] = q~[t,i] 2^(G[t,i]-rho[i]),   K'[s,i] = k~[s,i] 2^(rho[i]-G[s,i])
+//     U       = diag(2^(rho - G_chunk_start)) eta_chunk_start      (state, TMEM fp32)
+//     out     = mask_causal(Q' K'^T) V + Q' U                       (tcgen05, TMEM fp32)
+//     U      += K'^T V                                              (tcgen05, TMEM fp32)
 // The state never leaves the SM while a CTA walks its segment: it lives in
 // TMEM as the accumulator of the K'^T V products (the pages' kernels likewise
 // avoid expanding the state in HBM).
 //
-// CTA = one segment of one (row or packed sequence, head); 320 threads:
-//   warps 0-3  gate: per key, the lambda recursion over the chunk (a, qn stream
-//              through a TMA ring of three 16-token slots), log-gates, then Q'/K' written in
-//              place over the TMA-loaded q/k tiles (bf16, 128B-swizzled), and
-//              the bf16 remainder of K' for a two-term state update, slot by
-//              slot (the gate warps fold every slot themselves);
-//              isotropic mode runs a warp-level Moebius scan over the chunk;
-//   warps 4-7  epilogue: rescale U in TMEM and snapshot it to bf16 shared
-//              memory, mask the score tile into P, store the output rows;
-//   warp 8     TMA producer (q, k, v tiles double-buffered; a, qn ring);
-//   warp 9     TMEM owner and single-thread tcgen05.mma issuer.
+// The reference: every factor 2^(+-(G - rho)) must stay inside the fp32/bf16
+// exponent window. The gate warps compute the chunk's whole precision chain
+// first, so the chunk's actual G range per key is known before any operand is
+// folded. The reference stays where it is while that range fits within
+// kStick of it (then the state needs no rescale); otherwise it moves to the
+// range's midpoint. A chunk whose range spans more than 2 kLim for some key is
+// processed as two passes of 32 tokens or four of 16, each with its own
+// reference per key, the state rescaled between them (strong forgetting inside
+// a chunk). A 16-token quarter spanning more than 2 kLim is outside what the
+// factorised form represents: KLA_ERR_RANGE.
+//
+// CTA = one segment of one (row or packed sequence, head); 448 threads:
+//   warps 0-7   gate. Diagonal precision: thread = (key pair, sub-block of 16
+//               tokens at dk = 128, 8 at dk = 64). Each thread composes its
+//               sub-block's Moebius matrices for its two keys, the matrices
+//               are exchanged through shared memory, each thread walks its
+//               sub-block from the exact start precision and forms the raw
+//               operand factors, the per-key G ranges are exchanged, the
+//               references chosen, and the thread writes Q', K' (bf16 hi) and
+//               the bf16 remainder of K' over the TMA-loaded tiles.
+//               Isotropic precision: warp 0 scans the chunk's 64 Moebius maps
+//               with shuffles; all eight warps fold the rows.
+//   warps 8-11  epilogue: rescale U in TMEM and snapshot it to bf16 shared
+//               memory, mask the score tile into P, store the output rows;
+//   warp 12     TMA producer (q, k, v tiles double-buffered; L2 prefetch of
+//               later chunks, a and qn included);
+//   warp 13     TMEM owner and single-thread tcgen05.mma issuer.
 // mode 0 walks whole rows or packed sequences (from lambda0, eta0); mode 2
 // walks every segment of split rows from a zero state (segment 0 from eta0)
 // and exports what the correction pass needs. The kernel is instantiated per
-// (dk, dv, isotropic or diagonal precision), each variant with only its own
-// gate code.
+// (dk, dv, isotropic or diagonal precision, walk mode).
 //
 // Every wait is bounded: after kWaitLimitNs a waiter sets the abort flag and
 // the library status bit, all roles fall through to the teardown, the
@@ -49,29 +63,28 @@ using namespace ptx;
 
 namespace {
 
-constexpr int kC = 64;             // chunk tokens
-constexpr int kSlotTok = 8;        // tokens per gate slot (one pass of the chain and fold)
-constexpr int kSlotsPerChunk = kC / kSlotTok;
-constexpr int kRingTok = 16;       // tokens per a/qn ring slot (two gate slots per wait)
-constexpr int kRings = 3;          // ring depth (48 tokens of look-ahead)
-constexpr int kRingsPerChunk = kC / kRingTok;
-constexpr int kMaxOffset = 110;    // |G - R| (log2) kept inside the fp32/bf16 exponent range
-constexpr int kRebase = 64;        // diagonal mode: predicted |G - rho| that moves the reference
-// Warp roles. dk = 128: gate warps 0-3, epilogue 4-7, TMA producer 8, MMA 9.
-// dk = 64: gate warps 0 and 2, producer 1, MMA 3, epilogue 4-7 (8 warps, so
-// two CTAs fit on one SM when dv = 64 as well).
+constexpr int kC = 64;        // chunk tokens
+constexpr int kQ = 16;        // tokens per pass quarter
+constexpr int kLim = 80;      // |G - rho| (log2) a pass keeps inside the exponent window
+constexpr int kStick = 48;    // the reference stays while the range fits [rho - kStick, rho + kStick]
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr int kGateBar = 1;   // named barrier of the gate warps
+constexpr int kEpiBar = 2;    // named barrier of the epilogue warps
+
 template <int DK, int DV>
 struct Roles {
-    static constexpr int NGW = (DK == 64) ? 2 : 4;
-    static constexpr int THREADS = (NGW + 6) * 32;
-    static constexpr int MIN_BLOCKS = (DK == 64 && DV == 64) ? 2 : 1;
-    static constexpr int PRODW = (NGW == 2) ? 1 : 8;
-    static constexpr int MMAW = (NGW == 2) ? 3 : 9;
+    static constexpr int NGW = 8;                     // gate warps
+    static constexpr int GT = NGW * 32;               // gate threads
+    static constexpr int EPIW = 8;                    // first epilogue warp (TMEM lane quarter 0)
+    static constexpr int THREADS = 12 * 32;           // 12 warps: up to 168 registers per thread
+    static constexpr int MIN_BLOCKS = 1;
+    // diagonal gate: sub-blocks per chunk and their length
+    static constexpr int NSUB = (DK == 128) ? 4 : 8;
+    static constexpr int SL = kC / NSUB;
 };
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 struct TcArgs {
-    int N, H, P, NB, seg_blocks, iso, mode;
+    int N, H, P, NB, seg_blocks, NC;
     long long T, Lseg;
     const int *cu, *perm;
     const float *a, *qn, *beta;
@@ -81,12 +94,9 @@ struct TcArgs {
     __nv_bfloat16 *out;
     float *final_lambda, *final_eta;
     int *status;
-    // mode 2 (segments from a zero state): per chunk and key, the log2 factor
-    // that takes the folded q' of the chunk to the segment-start frame,
-    // rlog[(u * NC + chunk of the row) * DK + key]; the folded q tiles go to
-    // the tensor map of the q' buffer
+    // mode 2: per chunk, pass quarter and key, the reference rho of the folded
+    // q' (segment-start frame): rlog[((u * NC + chunk of the row) * 4 + quarter) * DK + key]
     float *rlog;
-    int NC;
 };
 
 template <int DK, int DV>
@@ -95,23 +105,27 @@ struct Layout {
     static constexpr int V = kC * DV * 2;
     static constexpr int PT = kC * kC * 2;
     static constexpr int UB = DK * DV * 2;
-    static constexpr int RINGF = kRingTok * DK;   // floats of one of a / qn per ring slot
+    static constexpr int XN = 512;                   // sub-blocks x keys of the diagonal gate (NSUB * DK)
     static constexpr int q0 = 0;
     static constexpr int k0 = q0 + 2 * QK;
     static constexpr int v0 = k0 + 2 * QK;
-    static constexpr int p0 = v0 + 2 * V;
+    static constexpr int klo0 = v0 + 2 * V;          // low bf16 part of K' (state update), per stage
+    static constexpr int p0 = klo0 + 2 * QK;
     static constexpr int ub0 = p0 + PT;
-    static constexpr int klo0 = ub0 + UB;          // low bf16 part of K' (state update), per stage
-    static constexpr int ring0 = klo0 + 2 * QK;
-    static constexpr int fac0 = ring0 + kRings * 2 * RINGF * 4;
-    static constexpr int facf0 = fac0 + 2 * DK * 4;
-    static constexpr int isof0 = facf0 + DK * 4;   // iso: per-token factors (q, beta k) of a chunk
-    static constexpr int bar0 = ((isof0 + kC * 8) + 7) & ~7;
-    static constexpr int NBAR = 6 + 2 * kRings + 9;
+    static constexpr int xch0 = ub0 + UB;            // [NSUB][DK] {float4 matrix, float4 {PA, EM, FM, -}}
+    static constexpr int rng0 = xch0 + XN * 32;      // [NSUB][DK] int2 G range
+    static constexpr int car0 = rng0 + XN * 8;       // [2][DK] chunk-start state {float4 n,d,pa; int4 E,F}
+    static constexpr int fac0 = car0 + 2 * DK * 32;  // [2][4][DK] int: U rescale exponent at each pass quarter
+    static constexpr int facf0 = fac0 + 2 * kQuarters * DK * 4;   // [DK] float: 2^(G_end - rho_end)
+    static constexpr int isof0 = facf0 + DK * 4;     // [2][kC] float2: iso per-token factors
+    static constexpr int lvl0 = isof0 + 2 * kC * 8;  // int[2]: pass level of the chunk, tagged with its index
+    static constexpr int bar0 = lvl0 + 16;
+    static constexpr int NBAR = 8;
     static constexpr int hold0 = bar0 + NBAR * 8;
     static constexpr int bytes = hold0 + 16;
     static constexpr int alloc = bytes + 1024;
     static_assert(alloc <= 232448, "shared memory per CTA");
+    static_assert(Roles<DK, DV>::MIN_BLOCKS == 1 || 2 * (alloc + 1024) <= 233472, "two CTAs per SM");
     static constexpr uint32_t NCOLS = (2 * DV + 64 <= 256) ? 256u : 512u;
     static constexpr uint32_t colU = 0, colO = DV, colS = 2 * DV;
 };
@@ -122,15 +136,27 @@ __device__ __forceinline__ int sw_off(int row, int col, int rows) {
     return (col >> 6) * (rows * 128) + row * 128 + ((((col & 63) >> 3) ^ (row & 7)) << 4) + ((col & 7) << 1);
 }
 
-__device__ __forceinline__ float bf_at(const uint8_t *base, int off) {
-    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(base + off));
-}
-__device__ __forceinline__ void bf_put(uint8_t *base, int off, float x) {
-    *reinterpret_cast<__nv_bfloat16 *>(base + off) = __float2bfloat16_rn(x);
-}
 __device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
+}
+__device__ __forceinline__ float2 unpack_bf2(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+__device__ __forceinline__ float2 f2mul(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 f2fma(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ int expo(float x) { return ((__float_as_int(x) >> 23) & 0xff) - 127; }
+// 2^e for e in [-126, 127]
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
+__device__ __forceinline__ int clampe(int e) { return max(-126, min(126, e)); }
+// R[q] for a runtime q without indexing the array (it stays in registers)
+__device__ __forceinline__ int pick4(const int (&R)[4], int q) {
+    return q == 0 ? R[0] : (q == 1 ? R[1] : (q == 2 ? R[2] : R[3]));
+}
+// x * 2^e for |e| <= 252, exact while the result is a normal float
+__device__ __forceinline__ float scale2(float x, int e) {
+    const int e1 = e / 2;
+    return x * pow2i(e1) * pow2i(e - e1);
 }
 
 __device__ __noinline__ bool wait_slow(uint64_t *bar, uint32_t parity, volatile int *abort_flag, int *status,
@@ -169,10 +195,10 @@ __device__ __forceinline__ float row_sumsq(const uint8_t *ktile, int row) {
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
             uint4 x = *reinterpret_cast<const uint4 *>(ktile + a * kC * 128 + row * 128 + ch * 16);
-            const __nv_bfloat162 *b = reinterpret_cast<const __nv_bfloat162 *>(&x);
+            const uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                float2 f = __bfloat1622float2(b[e]);
+                const float2 f = unpack_bf2(w[e]);
                 s = fmaf(f.x, f.x, s);
                 s = fmaf(f.y, f.y, s);
             }
@@ -181,75 +207,62 @@ __device__ __forceinline__ float row_sumsq(const uint8_t *ktile, int row) {
     return s;
 }
 
-// One 8-token slot (rows 8j .. 8j+7 of the chunk) of the diagonal gate for the
-// key i of this thread. The precision runs in projective form, lambda = n/d:
-//   d <- a^2 d + qn n,   n <- n + b d   (b = beta k^2),   PA <- PA a,
-// two FMAs per token on the serial chain; with G the cumulative log2 gate,
-// 2^G = PA/d and 2^G / lambda = PA/n (n, d, PA carry exponents E, E, F). The
-// slot's operands are then written over the q/k tiles:
-//   K' = beta k 2^(R - G) = beta k (d/PA) mk   (bf16 hi + bf16 remainder)
-//   Q' = q / lambda 2^(G - R) = q (PA/n) mq    (bf16)
-// (mk = 2^(R - (F - E)), mq = 1/mk), packed to bf16 by integer rounding. The
-// chain runs first, then every token's reciprocals and stores, which are
-// independent of one another. Ends with the exact power-of-two rescale.
-// a and qn come from the ring slot ra.
-template <int DK>
-__device__ __forceinline__ void gate_slot(int j, const float *ra, uint8_t *qt, uint8_t *kt, uint8_t *klo,
-                                          const int (&offr)[kSlotTok], float bsrc, bool state_mode, int R,
-                                          float &nn, float &dd, float &pa, int &E, int &F, float &mq, float &mk,
-                                          float &rkmin, float &rkmax) {
-    constexpr int RINGF = kRingTok * DK;    // qn follows a in the ring slot
-    float xa[kSlotTok], xn[kSlotTok], xk[kSlotTok], xq[kSlotTok];
-#pragma unroll
-    for (int r = 0; r < kSlotTok; ++r) {
-        xa[r] = ra[r * DK];
-        xn[r] = ra[RINGF + r * DK];
-        xk[r] = bf_at(kt, j * 1024 + offr[r]);
-        xq[r] = state_mode ? 0.f : bf_at(qt, j * 1024 + offr[r]);
+// ---- reference choice ------------------------------------------------------
+
+__device__ __forceinline__ int2 runion(int2 a, int2 b) { return make_int2(min(a.x, b.x), max(a.y, b.y)); }
+__device__ __forceinline__ int rspan(int2 a) { return a.y - a.x; }
+__device__ __forceinline__ bool rfits(int2 a, int r) { return a.x >= r - kStick && a.y <= r + kStick; }
+__device__ __forceinline__ int rmid(int2 a) { return (a.x + a.y) >> 1; }
+
+// The references of one key for the four pass quarters of a chunk, from the
+// integer bounds qr[q] of G over each quarter (including the value just before
+// it) and the reference rho in force: level 0 = one pass (span <= 2 kLim),
+// 1 = two passes of 32 tokens, 2 = four passes of 16. `bad` when a quarter's
+// own span exceeds the window.
+__device__ __forceinline__ int choose_refs(const int2 (&qr)[4], int rho, int (&R)[4], bool &bad) {
+    const int2 h0 = runion(qr[0], qr[1]), h1 = runion(qr[2], qr[3]);
+    const int2 all = runion(h0, h1);
+    bad = false;
+    if (rspan(all) <= 2 * kLim) {
+        const int r = rfits(all, rho) ? rho : rmid(all);
+        R[0] = R[1] = R[2] = R[3] = r;
+        return 0;
     }
-    float bk[kSlotTok], nt[kSlotTok], pt[kSlotTok], dt[kSlotTok];
-#pragma unroll
-    for (int r = 0; r < kSlotTok; ++r) bk[r] = __shfl_sync(0xffffffffu, bsrc, (kSlotTok * j + r) & 31) * xk[r];
-#pragma unroll
-    for (int r = 0; r < kSlotTok; ++r) {
-        const float at = xa[r];
-        dd = fmaf(at * at, dd, xn[r] * nn);
-        nn = fmaf(bk[r] * xk[r], dd, nn);
-        pa *= at;
-        nt[r] = nn;
-        pt[r] = pa;
-        dt[r] = dd;
+    if (rspan(h0) <= 2 * kLim && rspan(h1) <= 2 * kLim) {
+        const int ra = rfits(h0, rho) ? rho : rmid(h0);
+        const int rb = rfits(h1, ra) ? ra : rmid(h1);
+        R[0] = R[1] = ra;
+        R[2] = R[3] = rb;
+        return 1;
     }
+    int prev = rho;
 #pragma unroll
-    for (int r = 0; r < kSlotTok; ++r) {
-        const float rkm = (dt[r] * mk) * rcp_approx(pt[r]);      // 2^(R - G)
-        rkmin = fminf(rkmin, rkm);
-        rkmax = fmaxf(rkmax, rkm);
-        const float ko = bk[r] * rkm;
-        const uint32_t t = __float_as_uint(ko) + 0x8000u;         // K' hi, rounded
-        const int off = j * 1024 + offr[r];
-        *reinterpret_cast<uint16_t *>(kt + off) = (uint16_t)(t >> 16);
-        *reinterpret_cast<uint16_t *>(klo + off) =
-            (uint16_t)(__float_as_uint(ko - __uint_as_float(t & 0xffff0000u)) >> 16);
+    for (int q = 0; q < 4; ++q) {
+        R[q] = rfits(qr[q], prev) ? prev : rmid(qr[q]);
+        prev = R[q];
+        bad |= rspan(qr[q]) > 2 * kLim;
     }
-    if (!state_mode) {
-#pragma unroll
-        for (int r = 0; r < kSlotTok; ++r) {
-            const float qo = xq[r] * ((pt[r] * mq) * rcp_approx(nt[r]));
-            *reinterpret_cast<uint16_t *>(qt + j * 1024 + offr[r]) = (uint16_t)((__float_as_uint(qo) + 0x8000u) >> 16);
-        }
-    }
-    const int e = ((__float_as_int(dd) >> 23) & 0xff) - 127;
-    const int f = ((__float_as_int(pa) >> 23) & 0xff) - 127;
-    const float se = __int_as_float((127 - e) << 23);
-    nn *= se;
-    dd *= se;
-    pa *= __int_as_float((127 - f) << 23);
+    return 2;
+}
+
+// Normalises a 2x2 map (two columns) of one key by the power of two of its
+// largest entry; the exponent goes to `e`.
+__device__ __forceinline__ void norm_cols(float &n1, float &n2, float &d1, float &d2, int &e) {
+    const int x = clampe(expo(fmaxf(fmaxf(n1, n2), fmaxf(d1, d2))));
+    const float s = pow2i(-x);
+    n1 *= s; n2 *= s; d1 *= s; d2 *= s;
+    e += x;
+}
+// Normalises the projective precision (n, d) by the power of two of d and the
+// gate product pa by its own.
+__device__ __forceinline__ void norm_state(float &n, float &d, float &pa, int &E, int &F) {
+    const int e = clampe(expo(d)), f = clampe(expo(pa));
+    const float se = pow2i(-e);
+    n *= se;
+    d *= se;
+    pa *= pow2i(-f);
     E += e;
     F += f;
-    const int sh = max(-126, min(127, (F - E) - R));
-    mq = __int_as_float((127 + sh) << 23);
-    mk = __int_as_float((127 - sh) << 23);
 }
 
 }  // namespace
@@ -267,69 +280,44 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // on the shared array so that every tile access stays a shared-space access
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::bar0);
-    uint64_t *stage_full = bars + 0, *stage_empty = bars + 2, *qk_ready = bars + 4;
-    uint64_t *ring_full = bars + 6, *ring_empty = bars + 6 + kRings;
-    uint64_t *s_full = bars + 6 + 2 * kRings, *u_ready = s_full + 1, *u_done = s_full + 2, *p_full = s_full + 3;
-    uint64_t *o_full = s_full + 4, *o_empty = s_full + 5, *td_bar = s_full + 6, *gate_sync = s_full + 7;
-    uint64_t *gate_sync2 = s_full + 8;   // iso: the chunk's per-token factors are in shared memory
+    uint64_t *stage_full = bars + 0, *qk_ready = bars + 2;
+    uint64_t *s_full = bars + 4, *u_done = bars + 5, *o_full = bars + 6, *td_bar = bars + 7;
     uint32_t *tmem_hold = reinterpret_cast<uint32_t *>(sm + L::hold0);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::hold0 + 4);
-    float *fac = reinterpret_cast<float *>(sm + L::fac0);
-    float *fac_final = reinterpret_cast<float *>(sm + L::facf0);
-    float2 *isof = reinterpret_cast<float2 *>(sm + L::isof0);
+    int *lvl = reinterpret_cast<int *>(sm + L::lvl0);
+    int *facd = reinterpret_cast<int *>(sm + L::fac0);
+    float *facf = reinterpret_cast<float *>(sm + L::facf0);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // the transfer-only pass (mode 1) runs on the CUDA-core walk; this kernel
-    // takes modes 0 and 2 and is instantiated per precision mode (ISO) and walk
-    // mode (LOCAL), so that each variant holds only its own code
-    constexpr bool state_mode = false;
-    // mode 2: every segment walks from a zero state (segment 0 from eta0), writes
-    // its transfer and decay, and segments p > 0 export their folded q tiles and
-    // chunk references for the correction pass that adds the carried state
-    constexpr bool local_mode = LOCAL;
-    // one gate thread per key: each reads and rewrites only its own key column
-    const int gate_threads = DK;
-    const bool is_gate = (RL::NGW == 4) ? (warp < 4) : (warp == 0 || warp == 2);
-    const int gt = (RL::NGW == 4) ? tid : ((warp >> 1) * 32 + lane);   // gate rank
 
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(&stage_full[s], 1);
-            mbar_init(&stage_empty[s], 1);
-            mbar_init(&qk_ready[s], gate_threads);
-        }
-        for (int j = 0; j < kRings; ++j) {
-            mbar_init(&ring_full[j], 1);
-            mbar_init(&ring_empty[j], gate_threads);
+            mbar_init(&qk_ready[s], RL::GT);
+            lvl[s] = -1;
         }
         mbar_init(s_full, 1);
-        mbar_init(u_ready, 128);
         mbar_init(u_done, 1);
-        mbar_init(p_full, 128);
         mbar_init(o_full, 1);
-        mbar_init(o_empty, 128);
         mbar_init(td_bar, 1);
-        mbar_init(gate_sync, gate_threads);
-        mbar_init(gate_sync2, gate_threads);
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == RL::PRODW && lane == 0) {
+    if (warp == RL::EPIW && lane == 0) {
         prefetch_map(&tm_q); prefetch_map(&tm_k); prefetch_map(&tm_v);
         if (!ISO) { prefetch_map(&tm_a); prefetch_map(&tm_qn); }
     }
-    if (warp == RL::MMAW) tmem_alloc(tmem_hold, L::NCOLS);
+    if (warp == RL::EPIW) tmem_alloc(tmem_hold, L::NCOLS);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = *tmem_hold;
     pdl_release();
     pdl_wait();
-    const int P_eff = state_mode ? g.P - 1 : g.P;
     // unit u = (row or packed sequence n, head h); packed sequences in the
     // longest-first order when one is given
-    const long long ur = blockIdx.x / P_eff;
-    const int p = (int)(blockIdx.x % P_eff);
+    const long long ur = blockIdx.x / g.P;
+    const int p = (int)(blockIdx.x % g.P);
     const int h = (int)(ur % g.H);
     const int n = g.perm ? g.perm[ur / g.H] : (int)(ur / g.H);
     const long long u = (long long)n * g.H + h;
@@ -340,491 +328,691 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         te = (long long)n * g.T + min((long long)(p + 1) * g.Lseg, g.T);
     }
     const int nchunks = te > tb ? (int)((te - tb + kC - 1) / kC) : 0;
-    const bool last_seg = p == P_eff - 1;
+    const bool last_seg = p == g.P - 1;
+    // chunk index of the row (for the exported references)
+    const long long chunk_base = (long long)p * g.seg_blocks;
 
-    if (is_gate) {
-      {
+    // precision at the segment start, key i (iso: i = 0)
+    auto seg_lambda = [&](int i) -> float {
+        const int nl = ISO ? 1 : DK;
+        float lam = g.lambda0 ? g.lambda0[u * nl + i] : 1.0f;
+        if (p > 0 && g.agg) {
+            // compose the Moebius aggregates of the blocks before this segment
+            // (in order) and apply them to lambda0
+            const float4 *src = g.agg + u * g.NB * nl + i;
+            const int nb = p * g.seg_blocks;
+            Mob M{1.f, 0.f, 0.f, 1.f};
+            for (int b0 = 0; b0 < nb; b0 += 8) {
+                float4 m[8];
+#pragma unroll
+                for (int r = 0; r < 8; ++r)
+                    if (b0 + r < nb) m[r] = __ldg(src + (long long)(b0 + r) * nl);
+#pragma unroll
+                for (int r = 0; r < 8; ++r)
+                    if (b0 + r < nb) M = mob_norm(mob_mul(Mob{m[r].x, m[r].y, m[r].z, m[r].w}, M));
+            }
+            lam = mob_apply(M, lam);
+        } else if (p > 0) {
+            lam = g.lam_blk[(u * g.NB + (long long)p * g.seg_blocks) * nl + i];
+        }
+        return lam;
+    };
+
+    if (warp < RL::NGW) {
         // ================= gate warps: precision path and operand folding =====
-        const int i = gt;                    // key owned by this thread
-        const bool key = true;
-        // byte offset of (row r of an 8-row group, key i) in a 64-row 128B-swizzled
-        // tile; row 8j + r of the chunk is at j * 1024 + offr[r]
-        int offr[kSlotTok];
-#pragma unroll
-        for (int r = 0; r < kSlotTok; ++r) offr[r] = sw_off(r, i, kC);
-        float lam = 1.0f;
-        {
-            const int il = ISO ? 0 : i;
-            if (key || ISO) {
-                const int nl = ISO ? 1 : DK;
-                lam = g.lambda0 ? g.lambda0[u * nl + il] : 1.0f;
-                if (p > 0 && g.agg) {
-                    // compose the Moebius aggregates of the blocks before this segment
-                    // (in order) and apply them to lambda0
-                    const float4 *src = g.agg + u * g.NB * nl + il;
-                    const int nb = p * g.seg_blocks;
-                    Mob M{1.f, 0.f, 0.f, 1.f};
-                    for (int b0 = 0; b0 < nb; b0 += 16) {
-                        float4 m[16];
-#pragma unroll
-                        for (int r = 0; r < 16; ++r)
-                            if (b0 + r < nb) m[r] = __ldg(src + (long long)(b0 + r) * nl);
-#pragma unroll
-                        for (int r = 0; r < 16; ++r)
-                            if (b0 + r < nb) M = mob_norm(mob_mul(Mob{m[r].x, m[r].y, m[r].z, m[r].w}, M));
-                    }
-                    lam = mob_apply(M, lam);
-                } else if (p > 0) {
-                    lam = g.lam_blk[(u * g.NB + (long long)p * g.seg_blocks) * nl + il];
+        bool ok = true;
+        if constexpr (!ISO) {
+            constexpr int NSUB = RL::NSUB, SL = RL::SL;
+            float4 *xch = reinterpret_cast<float4 *>(sm + L::xch0);   // [(s*DK + i)*2 + {0,1}]
+            int2 *rng = reinterpret_cast<int2 *>(sm + L::rng0);        // [s*DK + i]
+            float4 *carf = reinterpret_cast<float4 *>(sm + L::car0);   // [(par*DK + i)*2]
+            int4 *cari = reinterpret_cast<int4 *>(sm + L::car0);       // [(par*DK + i)*2 + 1]
+            const int s = (DK == 128) ? (warp >> 1) : warp;           // sub-block
+            const int i0 = 2 * ((DK == 128) ? ((warp & 1) * 32 + lane) : lane);   // first key of the pair
+            const int quarter = (SL * s) / kQ;                        // pass quarter of this sub-block
+            // byte offset of (row SL*s + r, keys i0, i0+1) in a swizzled tile: the
+            // sub-block starts on a multiple of 8 rows, so row & 7 = r & 7
+            const int obase = (i0 >> 6) * (kC * 128) + (SL * s) * 128 + ((i0 & 7) << 1);
+            const int ochunk = ((i0 & 63) >> 3) << 4;
+            auto offr = [&](int r) { return obase + r * 128 + ((ochunk ^ ((r & 7) << 4)) & 0x70); };
+            if (s == 0) {
+                // the belief at the segment start, as the first chunk's start state
+                for (int j = 0; j < 2; ++j) {
+                    carf[(0 * DK + i0 + j) * 2] = make_float4(seg_lambda(i0 + j), 1.f, 1.f, 0.f);
+                    cari[(0 * DK + i0 + j) * 2 + 1] = make_int4(0, 0, 0, 0);
                 }
             }
-        }
-        float e_prev = 1.f, log_decay = 0.f;   // e_prev = 2^(G_last - R) of the previous chunk
-        bool ok = true;
-        // Diagonal mode keeps the precision chain and the log-gate reference across
-        // chunks: G is the cumulative log2 gate since the segment start, rho a
-        // per-key integer reference that moves only when the next chunk's predicted
-        // G range would leave [rho - kRebase, rho + kRebase]. The state in TMEM is
-        // U = diag(2^(rho - G)) eta, so it needs no rescale while rho stays put.
-        float nn = lam, dd = 1.0f, pa = 1.0f;
-        int E = 0, F = 0, rho = 0, dpred = 0;
-        float gprev = 0.f;
-        // Per-token scalars of a chunk are loaded one chunk ahead into registers
-        // and broadcast with shuffles (no global load sits on the recursion).
-        // diag: beta of tokens (lane, lane+32); iso: a, qn, beta of (2 lane, 2 lane+1).
-        float nb0 = 0.f, nb1 = 0.f, na0 = 1.f, na1 = 1.f, nq0 = 0.f, nq1 = 0.f;
-        auto prefetch = [&](int c) {
-            const long long t0 = tb + (long long)c * kC;
-            const long long x0 = ISO ? t0 + 2 * lane : t0 + lane;
-            const long long x1 = ISO ? x0 + 1 : t0 + 32 + lane;
-            nb0 = x0 < te ? __ldg(g.beta + x0 * g.H + h) : 0.f;
-            nb1 = x1 < te ? __ldg(g.beta + x1 * g.H + h) : 0.f;
-            if (ISO) {
+            int rho0 = 0, rho1 = 0;          // references in force (segment-start frame)
+            float2 av[SL], qv[SL];           // a, qn of the sub-block
+            float bl = 0.f;                  // beta of token SL*s + lane (lanes < SL)
+            auto load_tok = [&](int c, int r) {
+                const long long tok = tb + (long long)c * kC + SL * s + r;
+                if (tok < te) {
+                    const long long off = (tok * g.H + h) * DK + i0;
+                    av[r] = __ldg(reinterpret_cast<const float2 *>(g.a + off));
+                    qv[r] = __ldg(reinterpret_cast<const float2 *>(g.qn + off));
+                } else {
+                    av[r] = make_float2(1.f, 1.f);
+                    qv[r] = make_float2(0.f, 0.f);
+                }
+            };
+            auto load_beta = [&](int c) {
+                const long long tok = tb + (long long)c * kC + SL * s + lane;
+                bl = (lane < SL && tok < te) ? __ldg(g.beta + tok * g.H + h) : 0.f;
+            };
+            if (nchunks > 0) {
+#pragma unroll
+                for (int r = 0; r < SL; ++r) load_tok(0, r);
+                load_beta(0);
+            }
+            float lam_end0 = 0.f, lam_end1 = 0.f, gend0 = 1.f, gend1 = 1.f;
+            int xend0 = 0, xend1 = 0;
+            for (int c = 0; c < nchunks; ++c) {
+                const int st = c & 1;
+                const long long tok0 = tb + (long long)c * kC;
+                uint8_t *qt = sm + L::q0 + st * L::QK;
+                uint8_t *kt = sm + L::k0 + st * L::QK;
+                uint8_t *klo = sm + L::klo0 + st * L::QK;
+                const bool okw = waitw(&stage_full[st], (c >> 1) & 1, abort_flag, g.status);
+                // ---- step 1: the sub-block's Moebius maps for both keys (columns
+                // are the images of (1, 0) and (0, 1); chain d <- a^2 d + qn n,
+                // n <- n + b d with b = beta k^2), and its product of a
+                float2 n1 = make_float2(1.f, 1.f), d1 = make_float2(0.f, 0.f);
+                float2 n2 = make_float2(0.f, 0.f), d2 = make_float2(1.f, 1.f), PA = make_float2(1.f, 1.f);
+                int em0 = 0, em1 = 0, fm0 = 0, fm1 = 0;
+                if (okw) {
+#pragma unroll
+                    for (int r = 0; r < SL; ++r) {
+                        const float2 kf = unpack_bf2(*reinterpret_cast<const uint32_t *>(kt + offr(r)));
+                        const float be = __shfl_sync(0xffffffffu, bl, r);
+                        const float2 a2 = f2mul(av[r], av[r]);
+                        const float2 b = f2mul(f2mul(make_float2(be, be), kf), kf);
+                        d1 = f2fma(a2, d1, f2mul(qv[r], n1));
+                        n1 = f2fma(b, d1, n1);
+                        d2 = f2fma(a2, d2, f2mul(qv[r], n2));
+                        n2 = f2fma(b, d2, n2);
+                        PA = f2mul(PA, av[r]);
+                        if ((r & 7) == 7) {
+                            norm_cols(n1.x, n2.x, d1.x, d2.x, em0);
+                            norm_cols(n1.y, n2.y, d1.y, d2.y, em1);
+                            const int f0 = clampe(expo(PA.x)), f1 = clampe(expo(PA.y));
+                            PA.x *= pow2i(-f0); PA.y *= pow2i(-f1);
+                            fm0 += f0; fm1 += f1;
+                        }
+                    }
+                    xch[(s * DK + i0) * 2] = make_float4(n1.x, n2.x, d1.x, d2.x);
+                    xch[(s * DK + i0) * 2 + 1] = make_float4(PA.x, __int_as_float(em0), __int_as_float(fm0), 0.f);
+                    xch[(s * DK + i0 + 1) * 2] = make_float4(n1.y, n2.y, d1.y, d2.y);
+                    xch[(s * DK + i0 + 1) * 2 + 1] = make_float4(PA.y, __int_as_float(em1), __int_as_float(fm1), 0.f);
+                }
+                if (named_bar_or(kGateBar, RL::GT, !okw || *abort_flag)) { ok = false; break; }
+                // ---- step 2: the state at this sub-block's start: the chunk-start
+                // state with the maps of the sub-blocks before it applied
+                float nn[2], dd[2], pa[2];
+                int E[2], F[2];
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const float4 cf = carf[(st * DK + i0 + j) * 2];
+                    const int4 ci = cari[(st * DK + i0 + j) * 2 + 1];
+                    nn[j] = cf.x; dd[j] = cf.y; pa[j] = cf.z; E[j] = ci.x; F[j] = ci.y;
+                    for (int sj = 0; sj < s; ++sj) {
+                        const float4 m = xch[(sj * DK + i0 + j) * 2];
+                        const float4 x = xch[(sj * DK + i0 + j) * 2 + 1];
+                        const float n2v = fmaf(m.x, nn[j], m.y * dd[j]);
+                        const float d2v = fmaf(m.z, nn[j], m.w * dd[j]);
+                        nn[j] = n2v;
+                        dd[j] = d2v;
+                        pa[j] *= x.x;
+                        E[j] += __float_as_int(x.y);
+                        F[j] += __float_as_int(x.z);
+                        norm_state(nn[j], dd[j], pa[j], E[j], F[j]);
+                    }
+                }
+                // ---- step 3: walk the sub-block for its G range (projective
+                // precision and gate product only); the last sub-block's end state
+                // starts the next chunk
+                const float2 n2s0 = make_float2(nn[0], nn[1]), d2s0 = make_float2(dd[0], dd[1]);
+                const float2 p2s0 = make_float2(pa[0], pa[1]);
+                const int E00 = E[0], E01 = E[1], F00 = F[0], F01 = F[1];
+                int2 glo, ghi;
+                {
+                    float2 n2s = n2s0, d2s = d2s0, p2s = p2s0;
+                    // G just before the sub-block: (F - E) - log2(d/pa)
+                    int2 ge = make_int2(F[0] - E[0], F[1] - E[1]);
+                    const float r0 = dd[0] / pa[0], r1 = dd[1] / pa[1];
+                    glo = make_int2(ge.x - expo(r0) - 1, ge.y - expo(r1) - 1);
+                    ghi = make_int2(ge.x - expo(r0), ge.y - expo(r1));
+                    float2 rkmin = make_float2(3.0e38f, 3.0e38f), rkmax = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int r = 0; r < SL; ++r) {
+                        const float2 kf = unpack_bf2(*reinterpret_cast<const uint32_t *>(kt + offr(r)));
+                        const float be = __shfl_sync(0xffffffffu, bl, r);
+                        const float2 b = f2mul(f2mul(make_float2(be, be), kf), kf);
+                        d2s = f2fma(f2mul(av[r], av[r]), d2s, f2mul(qv[r], n2s));
+                        n2s = f2fma(b, d2s, n2s);
+                        p2s = f2mul(p2s, av[r]);
+                        const float2 rk = make_float2(__fdividef(d2s.x, p2s.x), __fdividef(d2s.y, p2s.y));
+                        rkmin = make_float2(fminf(rkmin.x, rk.x), fminf(rkmin.y, rk.y));
+                        rkmax = make_float2(fmaxf(rkmax.x, rk.x), fmaxf(rkmax.y, rk.y));
+                        if ((r & 7) == 7) {
+                            glo = make_int2(min(glo.x, ge.x - expo(rkmax.x) - 1), min(glo.y, ge.y - expo(rkmax.y) - 1));
+                            ghi = make_int2(max(ghi.x, ge.x - expo(rkmin.x)), max(ghi.y, ge.y - expo(rkmin.y)));
+                            rkmin = make_float2(3.0e38f, 3.0e38f);
+                            rkmax = make_float2(0.f, 0.f);
+                            norm_state(n2s.x, d2s.x, p2s.x, E[0], F[0]);
+                            norm_state(n2s.y, d2s.y, p2s.y, E[1], F[1]);
+                            ge = make_int2(F[0] - E[0], F[1] - E[1]);
+                        }
+                    }
+                    if (s == NSUB - 1) {
+                        // the chunk-end state starts the next chunk
+                        const int nst = (c + 1) & 1;
+                        carf[(nst * DK + i0) * 2] = make_float4(n2s.x, d2s.x, p2s.x, 0.f);
+                        cari[(nst * DK + i0) * 2 + 1] = make_int4(E[0], F[0], 0, 0);
+                        carf[(nst * DK + i0 + 1) * 2] = make_float4(n2s.y, d2s.y, p2s.y, 0.f);
+                        cari[(nst * DK + i0 + 1) * 2 + 1] = make_int4(E[1], F[1], 0, 0);
+                        if (c == nchunks - 1) {
+                            // final outputs of the segment (the references follow in step 4)
+                            lam_end0 = n2s.x / d2s.x;
+                            lam_end1 = n2s.y / d2s.y;
+                            gend0 = p2s.x / d2s.x;
+                            gend1 = p2s.y / d2s.y;
+                            xend0 = F[0] - E[0];
+                            xend1 = F[1] - E[1];
+                        }
+                    }
+                }
+                rng[s * DK + i0] = make_int2(glo.x, ghi.x);
+                rng[s * DK + i0 + 1] = make_int2(glo.y, ghi.y);
+                if (named_bar_or(kGateBar, RL::GT, *abort_flag != 0)) { ok = false; break; }
+                // ---- step 4: references of the pass quarters, from the G ranges
+                // of every sub-block of the chunk
+                int R0[4], R1[4];
+                int lv;
+                bool bad0, bad1;
+                {
+                    int2 qa[4], qb[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        constexpr int per = NSUB / 4;
+                        int2 ra = rng[(q * per) * DK + i0], rb = rng[(q * per) * DK + i0 + 1];
+#pragma unroll
+                        for (int x = 1; x < per; ++x) {
+                            ra = runion(ra, rng[(q * per + x) * DK + i0]);
+                            rb = runion(rb, rng[(q * per + x) * DK + i0 + 1]);
+                        }
+                        qa[q] = ra;
+                        qb[q] = rb;
+                    }
+                    const int l0 = choose_refs(qa, rho0, R0, bad0);
+                    const int l1 = choose_refs(qb, rho1, R1, bad1);
+                    lv = max(l0, l1);
+                }
+                if (s == 0) {
+                    atomicMax(&lvl[st], (c << 2) | lv);
+                    if (bad0 || bad1) atomicOr(g.status, kStatusRange);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        facd[(st * 4 + q) * DK + i0] = R0[q] - (q ? R0[q - 1] : rho0);
+                        facd[(st * 4 + q) * DK + i0 + 1] = R1[q] - (q ? R1[q - 1] : rho1);
+                    }
+                    if (LOCAL && p > 0) {
+                        float *rl = g.rlog + ((u * g.NC + chunk_base + c) * 4) * DK + i0;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            *reinterpret_cast<float2 *>(rl + q * DK) = make_float2((float)R0[q], (float)R1[q]);
+                    }
+                }
+                rho0 = R0[3];
+                rho1 = R1[3];
+                if (c == nchunks - 1 && s == NSUB - 1) {
+                    // final outputs of the segment: 2^(G_end - rho) for the state
+                    // export, the precision, and the segment's gate product
+                    facf[i0] = scale2(gend0, xend0 - rho0);
+                    facf[i0 + 1] = scale2(gend1, xend1 - rho1);
+                    if (LOCAL) {
+                        auto prod = [](float gm, int x) {
+                            return x < -250 ? 0.f : (x > 250 ? __int_as_float(0x7f800000) : scale2(gm, x));
+                        };
+                        g.decay[(u * g.P + p) * DK + i0] = prod(gend0, xend0);
+                        g.decay[(u * g.P + p) * DK + i0 + 1] = prod(gend1, xend1);
+                    }
+                    if (last_seg && g.final_lambda) {
+                        g.final_lambda[u * DK + i0] = lam_end0;
+                        g.final_lambda[u * DK + i0 + 1] = lam_end1;
+                    }
+                }
+                // ---- step 5: walk the sub-block again and fold each token:
+                //   Q' = q/lambda 2^(G - R) = q pa/n 2^((F-E) - R)
+                //   K' = beta k 2^(R - G)   = beta k d/pa 2^(R - (F-E))
+                // then load the next chunk's a, qn into the freed registers
+                {
+                    const int ra = pick4(R0, quarter), rb = pick4(R1, quarter);
+                    float2 n2s = n2s0, d2s = d2s0, p2s = p2s0;
+                    int e0 = clampe(F00 - E00 - ra), e1 = clampe(F01 - E01 - rb);
+                    int Ew0 = E00, Ew1 = E01, Fw0 = F00, Fw1 = F01;
+                    float2 mq = make_float2(pow2i(e0), pow2i(e1)), mk = make_float2(pow2i(-e0), pow2i(-e1));
+#pragma unroll
+                    for (int r = 0; r < SL; ++r) {
+                        const uint32_t kw = *reinterpret_cast<const uint32_t *>(kt + offr(r));
+                        const uint32_t qw = *reinterpret_cast<const uint32_t *>(qt + offr(r));
+                        const bool valid = tok0 + SL * s + r < te;
+                        const float2 kf = unpack_bf2(kw);
+                        const float2 qf = valid ? unpack_bf2(qw) : make_float2(0.f, 0.f);
+                        const float be = __shfl_sync(0xffffffffu, bl, r);
+                        const float2 bk = f2mul(make_float2(be, be), kf);
+                        d2s = f2fma(f2mul(av[r], av[r]), d2s, f2mul(qv[r], n2s));
+                        n2s = f2fma(f2mul(bk, kf), d2s, n2s);
+                        p2s = f2mul(p2s, av[r]);
+                        const float2 pn = f2mul(p2s, n2s);
+                        const float2 rc = make_float2(rcp_approx(pn.x), rcp_approx(pn.y));
+                        const float2 qo = f2mul(f2mul(f2mul(qf, p2s), f2mul(p2s, rc)), mq);     // q pa/n
+                        const float2 ko = f2mul(f2mul(bk, f2mul(d2s, f2mul(n2s, rc))), mk);    // beta k d/pa
+                        const uint32_t kh = pack_bf2(ko.x, ko.y);
+                        const float2 khf = unpack_bf2(kh);
+                        *reinterpret_cast<uint32_t *>(qt + offr(r)) = pack_bf2(qo.x, qo.y);
+                        *reinterpret_cast<uint32_t *>(kt + offr(r)) = kh;
+                        *reinterpret_cast<uint32_t *>(klo + offr(r)) = pack_bf2(ko.x - khf.x, ko.y - khf.y);
+                        if (c + 1 < nchunks) load_tok(c + 1, r);
+                        if ((r & 7) == 7 && r + 1 < SL) {
+                            norm_state(n2s.x, d2s.x, p2s.x, Ew0, Fw0);
+                            norm_state(n2s.y, d2s.y, p2s.y, Ew1, Fw1);
+                            e0 = clampe(Fw0 - Ew0 - ra);
+                            e1 = clampe(Fw1 - Ew1 - rb);
+                            mq = make_float2(pow2i(e0), pow2i(e1));
+                            mk = make_float2(pow2i(-e0), pow2i(-e1));
+                        }
+                    }
+                }
+                if (c + 1 < nchunks) load_beta(c + 1);
+                fence_proxy_async();
+                mbar_arrive(&qk_ready[st]);
+            }
+            if (nchunks == 0 && s == 0 && last_seg && g.final_lambda) {
+                g.final_lambda[u * DK + i0] = carf[i0 * 2].x;
+                g.final_lambda[u * DK + i0 + 1] = carf[(i0 + 1) * 2].x;
+            }
+        } else {
+            // ---- isotropic: one precision per head ---------------------------
+            float2 *isof = reinterpret_cast<float2 *>(sm + L::isof0);
+            float lam = 0.f, D = 0.f, Gc = 0.f;   // warp 0: precision, G - rho and G at the chunk start
+            // per-token scalars of a chunk, loaded one chunk ahead (lane: tokens 2 lane, 2 lane + 1)
+            float nb0 = 0.f, nb1 = 0.f, na0 = 1.f, na1 = 1.f, nq0 = 0.f, nq1 = 0.f;
+            auto prefetch = [&](int c) {
+                const long long x0 = tb + (long long)c * kC + 2 * lane, x1 = x0 + 1;
+                nb0 = x0 < te ? __ldg(g.beta + x0 * g.H + h) : 0.f;
+                nb1 = x1 < te ? __ldg(g.beta + x1 * g.H + h) : 0.f;
                 na0 = x0 < te ? __ldg(g.a + x0 * g.H + h) : 1.f;
                 na1 = x1 < te ? __ldg(g.a + x1 * g.H + h) : 1.f;
                 nq0 = x0 < te ? __ldg(g.qn + x0 * g.H + h) : 0.f;
                 nq1 = x1 < te ? __ldg(g.qn + x1 * g.H + h) : 0.f;
+            };
+            if (warp == 0) {
+                lam = seg_lambda(0);
+                if (nchunks > 0) prefetch(0);
             }
-        };
-        if (nchunks > 0) prefetch(0);
-        for (int c = 0; c < nchunks && ok; ++c) {
-            const int s = c & 1;
-            const long long tok0 = tb + (long long)c * kC;
-            uint8_t *qt = sm + L::q0 + s * L::QK;
-            uint8_t *kt = sm + L::k0 + s * L::QK;
-            const float cb0 = nb0, cb1 = nb1, ca0 = na0, ca1 = na1, cq0 = nq0, cq1 = nq1;
-            if (c + 1 < nchunks) prefetch(c + 1);
-            if (!waitw(&stage_full[s], (c >> 1) & 1, abort_flag, g.status)) { ok = false; break; }
-            int R;                 // integer log2 reference of this chunk (per key)
-            float fac_c = 1.f;     // diagonal mode: rescale of U at this chunk's start
-            float e_cur;           // 2^(G_last - R)
-            float glast_log2;      // G_last
-            uint8_t *klo = sm + L::klo0 + s * L::QK;
-            if (!ISO) {
-                // One pass per chunk. Projective form of the precision: lambda = n/d with
-                //   d <- a^2 d + qn n,  n <- n + b d   (b = beta k^2),
-                // two FMAs per token on the serial chain. The gate is g = a d_prev / d,
-                // so with PA = prod a the cumulative gate telescopes (d = 1 at the chunk
-                // start): 2^G = PA/d and 2^G/lambda = PA/n. n, d and PA are floats times
-                // 2^E (n, d) and 2^F (PA), rescaled by exact powers of two every 8 tokens.
-                // The operands are written at once against the reference R predicted
-                // from the previous chunk's decay; the chunk's actual G range is checked.
-                const int nvalid = (int)min((long long)kC, te - tok0);
-                float mq, mk;
-                bool range_bad = false;
-                {
-                    // G at the chunk start is F - E to within one (n, d, PA are kept
-                    // in [1, 2) by the per-slot rescale); dpred = the last chunk's drift
-                    const int gs = F - E;
-                    const int lo = gs + min(0, dpred) - 2, hi = gs + max(0, dpred) + 2;
-                    int rnew = rho;
-                    if (hi - rho > kRebase || rho - lo > kRebase) rnew = gs + dpred / 2;
-                    fac_c = __int_as_float((127 + max(-126, min(127, rnew - rho))) << 23);
-                    rho = rnew;
-                    R = rho;
-                    if (local_mode && p > 0)
-                        g.rlog[(u * g.NC + (tok0 - tb) / kC + (long long)p * g.seg_blocks) * DK + i] = (float)R;
-                    const int sh0 = max(-126, min(127, gs - R));
-                    mq = __int_as_float((127 + sh0) << 23);
-                    mk = __int_as_float((127 - sh0) << 23);
-                }
-                const int gs_chunk = F - E;
-                if (nvalid == kC) {
-                    // Full chunk: the chain and the operands of every slot.
-                    float rkmin = 3.0e38f, rkmax = 0.f;
-                    // not unrolled: one slot's code stays resident in the instruction cache
-#pragma unroll 1
-                    for (int j = 0; j < kSlotsPerChunk; ++j) {
-                        const int n = c * kRingsPerChunk + (j >> 1), slot = n % kRings;
-                        // one wait per ring slot of two gate slots
-                        if (!(j & 1) && !waitw(&ring_full[slot], (n / kRings) & 1, abort_flag, g.status)) {
-                            ok = false;
-                            break;
-                        }
-                        const float *ra = reinterpret_cast<const float *>(sm + L::ring0) + slot * 2 * L::RINGF +
-                                          (j & 1) * kSlotTok * DK + i;
-                        const float bsrc = (j < 4) ? cb0 : cb1;
-                        gate_slot<DK>(j, ra, qt, kt, klo, offr, bsrc, state_mode, R, nn, dd, pa, E, F, mq, mk, rkmin,
-                                      rkmax);
-                        if (j & 1) {
-                            // ring slot read into registers: release it (generic reads
-                            // ordered before the TMA refill)
-                            fence_proxy_async();
-                            mbar_arrive(&ring_empty[slot]);
-                        }
-                    }
-                    if (!ok) break;
-                    // rk = 2^(R - G): |G - R| beyond the kept range leaves the exponent window
-                    range_bad = (((__float_as_int(rkmax) >> 23) & 0xff) - 127 >= kMaxOffset) ||
-                                (((__float_as_int(rkmin) >> 23) & 0xff) - 127 < -kMaxOffset);
-                } else {
-                    // Partial chunk (end of a segment or sequence): same recursion, one
-                    // slot at a time, with per-token validity.
-                    int gmin = F - E, gmax = F - E;     // G at the chunk start (absolute)
-#pragma unroll 1
-                    for (int j = 0; j < kSlotsPerChunk; ++j) {
-                        const int n = c * kRingsPerChunk + (j >> 1), slot = n % kRings;
-                        if (!(j & 1) && !waitw(&ring_full[slot], (n / kRings) & 1, abort_flag, g.status)) {
-                            ok = false;
-                            break;
-                        }
-                        const float *ra = reinterpret_cast<const float *>(sm + L::ring0) + slot * 2 * L::RINGF +
-                                          (j & 1) * kSlotTok * DK;
-                        const float *rq = ra + L::RINGF;
-                        const float bsrc = (j < 4) ? cb0 : cb1;
-                        float kr[kSlotTok], qr[kSlotTok], ar[kSlotTok], qnr[kSlotTok], br[kSlotTok];
-#pragma unroll
-                        for (int r = 0; r < kSlotTok; ++r) {
-                            const int off = j * 1024 + offr[r];
-                            kr[r] = bf_at(kt, off);
-                            qr[r] = state_mode ? 0.f : bf_at(qt, off);
-                            ar[r] = ra[r * DK + i];
-                            qnr[r] = rq[r * DK + i];
-                            br[r] = __shfl_sync(0xffffffffu, bsrc, (kSlotTok * j + r) & 31);
-                        }
-                        if (j & 1) {
-                            fence_proxy_async();
-                            mbar_arrive(&ring_empty[slot]);
-                        }
-                        float qo[kSlotTok], ko[kSlotTok];
-                        float rkmin = 3.0e38f, rkmax = 0.f;
-#pragma unroll
-                        for (int r = 0; r < kSlotTok; ++r) {
-                            const bool valid = kSlotTok * j + r < nvalid;
-                            const float at = valid ? ar[r] : 1.f;
-                            const float bk = valid ? br[r] * kr[r] : 0.f;
-                            dd = fmaf(at * at, dd, valid ? qnr[r] * nn : 0.f);
-                            nn = fmaf(bk * kr[r], dd, nn);
-                            pa *= at;
-                            const float rk = __fdividef(dd, pa);
-                            rkmin = fminf(rkmin, rk);
-                            rkmax = fmaxf(rkmax, rk);
-                            qo[r] = valid ? qr[r] * (__fdividef(pa, nn) * mq) : 0.f;
-                            ko[r] = bk * (rk * mk);
-                        }
-                        // G = (F - E) - log2(rk); integer bounds of this slot's G range
-                        gmin = min(gmin, (F - E) - (((__float_as_int(rkmax) >> 23) & 0xff) - 126));
-                        gmax = max(gmax, (F - E) - (((__float_as_int(rkmin) >> 23) & 0xff) - 127));
-#pragma unroll
-                        for (int r = 0; r < kSlotTok; ++r) {
-                            const int off = j * 1024 + offr[r];
-                            if (!state_mode) bf_put(qt, off, qo[r]);
-                            const __nv_bfloat16 khi = __float2bfloat16_rn(ko[r]);
-                            *reinterpret_cast<__nv_bfloat16 *>(kt + off) = khi;
-                            bf_put(klo, off, ko[r] - __bfloat162float(khi));
-                        }
-                        const int e = ((__float_as_int(dd) >> 23) & 0xff) - 127;
-                        const int f = ((__float_as_int(pa) >> 23) & 0xff) - 127;
-                        const float se = __int_as_float((127 - e) << 23);
-                        nn *= se;
-                        dd *= se;
-                        pa *= __int_as_float((127 - f) << 23);
-                        E += e;
-                        F += f;
-                        const int sh = max(-126, min(127, (F - E) - R));
-                        mq = __int_as_float((127 + sh) << 23);
-                        mk = __int_as_float((127 - sh) << 23);
-                    }
-                    if (!ok) break;
-                    range_bad = gmax - R > kMaxOffset || R - gmin > kMaxOffset;
-                }
-                lam = nn / dd;
-                const float gm = pa / dd;                 // 2^G = gm * 2^(F-E)
-                const int sl = F - E;
-                e_cur = gm * __int_as_float((127 + max(-126, min(127, sl - R))) << 23);   // 2^(G - rho)
-                const float gnow = (float)sl + __log2f(gm);
-                glast_log2 = gnow - gprev;                 // this chunk's log2 decay
-                gprev = gnow;
-                dpred = sl - gs_chunk;
-                if (range_bad) atomicOr(g.status, kStatusRange);
-            } else {
-                // isotropic: one precision per head; warp-level Moebius scan over
-                // the chunk (lane l owns tokens 2l, 2l+1), redundantly per warp.
-                const int t0i = 2 * lane, t1i = 2 * lane + 1;
-                const bool va = tok0 + t0i < te, vb = tok0 + t1i < te;
-                const float inv_dk = 1.0f / (float)DK;
-                const float a0 = ca0, q0 = cq0, a1 = ca1, q1 = cq1;
-                const float b0 = va ? cb0 * row_sumsq<DK>(kt, t0i) * inv_dk : 0.f;
-                const float b1 = vb ? cb1 * row_sumsq<DK>(kt, t1i) * inv_dk : 0.f;
-                Mob Mp = mob_norm(mob_mul(mob_step(a1, q1, b1), mob_step(a0, q0, b0)));
-#pragma unroll
-                for (int d = 1; d < 32; d <<= 1) {
-                    Mob o = shfl_up_mob(Mp, d);
-                    if (lane >= d) Mp = mob_norm(mob_mul(Mp, o));
-                }
-                Mob Ex = shfl_up_mob(Mp, 1);
-                if (lane == 0) Ex = Mob{1.f, 0.f, 0.f, 1.f};
-                const float lamA = mob_apply(Ex, lam);
-                float g0 = 1.f, lamB = lamA, g1 = 1.f, lamC;
-                if (va) { float rr = __frcp_rn(fmaf(a0, a0, q0 * lamA)); g0 = a0 * rr; lamB = fmaf(lamA, rr, b0); }
-                lamC = lamB;
-                if (vb) { float rr = __frcp_rn(fmaf(a1, a1, q1 * lamB)); g1 = a1 * rr; lamC = fmaf(lamB, rr, b1); }
-                const float l0 = __log2f(g0), l1 = __log2f(g1);
-                float sum = l0 + l1;
-#pragma unroll
-                for (int d = 1; d < 32; d <<= 1) {
-                    float o = __shfl_up_sync(0xffffffffu, sum, d);
-                    if (lane >= d) sum += o;
-                }
-                const float G1 = sum, G0 = sum - l1;
-                float mn = fminf(0.f, fminf(G0, G1)), mx = fmaxf(0.f, fmaxf(G0, G1));
-#pragma unroll
-                for (int d = 16; d > 0; d >>= 1) {
-                    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, d));
-                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, d));
-                }
-                const int gmin = (int)floorf(mn), gmax = (int)ceilf(mx);
-                R = (gmin + gmax) >> 1;
-                const float Rf = (float)R;
-                // G here runs from the chunk start: the segment-start frame adds the
-                // log2 decay of the segment's earlier chunks
-                if (local_mode && p > 0)
-                    g.rlog[(u * g.NC + (tok0 - tb) / kC + (long long)p * g.seg_blocks) * DK + i] = Rf + log_decay;
-                const float Glast = __shfl_sync(0xffffffffu, G1, 31);
-                e_cur = exp2f(Glast - Rf);
-                glast_log2 = Glast;
-                lam = __shfl_sync(0xffffffffu, lamC, 31);
-                // per-token factors, shared by all keys of the head
-                if (gmax - gmin > 2 * kMaxOffset) atomicOr(g.status, kStatusRange);
-                // every gate warp has read the raw k rows, and the previous chunk's
-                // factors, before any of them is overwritten
-                mbar_arrive(gate_sync);
-                if (!waitw(gate_sync, c & 1, abort_flag, g.status)) { ok = false; break; }
-                // per-token factors, shared by all keys of the head: q / lambda 2^(G-R)
-                // and beta 2^(R-G), zero past the end of the sequence
+            for (int c = 0; c < nchunks; ++c) {
+                const int st = c & 1;
+                const long long tok0 = tb + (long long)c * kC;
+                uint8_t *qt = sm + L::q0 + st * L::QK;
+                uint8_t *kt = sm + L::k0 + st * L::QK;
+                uint8_t *klo = sm + L::klo0 + st * L::QK;
+                bool okw = true;
                 if (warp == 0) {
-                    isof[t0i] = va ? make_float2(exp2f(G0 - Rf) / lamB, cb0 * exp2f(Rf - G0)) : make_float2(0.f, 0.f);
-                    isof[t1i] = vb ? make_float2(exp2f(G1 - Rf) / lamC, cb1 * exp2f(Rf - G1)) : make_float2(0.f, 0.f);
-                }
-                mbar_arrive(gate_sync2);
-                if (!waitw(gate_sync2, c & 1, abort_flag, g.status)) { ok = false; break; }
-#pragma unroll 1
-                for (int j = 0; j < kSlotsPerChunk; ++j) {
-                    float qr[kSlotTok], kr[kSlotTok];
-                    float2 fv[kSlotTok];
+                    const float cb0 = nb0, cb1 = nb1, a0 = na0, a1 = na1, q0 = nq0, q1 = nq1;
+                    if (c + 1 < nchunks) prefetch(c + 1);
+                    okw = waitw(&stage_full[st], (c >> 1) & 1, abort_flag, g.status);
+                    if (okw) {
+                        // warp-level Moebius scan of the chunk (lane: tokens 2l, 2l+1)
+                        const int t0i = 2 * lane, t1i = t0i + 1;
+                        const bool va = tok0 + t0i < te, vb = tok0 + t1i < te;
+                        const float inv_dk = 1.0f / (float)DK;
+                        const float b0 = va ? cb0 * row_sumsq<DK>(kt, t0i) * inv_dk : 0.f;
+                        const float b1 = vb ? cb1 * row_sumsq<DK>(kt, t1i) * inv_dk : 0.f;
+                        Mob Mp = mob_norm(mob_mul(mob_step(a1, q1, b1), mob_step(a0, q0, b0)));
 #pragma unroll
-                    for (int r = 0; r < kSlotTok; ++r) {
-                        const int off = j * 1024 + offr[r];
-                        qr[r] = state_mode ? 0.f : bf_at(qt, off);
-                        kr[r] = bf_at(kt, off);
-                        fv[r] = isof[kSlotTok * j + r];
-                    }
+                        for (int d = 1; d < 32; d <<= 1) {
+                            Mob o = shfl_up_mob(Mp, d);
+                            if (lane >= d) Mp = mob_norm(mob_mul(Mp, o));
+                        }
+                        Mob Ex = shfl_up_mob(Mp, 1);
+                        if (lane == 0) Ex = Mob{1.f, 0.f, 0.f, 1.f};
+                        const float lamA = mob_apply(Ex, lam);
+                        float g0 = 1.f, lamB = lamA, g1 = 1.f, lamC;
+                        if (va) { float rr = __frcp_rn(fmaf(a0, a0, q0 * lamA)); g0 = a0 * rr; lamB = fmaf(lamA, rr, b0); }
+                        lamC = lamB;
+                        if (vb) { float rr = __frcp_rn(fmaf(a1, a1, q1 * lamB)); g1 = a1 * rr; lamC = fmaf(lamB, rr, b1); }
+                        const float l0 = __log2f(g0), l1 = __log2f(g1);
+                        float sum = l0 + l1;
 #pragma unroll
-                    for (int r = 0; r < kSlotTok; ++r) {
-                        const int off = j * 1024 + offr[r];
-                        const float ko = kr[r] * fv[r].y;
-                        const uint32_t t = __float_as_uint(ko) + 0x8000u;         // K' hi, rounded
-                        *reinterpret_cast<uint16_t *>(kt + off) = (uint16_t)(t >> 16);
-                        *reinterpret_cast<uint16_t *>(klo + off) =
-                            (uint16_t)(__float_as_uint(ko - __uint_as_float(t & 0xffff0000u)) >> 16);
-                        if (!state_mode)
-                            *reinterpret_cast<uint16_t *>(qt + off) =
-                                (uint16_t)((__float_as_uint(qr[r] * fv[r].x) + 0x8000u) >> 16);
+                        for (int d = 1; d < 32; d <<= 1) {
+                            float o = __shfl_up_sync(0xffffffffu, sum, d);
+                            if (lane >= d) sum += o;
+                        }
+                        // G (relative to the chunk start) after tokens 2l and 2l+1, and
+                        // just before 2l; in the frame x = G_abs - rho: D + G
+                        const float G1 = sum, G0 = sum - l1, Gp = G0 - l0;
+                        float mn = fminf(Gp, fminf(G0, G1)), mx = fmaxf(Gp, fmaxf(G0, G1));
+                        // quarter q = lanes 8q .. 8q+7
+#pragma unroll
+                        for (int d = 1; d < 8; d <<= 1) {
+                            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, d));
+                            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, d));
+                        }
+                        int2 qr[4];
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const float lo = __shfl_sync(0xffffffffu, mn, 8 * q);
+                            const float hi = __shfl_sync(0xffffffffu, mx, 8 * q);
+                            qr[q] = make_int2((int)floorf(D + lo), (int)ceilf(D + hi));
+                        }
+                        int R[4];
+                        bool bad;
+                        const int lv = choose_refs(qr, 0, R, bad);
+                        const int myq = lane >> 3;
+                        const float Rq = (float)pick4(R, myq);
+                        // per-token factors: q / lambda 2^(G - rho_q), beta 2^(rho_q - G)
+                        const float e0 = D + G0 - Rq, e1 = D + G1 - Rq;
+                        isof[st * kC + t0i] = va ? make_float2(exp2f(e0) / lamB, cb0 * exp2f(-e0)) : make_float2(0.f, 0.f);
+                        isof[st * kC + t1i] = vb ? make_float2(exp2f(e1) / lamC, cb1 * exp2f(-e1)) : make_float2(0.f, 0.f);
+                        for (int i = lane; i < DK; i += 32) {
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) facd[(st * 4 + q) * DK + i] = R[q] - (q ? R[q - 1] : 0);
+                        }
+                        if (lane == 0) {
+                            lvl[st] = (c << 2) | lv;
+                            if (bad) atomicOr(g.status, kStatusRange);
+                        }
+                        if (LOCAL && p > 0) {
+                            // segment-start frame: rho_q = G_chunk_start - D + R_q
+                            float *rl = g.rlog + ((u * g.NC + chunk_base + c) * 4) * DK;
+                            for (int i = lane; i < DK; i += 32) {
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) rl[q * DK + i] = Gc - D + (float)R[q];
+                            }
+                        }
+                        const float Gend = __shfl_sync(0xffffffffu, G1, 31);
+                        lam = __shfl_sync(0xffffffffu, lamC, 31);
+                        D = D + Gend - (float)R[3];
+                        Gc += Gend;
+                        if (c == nchunks - 1) {
+                            for (int i = lane; i < DK; i += 32) facf[i] = exp2f(D);
+                            if (lane == 0) {
+                                if (LOCAL) g.decay[u * g.P + p] = exp2f(Gc);
+                                if (last_seg && g.final_lambda) g.final_lambda[u] = lam;
+                            }
+                        }
                     }
                 }
+                if (named_bar_or(kGateBar, RL::GT, !okw || *abort_flag)) { ok = false; break; }
+                // fold the rows: Q' = q fq, K' = k fk (hi + remainder); thread = (row, key pair)
+                constexpr int NP = DK / 2;
+#pragma unroll 4
+                for (int it = tid; it < kC * NP; it += RL::GT) {
+                    const int row = it / NP, i0 = 2 * (it % NP);
+                    const int off = sw_off(row, i0, kC);
+                    const float2 f = isof[st * kC + row];
+                    const float2 qf = unpack_bf2(*reinterpret_cast<const uint32_t *>(qt + off));
+                    const float2 kf = unpack_bf2(*reinterpret_cast<const uint32_t *>(kt + off));
+                    const float2 ko = make_float2(kf.x * f.y, kf.y * f.y);
+                    const uint32_t kh = pack_bf2(ko.x, ko.y);
+                    const float2 khf = unpack_bf2(kh);
+                    *reinterpret_cast<uint32_t *>(qt + off) = pack_bf2(qf.x * f.x, qf.y * f.x);
+                    *reinterpret_cast<uint32_t *>(kt + off) = kh;
+                    *reinterpret_cast<uint32_t *>(klo + off) = pack_bf2(ko.x - khf.x, ko.y - khf.y);
+                }
+                fence_proxy_async();
+                mbar_arrive(&qk_ready[st]);
             }
-            // state rescale factors: U_c = diag(2^R_c) S_c, S_{c+1} = diag(2^(G_last - R_c)) (U_c + K'^T V)
-            fac[s * DK + i] = ISO ? e_prev * __int_as_float((127 + max(-126, min(127, R))) << 23) : fac_c;
-            if (c == nchunks - 1) fac_final[i] = e_cur;
-            e_prev = e_cur;
-            log_decay += glast_log2;
-            fence_proxy_async();
-            mbar_arrive(&qk_ready[s]);
+            if (warp == 0 && lane == 0 && nchunks == 0 && last_seg && g.final_lambda) g.final_lambda[u] = lam;
         }
-        if (ok && !*abort_flag) {
-            if (state_mode || local_mode) {
-                if (ISO ? (gt == 0) : key) g.decay[(u * g.P + p) * (ISO ? 1 : DK) + (ISO ? 0 : i)] = exp2f(log_decay);
-            }
-            if (!state_mode && last_seg && g.final_lambda) {
-                if (ISO ? (gt == 0) : key) g.final_lambda[u * (ISO ? 1 : DK) + (ISO ? 0 : i)] = lam;
-            }
-        }
-      }
-    } else if (warp >= 4 && warp < 8) {
-        // ================= epilogue warps ====================================
-        const int e = tid - 128, we = e >> 5, le = e & 31;
+        (void)ok;
+    } else {
+        // ================= epilogue warps; thread 0 also issues the TMA loads and
+        // the tcgen05 MMAs at the points where the epilogue synchronises ========
+        const int we = warp - RL::EPIW;        // TMEM lane quarter (warp % 4)
+        const bool issuer = we == 0 && lane == 0;
         const uint32_t lane_base = (uint32_t)(32 * we) << 16;
-        const int row64 = 16 * we + le;
-        const bool v64 = le < 16;
-        const int rowU = (DK == 128) ? (32 * we + le) : row64;
+        const int row64 = 16 * we + lane;
+        const bool v64 = lane < 16;
+        const int rowU = (DK == 128) ? (32 * we + lane) : row64;
         const bool vU = (DK == 128) || v64;
         uint8_t *ub = sm + L::ub0;
         uint8_t *pt = sm + L::p0;
-        const float *eta0 = (!state_mode && (!local_mode || p == 0) && g.eta0) ? g.eta0 + u * DK * DV : nullptr;
+        const float *eta0 = ((!LOCAL || p == 0) && g.eta0) ? g.eta0 + u * DK * DV : nullptr;
         bool ok = true;
+        // q, k, v tiles of chunk c into stage c & 1, and an L2 prefetch of the
+        // chunk two ahead (its tiles, a and qn: the gate loads those itself)
+        auto load_chunk = [&](int c) {
+            const int tok0 = (int)(tb + (long long)c * kC);
+            const int s = c & 1;
+            mbar_expect_tx(&stage_full[s], 2 * L::QK + L::V);
+#pragma unroll
+            for (int a = 0; a < DK / 64; ++a) {
+                tma_load_3d(sm + L::q0 + s * L::QK + a * kC * 128, &tm_q, &stage_full[s], 64 * a, h, tok0);
+                tma_load_3d(sm + L::k0 + s * L::QK + a * kC * 128, &tm_k, &stage_full[s], 64 * a, h, tok0);
+            }
+#pragma unroll
+            for (int a = 0; a < DV / 64; ++a)
+                tma_load_3d(sm + L::v0 + s * L::V + a * kC * 128, &tm_v, &stage_full[s], 64 * a, h, tok0);
+            if (c + 2 < nchunks) {
+                const int tp = tok0 + 2 * kC;
+#pragma unroll
+                for (int a = 0; a < DK / 64; ++a) {
+                    tma_prefetch_3d(&tm_q, 64 * a, h, tp);
+                    tma_prefetch_3d(&tm_k, 64 * a, h, tp);
+                }
+#pragma unroll
+                for (int a = 0; a < DV / 64; ++a) tma_prefetch_3d(&tm_v, 64 * a, h, tp);
+                if (!ISO) {
+                    tma_prefetch_3d(&tm_a, 0, h, tp);
+                    tma_prefetch_3d(&tm_qn, 0, h, tp);
+                }
+            }
+        };
+        int loaded = 0;                                 // chunks whose loads were issued
+        if (issuer) {
+            // a and qn of chunk 1 (chunk 0 is read at once)
+            if (!ISO && nchunks > 1) {
+                tma_prefetch_3d(&tm_a, 0, h, (int)(tb + kC));
+                tma_prefetch_3d(&tm_qn, 0, h, (int)(tb + kC));
+            }
+            for (; loaded < 2 && loaded < nchunks; ++loaded) load_chunk(loaded);
+        }
         // Belief at the segment start, written into the U columns of TMEM before
         // the first chunk (while the gate works on it): eta0 for whole rows and
         // first segments, zero for the later segments of split rows (their
         // carried state is added by the correction pass)
-        if (!state_mode && nchunks > 0) {
+        if (nchunks > 0) {
 #pragma unroll
             for (int cb = 0; cb < DV / 32; ++cb) {
-                float acc[32];
+                uint32_t r[32];
 #pragma unroll
                 for (int x = 0; x < 32; x += 4) {
                     const float4 e4 = (vU && eta0) ? *reinterpret_cast<const float4 *>(eta0 + rowU * DV + cb * 32 + x)
                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
-                    acc[x] = e4.x; acc[x + 1] = e4.y; acc[x + 2] = e4.z; acc[x + 3] = e4.w;
+                    r[x] = __float_as_uint(e4.x); r[x + 1] = __float_as_uint(e4.y);
+                    r[x + 2] = __float_as_uint(e4.z); r[x + 3] = __float_as_uint(e4.w);
                 }
-                uint32_t r[32];
-#pragma unroll
-                for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(acc[x]);
                 tmem_st32(tbase + lane_base + L::colU + cb * 32, r);
             }
             tmem_wait_st();
         }
-        // output rows of chunk cc (TMEM O -> bf16 -> global)
-        auto emit_out = [&](int cc) -> bool {
-            if (!waitw(o_full, cc & 1, abort_flag, g.status)) return false;
+        constexpr uint32_t iS = idesc_bf16(64, 64, false, false);
+        constexpr uint32_t iO = idesc_bf16(64, DV, false, true);
+        constexpr uint32_t iU = idesc_bf16(DK, DV, true, true);
+        const uint32_t tS = tbase + L::colS, tO = tbase + L::colO, tU = tbase + L::colU;
+        const uint32_t pa_s = smem_u32(sm + L::p0), uba = smem_u32(sm + L::ub0);
+        int pc = 0;                                   // passes so far (barrier phases)
+        for (int c = 0; c < nchunks && ok; ++c) {
+            const int st = c & 1;
+            if (!waitw(&qk_ready[st], (c >> 1) & 1, abort_flag, g.status)) { ok = false; }
+            if (named_bar_or(kEpiBar, 128, !ok || *abort_flag)) { ok = false; break; }
             tc_fence_after();
-            const long long tok0 = tb + (long long)cc * kC;
-            const bool row_ok = v64 && (tok0 + row64 < te);
-            __nv_bfloat16 *orow = g.out + ((tok0 + row64) * g.H + h) * DV;
+            const int lv = lvl[st] & 3;
+            const int np = 1 << lv, qper = 4 >> lv;
+            const uint32_t qa = smem_u32(sm + L::q0 + st * L::QK);
+            const uint32_t ka = smem_u32(sm + L::k0 + st * L::QK);
+            const uint32_t va = smem_u32(sm + L::v0 + st * L::V);
+            const uint32_t kloa = smem_u32(sm + L::klo0 + st * L::QK);
+            if (issuer) {
+                if (LOCAL && p > 0) {
+                    // export the folded q tile (the correction pass multiplies it by
+                    // the carried segment-start state)
+                    const int tok0 = (int)(tb + (long long)c * kC);
 #pragma unroll
-            for (int cb = 0; cb < DV / 32; cb += 2) {
-                uint32_t rr[2][32];
-                tmem_ld32(tbase + lane_base + L::colO + cb * 32, rr[0]);
-                tmem_ld32(tbase + lane_base + L::colO + cb * 32 + 32, rr[1]);
-                tmem_wait_ld();
-                if (row_ok) {
+                    for (int a = 0; a < DK / 64; ++a)
+                        tma_store_3d(&tm_qs, sm + L::q0 + st * L::QK + a * kC * 128, 64 * a, h, tok0);
+                    tma_store_commit();
+                }
+                // scores of the whole chunk (each pass masks its own block)
 #pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const uint32_t *r = rr[hh];
+                for (int kk = 0; kk < DK / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * (kC * 128) + (kk & 3) * 32;
+                    mma_bf16(tS, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), iS, kk > 0);
+                }
+                mma_commit(s_full);
+            }
+            for (int k = 0; k < np; ++k) {
+                const int m0 = kQ * qper * k, m1 = m0 + kQ * qper;
+                const int s0 = k * qper, s1 = s0 + qper;      // 16-token slices of this pass
+                // ---- state: U <- 2^d U for this pass's reference, snapshot to bf16
+                if (pc > 0 && !waitw(u_done, (pc - 1) & 1, abort_flag, g.status)) ok = false;
+                tc_fence_after();
+                const int d = vU ? facd[(st * 4 + k * qper) * DK + rowU] : 0;
+                const bool rmw = __any_sync(0xffffffffu, d != 0);
+                if (ok) {
 #pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            uint4 w;
-                            w.x = pack_bf2(__uint_as_float(r[q4 * 8 + 0]), __uint_as_float(r[q4 * 8 + 1]));
-                            w.y = pack_bf2(__uint_as_float(r[q4 * 8 + 2]), __uint_as_float(r[q4 * 8 + 3]));
-                            w.z = pack_bf2(__uint_as_float(r[q4 * 8 + 4]), __uint_as_float(r[q4 * 8 + 5]));
-                            w.w = pack_bf2(__uint_as_float(r[q4 * 8 + 6]), __uint_as_float(r[q4 * 8 + 7]));
-                            *reinterpret_cast<uint4 *>(orow + (cb + hh) * 32 + q4 * 8) = w;
+                    for (int cb = 0; cb < DV / 32; ++cb) {
+                        uint32_t r[32];
+                        const uint32_t ta = tbase + lane_base + L::colU + cb * 32;
+                        tmem_ld32(ta, r);
+                        tmem_wait_ld();
+                        if (rmw) {
+#pragma unroll
+                            for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(scale2(__uint_as_float(r[x]), d));
+                            tmem_st32(ta, r);
+                        }
+                        if (vU) {
+#pragma unroll
+                            for (int q4 = 0; q4 < 4; ++q4) {
+                                uint4 w;
+                                w.x = pack_bf2(__uint_as_float(r[q4 * 8 + 0]), __uint_as_float(r[q4 * 8 + 1]));
+                                w.y = pack_bf2(__uint_as_float(r[q4 * 8 + 2]), __uint_as_float(r[q4 * 8 + 3]));
+                                w.z = pack_bf2(__uint_as_float(r[q4 * 8 + 4]), __uint_as_float(r[q4 * 8 + 5]));
+                                w.w = pack_bf2(__uint_as_float(r[q4 * 8 + 6]), __uint_as_float(r[q4 * 8 + 7]));
+                                *reinterpret_cast<uint4 *>(ub + sw_off(rowU, cb * 32 + q4 * 8, DK)) = w;
+                            }
+                        }
+                    }
+                    tmem_wait_st();
+                }
+                fence_proxy_async();
+                tc_fence_before();
+                if (named_bar_or(kEpiBar, 128, !ok || *abort_flag)) { ok = false; break; }
+                if (issuer) {
+                    tc_fence_after();
+                    // O = Q' U (the previous pass's O was read out before the barrier)
+#pragma unroll
+                    for (int kk = 0; kk < DK / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * (kC * 128) + (kk & 3) * 32;
+                        mma_bf16(tO, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(uba + kk * 2048, DK * 128, 1024), iO,
+                                 kk > 0);
+                    }
+                    // U += K'^T V over this pass's tokens (hi and remainder of K')
+                    for (int kk = s0; kk < s1; ++kk) {
+                        const uint64_t bv = sdesc_sw128(va + kk * 2048, kC * 128, 1024);
+                        mma_bf16(tU, sdesc_sw128(ka + kk * 2048, kC * 128, 1024), bv, iU, 1);
+                        mma_bf16(tU, sdesc_sw128(kloa + kk * 2048, kC * 128, 1024), bv, iU, 1);
+                    }
+                    mma_commit(u_done);
+                }
+                // ---- P = the pass's block of the causal score tile, bf16
+                if (k == 0 && !waitw(s_full, c & 1, abort_flag, g.status)) ok = false;
+                tc_fence_after();
+                if (ok) {
+#pragma unroll
+                    for (int hf = 0; hf < 2; ++hf) {
+                        uint32_t r[32];
+                        tmem_ld32(tbase + lane_base + L::colS + 32 * hf, r);
+                        tmem_wait_ld();
+                        if (v64) {
+                            const int tau = row64;
+                            const bool in_row = tau >= m0 && tau < m1;
+#pragma unroll
+                            for (int ch = 4 * hf; ch < 4 * hf + 4; ++ch) {
+                                float x[8];
+#pragma unroll
+                                for (int e2 = 0; e2 < 8; ++e2) {
+                                    const int sg = ch * 8 + e2;
+                                    const float sv = __uint_as_float(r[sg - 32 * hf]);
+                                    x[e2] = (in_row && sg >= m0 && sg <= tau) ? sv : 0.f;
+                                }
+                                uint4 w;
+                                w.x = pack_bf2(x[0], x[1]); w.y = pack_bf2(x[2], x[3]);
+                                w.z = pack_bf2(x[4], x[5]); w.w = pack_bf2(x[6], x[7]);
+                                *reinterpret_cast<uint4 *>(pt + tau * 128 + ((ch ^ (tau & 7)) << 4)) = w;
+                            }
                         }
                     }
                 }
-            }
-            tc_fence_before();
-            mbar_arrive(o_empty);
-            return true;
-        };
-        for (int c = 0; c < nchunks; ++c) {
-            const int s = c & 1;
-            // ---- output rows of the previous chunk (its MMAs finished meanwhile)
-            if (!state_mode && c > 0 && !emit_out(c - 1)) { ok = false; break; }
-            // ---- state U_c = diag(fac) * (eta_start or U_{c-1} + K'^T V)
-            if (!waitw(&qk_ready[s], (c >> 1) & 1, abort_flag, g.status)) { ok = false; break; }
-            if (c > 0 && !waitw(u_done, (c - 1) & 1, abort_flag, g.status)) { ok = false; break; }
-            tc_fence_after();
-            // diag: f = 1 unless the gate moved this key's reference; the warp then
-            // only snapshots U (bf16, for the readout MMA) without rewriting TMEM
-            const float f = vU ? fac[s * DK + rowU] : 1.f;
-            const bool rmw = (c == 0) || __any_sync(0xffffffffu, f != 1.0f);
-            auto snap = [&](const uint32_t (&r)[32], int cb) {
-                if (!state_mode && vU) {
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        uint4 w;
-                        w.x = pack_bf2(__uint_as_float(r[q4 * 8 + 0]), __uint_as_float(r[q4 * 8 + 1]));
-                        w.y = pack_bf2(__uint_as_float(r[q4 * 8 + 2]), __uint_as_float(r[q4 * 8 + 3]));
-                        w.z = pack_bf2(__uint_as_float(r[q4 * 8 + 4]), __uint_as_float(r[q4 * 8 + 5]));
-                        w.w = pack_bf2(__uint_as_float(r[q4 * 8 + 6]), __uint_as_float(r[q4 * 8 + 7]));
-                        *reinterpret_cast<uint4 *>(ub + sw_off(rowU, cb * 32 + q4 * 8, DK)) = w;
-                    }
+                fence_proxy_async();
+                tc_fence_before();
+                if (named_bar_or(kEpiBar, 128, !ok || *abort_flag)) { ok = false; break; }
+                if (issuer) {
+                    tc_fence_after();
+                    // O += P V over this pass's tokens
+                    for (int kk = s0; kk < s1; ++kk)
+                        mma_bf16(tO, sdesc_sw128(pa_s + kk * 32, 16, 1024), sdesc_sw128(va + kk * 2048, kC * 128, 1024),
+                                 iO, 1);
+                    mma_commit(o_full);
                 }
-            };
-            if (c == 0 && state_mode) {
+                // ---- output rows of this pass (a timeout here is seen by every
+                // epilogue warp at the next reducing barrier)
+                if (!waitw(o_full, pc & 1, abort_flag, g.status)) ok = false;
+                tc_fence_after();
+                if (ok) {
+                    const long long tok0 = tb + (long long)c * kC;
+                    const bool row_ok = v64 && row64 >= m0 && row64 < m1 && (tok0 + row64 < te);
+                    __nv_bfloat16 *orow = g.out + ((tok0 + row64) * g.H + h) * DV;
 #pragma unroll
-                for (int cb = 0; cb < DV / 32; ++cb) {
-                    uint32_t r[32];
+                    for (int cb = 0; cb < DV / 32; ++cb) {
+                        uint32_t r[32];
+                        tmem_ld32(tbase + lane_base + L::colO + cb * 32, r);
+                        tmem_wait_ld();
+                        if (row_ok) {
 #pragma unroll
-                    for (int x = 0; x < 32; ++x) r[x] = 0u;
-                    tmem_st32(tbase + lane_base + L::colU + cb * 32, r);
-                }
-            } else if (rmw || !state_mode) {
-#pragma unroll
-                for (int cb = 0; cb < DV / 32; cb += 2) {
-                    uint32_t r0[32], r1[32];
-                    const uint32_t ta = tbase + lane_base + L::colU + cb * 32;
-                    tmem_ld32(ta, r0);
-                    tmem_ld32(ta + 32, r1);
-                    tmem_wait_ld();
-                    if (rmw) {
-#pragma unroll
-                        for (int x = 0; x < 32; ++x) {
-                            r0[x] = __float_as_uint(__uint_as_float(r0[x]) * f);
-                            r1[x] = __float_as_uint(__uint_as_float(r1[x]) * f);
+                            for (int q4 = 0; q4 < 4; ++q4) {
+                                uint4 w;
+                                w.x = pack_bf2(__uint_as_float(r[q4 * 8 + 0]), __uint_as_float(r[q4 * 8 + 1]));
+                                w.y = pack_bf2(__uint_as_float(r[q4 * 8 + 2]), __uint_as_float(r[q4 * 8 + 3]));
+                                w.z = pack_bf2(__uint_as_float(r[q4 * 8 + 4]), __uint_as_float(r[q4 * 8 + 5]));
+                                w.w = pack_bf2(__uint_as_float(r[q4 * 8 + 6]), __uint_as_float(r[q4 * 8 + 7]));
+                                *reinterpret_cast<uint4 *>(orow + cb * 32 + q4 * 8) = w;
+                            }
                         }
-                        tmem_st32(ta, r0);
-                        tmem_st32(ta + 32, r1);
-                    }
-                    snap(r0, cb);
-                    snap(r1, cb + 1);
-                }
-            }
-            tmem_wait_st();
-            fence_proxy_async();
-            tc_fence_before();
-            mbar_arrive(u_ready);
-            if (state_mode) continue;
-            // ---- P = causal mask of the score tile, bf16
-            if (!waitw(s_full, c & 1, abort_flag, g.status)) { ok = false; break; }
-            tc_fence_after();
-            {
-                uint32_t r0[32], r1[32];
-                tmem_ld32(tbase + lane_base + L::colS, r0);
-                tmem_ld32(tbase + lane_base + L::colS + 32, r1);
-                tmem_wait_ld();
-                if (v64) {
-                    const int tau = row64;
-#pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) {
-                        float x[8];
-#pragma unroll
-                        for (int e2 = 0; e2 < 8; ++e2) {
-                            const int sg = ch * 8 + e2;
-                            const float sv = __uint_as_float(sg < 32 ? r0[sg] : r1[sg - 32]);
-                            x[e2] = sg <= tau ? sv : 0.f;
-                        }
-                        uint4 w;
-                        w.x = pack_bf2(x[0], x[1]); w.y = pack_bf2(x[2], x[3]);
-                        w.z = pack_bf2(x[4], x[5]); w.w = pack_bf2(x[6], x[7]);
-                        *reinterpret_cast<uint4 *>(pt + tau * 128 + ((ch ^ (tau & 7)) << 4)) = w;
                     }
                 }
+                tc_fence_before();
+                ++pc;
             }
-            fence_proxy_async();
-            tc_fence_before();
-            mbar_arrive(p_full);
+            if (named_bar_or(kEpiBar, 128, !ok || *abort_flag)) { ok = false; break; }
+            // every MMA of this chunk has completed (o_full of its last pass): the
+            // stage takes the chunk two ahead once the q' export has read it
+            if (issuer) {
+                if (LOCAL && p > 0) tma_store_wait_read();
+                if (loaded < nchunks) { load_chunk(loaded); ++loaded; }
+            }
         }
-        if (ok && !state_mode && nchunks > 0 && !emit_out(nchunks - 1)) ok = false;
-        // ---- final belief (last segment) or segment transfer (state mode)
+        // ---- final belief (last segment) or segment transfer (mode 2)
         float *dst = nullptr;
-        if (state_mode || local_mode) dst = g.S_io + (u * g.P + p) * DK * DV;
+        if (LOCAL) dst = g.S_io + (u * g.P + p) * DK * DV;
         else if (last_seg && g.final_eta) dst = g.final_eta + u * DK * DV;
         if (ok && dst && !*abort_flag) {
             if (nchunks > 0) {
-                if (waitw(u_done, (nchunks - 1) & 1, abort_flag, g.status)) {
+                if (waitw(u_done, (pc - 1) & 1, abort_flag, g.status)) {
                     tc_fence_after();
-                    const float ff = vU ? fac_final[rowU] : 0.f;
+                    const float ff = vU ? facf[rowU] : 0.f;
 #pragma unroll
                     for (int cb = 0; cb < DV / 32; ++cb) {
                         uint32_t r[32];
@@ -840,141 +1028,18 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     }
                 }
             } else if (vU) {
-                // no tokens (an empty packed sequence, a single segment): the belief is eta0
+                // no tokens (an empty packed sequence): the belief is eta0
                 for (int x = 0; x < DV; ++x) dst[rowU * DV + x] = eta0 ? eta0[rowU * DV + x] : 0.f;
             }
         }
-    } else if (warp == RL::PRODW) {
-        // ================= TMA producer =====================================
-        if (lane == 0) {
-            int last_ring[kRings], last_stage[2] = {-1, -1};
-            for (int j = 0; j < kRings; ++j) last_ring[j] = -1;
-            bool ok = true;
-            for (int c = 0; c < nchunks && ok; ++c) {
-                const int tok0 = (int)(tb + (long long)c * kC);
-                const int s = c & 1;
-                if (c >= 2 && !wait1(&stage_empty[s], ((c >> 1) - 1) & 1, abort_flag, g.status)) { ok = false; break; }
-                mbar_expect_tx(&stage_full[s], (state_mode ? 0 : L::QK) + L::QK + L::V);
-#pragma unroll
-                for (int a = 0; a < DK / 64; ++a) {
-                    if (!state_mode)
-                        tma_load_3d(sm + L::q0 + s * L::QK + a * kC * 128, &tm_q, &stage_full[s], 64 * a, h, tok0);
-                    tma_load_3d(sm + L::k0 + s * L::QK + a * kC * 128, &tm_k, &stage_full[s], 64 * a, h, tok0);
-                }
-#pragma unroll
-                for (int a = 0; a < DV / 64; ++a)
-                    tma_load_3d(sm + L::v0 + s * L::V + a * kC * 128, &tm_v, &stage_full[s], 64 * a, h, tok0);
-                last_stage[s] = c;
-                // L2 prefetch of the chunk two ahead, so that the TMA copies above
-                // and the ring refills below are served from L2
-                if (c + 2 < nchunks) {
-                    const int tp = tok0 + 2 * kC;
-#pragma unroll
-                    for (int a = 0; a < DK / 64; ++a) {
-                        if (!state_mode) tma_prefetch_3d(&tm_q, 64 * a, h, tp);
-                        tma_prefetch_3d(&tm_k, 64 * a, h, tp);
-                    }
-#pragma unroll
-                    for (int a = 0; a < DV / 64; ++a) tma_prefetch_3d(&tm_v, 64 * a, h, tp);
-                    if (!ISO)
-                        for (int j = 0; j < kRingsPerChunk; ++j) {
-                            tma_prefetch_3d(&tm_a, 0, h, tp + kRingTok * j);
-                            tma_prefetch_3d(&tm_qn, 0, h, tp + kRingTok * j);
-                        }
-                }
-                if (!ISO) {
-                    for (int j = 0; j < kRingsPerChunk; ++j) {
-                        const int n = c * kRingsPerChunk + j, slot = n % kRings;
-                        if (n >= kRings && !wait1(&ring_empty[slot], ((n / kRings) - 1) & 1, abort_flag, g.status)) {
-                            ok = false;
-                            break;
-                        }
-                        float *ra = reinterpret_cast<float *>(sm + L::ring0) + slot * 2 * L::RINGF;
-                        mbar_expect_tx(&ring_full[slot], 2 * L::RINGF * 4);
-                        tma_load_3d(ra, &tm_a, &ring_full[slot], 0, h, tok0 + kRingTok * j);
-                        tma_load_3d(ra + L::RINGF, &tm_qn, &ring_full[slot], 0, h, tok0 + kRingTok * j);
-                        last_ring[slot] = n;
-                    }
-                }
-            }
+        if (issuer) {
+            if (LOCAL && p > 0) tma_store_wait_all();
             if (!ok || *abort_flag) {
-                // wait (bounded) until every copy this thread issued has landed
-                for (int j = 0; j < kRings; ++j)
-                    if (last_ring[j] >= 0)
-                        wait_slow(&ring_full[j], (last_ring[j] / kRings) & 1, abort_flag, g.status, false);
-                for (int s = 0; s < 2; ++s)
-                    if (last_stage[s] >= 0)
-                        wait_slow(&stage_full[s], (last_stage[s] >> 1) & 1, abort_flag, g.status, false);
+                // wait (bounded) until every tile load issued has landed
+                for (int c = max(0, loaded - 2); c < loaded; ++c)
+                    wait_slow(&stage_full[c & 1], (c >> 1) & 1, abort_flag, g.status, false);
             }
-        }
-    } else if (warp == RL::MMAW) {
-        // ================= MMA issuer =======================================
-        if (lane == 0) {
-            constexpr uint32_t iS = idesc_bf16(64, 64, false, false);
-            constexpr uint32_t iO = idesc_bf16(64, DV, false, true);
-            constexpr uint32_t iU = idesc_bf16(DK, DV, true, true);
-            const uint32_t tS = tbase + L::colS, tO = tbase + L::colO, tU = tbase + L::colU;
-            const uint32_t pa = smem_u32(sm + L::p0), uba = smem_u32(sm + L::ub0);
-            for (int c = 0; c < nchunks; ++c) {
-                const int s = c & 1;
-                if (!wait1(&qk_ready[s], (c >> 1) & 1, abort_flag, g.status)) break;
-                tc_fence_after();
-                const uint32_t qa = smem_u32(sm + L::q0 + s * L::QK);
-                const uint32_t ka = smem_u32(sm + L::k0 + s * L::QK);
-                const uint32_t va = smem_u32(sm + L::v0 + s * L::V);
-                const uint32_t kloa = smem_u32(sm + L::klo0 + s * L::QK);
-                if (local_mode && p > 0) {
-                    // export the folded q tile (the correction pass multiplies it by the
-                    // carried segment-start state)
-                    const int tok0 = (int)(tb + (long long)c * kC);
-#pragma unroll
-                    for (int a = 0; a < DK / 64; ++a)
-                        tma_store_3d(&tm_qs, sm + L::q0 + s * L::QK + a * kC * 128, 64 * a, h, tok0);
-                    tma_store_commit();
-                }
-                if (!state_mode) {
-#pragma unroll
-                    for (int kk = 0; kk < DK / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * (kC * 128) + (kk & 3) * 32;
-                        mma_bf16(tS, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), iS, kk > 0);
-                    }
-                    mma_commit(s_full);
-                }
-                if (!wait1(u_ready, c & 1, abort_flag, g.status)) break;
-                tc_fence_after();
-                if (!state_mode) {
-                    // O of the previous chunk has been read out by the epilogue
-                    if (c > 0 && !wait1(o_empty, (c - 1) & 1, abort_flag, g.status)) break;
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < DK / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * (kC * 128) + (kk & 3) * 32;
-                        mma_bf16(tO, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(uba + kk * 2048, DK * 128, 1024), iO,
-                                 kk > 0);
-                    }
-                }
-#pragma unroll
-                for (int kk = 0; kk < kC / 16; ++kk) {
-                    const uint64_t bv = sdesc_sw128(va + kk * 2048, kC * 128, 1024);
-                    mma_bf16(tU, sdesc_sw128(ka + kk * 2048, kC * 128, 1024), bv, iU, 1);
-                    mma_bf16(tU, sdesc_sw128(kloa + kk * 2048, kC * 128, 1024), bv, iU, 1);
-                }
-                mma_commit(u_done);
-                if (!state_mode) {
-                    if (!wait1(p_full, c & 1, abort_flag, g.status)) break;
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < kC / 16; ++kk)
-                        mma_bf16(tO, sdesc_sw128(pa + kk * 32, 16, 1024), sdesc_sw128(va + kk * 2048, kC * 128, 1024),
-                                 iO, 1);
-                    mma_commit(o_full);
-                }
-                // the stage is refilled only after the q' export read it
-                if (local_mode && p > 0) tma_store_wait_read();
-                mma_commit(&stage_empty[s]);
-            }
-            if (local_mode && p > 0) tma_store_wait_all();
-            // all MMAs this thread issued have completed before TMEM is released
+            // all MMAs issued have completed before TMEM is released
             mma_commit(td_bar);
             wait_slow(td_bar, 0, abort_flag, g.status, false);
         }
@@ -983,7 +1048,7 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == RL::MMAW) tmem_dealloc(tbase, L::NCOLS);
+    if (warp == RL::EPIW) tmem_dealloc(tbase, L::NCOLS);
 }
 
 // ---- host side ---------------------------------------------------------------
@@ -995,15 +1060,18 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
+    static std::atomic<EncodeTiledFn> fn{nullptr};
+    EncodeTiledFn f = fn.load(std::memory_order_acquire);
+    if (!f) {
         void *ptr = nullptr;
         cudaDriverEntryPointQueryResult qr;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &qr) == cudaSuccess &&
-            qr == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+            qr == cudaDriverEntryPointSuccess) {
+            f = reinterpret_cast<EncodeTiledFn>(ptr);
+            fn.store(f, std::memory_order_release);
+        }
     }
-    return fn;
+    return f;
 }
 
 }  // namespace
@@ -1036,45 +1104,35 @@ cudaError_t launch_t(const Plan &p, const int *cu, int mode, const void *q, cons
     bool ok = make_tma_map(&mq, q, BF, 2, DK, p.H, p.ntok, 64, kC, true) &&
               make_tma_map(&mk, k, BF, 2, DK, p.H, p.ntok, 64, kC, true) &&
               make_tma_map(&mv, v, BF, 2, DV, p.H, p.ntok, 64, kC, true);
+    // a and qn: L2 prefetch boxes of a whole chunk (the gate loads them itself)
     if (ok && !p.iso)
-        ok = make_tma_map(&ma, a, F32, 4, DK, p.H, p.ntok, DK, kRingTok, false) &&
-             make_tma_map(&mqn, qn, F32, 4, DK, p.H, p.ntok, DK, kRingTok, false);
+        ok = make_tma_map(&ma, a, F32, 4, DK, p.H, p.ntok, DK, kC, false) &&
+             make_tma_map(&mqn, qn, F32, 4, DK, p.H, p.ntok, DK, kC, false);
     else { ma = mq; mqn = mq; }
     if (ok && mode == 2) ok = make_tma_map(&mqs, p.qbuf, BF, 2, DK, p.H, p.ntok, 64, kC, true);
     else mqs = mq;
     if (!ok) return cudaErrorInvalidValue;
     if (mode != 0 && mode != 2) return cudaErrorInvalidValue;
-    static bool attr[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr[dev]) {
-        void (*const kerns[4])(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap,
-                               TcArgs) = {kla_chunk_tc_kernel<DK, DV, false, false>,
-                                          kla_chunk_tc_kernel<DK, DV, false, true>,
-                                          kla_chunk_tc_kernel<DK, DV, true, false>,
-                                          kla_chunk_tc_kernel<DK, DV, true, true>};
-        for (auto kern : kerns) {
-            const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::alloc);
-            if (e != cudaSuccess) return e;
-        }
-        attr[dev] = true;
-    }
+    static PerDevice<bool> attr[4];
+    void (*const kerns[4])(CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap, CUtensorMap,
+                           TcArgs) = {kla_chunk_tc_kernel<DK, DV, false, false>,
+                                      kla_chunk_tc_kernel<DK, DV, false, true>,
+                                      kla_chunk_tc_kernel<DK, DV, true, false>,
+                                      kla_chunk_tc_kernel<DK, DV, true, true>};
+    const int which = (p.iso ? 2 : 0) + (mode == 2 ? 1 : 0);
+    const cudaError_t e = ensure_smem_attr(attr[which], kerns[which], L::alloc);
+    if (e != cudaSuccess) return e;
     TcArgs g;
-    g.N = p.N; g.H = p.H; g.P = p.P; g.NB = p.NB; g.seg_blocks = p.seg_blocks; g.iso = p.iso; g.mode = mode;
+    g.N = p.N; g.H = p.H; g.P = p.P; g.NB = p.NB; g.seg_blocks = p.seg_blocks; g.NC = p.NB;
     g.T = p.T; g.Lseg = p.Lseg; g.cu = cu; g.perm = cu ? p.perm : nullptr;
     g.a = a; g.qn = qn; g.beta = beta; g.lambda0 = lambda0; g.eta0 = eta0; g.lam_blk = lam_blk;
     g.agg = p.inline_carry ? p.agg : nullptr;
-    g.rlog = p.rlog; g.NC = p.NB;
+    g.rlog = p.rlog;
     g.S_io = S_io; g.decay = decay; g.out = (__nv_bfloat16 *)out;
     g.final_lambda = final_lambda; g.final_eta = final_eta; g.status = status;
-    const long long segs = p.P;
-    const unsigned grid = (unsigned)((long long)p.N * p.H * segs);
+    const unsigned grid = (unsigned)((long long)p.N * p.H * p.P);
     if (grid == 0) return cudaSuccess;
-    auto kern = p.iso ? (mode == 2 ? kla_chunk_tc_kernel<DK, DV, true, true> : kla_chunk_tc_kernel<DK, DV, true, false>)
-                      : (mode == 2 ? kla_chunk_tc_kernel<DK, DV, false, true>
-                                   : kla_chunk_tc_kernel<DK, DV, false, false>);
-    return launch_pdl(kern, grid, Roles<DK, DV>::THREADS, L::alloc, st, mq, mk, mv, ma, mqn,
-                      mqs, g);
+    return launch_pdl(kerns[which], grid, Roles<DK, DV>::THREADS, L::alloc, st, mq, mk, mv, ma, mqn, mqs, g);
 }
 
 }  // namespace

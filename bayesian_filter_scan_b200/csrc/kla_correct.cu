@@ -8,20 +8,23 @@
 // G the cumulative log2 gate from the segment start. The chunk kernel (mode 2)
 // walks every segment from a zero start, writes the segment's transfer and gate
 // product, and exports its folded q tiles Q' = q/lambda 2^(G - rho) with the
-// log2 factor rlog = rho (per chunk and key) that takes them to the segment
-// start. Here: first the segment-start beliefs of every row,
+// log2 factor rlog = rho (per chunk, 16-token pass quarter and key) that takes
+// them to the segment start. Here: first the segment-start beliefs of every row,
 //     eta_start(1) = T_0, eta_start(q+1) = D_q eta_start(q) + T_q,
 // and the final belief D_{P-1} eta_start(P-1) + T_{P-1} (T_0 is segment 0's
 // end state from eta0; T_q, D_q the transfers and gate products); then, per
 // chunk of every segment p >= 1, on the tensor cores,
-//     out[chunk rows] += Q' (64 x dk) . diag(2^rlog) eta_start(p) (dk x dv).
+//     out[chunk rows] += Q' (64 x dk) . diag(2^rlog) eta_start(p) (dk x dv),
+// one product per chunk when its four quarters share their references (a
+// chunk the walk took in one pass), else one per quarter, each adding only its
+// quarter's rows.
 //
 // Correction CTA = a range of chunks of one (row, head, segment p >= 1), 128
 // threads, two per SM. Chunks whose operand diag(2^rlog) eta_start rounds to
 // zero for every key (the carried state has decayed below bf16 range there) add
 // exactly zero and are skipped. The Q' and output tiles of the others stream
 // through a 2-stage TMA ring; thread 0 issues the copies and the tcgen05 MMAs
-// into two TMEM accumulators; the operand is rebuilt in shared memory (bf16),
+// into a TMEM accumulator; the operand is rebuilt in shared memory (bf16),
 // the rows of the keys whose factor changed; all threads add the TMEM result to
 // the output tile in shared memory, which a TMA store writes back.
 // Every wait is bounded: on a timeout the status bit is set and the CTA stops
@@ -37,6 +40,7 @@ using namespace ptx;
 namespace {
 
 constexpr int kCC = 64;   // chunk tokens (the chunk kernel's)
+constexpr int kQ = 16;    // tokens per pass quarter (the chunk kernel's)
 constexpr uint64_t kCorrWaitNs = 2000000000ull;
 constexpr int kMaxRange = 256;   // chunks per correction CTA at most
 // log2 of a size below which bf16(2^rlog eta) rounds to zero, with margin
@@ -64,7 +68,7 @@ struct CLayout {
     static constexpr int bytes = bar0 + 8 * 8;
     static constexpr int alloc = bytes + 1024;
     static_assert(2 * (alloc + 1024) <= 233472, "two CTAs per SM");
-    static constexpr uint32_t NCOLS = 2 * DV;      // two fp32 accumulators (64 or 128 columns each)
+    static constexpr uint32_t NCOLS = (DV <= 32) ? 32u : (uint32_t)DV;   // one fp32 accumulator
 };
 
 __device__ __forceinline__ int csw_off(int row, int col, int rows) {
@@ -172,7 +176,8 @@ kla_correct_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
 
     float *lmax = reinterpret_cast<float *>(sm + L::m0);
     int *list = reinterpret_cast<int *>(sm + L::l0);
-    const float *rl = g.rlog + (u * g.NB + (long long)p * g.seg_blocks + c0) * DK;
+    // references of this range's chunks: rl[(chunk * kQuarters + quarter) * DK + key]
+    const float *rl = g.rlog + ((u * g.NB + (long long)p * g.seg_blocks + c0) * kQuarters) * DK;
     // short ranges take every chunk (the zero test would cost more than it saves)
     const bool test = nch > 2;
     // log2 max |eta_start| per key
@@ -187,7 +192,8 @@ kla_correct_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
     }
     __syncthreads();
     // The chunks whose operand diag(2^rlog) eta_start is not zero in bf16 for
-    // some key; the others add exactly zero and are skipped. list[0] = count.
+    // some key and quarter; the others add exactly zero and are skipped.
+    // list[0] = count.
     if (!test) {
         if (tid == 0) list[0] = nch;
         if (tid < nch) list[1 + tid] = tid;
@@ -197,7 +203,8 @@ kla_correct_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
             const int jj = j0 + lane;
             bool need = false;
             if (jj < nch)
-                for (int i = 0; i < DK; ++i) need |= __ldg(rl + jj * DK + i) + lmax[i] >= kZeroLog2;
+                for (int x = 0; x < kQuarters * DK; ++x)
+                    need |= __ldg(rl + (long long)jj * kQuarters * DK + x) + lmax[x % DK] >= kZeroLog2;
             const unsigned m = __ballot_sync(0xffffffffu, need);
             if (need) list[1 + cnt + __popc(m & ((1u << lane) - 1u))] = jj;
             cnt += __popc(m);
@@ -229,84 +236,96 @@ kla_correct_kernel(const __grid_constant__ CUtensorMap tm_qs, const __grid_const
     const int row64 = 16 * warp + lane;
     const bool v64 = lane < 16;
     bool ok = true;
-    float rnext = (tid < DK && nl2 > 0) ? __ldg(rl + list[1] * DK + tid) : 0.f;
+    int nmma = 0;   // MMAs committed so far (phases of mma_done[0])
     for (int k = 0; k < nl2; ++k) {
         const int s = k & 1, c = c0 + list[1 + k];
-        // rebuild the operand rows of the keys whose factor moved (thread = key);
-        // the previous chunk's MMA, the last reader, has completed
-        const float rnew = rnext;
-        if (tid < DK && k + 1 < nl2) rnext = __ldg(rl + list[2 + k] * DK + tid);
-        const bool changed = tid < DK && !(rnew == rcur[tid]);
-        if (__syncthreads_or(changed)) {
-            if (changed) {
-                rcur[tid] = rnew;
-                const float f = exp2f(rnew);
-                const float4 *src = reinterpret_cast<const float4 *>(Sst + tid * DV);
+        const float *rc = rl + (long long)list[1 + k] * kQuarters * DK;
+        // one group when the four quarters share their references, else one per quarter
+        bool same = true;
+        if (tid < DK)
+            for (int q = 1; q < kQuarters; ++q) same &= rc[q * DK + tid] == rc[tid];
+        const int ngr = __syncthreads_and(same) ? 1 : kQuarters;
+        if (!__syncthreads_and(cwait(&full[s], (k >> 1) & 1, g.status))) { ok = false; break; }
+        uint8_t *ot = sm + L::st0 + s * L::ST + L::QT;
+        for (int gi = 0; gi < ngr; ++gi) {
+            const int q0 = ngr == 1 ? 0 : gi, q1 = ngr == 1 ? kQuarters : gi + 1;
+            // rebuild the operand rows of the keys whose reference moved (thread =
+            // key); the previous MMA, the last reader, has completed
+            const float rnew = tid < DK ? rc[q0 * DK + tid] : 0.f;
+            const bool changed = tid < DK && !(rnew == rcur[tid]);
+            if (__syncthreads_or(changed)) {
+                if (changed) {
+                    rcur[tid] = rnew;
+                    const float f = exp2f(rnew);
+                    const float4 *src = reinterpret_cast<const float4 *>(Sst + tid * DV);
 #pragma unroll 4
-                for (int jj = 0; jj < DV; jj += 8) {
-                    const float4 a = __ldg(src + jj / 4), b = __ldg(src + jj / 4 + 1);
-                    uint4 w;
-                    w.x = cpack_bf2(f * a.x, f * a.y); w.y = cpack_bf2(f * a.z, f * a.w);
-                    w.z = cpack_bf2(f * b.x, f * b.y); w.w = cpack_bf2(f * b.z, f * b.w);
-                    *reinterpret_cast<uint4 *>(Bt + csw_off(tid, jj, DK)) = w;
+                    for (int jj = 0; jj < DV; jj += 8) {
+                        const float4 a = __ldg(src + jj / 4), b = __ldg(src + jj / 4 + 1);
+                        uint4 w;
+                        w.x = cpack_bf2(f * a.x, f * a.y); w.y = cpack_bf2(f * a.z, f * a.w);
+                        w.z = cpack_bf2(f * b.x, f * b.y); w.w = cpack_bf2(f * b.z, f * b.w);
+                        *reinterpret_cast<uint4 *>(Bt + csw_off(tid, jj, DK)) = w;
+                    }
                 }
+                fence_proxy_async();
+                __syncthreads();
             }
-            fence_proxy_async();
-            __syncthreads();
-        }
-        // D_s[64 x DV] = Q'[64 x DK] . B[DK x DV]
-        if (tid == 0) {
-            if (!cwait(&full[s], (k >> 1) & 1, g.status)) ok = false;
-            else {
+            // D[64 x DV] = Q'[64 x DK] . B[DK x DV]
+            if (tid == 0) {
                 tc_fence_after();
                 const uint32_t qa = smem_u32(sm + L::st0 + s * L::ST), ba = smem_u32(Bt);
 #pragma unroll
                 for (int kk = 0; kk < DK / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * (kCC * 128) + (kk & 3) * 32;
-                    mma_bf16(tbase + s * DV, sdesc_sw128(qa + off, 16, 1024),
-                             sdesc_sw128(ba + kk * 2048, DK * 128, 1024), idesc, kk > 0);
+                    mma_bf16(tbase, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ba + kk * 2048, DK * 128, 1024),
+                             idesc, kk > 0);
                 }
-                mma_commit(&mma_done[s]);
+                mma_commit(&mma_done[0]);
             }
-        }
-        if (!__syncthreads_and(ok)) break;
-        if (!__syncthreads_and(cwait(&mma_done[s], (k >> 1) & 1, g.status))) { ok = false; break; }
-        tc_fence_after();
-        // add the carried-state readout to the output tile in shared memory
-        uint8_t *ot = sm + L::st0 + s * L::ST + L::QT;
-        const bool row_ok = v64 && tb + (long long)c * kCC + row64 < te;
+            if (!__syncthreads_and(cwait(&mma_done[0], nmma & 1, g.status))) { ok = false; break; }
+            ++nmma;
+            tc_fence_after();
+            // add the carried-state readout of this group's rows to the output tile
+            const bool row_ok = v64 && row64 >= kQ * q0 && row64 < kQ * q1 && tb + (long long)c * kCC + row64 < te;
 #pragma unroll
-        for (int cb = 0; cb < DV / 32; cb += 2) {
-            uint32_t rr[2][32];
-            tmem_ld32(tbase + s * DV + lane_base + cb * 32, rr[0]);
-            tmem_ld32(tbase + s * DV + lane_base + cb * 32 + 32, rr[1]);
-            tmem_wait_ld();
-            if (row_ok) {
+            for (int cb = 0; cb < DV / 32; cb += 2) {
+                uint32_t rr[2][32];
+                tmem_ld32(tbase + lane_base + cb * 32, rr[0]);
+                tmem_ld32(tbase + lane_base + cb * 32 + 32, rr[1]);
+                tmem_wait_ld();
+                if (row_ok) {
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
+                    for (int hh = 0; hh < 2; ++hh) {
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(ot + csw_off(row64, (cb + hh) * 32 + q4 * 8, kCC));
-                        const uint4 o = *dst;
-                        const uint32_t ow[4] = {o.x, o.y, o.z, o.w};
-                        uint32_t nw[4];
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            uint4 *dst = reinterpret_cast<uint4 *>(ot + csw_off(row64, (cb + hh) * 32 + q4 * 8, kCC));
+                            const uint4 o = *dst;
+                            const uint32_t ow[4] = {o.x, o.y, o.z, o.w};
+                            uint32_t nw[4];
 #pragma unroll
-                        for (int x = 0; x < 4; ++x) {
-                            const float lo = __uint_as_float(ow[x] << 16) + __uint_as_float(rr[hh][q4 * 8 + 2 * x]);
-                            const float hi =
-                                __uint_as_float(ow[x] & 0xffff0000u) + __uint_as_float(rr[hh][q4 * 8 + 2 * x + 1]);
-                            nw[x] = cpack_bf2(lo, hi);
+                            for (int x = 0; x < 4; ++x) {
+                                const float lo = __uint_as_float(ow[x] << 16) + __uint_as_float(rr[hh][q4 * 8 + 2 * x]);
+                                const float hi =
+                                    __uint_as_float(ow[x] & 0xffff0000u) + __uint_as_float(rr[hh][q4 * 8 + 2 * x + 1]);
+                                nw[x] = cpack_bf2(lo, hi);
+                            }
+                            *dst = make_uint4(nw[0], nw[1], nw[2], nw[3]);
                         }
-                        *dst = make_uint4(nw[0], nw[1], nw[2], nw[3]);
                     }
                 }
             }
+            tc_fence_before();
+            __syncthreads();
         }
-        tc_fence_before();
+        if (!ok) break;
         fence_proxy_async();
         __syncthreads();
         if (tid == 0) {
-            // write the tile back; its stage is reloaded once the store has read it
+            // Write the tile back; its stage is reloaded once the store has read it.
+            // The tile's rows past the segment end (a last partial chunk) were
+            // loaded and are stored back unchanged: they are the first tokens of
+            // the next row, which only segment 0 of that row writes, in the walk
+            // launch that finished before this one.
             const int tok = (int)(tb + (long long)c * kCC);
 #pragma unroll
             for (int a = 0; a < DV / 64; ++a) tma_store_3d(&tm_o, ot + a * kCC * 128, 64 * a, h, tok);
@@ -339,15 +358,9 @@ cudaError_t launch_correct_t(const Plan &p, const float *S_io, void *out, int *s
     if (!make_tma_map(&mqs, p.qbuf, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DK, p.H, p.ntok, 64, kCC, true) ||
         !make_tma_map(&mo, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, DV, p.H, p.ntok, 64, kCC, true))
         return cudaErrorInvalidValue;
-    static bool attr[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(kla_correct_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             L::alloc);
-        if (e != cudaSuccess) return e;
-        attr[dev] = true;
-    }
+    static PerDevice<bool> attr;
+    const cudaError_t ea = ensure_smem_attr(attr, kla_correct_kernel<DK, DV>, L::alloc);
+    if (ea != cudaSuccess) return ea;
     CorrArgs g;
     g.H = p.H; g.P = p.P; g.NB = p.NB; g.seg_blocks = p.seg_blocks; g.iso = p.iso;
     g.T = p.T; g.Lseg = p.Lseg;

@@ -16,6 +16,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <utility>
 
 namespace kla {
@@ -24,6 +25,37 @@ constexpr int kBlockTokens = 64;   // Lb: tokens per Moebius-reduction block (on
 constexpr int kChunk = 64;         // C: tokens per chunk of the chunked form
 constexpr int kMaxOrderSeqs = 1024; // packed sequences ranked by length for the launch order
 constexpr int kInlineCarryBlocks = 64; // at most this many blocks before a segment: carry in the walk kernel
+constexpr int kQuarters = 4;       // pass quarters per chunk: the chunk kernel's finest reference granularity
+                                   // (16 tokens, the token step of its tensor-core contractions)
+constexpr int kMaxDevices = 64;
+
+// Host state kept once per device (symbol addresses, function attributes).
+// Entries are atomics, so first calls that race from several host threads
+// store the same value without a data race.
+template <typename T>
+struct PerDevice {
+    std::atomic<T> v[kMaxDevices];
+    PerDevice() {
+        for (auto &x : v) x.store(T{}, std::memory_order_relaxed);
+    }
+};
+
+// The current device, or -1 if there is none or its index is out of range.
+inline int current_device() {
+    int d = -1;
+    if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kMaxDevices) return -1;
+    return d;
+}
+
+// Sets the dynamic shared-memory limit of `kern` once per device.
+template <typename K>
+inline cudaError_t ensure_smem_attr(PerDevice<bool> &done, K kern, int bytes) {
+    const int dev = current_device();
+    if (dev >= 0 && done.v[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess && dev >= 0) done.v[dev].store(true, std::memory_order_release);
+    return e;
+}
 
 // Bits of the library's device status word (kla_check reads and clears it);
 // kernels that can detect an error receive its address and OR a bit into it.
@@ -55,8 +87,9 @@ struct Plan {
     const float4 *agg;
     // split rows on the tensor-core path: segments walk from a zero state and a
     // correction pass adds the carried state; the walk exports its folded q
-    // tiles (qbuf [Ntok, H, dk] bf16) and per-chunk log2 factors (rlog
-    // [N*H][NB][dk] fp32), in the workspace at off_qbuf / off_rlog
+    // tiles (qbuf [Ntok, H, dk] bf16) and the log2 reference of every pass
+    // quarter of every chunk (rlog [N*H][NB][kQuarters][dk] fp32), in the
+    // workspace at off_qbuf / off_rlog
     bool local;
     size_t off_qbuf, off_rlog;
     void *qbuf;

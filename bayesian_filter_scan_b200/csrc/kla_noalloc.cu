@@ -20,15 +20,15 @@ __device__ __align__(256) unsigned char g_noalloc_scratch[KLA_NOALLOC_SCRATCH_BY
 // the array's name is only a host-side stand-in, so its device address must be
 // taken with cudaGetSymbolAddress while that device is current.
 void *scratch_address() {
-    static void *addr[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (!addr[dev]) {
-        void *p = nullptr;
+    static kla::PerDevice<void *> addr;
+    const int dev = kla::current_device();
+    if (dev < 0) return nullptr;
+    void *p = addr.v[dev].load(std::memory_order_acquire);
+    if (!p) {
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
-        addr[dev] = p;
+        addr.v[dev].store(p, std::memory_order_release);
     }
-    return addr[dev];
+    return p;
 }
 
 }  // namespace

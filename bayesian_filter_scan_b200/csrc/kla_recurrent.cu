@@ -213,15 +213,9 @@ kla_walk_simt(WalkArgs w) {
 template <typename TIn, int KPG>
 static cudaError_t launch_walk_t(const WalkArgs &w, unsigned grid, cudaStream_t st) {
     size_t smem = walk_smem_bytes(w.dk, w.dv);
-    static bool attr_set[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr_set[dev]) {
-        cudaError_t e = cudaFuncSetAttribute(kla_walk_simt<TIn, KPG>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, 64 * 1024);
-        if (e != cudaSuccess) return e;
-        attr_set[dev] = true;
-    }
+    static PerDevice<bool> attr;
+    const cudaError_t e = ensure_smem_attr(attr, kla_walk_simt<TIn, KPG>, 64 * 1024);
+    if (e != cudaSuccess) return e;
     return launch_pdl(kla_walk_simt<TIn, KPG>, grid, kWalkThreads, smem, st, w);
 }
 

@@ -496,16 +496,11 @@ cudaError_t launch_mobius_reduce(const Plan &p, const void *k, const float *a, c
         !make_tma_map(&mk, k, KT, kes, p.dk, p.H, p.ntok, dki, kBlockTokens, false))
         return cudaErrorInvalidValue;
     const int smem = kRedStages * red_stage_bytes(dki, kes) + kRedSub * 64 * 16 + 2 * kRedStages * 8;
-    static bool attr[2][64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 64 && !attr[kes == 2][dev]) {
-        // the largest request (64-key items) once per device and input type
-        const int smax = kRedStages * red_stage_bytes(64, kes) + kRedSub * 64 * 16 + 2 * kRedStages * 8;
-        cudaError_t e = cudaFuncSetAttribute(mobius_reduce_tma<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, smax);
-        if (e != cudaSuccess) return e;
-        attr[kes == 2][dev] = true;
-    }
+    // the largest request (64-key items) once per device and input type
+    static PerDevice<bool> attr;
+    const int smax = kRedStages * red_stage_bytes(64, kes) + kRedSub * 64 * 16 + 2 * kRedStages * 8;
+    const cudaError_t ea = ensure_smem_attr(attr, mobius_reduce_tma<TIn>, smax);
+    if (ea != cudaSuccess) return ea;
     const long long nitems = pairs * nhalf;
     // the kernel indexes items and tokens in 32 bits (TMA coordinates are 32-bit too)
     if (nitems >= (1LL << 31) || p.ntok >= (1LL << 31)) return cudaErrorInvalidValue;

@@ -46,6 +46,8 @@ class Workload:
     len_hi: int = 8192
     final_state: bool = False    # the workload asks for final_lambda/final_eta
     seed: int = 0
+    iso_sigmoid: bool = False    # isotropic mode: a = sigmoid(N(a_mu, 1)), qn = softplus(N(qn_mu, 1))
+                                 # per (t,h) instead of the near-unit stress gates
 
     @property
     def tokens(self) -> int:
@@ -101,7 +103,11 @@ def make_inputs(w: Workload, seed: Optional[int] = None) -> dict:
     q = unit_rows(torch.randn(N_tok, H, dk, generator=gen)).to(io)
     k = unit_rows(torch.randn(N_tok, H, dk, generator=gen)).to(io)
     v = torch.randn(N_tok, H, dv, generator=gen).to(io)
-    if w.mode == "iso":
+    if w.mode == "iso" and w.iso_sigmoid:
+        a = torch.sigmoid(w.a_mu + torch.randn(N_tok, H, generator=gen))
+        qn = torch.nn.functional.softplus(w.qn_mu + torch.randn(N_tok, H, generator=gen))
+        beta = torch.sigmoid(torch.randn(N_tok, H, generator=gen))
+    elif w.mode == "iso":
         a = 1.0 - 1e-4 * torch.rand(N_tok, H, generator=gen)
         qn = torch.full((N_tok, H), 1e-4)
         lo, hi = math.log(0.5), math.log(8.0)

@@ -6,6 +6,8 @@ Bar (per element, out / final_lambda / final_eta / lambda trajectory):
 with tol = 2e-2 for bf16 inputs (fp32 accumulation, bf16 tensor-core operands)
 and tol = 1e-4 for fp32 inputs.
 """
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -19,9 +21,15 @@ pytestmark = pytest.mark.gpu
 TOL = {"bf16": 2e-2, "fp32": 1e-4}
 
 
+# max scaled error of every comparison, printed in the session summary
+ERRORS = []
+
+
 def close(got, want, tol, what=""):
     got = got.detach().float().cpu().numpy().astype(np.float64) if hasattr(got, "detach") else got
     err = np.abs(got - want) / (1.0 + np.abs(want))
+    test = os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0].split("::")[-1]
+    ERRORS.append((test, what, float(np.nanmax(err)) if err.size else 0.0, tol))
     bad = ~(err <= tol)
     assert not bad.any(), "%s: %d/%d elements off, max scaled err %.3g at %s" % (
         what, int(bad.sum()), bad.size, float(np.nanmax(err)), np.unravel_index(np.nanargmax(err), err.shape))
