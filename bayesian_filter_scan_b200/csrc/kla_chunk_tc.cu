@@ -67,6 +67,7 @@ constexpr int kC = 64;        // chunk tokens
 constexpr int kQ = 16;        // tokens per pass quarter
 constexpr int kLim = 80;      // |G - rho| (log2) a pass keeps inside the exponent window
 constexpr int kStick = 48;    // the reference stays while the range fits [rho - kStick, rho + kStick]
+constexpr int kLost = 100;    // the fold against the reference in force is exact while |G - rho| <= kLost
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kGateBar = 1;   // named barrier of the gate warps
 constexpr int kEpiBar = 2;    // named barrier of the epilogue warps
@@ -89,6 +90,7 @@ struct TcArgs {
     const int *cu, *perm;
     const float *a, *qn, *beta;
     const float *lambda0, *eta0, *lam_blk;
+    const void *q, *k;   // inputs (the strong-forgetting re-walk reloads them)
     const float4 *agg;   // block aggregates when the segment-start precision is composed here
     float *S_io, *decay;
     __nv_bfloat16 *out;
@@ -111,7 +113,7 @@ struct Layout {
     static constexpr int v0 = k0 + 2 * QK;
     static constexpr int klo0 = v0 + 2 * V;          // low bf16 part of K' (state update), per stage
     static constexpr int p0 = klo0 + 2 * QK;
-    static constexpr int ub0 = p0 + PT;
+    static constexpr int ub0 = p0 + 2 * PT;         // (P double-buffered by pass)
     static constexpr int xch0 = ub0 + UB;            // [NSUB][DK] {float4 matrix, float4 {PA, EM, FM, -}}
     static constexpr int rng0 = xch0 + XN * 32;      // [NSUB][DK] int2 G range
     static constexpr int car0 = rng0 + XN * 8;       // [2][DK] chunk-start state {float4 n,d,pa; int4 E,F}
@@ -120,14 +122,15 @@ struct Layout {
     static constexpr int isof0 = facf0 + DK * 4;     // [2][kC] float2: iso per-token factors
     static constexpr int lvl0 = isof0 + 2 * kC * 8;  // int[2]: pass level of the chunk, tagged with its index
     static constexpr int bar0 = lvl0 + 16;
-    static constexpr int NBAR = 8;
+    static constexpr int NBAR = 9;
     static constexpr int hold0 = bar0 + NBAR * 8;
     static constexpr int bytes = hold0 + 16;
     static constexpr int alloc = bytes + 1024;
     static_assert(alloc <= 232448, "shared memory per CTA");
     static_assert(Roles<DK, DV>::MIN_BLOCKS == 1 || 2 * (alloc + 1024) <= 233472, "two CTAs per SM");
-    static constexpr uint32_t NCOLS = (2 * DV + 64 <= 256) ? 256u : 512u;
-    static constexpr uint32_t colU = 0, colO = DV, colS = 2 * DV;
+    // TMEM columns: the state U, two output accumulators (by pass), the scores
+    static constexpr uint32_t NCOLS = (3 * DV + 64 <= 256) ? 256u : 512u;
+    static constexpr uint32_t colU = 0, colO = DV, colS = 3 * DV;
 };
 
 // Byte offset of element (row, col) in a 128B-swizzled bf16 tile stored as
@@ -149,6 +152,25 @@ __device__ __forceinline__ int expo(float x) { return ((__float_as_int(x) >> 23)
 // 2^e for e in [-126, 127]
 __device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
 __device__ __forceinline__ int clampe(int e) { return max(-126, min(126, e)); }
+// Multiplies the DV state columns of this thread's TMEM lane by 2^d (the
+// reference of the lane's key moved). Warp-collective (every lane calls it, d
+// = 0 where nothing moves). Out of line: it is rare, and keeping it out of
+// the epilogue's loop body keeps the hot code small.
+template <int DV>
+__device__ __noinline__ void tmem_scale_lane(uint32_t taddr, int d) {
+    const float f1 = pow2i(d / 2), f2 = pow2i(d - d / 2);
+#pragma unroll 1
+    for (int cb = 0; cb < DV / 32; ++cb) {
+        uint32_t r[32];
+        tmem_ld32(taddr + cb * 32, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(__uint_as_float(r[x]) * f1 * f2);
+        tmem_st32(taddr + cb * 32, r);
+    }
+    tmem_wait_st();
+}
+
 // R[q] for a runtime q without indexing the array (it stays in registers)
 __device__ __forceinline__ int pick4(const int (&R)[4], int q) {
     return q == 0 ? R[0] : (q == 1 ? R[1] : (q == 2 ? R[2] : R[3]));
@@ -265,6 +287,56 @@ __device__ __forceinline__ void norm_state(float &n, float &d, float &pa, int &E
     F += f;
 }
 
+// The strong-forgetting path of the diagonal gate: walks a sub-block of SL
+// tokens again from its start state and folds every token against the
+// references R0, R1 of its two keys (a, qn, beta, q, k reloaded from global
+// memory: the tile words were overwritten by the provisional fold). Out of line:
+// it runs only when a provisional fold lost bits.
+template <int DK, int SL>
+__device__ __noinline__ void rewalk_fold(uint8_t *qt, uint8_t *kt, uint8_t *klo, int cbase, float2 n2s, float2 d2s,
+                                         float2 p2s, int Ew0, int Ew1, int Fw0, int Fw1, int R0, int R1,
+                                         const float *a, const float *qn, const float *beta, const __nv_bfloat16 *q,
+                                         const __nv_bfloat16 *k, long long tok0, int nval, int H, int h, int i0) {
+    int e0 = clampe(Fw0 - Ew0 - R0), e1 = clampe(Fw1 - Ew1 - R1);
+    float2 mq = make_float2(pow2i(e0), pow2i(e1)), mk = make_float2(pow2i(-e0), pow2i(-e1));
+#pragma unroll 1
+    for (int r = 0; r < SL; ++r) {
+        const long long tok = tok0 + r;
+        const long long off = (tok * H + h) * DK + i0;
+        float2 ar = make_float2(1.f, 1.f), qr = make_float2(0.f, 0.f), kf = qr, qf = qr;
+        float be = 0.f;
+        if (r < nval) {
+            ar = __ldg(reinterpret_cast<const float2 *>(a + off));
+            qr = __ldg(reinterpret_cast<const float2 *>(qn + off));
+            kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(k + off));
+            qf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(q + off));
+            be = __ldg(beta + tok * H + h);
+        }
+        const float2 bk = f2mul(make_float2(be, be), kf);
+        d2s = f2fma(f2mul(ar, ar), d2s, f2mul(qr, n2s));
+        n2s = f2fma(f2mul(bk, kf), d2s, n2s);
+        p2s = f2mul(p2s, ar);
+        const float2 pn = f2mul(p2s, n2s);
+        const float2 rc = make_float2(__frcp_rn(pn.x), __frcp_rn(pn.y));
+        const float2 qo = f2mul(f2mul(f2mul(qf, p2s), f2mul(p2s, rc)), mq);
+        const float2 ko = f2mul(bk, f2mul(f2mul(d2s, f2mul(n2s, rc)), mk));
+        const uint32_t kh = pack_bf2(ko.x, ko.y);
+        const float2 khf = unpack_bf2(kh);
+        const int o = (cbase + r * 128) ^ ((r & 7) << 4);
+        *reinterpret_cast<uint32_t *>(qt + o) = pack_bf2(qo.x, qo.y);
+        *reinterpret_cast<uint32_t *>(kt + o) = kh;
+        *reinterpret_cast<uint32_t *>(klo + o) = pack_bf2(ko.x - khf.x, ko.y - khf.y);
+        if ((r & 7) == 7) {
+            norm_state(n2s.x, d2s.x, p2s.x, Ew0, Fw0);
+            norm_state(n2s.y, d2s.y, p2s.y, Ew1, Fw1);
+            e0 = clampe(Fw0 - Ew0 - R0);
+            e1 = clampe(Fw1 - Ew1 - R1);
+            mq = make_float2(pow2i(e0), pow2i(e1));
+            mk = make_float2(pow2i(-e0), pow2i(-e1));
+        }
+    }
+}
+
 }  // namespace
 
 template <int DK, int DV, bool ISO, bool LOCAL>
@@ -281,7 +353,10 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::bar0);
     uint64_t *stage_full = bars + 0, *qk_ready = bars + 2;
-    uint64_t *s_full = bars + 4, *u_done = bars + 5, *o_full = bars + 6, *td_bar = bars + 7;
+    // o_full[b]: the MMAs of the pass that used output accumulator b (one barrier
+    // per accumulator, so that a pass's completion is waited for before the
+    // barrier can complete again)
+    uint64_t *s_full = bars + 4, *u_done = bars + 5, *td_bar = bars + 6, *o_full = bars + 7;
     uint32_t *tmem_hold = reinterpret_cast<uint32_t *>(sm + L::hold0);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::hold0 + 4);
     int *lvl = reinterpret_cast<int *>(sm + L::lvl0);
@@ -298,7 +373,8 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
         mbar_init(s_full, 1);
         mbar_init(u_done, 1);
-        mbar_init(o_full, 1);
+        mbar_init(&o_full[0], 1);
+        mbar_init(&o_full[1], 1);
         mbar_init(td_bar, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -362,54 +438,68 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // ================= gate warps: precision path and operand folding =====
         bool ok = true;
         if constexpr (!ISO) {
-            constexpr int NSUB = RL::NSUB, SL = RL::SL;
-            float4 *xch = reinterpret_cast<float4 *>(sm + L::xch0);   // [(s*DK + i)*2 + {0,1}]
-            int2 *rng = reinterpret_cast<int2 *>(sm + L::rng0);        // [s*DK + i]
-            float4 *carf = reinterpret_cast<float4 *>(sm + L::car0);   // [(par*DK + i)*2]
-            int4 *cari = reinterpret_cast<int4 *>(sm + L::car0);       // [(par*DK + i)*2 + 1]
+            constexpr int NSUB = RL::NSUB, SL = RL::SL, NP = DK / 2;
             const int s = (DK == 128) ? (warp >> 1) : warp;           // sub-block
-            const int i0 = 2 * ((DK == 128) ? ((warp & 1) * 32 + lane) : lane);   // first key of the pair
+            const int pr = (DK == 128) ? ((warp & 1) * 32 + lane) : lane;   // key pair
+            const int i0 = 2 * pr;
             const int quarter = (SL * s) / kQ;                        // pass quarter of this sub-block
+            // exchange buffers, one float2 (the pair's two keys) per entry, so that a
+            // warp's accesses are consecutive 8-byte words:
+            //   sub-block maps  xch[(comp * NSUB + sub) * NP + pair], comp = n1 n2 d1 d2 PA EM FM
+            //   chunk-start state car[(comp * 2 + parity) * NP + pair], comp = n d pa E F
+            //   G ranges        rng[sub * NP + pair] = {lo, hi} of both keys, relative to rho
+            float2 *xch = reinterpret_cast<float2 *>(sm + L::xch0);
+            float2 *car = reinterpret_cast<float2 *>(sm + L::car0);
+            int4 *rng = reinterpret_cast<int4 *>(sm + L::rng0);
+            auto X = [&](int comp, int sj) -> float2 & { return xch[(comp * NSUB + sj) * NP + pr]; };
+            auto CAR = [&](int comp, int par) -> float2 & { return car[(comp * 2 + par) * NP + pr]; };
+            auto i2f = [](int x, int y) { return make_float2(__int_as_float(x), __int_as_float(y)); };
             // byte offset of (row SL*s + r, keys i0, i0+1) in a swizzled tile: the
             // sub-block starts on a multiple of 8 rows, so row & 7 = r & 7
-            const int obase = (i0 >> 6) * (kC * 128) + (SL * s) * 128 + ((i0 & 7) << 1);
-            const int ochunk = ((i0 & 63) >> 3) << 4;
-            auto offr = [&](int r) { return obase + r * 128 + ((ochunk ^ ((r & 7) << 4)) & 0x70); };
+            // (bits 4-6 of a row's base are zero, so the swizzled 16-byte chunk
+            // index can be XORed into the sum)
+            const int cbase = ((i0 >> 6) * (kC * 128) + (SL * s) * 128 + ((i0 & 7) << 1)) | (((i0 & 63) >> 3) << 4);
+            auto offr = [&](int r) { return (cbase + r * 128) ^ ((r & 7) << 4); };
             if (s == 0) {
                 // the belief at the segment start, as the first chunk's start state
-                for (int j = 0; j < 2; ++j) {
-                    carf[(0 * DK + i0 + j) * 2] = make_float4(seg_lambda(i0 + j), 1.f, 1.f, 0.f);
-                    cari[(0 * DK + i0 + j) * 2 + 1] = make_int4(0, 0, 0, 0);
-                }
+                CAR(0, 0) = make_float2(seg_lambda(i0), seg_lambda(i0 + 1));
+                CAR(1, 0) = make_float2(1.f, 1.f);
+                CAR(2, 0) = make_float2(1.f, 1.f);
+                CAR(3, 0) = i2f(0, 0);
+                CAR(4, 0) = i2f(0, 0);
             }
             int rho0 = 0, rho1 = 0;          // references in force (segment-start frame)
-            float2 av[SL], qv[SL];           // a, qn of the sub-block
-            float bl = 0.f;                  // beta of token SL*s + lane (lanes < SL)
-            auto load_tok = [&](int c, int r) {
-                const long long tok = tb + (long long)c * kC + SL * s + r;
-                if (tok < te) {
-                    const long long off = (tok * g.H + h) * DK + i0;
-                    av[r] = __ldg(reinterpret_cast<const float2 *>(g.a + off));
-                    qv[r] = __ldg(reinterpret_cast<const float2 *>(g.qn + off));
+            float2 av[SL], qv[SL];           // a, qn of the sub-block's tokens
+            float bl = 0.f, bln = 0.f;       // beta of token SL*s + lane (lanes < SL): this chunk, next
+            // a, qn of token r of this thread's sub-block in chunk c (identity step
+            // past the segment end); the addresses step by H * DK floats per token
+            const long long tstep = (long long)g.H * (DK / 2);   // in float2
+            auto load_tok = [&](int c, int r, float2 &ra, float2 &rq) {
+                const long long t0s = tb + (long long)c * kC + SL * s;
+                const long long off = ((t0s * g.H + h) * DK + i0) / 2 + r * tstep;
+                if (t0s + r < te) {
+                    ra = __ldg(reinterpret_cast<const float2 *>(g.a) + off);
+                    rq = __ldg(reinterpret_cast<const float2 *>(g.qn) + off);
                 } else {
-                    av[r] = make_float2(1.f, 1.f);
-                    qv[r] = make_float2(0.f, 0.f);
+                    ra = make_float2(1.f, 1.f);
+                    rq = make_float2(0.f, 0.f);
                 }
             };
             auto load_beta = [&](int c) {
                 const long long tok = tb + (long long)c * kC + SL * s + lane;
-                bl = (lane < SL && tok < te) ? __ldg(g.beta + tok * g.H + h) : 0.f;
+                return (lane < SL && tok < te) ? __ldg(g.beta + tok * g.H + h) : 0.f;
             };
             if (nchunks > 0) {
 #pragma unroll
-                for (int r = 0; r < SL; ++r) load_tok(0, r);
-                load_beta(0);
+                for (int r = 0; r < SL; ++r) load_tok(0, r, av[r], qv[r]);
+                bl = load_beta(0);
             }
             float lam_end0 = 0.f, lam_end1 = 0.f, gend0 = 1.f, gend1 = 1.f;
             int xend0 = 0, xend1 = 0;
             for (int c = 0; c < nchunks; ++c) {
                 const int st = c & 1;
                 const long long tok0 = tb + (long long)c * kC;
+                const int nval = (int)min((long long)SL, max(0LL, te - (tok0 + SL * s)));   // valid tokens of the sub-block
                 uint8_t *qt = sm + L::q0 + st * L::QK;
                 uint8_t *kt = sm + L::k0 + st * L::QK;
                 uint8_t *klo = sm + L::klo0 + st * L::QK;
@@ -417,116 +507,170 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 // ---- step 1: the sub-block's Moebius maps for both keys (columns
                 // are the images of (1, 0) and (0, 1); chain d <- a^2 d + qn n,
                 // n <- n + b d with b = beta k^2), and its product of a
-                float2 n1 = make_float2(1.f, 1.f), d1 = make_float2(0.f, 0.f);
-                float2 n2 = make_float2(0.f, 0.f), d2 = make_float2(1.f, 1.f), PA = make_float2(1.f, 1.f);
-                int em0 = 0, em1 = 0, fm0 = 0, fm1 = 0;
                 if (okw) {
+                    float2 n1 = make_float2(1.f, 1.f), d1 = make_float2(0.f, 0.f);
+                    float2 n2 = make_float2(0.f, 0.f), d2 = make_float2(1.f, 1.f), PA = make_float2(1.f, 1.f);
+                    int em0 = 0, em1 = 0, fm0 = 0, fm1 = 0;
 #pragma unroll
-                    for (int r = 0; r < SL; ++r) {
-                        const float2 kf = unpack_bf2(*reinterpret_cast<const uint32_t *>(kt + offr(r)));
-                        const float be = __shfl_sync(0xffffffffu, bl, r);
-                        const float2 a2 = f2mul(av[r], av[r]);
-                        const float2 b = f2mul(f2mul(make_float2(be, be), kf), kf);
-                        d1 = f2fma(a2, d1, f2mul(qv[r], n1));
-                        n1 = f2fma(b, d1, n1);
-                        d2 = f2fma(a2, d2, f2mul(qv[r], n2));
-                        n2 = f2fma(b, d2, n2);
-                        PA = f2mul(PA, av[r]);
-                        if ((r & 7) == 7) {
-                            norm_cols(n1.x, n2.x, d1.x, d2.x, em0);
-                            norm_cols(n1.y, n2.y, d1.y, d2.y, em1);
-                            const int f0 = clampe(expo(PA.x)), f1 = clampe(expo(PA.y));
-                            PA.x *= pow2i(-f0); PA.y *= pow2i(-f1);
-                            fm0 += f0; fm1 += f1;
+                    for (int b8 = 0; b8 < SL; b8 += 8) {
+                        uint32_t kwb[8];
+#pragma unroll
+                        for (int x = 0; x < 8; ++x) kwb[x] = *reinterpret_cast<const uint32_t *>(kt + offr(b8 + x));
+#pragma unroll
+                        for (int x = 0; x < 8; ++x) {
+                            const int r = b8 + x;
+                            const float2 kf = unpack_bf2(kwb[x]);
+                            const float be = __shfl_sync(0xffffffffu, bl, r);
+                            const float2 a2 = f2mul(av[r], av[r]);
+                            const float2 b = f2mul(f2mul(make_float2(be, be), kf), kf);
+                            d1 = f2fma(a2, d1, f2mul(qv[r], n1));
+                            n1 = f2fma(b, d1, n1);
+                            d2 = f2fma(a2, d2, f2mul(qv[r], n2));
+                            n2 = f2fma(b, d2, n2);
+                            PA = f2mul(PA, av[r]);
                         }
+                        norm_cols(n1.x, n2.x, d1.x, d2.x, em0);
+                        norm_cols(n1.y, n2.y, d1.y, d2.y, em1);
+                        const int f0 = clampe(expo(PA.x)), f1 = clampe(expo(PA.y));
+                        PA.x *= pow2i(-f0); PA.y *= pow2i(-f1);
+                        fm0 += f0; fm1 += f1;
                     }
-                    xch[(s * DK + i0) * 2] = make_float4(n1.x, n2.x, d1.x, d2.x);
-                    xch[(s * DK + i0) * 2 + 1] = make_float4(PA.x, __int_as_float(em0), __int_as_float(fm0), 0.f);
-                    xch[(s * DK + i0 + 1) * 2] = make_float4(n1.y, n2.y, d1.y, d2.y);
-                    xch[(s * DK + i0 + 1) * 2 + 1] = make_float4(PA.y, __int_as_float(em1), __int_as_float(fm1), 0.f);
+                    X(0, s) = n1; X(1, s) = n2; X(2, s) = d1; X(3, s) = d2; X(4, s) = PA;
+                    X(5, s) = i2f(em0, em1);
+                    X(6, s) = i2f(fm0, fm1);
                 }
                 if (named_bar_or(kGateBar, RL::GT, !okw || *abort_flag)) { ok = false; break; }
                 // ---- step 2: the state at this sub-block's start: the chunk-start
                 // state with the maps of the sub-blocks before it applied
                 float nn[2], dd[2], pa[2];
                 int E[2], F[2];
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const float4 cf = carf[(st * DK + i0 + j) * 2];
-                    const int4 ci = cari[(st * DK + i0 + j) * 2 + 1];
-                    nn[j] = cf.x; dd[j] = cf.y; pa[j] = cf.z; E[j] = ci.x; F[j] = ci.y;
-                    for (int sj = 0; sj < s; ++sj) {
-                        const float4 m = xch[(sj * DK + i0 + j) * 2];
-                        const float4 x = xch[(sj * DK + i0 + j) * 2 + 1];
-                        const float n2v = fmaf(m.x, nn[j], m.y * dd[j]);
-                        const float d2v = fmaf(m.z, nn[j], m.w * dd[j]);
-                        nn[j] = n2v;
-                        dd[j] = d2v;
-                        pa[j] *= x.x;
-                        E[j] += __float_as_int(x.y);
-                        F[j] += __float_as_int(x.z);
-                        norm_state(nn[j], dd[j], pa[j], E[j], F[j]);
-                    }
+                {
+                    const float2 cn = CAR(0, st), cd = CAR(1, st), cp = CAR(2, st), cE = CAR(3, st), cF = CAR(4, st);
+                    nn[0] = cn.x; nn[1] = cn.y; dd[0] = cd.x; dd[1] = cd.y; pa[0] = cp.x; pa[1] = cp.y;
+                    E[0] = __float_as_int(cE.x); E[1] = __float_as_int(cE.y);
+                    F[0] = __float_as_int(cF.x); F[1] = __float_as_int(cF.y);
                 }
-                // ---- step 3: walk the sub-block for its G range (projective
-                // precision and gate product only); the last sub-block's end state
-                // starts the next chunk
+                for (int sj = 0; sj < s; ++sj) {
+                    const float2 m00 = X(0, sj), m01 = X(1, sj), m10 = X(2, sj), m11 = X(3, sj), mp = X(4, sj);
+                    const float2 me = X(5, sj), mf = X(6, sj);
+                    const float n0v = fmaf(m00.x, nn[0], m01.x * dd[0]), d0v = fmaf(m10.x, nn[0], m11.x * dd[0]);
+                    const float n1v = fmaf(m00.y, nn[1], m01.y * dd[1]), d1v = fmaf(m10.y, nn[1], m11.y * dd[1]);
+                    nn[0] = n0v; dd[0] = d0v; nn[1] = n1v; dd[1] = d1v;
+                    pa[0] *= mp.x; pa[1] *= mp.y;
+                    E[0] += __float_as_int(me.x); E[1] += __float_as_int(me.y);
+                    F[0] += __float_as_int(mf.x); F[1] += __float_as_int(mf.y);
+                    norm_state(nn[0], dd[0], pa[0], E[0], F[0]);
+                    norm_state(nn[1], dd[1], pa[1], E[1], F[1]);
+                }
+                // the sub-block's start state, kept for a re-walk
                 const float2 n2s0 = make_float2(nn[0], nn[1]), d2s0 = make_float2(dd[0], dd[1]);
                 const float2 p2s0 = make_float2(pa[0], pa[1]);
                 const int E00 = E[0], E01 = E[1], F00 = F[0], F01 = F[1];
+                bln = (c + 1 < nchunks) ? load_beta(c + 1) : 0.f;
+                // ---- step 3: walk the sub-block and fold every token against the
+                // reference in force (exact while |G - rho| stays within kLost):
+                //   Q' = q/lambda 2^(G - rho) = q pa/n 2^((F-E) - rho)
+                //   K' = beta k 2^(rho - G)   = beta k d/pa 2^(rho - (F-E))
+                // tracking fk = 2^(rho - G) for the chunk's G range; the next chunk's
+                // a, qn go into the freed registers
                 int2 glo, ghi;
+                bool clamped = false;
                 {
                     float2 n2s = n2s0, d2s = d2s0, p2s = p2s0;
-                    // G just before the sub-block: (F - E) - log2(d/pa)
-                    int2 ge = make_int2(F[0] - E[0], F[1] - E[1]);
-                    const float r0 = dd[0] / pa[0], r1 = dd[1] / pa[1];
-                    glo = make_int2(ge.x - expo(r0) - 1, ge.y - expo(r1) - 1);
-                    ghi = make_int2(ge.x - expo(r0), ge.y - expo(r1));
-                    float2 rkmin = make_float2(3.0e38f, 3.0e38f), rkmax = make_float2(0.f, 0.f);
+                    int Ew0 = E00, Ew1 = E01, Fw0 = F00, Fw1 = F01;
+                    // x = (F - E) - rho of the current 8-token group (unclamped): with
+                    // rk = d/pa, G - rho lies in (x - expo(rk) - 1, x - expo(rk)]
+                    int x0 = Fw0 - Ew0 - rho0, x1 = Fw1 - Ew1 - rho1;
+                    clamped = x0 != clampe(x0) || x1 != clampe(x1);
+                    float2 mq = make_float2(pow2i(clampe(x0)), pow2i(clampe(x1)));
+                    float2 mk = make_float2(pow2i(-clampe(x0)), pow2i(-clampe(x1)));
+                    // G just before the sub-block
+                    float2 rkmin = make_float2(__fdividef(d2s.x, p2s.x), __fdividef(d2s.y, p2s.y));
+                    float2 rkmax = rkmin;
+                    // four tokens at a time: their chain steps (the serial part), then
+                    // their folds, which are independent of one another; each token's
+                    // a, qn registers take the next chunk's once it is folded
+                    constexpr int TG = 4;
 #pragma unroll
-                    for (int r = 0; r < SL; ++r) {
-                        const float2 kf = unpack_bf2(*reinterpret_cast<const uint32_t *>(kt + offr(r)));
-                        const float be = __shfl_sync(0xffffffffu, bl, r);
-                        const float2 b = f2mul(f2mul(make_float2(be, be), kf), kf);
-                        d2s = f2fma(f2mul(av[r], av[r]), d2s, f2mul(qv[r], n2s));
-                        n2s = f2fma(b, d2s, n2s);
-                        p2s = f2mul(p2s, av[r]);
-                        const float2 rk = make_float2(__fdividef(d2s.x, p2s.x), __fdividef(d2s.y, p2s.y));
-                        rkmin = make_float2(fminf(rkmin.x, rk.x), fminf(rkmin.y, rk.y));
-                        rkmax = make_float2(fmaxf(rkmax.x, rk.x), fmaxf(rkmax.y, rk.y));
-                        if ((r & 7) == 7) {
-                            glo = make_int2(min(glo.x, ge.x - expo(rkmax.x) - 1), min(glo.y, ge.y - expo(rkmax.y) - 1));
-                            ghi = make_int2(max(ghi.x, ge.x - expo(rkmin.x)), max(ghi.y, ge.y - expo(rkmin.y)));
+                    for (int r0 = 0; r0 < SL; r0 += TG) {
+                        uint32_t kwb[TG], qwb[TG];
+#pragma unroll
+                        for (int x = 0; x < TG; ++x) {
+                            kwb[x] = *reinterpret_cast<const uint32_t *>(kt + offr(r0 + x));
+                            qwb[x] = *reinterpret_cast<const uint32_t *>(qt + offr(r0 + x));
+                        }
+                        float2 nt[TG], dt[TG], pt2[TG], bkt[TG];
+#pragma unroll
+                        for (int x = 0; x < TG; ++x) {
+                            const int r = r0 + x;
+                            const float2 kf = unpack_bf2(kwb[x]);
+                            const float be = __shfl_sync(0xffffffffu, bl, r);
+                            bkt[x] = f2mul(make_float2(be, be), kf);
+                            d2s = f2fma(f2mul(av[r], av[r]), d2s, f2mul(qv[r], n2s));
+                            n2s = f2fma(f2mul(bkt[x], kf), d2s, n2s);
+                            p2s = f2mul(p2s, av[r]);
+                            nt[x] = n2s; dt[x] = d2s; pt2[x] = p2s;
+                        }
+#pragma unroll
+                        for (int x = 0; x < TG; ++x) {
+                            const int r = r0 + x;
+                            // (rows past the segment end are never stored and their K' is
+                            // zero, so their Q' needs no masking)
+                            const float2 qf = unpack_bf2(qwb[x]);
+                            const float2 pn = f2mul(pt2[x], nt[x]);
+                            const float2 rc = make_float2(rcp_approx(pn.x), rcp_approx(pn.y));
+                            const float2 qo = f2mul(f2mul(qf, f2mul(pt2[x], mq)), f2mul(pt2[x], rc));   // q pa/n 2^x
+                            const float2 rk = f2mul(dt[x], f2mul(nt[x], rc));                         // d/pa
+                            const float2 ko = f2mul(bkt[x], f2mul(rk, mk));                            // beta k d/pa 2^-x
+                            rkmin = make_float2(fminf(rkmin.x, rk.x), fminf(rkmin.y, rk.y));
+                            rkmax = make_float2(fmaxf(rkmax.x, rk.x), fmaxf(rkmax.y, rk.y));
+                            const uint32_t kh = pack_bf2(ko.x, ko.y);
+                            const float2 khf = unpack_bf2(kh);
+                            *reinterpret_cast<uint32_t *>(qt + offr(r)) = pack_bf2(qo.x, qo.y);
+                            *reinterpret_cast<uint32_t *>(kt + offr(r)) = kh;
+                            *reinterpret_cast<uint32_t *>(klo + offr(r)) = pack_bf2(ko.x - khf.x, ko.y - khf.y);
+                            if (c + 1 < nchunks) load_tok(c + 1, r, av[r], qv[r]);
+                        }
+                        if (((r0 + TG) & 7) == 0) {
+                            // the 8-token group's G range, renormalisation, next factors
+                            const int r = r0 + TG - 1;
+                            const int lo0 = x0 - expo(rkmax.x) - 1, lo1 = x1 - expo(rkmax.y) - 1;
+                            const int hi0 = x0 - expo(rkmin.x), hi1 = x1 - expo(rkmin.y);
+                            glo = (r == 7) ? make_int2(lo0, lo1) : make_int2(min(glo.x, lo0), min(glo.y, lo1));
+                            ghi = (r == 7) ? make_int2(hi0, hi1) : make_int2(max(ghi.x, hi0), max(ghi.y, hi1));
+                            norm_state(n2s.x, d2s.x, p2s.x, Ew0, Fw0);
+                            norm_state(n2s.y, d2s.y, p2s.y, Ew1, Fw1);
                             rkmin = make_float2(3.0e38f, 3.0e38f);
                             rkmax = make_float2(0.f, 0.f);
-                            norm_state(n2s.x, d2s.x, p2s.x, E[0], F[0]);
-                            norm_state(n2s.y, d2s.y, p2s.y, E[1], F[1]);
-                            ge = make_int2(F[0] - E[0], F[1] - E[1]);
+                            if (r + 1 < SL) {
+                                x0 = Fw0 - Ew0 - rho0;
+                                x1 = Fw1 - Ew1 - rho1;
+                                clamped |= x0 != clampe(x0) || x1 != clampe(x1);
+                                mq = make_float2(pow2i(clampe(x0)), pow2i(clampe(x1)));
+                                mk = make_float2(pow2i(-clampe(x0)), pow2i(-clampe(x1)));
+                            }
                         }
                     }
                     if (s == NSUB - 1) {
                         // the chunk-end state starts the next chunk
                         const int nst = (c + 1) & 1;
-                        carf[(nst * DK + i0) * 2] = make_float4(n2s.x, d2s.x, p2s.x, 0.f);
-                        cari[(nst * DK + i0) * 2 + 1] = make_int4(E[0], F[0], 0, 0);
-                        carf[(nst * DK + i0 + 1) * 2] = make_float4(n2s.y, d2s.y, p2s.y, 0.f);
-                        cari[(nst * DK + i0 + 1) * 2 + 1] = make_int4(E[1], F[1], 0, 0);
+                        CAR(0, nst) = n2s; CAR(1, nst) = d2s; CAR(2, nst) = p2s;
+                        CAR(3, nst) = i2f(Ew0, Ew1);
+                        CAR(4, nst) = i2f(Fw0, Fw1);
                         if (c == nchunks - 1) {
-                            // final outputs of the segment (the references follow in step 4)
                             lam_end0 = n2s.x / d2s.x;
                             lam_end1 = n2s.y / d2s.y;
                             gend0 = p2s.x / d2s.x;
                             gend1 = p2s.y / d2s.y;
-                            xend0 = F[0] - E[0];
-                            xend1 = F[1] - E[1];
+                            xend0 = Fw0 - Ew0;
+                            xend1 = Fw1 - Ew1;
                         }
                     }
                 }
-                rng[s * DK + i0] = make_int2(glo.x, ghi.x);
-                rng[s * DK + i0 + 1] = make_int2(glo.y, ghi.y);
+                rng[s * NP + pr] = make_int4(glo.x, ghi.x, glo.y, ghi.y);
                 if (named_bar_or(kGateBar, RL::GT, *abort_flag != 0)) { ok = false; break; }
-                // ---- step 4: references of the pass quarters, from the G ranges
-                // of every sub-block of the chunk
+                // ---- step 4: references of the pass quarters from the G ranges of
+                // every sub-block (relative to rho): R = 0 keeps the reference
                 int R0[4], R1[4];
                 int lv;
                 bool bad0, bad1;
@@ -535,36 +679,66 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         constexpr int per = NSUB / 4;
-                        int2 ra = rng[(q * per) * DK + i0], rb = rng[(q * per) * DK + i0 + 1];
+                        int4 x = rng[(q * per) * NP + pr];
+                        int2 ra = make_int2(x.x, x.y), rb = make_int2(x.z, x.w);
 #pragma unroll
-                        for (int x = 1; x < per; ++x) {
-                            ra = runion(ra, rng[(q * per + x) * DK + i0]);
-                            rb = runion(rb, rng[(q * per + x) * DK + i0 + 1]);
+                        for (int y = 1; y < per; ++y) {
+                            x = rng[(q * per + y) * NP + pr];
+                            ra = runion(ra, make_int2(x.x, x.y));
+                            rb = runion(rb, make_int2(x.z, x.w));
                         }
                         qa[q] = ra;
                         qb[q] = rb;
                     }
-                    const int l0 = choose_refs(qa, rho0, R0, bad0);
-                    const int l1 = choose_refs(qb, rho1, R1, bad1);
+                    const int l0 = choose_refs(qa, 0, R0, bad0);
+                    const int l1 = choose_refs(qb, 0, R1, bad1);
                     lv = max(l0, l1);
                 }
+                const int ra = pick4(R0, quarter), rb = pick4(R1, quarter);
+                // the provisional fold of this sub-block is exact while its |G - rho|
+                // stays within kLost and no exponent was clamped; a rescale by more
+                // than 2^100 is not taken in one step either: re-walk instead
+                const bool lost = clamped || glo.x < -kLost || ghi.x > kLost || glo.y < -kLost || ghi.y > kLost ||
+                                  abs(ra) > kLost || abs(rb) > kLost;
                 if (s == 0) {
                     atomicMax(&lvl[st], (c << 2) | lv);
                     if (bad0 || bad1) atomicOr(g.status, kStatusRange);
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
-                        facd[(st * 4 + q) * DK + i0] = R0[q] - (q ? R0[q - 1] : rho0);
-                        facd[(st * 4 + q) * DK + i0 + 1] = R1[q] - (q ? R1[q - 1] : rho1);
+                        facd[(st * 4 + q) * DK + i0] = R0[q] - (q ? R0[q - 1] : 0);
+                        facd[(st * 4 + q) * DK + i0 + 1] = R1[q] - (q ? R1[q - 1] : 0);
                     }
                     if (LOCAL && p > 0) {
                         float *rl = g.rlog + ((u * g.NC + chunk_base + c) * 4) * DK + i0;
 #pragma unroll
                         for (int q = 0; q < 4; ++q)
-                            *reinterpret_cast<float2 *>(rl + q * DK) = make_float2((float)R0[q], (float)R1[q]);
+                            *reinterpret_cast<float2 *>(rl + q * DK) =
+                                make_float2((float)(rho0 + R0[q]), (float)(rho1 + R1[q]));
                     }
                 }
-                rho0 = R0[3];
-                rho1 = R1[3];
+                if (lost) {
+                    // ---- step 5a (strong forgetting): walk the sub-block again from its
+                    // start and fold against the pass reference (a, qn reloaded)
+                    rewalk_fold<DK, SL>(qt, kt, klo, cbase, n2s0, d2s0, p2s0, E00, E01, F00, F01, rho0 + ra, rho1 + rb,
+                                        g.a, g.qn, g.beta, reinterpret_cast<const __nv_bfloat16 *>(g.q),
+                                        reinterpret_cast<const __nv_bfloat16 *>(g.k), tok0 + SL * s, nval, g.H, h, i0);
+                } else if (ra != 0 || rb != 0) {
+                    // ---- step 5b: the reference moved: rescale the folded bf16 words
+                    // exactly by powers of two (Q' by 2^-R, K' by 2^R)
+                    const __nv_bfloat162 sq = __floats2bfloat162_rn(pow2i(-ra), pow2i(-rb));
+                    const __nv_bfloat162 sk = __floats2bfloat162_rn(pow2i(ra), pow2i(rb));
+#pragma unroll 1
+                    for (int r = 0; r < SL; ++r) {
+                        __nv_bfloat162 *wq = reinterpret_cast<__nv_bfloat162 *>(qt + offr(r));
+                        __nv_bfloat162 *wk = reinterpret_cast<__nv_bfloat162 *>(kt + offr(r));
+                        __nv_bfloat162 *wl = reinterpret_cast<__nv_bfloat162 *>(klo + offr(r));
+                        *wq = __hmul2(*wq, sq);
+                        *wk = __hmul2(*wk, sk);
+                        *wl = __hmul2(*wl, sk);
+                    }
+                }
+                rho0 += R0[3];
+                rho1 += R1[3];
                 if (c == nchunks - 1 && s == NSUB - 1) {
                     // final outputs of the segment: 2^(G_end - rho) for the state
                     // export, the precision, and the segment's gate product
@@ -582,55 +756,14 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         g.final_lambda[u * DK + i0 + 1] = lam_end1;
                     }
                 }
-                // ---- step 5: walk the sub-block again and fold each token:
-                //   Q' = q/lambda 2^(G - R) = q pa/n 2^((F-E) - R)
-                //   K' = beta k 2^(R - G)   = beta k d/pa 2^(R - (F-E))
-                // then load the next chunk's a, qn into the freed registers
-                {
-                    const int ra = pick4(R0, quarter), rb = pick4(R1, quarter);
-                    float2 n2s = n2s0, d2s = d2s0, p2s = p2s0;
-                    int e0 = clampe(F00 - E00 - ra), e1 = clampe(F01 - E01 - rb);
-                    int Ew0 = E00, Ew1 = E01, Fw0 = F00, Fw1 = F01;
-                    float2 mq = make_float2(pow2i(e0), pow2i(e1)), mk = make_float2(pow2i(-e0), pow2i(-e1));
-#pragma unroll
-                    for (int r = 0; r < SL; ++r) {
-                        const uint32_t kw = *reinterpret_cast<const uint32_t *>(kt + offr(r));
-                        const uint32_t qw = *reinterpret_cast<const uint32_t *>(qt + offr(r));
-                        const bool valid = tok0 + SL * s + r < te;
-                        const float2 kf = unpack_bf2(kw);
-                        const float2 qf = valid ? unpack_bf2(qw) : make_float2(0.f, 0.f);
-                        const float be = __shfl_sync(0xffffffffu, bl, r);
-                        const float2 bk = f2mul(make_float2(be, be), kf);
-                        d2s = f2fma(f2mul(av[r], av[r]), d2s, f2mul(qv[r], n2s));
-                        n2s = f2fma(f2mul(bk, kf), d2s, n2s);
-                        p2s = f2mul(p2s, av[r]);
-                        const float2 pn = f2mul(p2s, n2s);
-                        const float2 rc = make_float2(rcp_approx(pn.x), rcp_approx(pn.y));
-                        const float2 qo = f2mul(f2mul(f2mul(qf, p2s), f2mul(p2s, rc)), mq);     // q pa/n
-                        const float2 ko = f2mul(f2mul(bk, f2mul(d2s, f2mul(n2s, rc))), mk);    // beta k d/pa
-                        const uint32_t kh = pack_bf2(ko.x, ko.y);
-                        const float2 khf = unpack_bf2(kh);
-                        *reinterpret_cast<uint32_t *>(qt + offr(r)) = pack_bf2(qo.x, qo.y);
-                        *reinterpret_cast<uint32_t *>(kt + offr(r)) = kh;
-                        *reinterpret_cast<uint32_t *>(klo + offr(r)) = pack_bf2(ko.x - khf.x, ko.y - khf.y);
-                        if (c + 1 < nchunks) load_tok(c + 1, r);
-                        if ((r & 7) == 7 && r + 1 < SL) {
-                            norm_state(n2s.x, d2s.x, p2s.x, Ew0, Fw0);
-                            norm_state(n2s.y, d2s.y, p2s.y, Ew1, Fw1);
-                            e0 = clampe(Fw0 - Ew0 - ra);
-                            e1 = clampe(Fw1 - Ew1 - rb);
-                            mq = make_float2(pow2i(e0), pow2i(e1));
-                            mk = make_float2(pow2i(-e0), pow2i(-e1));
-                        }
-                    }
-                }
-                if (c + 1 < nchunks) load_beta(c + 1);
+                bl = bln;
                 fence_proxy_async();
                 mbar_arrive(&qk_ready[st]);
             }
             if (nchunks == 0 && s == 0 && last_seg && g.final_lambda) {
-                g.final_lambda[u * DK + i0] = carf[i0 * 2].x;
-                g.final_lambda[u * DK + i0 + 1] = carf[(i0 + 1) * 2].x;
+                const float2 l0 = CAR(0, 0);
+                g.final_lambda[u * DK + i0] = l0.x;
+                g.final_lambda[u * DK + i0 + 1] = l0.y;
             }
         } else {
             // ---- isotropic: one precision per head ---------------------------
@@ -842,9 +975,43 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         constexpr uint32_t iO = idesc_bf16(64, DV, false, true);
         constexpr uint32_t iU = idesc_bf16(DK, DV, true, true);
         const uint32_t tS = tbase + L::colS, tO = tbase + L::colO, tU = tbase + L::colU;
-        const uint32_t pa_s = smem_u32(sm + L::p0), uba = smem_u32(sm + L::ub0);
+        const uint32_t uba = smem_u32(sm + L::ub0);
         int pc = 0;                                   // passes so far (barrier phases)
-        for (int c = 0; c < nchunks && ok; ++c) {
+        // The output rows of a pass are read out during the next pass (after its
+        // P mask), from the other of two output accumulators, so the epilogue
+        // does not wait for the pass's last MMAs; P is double-buffered likewise.
+        int pend_c = -1, pend_m0 = 0, pend_m1 = 0;    // the pass whose rows are pending
+        auto emit = [&](int pcx, int cc, int m0, int m1) {
+            if (!waitw(&o_full[pcx & 1], (pcx >> 1) & 1, abort_flag, g.status)) { ok = false; return; }
+            tc_fence_after();
+            const long long tok0 = tb + (long long)cc * kC;
+            const bool row_ok = v64 && row64 >= m0 && row64 < m1 && (tok0 + row64 < te);
+            __nv_bfloat16 *orow = g.out + ((tok0 + row64) * g.H + h) * DV;
+            const uint32_t to = tbase + lane_base + L::colO + (pcx & 1) * DV;
+            uint32_t r2[DV / 32][32];
+#pragma unroll
+            for (int cb = 0; cb < DV / 32; ++cb) tmem_ld32(to + cb * 32, r2[cb]);
+            tmem_wait_ld();
+            if (row_ok) {
+#pragma unroll
+                for (int hh = 0; hh < DV / 32; ++hh) {
+                    const uint32_t *r = r2[hh];
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        uint4 w;
+                        w.x = pack_bf2(__uint_as_float(r[q4 * 8 + 0]), __uint_as_float(r[q4 * 8 + 1]));
+                        w.y = pack_bf2(__uint_as_float(r[q4 * 8 + 2]), __uint_as_float(r[q4 * 8 + 3]));
+                        w.z = pack_bf2(__uint_as_float(r[q4 * 8 + 4]), __uint_as_float(r[q4 * 8 + 5]));
+                        w.w = pack_bf2(__uint_as_float(r[q4 * 8 + 6]), __uint_as_float(r[q4 * 8 + 7]));
+                        *reinterpret_cast<uint4 *>(orow + hh * 32 + q4 * 8) = w;
+                    }
+                }
+            }
+            tc_fence_before();
+        };
+        // every exit from this loop goes through a reducing barrier, so that the
+        // four warps leave it together
+        for (int c = 0; c < nchunks; ++c) {
             const int st = c & 1;
             if (!waitw(&qk_ready[st], (c >> 1) & 1, abort_flag, g.status)) { ok = false; }
             if (named_bar_or(kEpiBar, 128, !ok || *abort_flag)) { ok = false; break; }
@@ -865,35 +1032,36 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         tma_store_3d(&tm_qs, sm + L::q0 + st * L::QK + a * kC * 128, 64 * a, h, tok0);
                     tma_store_commit();
                 }
-                // scores of the whole chunk (each pass masks its own block)
-#pragma unroll
+                // scores of the whole chunk (each pass masks its own block); the
+                // K step moves a descriptor's start address by (bytes >> 4)
+                const uint64_t dq = sdesc_sw128(qa, 16, 1024), dk = sdesc_sw128(ka, 16, 1024);
+#pragma unroll 1
                 for (int kk = 0; kk < DK / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * (kC * 128) + (kk & 3) * 32;
-                    mma_bf16(tS, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), iS, kk > 0);
+                    const uint32_t off = ((kk >> 2) * (kC * 128) + (kk & 3) * 32) >> 4;
+                    mma_bf16(tS, dq + off, dk + off, iS, kk > 0);
                 }
                 mma_commit(s_full);
             }
             for (int k = 0; k < np; ++k) {
                 const int m0 = kQ * qper * k, m1 = m0 + kQ * qper;
                 const int s0 = k * qper, s1 = s0 + qper;      // 16-token slices of this pass
+                const uint32_t tOp = tO + (pc & 1) * DV;      // this pass's output accumulator
+                uint8_t *ptp = pt + (pc & 1) * L::PT;         // and its P buffer
                 // ---- state: U <- 2^d U for this pass's reference, snapshot to bf16
                 if (pc > 0 && !waitw(u_done, (pc - 1) & 1, abort_flag, g.status)) ok = false;
                 tc_fence_after();
                 const int d = vU ? facd[(st * 4 + k * qper) * DK + rowU] : 0;
                 const bool rmw = __any_sync(0xffffffffu, d != 0);
                 if (ok) {
+                    if (rmw) tmem_scale_lane<DV>(tbase + lane_base + L::colU, d);
+                    uint32_t r2[DV / 32][32];
 #pragma unroll
-                    for (int cb = 0; cb < DV / 32; ++cb) {
-                        uint32_t r[32];
-                        const uint32_t ta = tbase + lane_base + L::colU + cb * 32;
-                        tmem_ld32(ta, r);
-                        tmem_wait_ld();
-                        if (rmw) {
+                    for (int cb = 0; cb < DV / 32; ++cb) tmem_ld32(tbase + lane_base + L::colU + cb * 32, r2[cb]);
+                    tmem_wait_ld();
+                    if (vU) {
 #pragma unroll
-                            for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(scale2(__uint_as_float(r[x]), d));
-                            tmem_st32(ta, r);
-                        }
-                        if (vU) {
+                        for (int hh = 0; hh < DV / 32; ++hh) {
+                            const uint32_t *r = r2[hh];
 #pragma unroll
                             for (int q4 = 0; q4 < 4; ++q4) {
                                 uint4 w;
@@ -901,58 +1069,49 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                                 w.y = pack_bf2(__uint_as_float(r[q4 * 8 + 2]), __uint_as_float(r[q4 * 8 + 3]));
                                 w.z = pack_bf2(__uint_as_float(r[q4 * 8 + 4]), __uint_as_float(r[q4 * 8 + 5]));
                                 w.w = pack_bf2(__uint_as_float(r[q4 * 8 + 6]), __uint_as_float(r[q4 * 8 + 7]));
-                                *reinterpret_cast<uint4 *>(ub + sw_off(rowU, cb * 32 + q4 * 8, DK)) = w;
+                                *reinterpret_cast<uint4 *>(ub + sw_off(rowU, hh * 32 + q4 * 8, DK)) = w;
                             }
                         }
                     }
-                    tmem_wait_st();
                 }
                 fence_proxy_async();
                 tc_fence_before();
                 if (named_bar_or(kEpiBar, 128, !ok || *abort_flag)) { ok = false; break; }
                 if (issuer) {
                     tc_fence_after();
-                    // O = Q' U (the previous pass's O was read out before the barrier)
-#pragma unroll
+                    // O = Q' U into this pass's accumulator (its previous contents, two
+                    // passes back, were read out before the barrier)
+                    const uint64_t dq = sdesc_sw128(qa, 16, 1024), du = sdesc_sw128(uba, DK * 128, 1024);
+#pragma unroll 1
                     for (int kk = 0; kk < DK / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * (kC * 128) + (kk & 3) * 32;
-                        mma_bf16(tO, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(uba + kk * 2048, DK * 128, 1024), iO,
-                                 kk > 0);
+                        const uint32_t off = ((kk >> 2) * (kC * 128) + (kk & 3) * 32) >> 4;
+                        mma_bf16(tOp, dq + off, du + kk * (2048 >> 4), iO, kk > 0);
                     }
-                    // U += K'^T V over this pass's tokens (hi and remainder of K')
-                    for (int kk = s0; kk < s1; ++kk) {
-                        const uint64_t bv = sdesc_sw128(va + kk * 2048, kC * 128, 1024);
-                        mma_bf16(tU, sdesc_sw128(ka + kk * 2048, kC * 128, 1024), bv, iU, 1);
-                        mma_bf16(tU, sdesc_sw128(kloa + kk * 2048, kC * 128, 1024), bv, iU, 1);
-                    }
-                    mma_commit(u_done);
                 }
                 // ---- P = the pass's block of the causal score tile, bf16
                 if (k == 0 && !waitw(s_full, c & 1, abort_flag, g.status)) ok = false;
                 tc_fence_after();
                 if (ok) {
+                    uint32_t r2[2][32];
+                    tmem_ld32(tbase + lane_base + L::colS, r2[0]);
+                    tmem_ld32(tbase + lane_base + L::colS + 32, r2[1]);
+                    tmem_wait_ld();
+                    if (v64) {
+                        const int tau = row64;
+                        const bool in_row = tau >= m0 && tau < m1;
 #pragma unroll
-                    for (int hf = 0; hf < 2; ++hf) {
-                        uint32_t r[32];
-                        tmem_ld32(tbase + lane_base + L::colS + 32 * hf, r);
-                        tmem_wait_ld();
-                        if (v64) {
-                            const int tau = row64;
-                            const bool in_row = tau >= m0 && tau < m1;
+                        for (int ch = 0; ch < 8; ++ch) {
+                            float x[8];
 #pragma unroll
-                            for (int ch = 4 * hf; ch < 4 * hf + 4; ++ch) {
-                                float x[8];
-#pragma unroll
-                                for (int e2 = 0; e2 < 8; ++e2) {
-                                    const int sg = ch * 8 + e2;
-                                    const float sv = __uint_as_float(r[sg - 32 * hf]);
-                                    x[e2] = (in_row && sg >= m0 && sg <= tau) ? sv : 0.f;
-                                }
-                                uint4 w;
-                                w.x = pack_bf2(x[0], x[1]); w.y = pack_bf2(x[2], x[3]);
-                                w.z = pack_bf2(x[4], x[5]); w.w = pack_bf2(x[6], x[7]);
-                                *reinterpret_cast<uint4 *>(pt + tau * 128 + ((ch ^ (tau & 7)) << 4)) = w;
+                            for (int e2 = 0; e2 < 8; ++e2) {
+                                const int sg = ch * 8 + e2;
+                                const float sv = __uint_as_float(r2[sg >> 5][sg & 31]);
+                                x[e2] = (in_row && sg >= m0 && sg <= tau) ? sv : 0.f;
                             }
+                            uint4 w;
+                            w.x = pack_bf2(x[0], x[1]); w.y = pack_bf2(x[2], x[3]);
+                            w.z = pack_bf2(x[4], x[5]); w.w = pack_bf2(x[6], x[7]);
+                            *reinterpret_cast<uint4 *>(ptp + tau * 128 + ((ch ^ (tau & 7)) << 4)) = w;
                         }
                     }
                 }
@@ -961,49 +1120,39 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 if (named_bar_or(kEpiBar, 128, !ok || *abort_flag)) { ok = false; break; }
                 if (issuer) {
                     tc_fence_after();
-                    // O += P V over this pass's tokens
-                    for (int kk = s0; kk < s1; ++kk)
-                        mma_bf16(tO, sdesc_sw128(pa_s + kk * 32, 16, 1024), sdesc_sw128(va + kk * 2048, kC * 128, 1024),
-                                 iO, 1);
-                    mma_commit(o_full);
-                }
-                // ---- output rows of this pass (a timeout here is seen by every
-                // epilogue warp at the next reducing barrier)
-                if (!waitw(o_full, pc & 1, abort_flag, g.status)) ok = false;
-                tc_fence_after();
-                if (ok) {
-                    const long long tok0 = tb + (long long)c * kC;
-                    const bool row_ok = v64 && row64 >= m0 && row64 < m1 && (tok0 + row64 < te);
-                    __nv_bfloat16 *orow = g.out + ((tok0 + row64) * g.H + h) * DV;
-#pragma unroll
-                    for (int cb = 0; cb < DV / 32; ++cb) {
-                        uint32_t r[32];
-                        tmem_ld32(tbase + lane_base + L::colO + cb * 32, r);
-                        tmem_wait_ld();
-                        if (row_ok) {
-#pragma unroll
-                            for (int q4 = 0; q4 < 4; ++q4) {
-                                uint4 w;
-                                w.x = pack_bf2(__uint_as_float(r[q4 * 8 + 0]), __uint_as_float(r[q4 * 8 + 1]));
-                                w.y = pack_bf2(__uint_as_float(r[q4 * 8 + 2]), __uint_as_float(r[q4 * 8 + 3]));
-                                w.z = pack_bf2(__uint_as_float(r[q4 * 8 + 4]), __uint_as_float(r[q4 * 8 + 5]));
-                                w.w = pack_bf2(__uint_as_float(r[q4 * 8 + 6]), __uint_as_float(r[q4 * 8 + 7]));
-                                *reinterpret_cast<uint4 *>(orow + cb * 32 + q4 * 8) = w;
-                            }
-                        }
+                    // O += P V over this pass's tokens; then the state update, whose
+                    // completion (u_done) the next pass's snapshot waits for
+                    const uint64_t dp = sdesc_sw128(smem_u32(ptp), 16, 1024), dv = sdesc_sw128(va, kC * 128, 1024);
+                    const uint64_t dk = sdesc_sw128(ka, kC * 128, 1024), dl = sdesc_sw128(kloa, kC * 128, 1024);
+#pragma unroll 1
+                    for (int kk = s0; kk < s1; ++kk) mma_bf16(tOp, dp + kk * (32 >> 4), dv + kk * (2048 >> 4), iO, 1);
+                    mma_commit(&o_full[pc & 1]);
+                    // U += K'^T V over this pass's tokens (hi and remainder of K')
+#pragma unroll 1
+                    for (int kk = s0; kk < s1; ++kk) {
+                        mma_bf16(tU, dk + kk * (2048 >> 4), dv + kk * (2048 >> 4), iU, 1);
+                        mma_bf16(tU, dl + kk * (2048 >> 4), dv + kk * (2048 >> 4), iU, 1);
                     }
+                    mma_commit(u_done);
                 }
-                tc_fence_before();
+                // ---- output rows of the previous pass (its MMAs have finished
+                // while this pass was prepared)
+                if (ok && pend_c >= 0) emit(pc - 1, pend_c, pend_m0, pend_m1);
+                pend_c = c; pend_m0 = m0; pend_m1 = m1;
                 ++pc;
             }
             if (named_bar_or(kEpiBar, 128, !ok || *abort_flag)) { ok = false; break; }
-            // every MMA of this chunk has completed (o_full of its last pass): the
-            // stage takes the chunk two ahead once the q' export has read it
+            // every MMA of this chunk has completed once its last u_done has (the
+            // state update is the last reader of K' and V): the stage takes the
+            // chunk two ahead once the q' export has read it. Only the issuing
+            // thread waits; the other warps go on to the next chunk.
             if (issuer) {
+                ok = wait_slow(u_done, (pc - 1) & 1, abort_flag, g.status, true) && ok;
                 if (LOCAL && p > 0) tma_store_wait_read();
-                if (loaded < nchunks) { load_chunk(loaded); ++loaded; }
+                if (ok && loaded < nchunks) { load_chunk(loaded); ++loaded; }
             }
         }
+        if (ok && pend_c >= 0) emit(pc - 1, pend_c, pend_m0, pend_m1);
         // ---- final belief (last segment) or segment transfer (mode 2)
         float *dst = nullptr;
         if (LOCAL) dst = g.S_io + (u * g.P + p) * DK * DV;
@@ -1126,6 +1275,7 @@ cudaError_t launch_t(const Plan &p, const int *cu, int mode, const void *q, cons
     g.N = p.N; g.H = p.H; g.P = p.P; g.NB = p.NB; g.seg_blocks = p.seg_blocks; g.NC = p.NB;
     g.T = p.T; g.Lseg = p.Lseg; g.cu = cu; g.perm = cu ? p.perm : nullptr;
     g.a = a; g.qn = qn; g.beta = beta; g.lambda0 = lambda0; g.eta0 = eta0; g.lam_blk = lam_blk;
+    g.q = q; g.k = k;
     g.agg = p.inline_carry ? p.agg : nullptr;
     g.rlog = p.rlog;
     g.S_io = S_io; g.decay = decay; g.out = (__nv_bfloat16 *)out;
