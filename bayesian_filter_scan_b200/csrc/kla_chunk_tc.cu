@@ -28,22 +28,26 @@
 // a chunk). A 16-token quarter spanning more than 2 kLim is outside what the
 // factorised form represents: KLA_ERR_RANGE.
 //
-// CTA = one segment of one (row or packed sequence, head); 448 threads:
-//   warps 0-7   gate. Diagonal precision: thread = (key pair, sub-block of 16
-//               tokens at dk = 128, 8 at dk = 64). Each thread composes its
-//               sub-block's Moebius matrices for its two keys, the matrices
-//               are exchanged through shared memory, each thread walks its
-//               sub-block from the exact start precision and forms the raw
-//               operand factors, the per-key G ranges are exchanged, the
-//               references chosen, and the thread writes Q', K' (bf16 hi) and
-//               the bf16 remainder of K' over the TMA-loaded tiles.
-//               Isotropic precision: warp 0 scans the chunk's 64 Moebius maps
-//               with shuffles; all eight warps fold the rows.
-//   warps 8-11  epilogue: rescale U in TMEM and snapshot it to bf16 shared
-//               memory, mask the score tile into P, store the output rows;
-//   warp 12     TMA producer (q, k, v tiles double-buffered; L2 prefetch of
-//               later chunks, a and qn included);
-//   warp 13     TMEM owner and single-thread tcgen05.mma issuer.
+// CTA = one segment of one (row or packed sequence, head), warp-specialised:
+//   gate        Diagonal precision: dk / 32 warps, thread = key. Each thread
+//               walks its key through every token of the segment (precision
+//               chain and exponents in registers), folding each token's Q',
+//               K' (bf16 hi) and the bf16 remainder of K' over the TMA-loaded
+//               tiles against the reference in force; then the chunk's G
+//               ranges per pass quarter fix the references, and rows whose
+//               reference moved are rescaled exactly (or re-walked where the
+//               provisional fold lost bits).
+//               Isotropic precision: three warps; warp 0 scans the chunk's 64
+//               Moebius maps with shuffles, all three fold the rows.
+//   epilogue    four warps (TMEM lane quarter = warp % 4): rescale U in TMEM
+//               and snapshot it to bf16 shared memory, mask the score tile into
+//               P, store the output rows;
+//   producer    (diagonal) streams a and qn into the gate's ring of 16-token
+//               slots, with an L2 prefetch two chunks ahead;
+//   MMA warp    TMEM owner; lane 0 loads the q, k, v tiles (double-buffered,
+//               L2 prefetch of later chunks), exports q' of split rows, and
+//               issues every tcgen05.mma, synchronised with the gate and the
+//               epilogue through mbarriers only.
 // mode 0 walks whole rows or packed sequences (from lambda0, eta0); mode 2
 // walks every segment of split rows from a zero state (segment 0 from eta0)
 // and exports what the correction pass needs. The kernel is instantiated per
@@ -51,8 +55,8 @@
 //
 // Every wait is bounded: after kWaitLimitNs a waiter sets the abort flag and
 // the library status bit, all roles fall through to the teardown, the
-// producer waits (bounded) for its outstanding copies, the MMA thread for its
-// outstanding MMAs, and the TMEM is released.
+// producer and the MMA thread wait (bounded) for their outstanding copies, the
+// MMA thread for its outstanding MMAs, and the TMEM is released.
 #include <cstdlib>
 
 #include "kla_internal.cuh"
@@ -68,20 +72,27 @@ constexpr int kQ = 16;        // tokens per pass quarter
 constexpr int kLim = 80;      // |G - rho| (log2) a pass keeps inside the exponent window
 constexpr int kStick = 48;    // the reference stays while the range fits [rho - kStick, rho + kStick]
 constexpr int kLost = 100;    // the fold against the reference in force is exact while |G - rho| <= kLost
+constexpr int kMove = 32;     // the reference moves to a chunk's start once G has drifted beyond kMove from it
+constexpr int kSl = 8;        // tokens per slice of the diagonal gate's walk
+constexpr int kRt = 16;       // tokens per a / qn ring slot of the diagonal gate (two slices)
+constexpr int kRpc = kC / kRt;             // ring slots per chunk
+constexpr int kRs = 2;                     // ring slots
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr int kGateBar = 1;   // named barrier of the gate warps
-constexpr int kEpiBar = 2;    // named barrier of the epilogue warps
 
-template <int DK, int DV>
+// Gate warps first, then the four epilogue warps (TMEM lane quarter = warp % 4),
+// the warp that streams a and qn into the diagonal gate's ring (diagonal only),
+// and the MMA warp. Diagonal precision: one gate thread per key (dk / 32
+// warps); isotropic: three gate warps (warp 0 scans, all three fold), so that
+// no scheduler holds more than two warps' registers.
+template <int DK, int DV, bool ISO>
 struct Roles {
-    static constexpr int NGW = 8;                     // gate warps
+    static constexpr int NGW = ISO ? 3 : DK / 32;     // gate warps
     static constexpr int GT = NGW * 32;               // gate threads
-    static constexpr int EPIW = 8;                    // first epilogue warp (TMEM lane quarter 0)
-    static constexpr int THREADS = 12 * 32;           // 12 warps: up to 168 registers per thread
+    static constexpr int EPIW = NGW;                  // first epilogue warp
+    static constexpr int MMAW = NGW + (ISO ? 4 : 5);  // TMEM owner, tile loads, MMA issue
+    static constexpr int THREADS = (MMAW + 1) * 32;
     static constexpr int MIN_BLOCKS = 1;
-    // diagonal gate: sub-blocks per chunk and their length
-    static constexpr int NSUB = (DK == 128) ? 4 : 8;
-    static constexpr int SL = kC / NSUB;
 };
 
 struct TcArgs {
@@ -107,27 +118,24 @@ struct Layout {
     static constexpr int V = kC * DV * 2;
     static constexpr int PT = kC * kC * 2;
     static constexpr int UB = DK * DV * 2;
-    static constexpr int XN = 512;                   // sub-blocks x keys of the diagonal gate (NSUB * DK)
+    static constexpr int RSLOT = 2 * kRt * DK * 4;   // a / qn ring slot: [a: kRt x DK][qn: kRt x DK] floats
     static constexpr int q0 = 0;
     static constexpr int k0 = q0 + 2 * QK;
     static constexpr int v0 = k0 + 2 * QK;
     static constexpr int klo0 = v0 + 2 * V;          // low bf16 part of K' (state update), per stage
     static constexpr int p0 = klo0 + 2 * QK;
     static constexpr int ub0 = p0 + 2 * PT;         // (P double-buffered by pass)
-    static constexpr int xch0 = ub0 + UB;            // [NSUB][DK] {float4 matrix, float4 {PA, EM, FM, -}}
-    static constexpr int rng0 = xch0 + XN * 32;      // [NSUB][DK] int2 G range
-    static constexpr int car0 = rng0 + XN * 8;       // [2][DK] chunk-start state {float4 n,d,pa; int4 E,F}
-    static constexpr int fac0 = car0 + 2 * DK * 32;  // [2][4][DK] int: U rescale exponent at each pass quarter
+    static constexpr int ring0 = ub0 + UB;           // [kRs] a / qn ring slots of the diagonal gate
+    static constexpr int fac0 = ring0 + kRs * RSLOT; // [2][4][DK] int: U rescale exponent at each pass quarter
     static constexpr int facf0 = fac0 + 2 * kQuarters * DK * 4;   // [DK] float: 2^(G_end - rho_end)
     static constexpr int isof0 = facf0 + DK * 4;     // [2][kC] float2: iso per-token factors
     static constexpr int lvl0 = isof0 + 2 * kC * 8;  // int[2]: pass level of the chunk, tagged with its index
     static constexpr int bar0 = lvl0 + 16;
-    static constexpr int NBAR = 9;
+    static constexpr int NBAR = 12 + 2 * kRs;
     static constexpr int hold0 = bar0 + NBAR * 8;
     static constexpr int bytes = hold0 + 16;
     static constexpr int alloc = bytes + 1024;
     static_assert(alloc <= 232448, "shared memory per CTA");
-    static_assert(Roles<DK, DV>::MIN_BLOCKS == 1 || 2 * (alloc + 1024) <= 233472, "two CTAs per SM");
     // TMEM columns: the state U, two output accumulators (by pass), the scores
     static constexpr uint32_t NCOLS = (3 * DV + 64 <= 256) ? 256u : 512u;
     static constexpr uint32_t colU = 0, colO = DV, colS = 3 * DV;
@@ -146,8 +154,6 @@ __device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
 __device__ __forceinline__ float2 unpack_bf2(uint32_t w) {
     return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
-__device__ __forceinline__ float2 f2mul(float2 a, float2 b) { return __fmul2_rn(a, b); }
-__device__ __forceinline__ float2 f2fma(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 __device__ __forceinline__ int expo(float x) { return ((__float_as_int(x) >> 23) & 0xff) - 127; }
 // 2^e for e in [-126, 127]
 __device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
@@ -267,14 +273,6 @@ __device__ __forceinline__ int choose_refs(const int2 (&qr)[4], int rho, int (&R
     return 2;
 }
 
-// Normalises a 2x2 map (two columns) of one key by the power of two of its
-// largest entry; the exponent goes to `e`.
-__device__ __forceinline__ void norm_cols(float &n1, float &n2, float &d1, float &d2, int &e) {
-    const int x = clampe(expo(fmaxf(fmaxf(n1, n2), fmaxf(d1, d2))));
-    const float s = pow2i(-x);
-    n1 *= s; n2 *= s; d1 *= s; d2 *= s;
-    e += x;
-}
 // Normalises the projective precision (n, d) by the power of two of d and the
 // gate product pa by its own.
 __device__ __forceinline__ void norm_state(float &n, float &d, float &pa, int &E, int &F) {
@@ -287,66 +285,138 @@ __device__ __forceinline__ void norm_state(float &n, float &d, float &pa, int &E
     F += f;
 }
 
-// The strong-forgetting path of the diagonal gate: walks a sub-block of SL
-// tokens again from its start state and folds every token against the
-// references R0, R1 of its two keys (a, qn, beta, q, k reloaded from global
-// memory: the tile words were overwritten by the provisional fold). Out of line:
-// it runs only when a provisional fold lost bits.
-template <int DK, int SL>
-__device__ __noinline__ void rewalk_fold(uint8_t *qt, uint8_t *kt, uint8_t *klo, int cbase, float2 n2s, float2 d2s,
-                                         float2 p2s, int Ew0, int Ew1, int Fw0, int Fw1, int R0, int R1,
-                                         const float *a, const float *qn, const float *beta, const __nv_bfloat16 *q,
-                                         const __nv_bfloat16 *k, long long tok0, int nval, int H, int h, int i0) {
-    int e0 = clampe(Fw0 - Ew0 - R0), e1 = clampe(Fw1 - Ew1 - R1);
-    float2 mq = make_float2(pow2i(e0), pow2i(e1)), mk = make_float2(pow2i(-e0), pow2i(-e1));
+__device__ __forceinline__ uint16_t bf16_bits(float f) { return __bfloat16_as_ushort(__float2bfloat16_rn(f)); }
+__device__ __forceinline__ float bf16_val(uint32_t bits) { return __uint_as_float(bits << 16); }
+
+// One key's walk in the diagonal gate. The projective precision lambda = n/d
+// and the gate product p are renormalised at every slice end, their exponents
+// kept in E and F, so that G = log2(p/d) + F - E.
+struct KeyWalk {
+    float n, d, p;
+    int E, F;
+    int x;                  // F - E - rho at the slice start (unclamped)
+    float mq, mk;           // 2^clamp(x), 2^-clamp(x)
+    float rkmin, rkmax;     // range of d/p over the slice
+    bool clamped;           // some slice's x left the exponent window
+    int2 cl, q0, q1, q2, q3;   // integer bounds of G - rho: this quarter, the completed ones
+};
+
+// Walks the kSl tokens of slice s8 for one key (a, qn at ra[x * DK], rq[x * DK]
+// for token x of the slice): per token the precision step
+// (the serial part) and the provisional fold against the reference rho, exact
+// while |G - rho| stays within kLost and no exponent clamps:
+//   Q' = q/lambda 2^(G - rho) = q p/n 2^x,   K' = beta k 2^(rho - G) = beta k d/p 2^-x
+// written over the q and k tiles (bf16; the K' remainder into the klo tile).
+// The slice's G range is folded into the quarter's (the first slice of a
+// quarter also counts G just before it); then the state is renormalised.
+template <bool SECOND, int DK>
+__device__ __forceinline__ void walk_slice(KeyWalk &w, uint8_t *qt, uint8_t *kt, uint8_t *klo, const int (&sw)[8],
+                                           int s8, float bsrc, const float *ra, const float *rq, int rho) {
+    const int rb = s8 * kSl * 128, bl0 = (s8 * kSl) & 31;
+    if (!SECOND) {
+        w.rkmin = __fdividef(w.d, w.p);
+        w.rkmax = w.rkmin;
+    }
+    uint32_t kw[kSl], qw[kSl];
+    float be[kSl], A[kSl], Q[kSl];
+#pragma unroll
+    for (int x = 0; x < kSl; ++x) {
+        A[x] = ra[x * DK];
+        Q[x] = rq[x * DK];
+        kw[x] = *reinterpret_cast<const uint16_t *>(kt + sw[x] + rb + x * 128);
+        qw[x] = *reinterpret_cast<const uint16_t *>(qt + sw[x] + rb + x * 128);
+        be[x] = __shfl_sync(0xffffffffu, bsrc, bl0 + x);
+    }
+#pragma unroll
+    for (int x = 0; x < kSl; ++x) {
+        const int o = sw[x] + rb + x * 128;
+        const float kf = bf16_val(kw[x]);
+        const float bk = be[x] * kf;
+        w.d = fmaf(A[x] * A[x], w.d, Q[x] * w.n);
+        w.n = fmaf(bk * kf, w.d, w.n);
+        w.p *= A[x];
+        const float rc = rcp_approx(w.p * w.n);
+        const float qo = (bf16_val(qw[x]) * (w.p * w.mq)) * (w.p * rc);
+        const float rk = w.d * (w.n * rc);
+        const float ko = bk * (rk * w.mk);
+        w.rkmin = fminf(w.rkmin, rk);
+        w.rkmax = fmaxf(w.rkmax, rk);
+        const uint16_t kh = bf16_bits(ko);
+        *reinterpret_cast<uint16_t *>(qt + o) = bf16_bits(qo);
+        *reinterpret_cast<uint16_t *>(kt + o) = kh;
+        *reinterpret_cast<uint16_t *>(klo + o) = bf16_bits(ko - bf16_val(kh));
+    }
+    // with d/p in [2^e, 2^(e+1)), G - rho lies in (x - e - 1, x - e]
+    const int2 gr = make_int2(w.x - expo(w.rkmax) - 1, w.x - expo(w.rkmin));
+    if (!SECOND) {
+        w.cl = gr;
+    } else {
+        w.cl = runion(w.cl, gr);
+        w.q0 = w.q1; w.q1 = w.q2; w.q2 = w.q3; w.q3 = w.cl;
+    }
+    norm_state(w.n, w.d, w.p, w.E, w.F);
+    w.x = w.F - w.E - rho;
+    w.clamped |= w.x != clampe(w.x);
+    w.mq = pow2i(clampe(w.x));
+    w.mk = pow2i(-clampe(w.x));
+}
+
+// The strong-forgetting path of the diagonal gate: walks one key through the
+// chunk again from its start state and folds every token of quarter q against
+// the reference ref[q] (a, qn, beta, q, k reloaded from global memory: the tile
+// words were overwritten by the provisional fold). Out of line: it runs only
+// when a provisional fold lost bits.
+template <int DK>
+__device__ __noinline__ void rewalk_key(uint8_t *qt, uint8_t *kt, uint8_t *klo, int cb, float n, float d, float p,
+                                        int E, int F, int4 ref, const float *a, const float *qn, const float *beta,
+                                        const __nv_bfloat16 *q, const __nv_bfloat16 *k, long long tok0, int nval,
+                                        int H, int h, int i) {
+    float mq = 1.f, mk = 1.f;
 #pragma unroll 1
-    for (int r = 0; r < SL; ++r) {
+    for (int r = 0; r < kC; ++r) {
+        if ((r & 7) == 0) {
+            const int qq = r >> 4;
+            const int rr = qq == 0 ? ref.x : qq == 1 ? ref.y : qq == 2 ? ref.z : ref.w;
+            const int e = clampe(F - E - rr);
+            mq = pow2i(e);
+            mk = pow2i(-e);
+        }
         const long long tok = tok0 + r;
-        const long long off = (tok * H + h) * DK + i0;
-        float2 ar = make_float2(1.f, 1.f), qr = make_float2(0.f, 0.f), kf = qr, qf = qr;
-        float be = 0.f;
+        const long long off = (tok * H + h) * DK + i;
+        float ar = 1.f, qr = 0.f, kf = 0.f, qf = 0.f, be = 0.f;
         if (r < nval) {
-            ar = __ldg(reinterpret_cast<const float2 *>(a + off));
-            qr = __ldg(reinterpret_cast<const float2 *>(qn + off));
-            kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(k + off));
-            qf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(q + off));
+            ar = __ldg(a + off);
+            qr = __ldg(qn + off);
+            kf = __bfloat162float(k[off]);
+            qf = __bfloat162float(q[off]);
             be = __ldg(beta + tok * H + h);
         }
-        const float2 bk = f2mul(make_float2(be, be), kf);
-        d2s = f2fma(f2mul(ar, ar), d2s, f2mul(qr, n2s));
-        n2s = f2fma(f2mul(bk, kf), d2s, n2s);
-        p2s = f2mul(p2s, ar);
-        const float2 pn = f2mul(p2s, n2s);
-        const float2 rc = make_float2(__frcp_rn(pn.x), __frcp_rn(pn.y));
-        const float2 qo = f2mul(f2mul(f2mul(qf, p2s), f2mul(p2s, rc)), mq);
-        const float2 ko = f2mul(bk, f2mul(f2mul(d2s, f2mul(n2s, rc)), mk));
-        const uint32_t kh = pack_bf2(ko.x, ko.y);
-        const float2 khf = unpack_bf2(kh);
-        const int o = (cbase + r * 128) ^ ((r & 7) << 4);
-        *reinterpret_cast<uint32_t *>(qt + o) = pack_bf2(qo.x, qo.y);
-        *reinterpret_cast<uint32_t *>(kt + o) = kh;
-        *reinterpret_cast<uint32_t *>(klo + o) = pack_bf2(ko.x - khf.x, ko.y - khf.y);
-        if ((r & 7) == 7) {
-            norm_state(n2s.x, d2s.x, p2s.x, Ew0, Fw0);
-            norm_state(n2s.y, d2s.y, p2s.y, Ew1, Fw1);
-            e0 = clampe(Fw0 - Ew0 - R0);
-            e1 = clampe(Fw1 - Ew1 - R1);
-            mq = make_float2(pow2i(e0), pow2i(e1));
-            mk = make_float2(pow2i(-e0), pow2i(-e1));
-        }
+        const float bk = be * kf;
+        d = fmaf(ar * ar, d, qr * n);
+        n = fmaf(bk * kf, d, n);
+        p *= ar;
+        const float rc = __frcp_rn(p * n);
+        const float qo = ((qf * p) * (p * rc)) * mq;
+        const float ko = bk * ((d * (n * rc)) * mk);
+        const uint16_t kh = bf16_bits(ko);
+        const int o = (cb + r * 128) ^ ((r & 7) << 4);
+        *reinterpret_cast<uint16_t *>(qt + o) = bf16_bits(qo);
+        *reinterpret_cast<uint16_t *>(kt + o) = kh;
+        *reinterpret_cast<uint16_t *>(klo + o) = bf16_bits(ko - bf16_val(kh));
+        if ((r & 7) == 7) norm_state(n, d, p, E, F);
     }
 }
 
 }  // namespace
 
 template <int DK, int DV, bool ISO, bool LOCAL>
-__global__ void __launch_bounds__(Roles<DK, DV>::THREADS, Roles<DK, DV>::MIN_BLOCKS)
+__global__ void __launch_bounds__(Roles<DK, DV, ISO>::THREADS, Roles<DK, DV, ISO>::MIN_BLOCKS)
 kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_a,
                     const __grid_constant__ CUtensorMap tm_qn, const __grid_constant__ CUtensorMap tm_qs,
                     const TcArgs g) {
     using L = Layout<DK, DV>;
-    using RL = Roles<DK, DV>;
+    using RL = Roles<DK, DV, ISO>;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     // 1024-byte aligned base (128B-swizzle atoms), derived by pointer arithmetic
     // on the shared array so that every tile access stays a shared-space access
@@ -357,6 +427,12 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // per accumulator, so that a pass's completion is waited for before the
     // barrier can complete again)
     uint64_t *s_full = bars + 4, *u_done = bars + 5, *td_bar = bars + 6, *o_full = bars + 7;
+    // the epilogue's hand-offs to the MMA warp: the pass's state snapshot is in
+    // shared memory; its P tile is (one barrier per P buffer, so that a phase is
+    // seen before the barrier can complete again)
+    uint64_t *snap_ready = bars + 9, *p_ready = bars + 10;
+    // a / qn ring of the diagonal gate: slot landed, slot read by every gate warp
+    uint64_t *ring_full = bars + 12, *ring_empty = bars + 12 + kRs;
     uint32_t *tmem_hold = reinterpret_cast<uint32_t *>(sm + L::hold0);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::hold0 + 4);
     int *lvl = reinterpret_cast<int *>(sm + L::lvl0);
@@ -376,14 +452,22 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mbar_init(&o_full[0], 1);
         mbar_init(&o_full[1], 1);
         mbar_init(td_bar, 1);
+        mbar_init(snap_ready, 128);
+        mbar_init(&p_ready[0], 128);
+        mbar_init(&p_ready[1], 128);
+        if (!ISO)
+            for (int r = 0; r < kRs; ++r) {
+                mbar_init(&ring_full[r], 1);
+                mbar_init(&ring_empty[r], RL::NGW);
+            }
         *abort_flag = 0;
         fence_mbar_init();
     }
-    if (warp == RL::EPIW && lane == 0) {
+    if (warp == RL::MMAW && lane == 0) {
         prefetch_map(&tm_q); prefetch_map(&tm_k); prefetch_map(&tm_v);
         if (!ISO) { prefetch_map(&tm_a); prefetch_map(&tm_qn); }
     }
-    if (warp == RL::EPIW) tmem_alloc(tmem_hold, L::NCOLS);
+    if (warp == RL::MMAW) tmem_alloc(tmem_hold, L::NCOLS);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -438,333 +522,154 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         // ================= gate warps: precision path and operand folding =====
         bool ok = true;
         if constexpr (!ISO) {
-            constexpr int NSUB = RL::NSUB, SL = RL::SL, NP = DK / 2;
-            const int s = (DK == 128) ? (warp >> 1) : warp;           // sub-block
-            const int pr = (DK == 128) ? ((warp & 1) * 32 + lane) : lane;   // key pair
-            const int i0 = 2 * pr;
-            const int quarter = (SL * s) / kQ;                        // pass quarter of this sub-block
-            // exchange buffers, one float2 (the pair's two keys) per entry, so that a
-            // warp's accesses are consecutive 8-byte words:
-            //   sub-block maps  xch[(comp * NSUB + sub) * NP + pair], comp = n1 n2 d1 d2 PA EM FM
-            //   chunk-start state car[(comp * 2 + parity) * NP + pair], comp = n d pa E F
-            //   G ranges        rng[sub * NP + pair] = {lo, hi} of both keys, relative to rho
-            float2 *xch = reinterpret_cast<float2 *>(sm + L::xch0);
-            float2 *car = reinterpret_cast<float2 *>(sm + L::car0);
-            int4 *rng = reinterpret_cast<int4 *>(sm + L::rng0);
-            auto X = [&](int comp, int sj) -> float2 & { return xch[(comp * NSUB + sj) * NP + pr]; };
-            auto CAR = [&](int comp, int par) -> float2 & { return car[(comp * 2 + par) * NP + pr]; };
-            auto i2f = [](int x, int y) { return make_float2(__int_as_float(x), __int_as_float(y)); };
-            // byte offset of (row SL*s + r, keys i0, i0+1) in a swizzled tile: the
-            // sub-block starts on a multiple of 8 rows, so row & 7 = r & 7
-            // (bits 4-6 of a row's base are zero, so the swizzled 16-byte chunk
-            // index can be XORed into the sum)
-            const int cbase = ((i0 >> 6) * (kC * 128) + (SL * s) * 128 + ((i0 & 7) << 1)) | (((i0 & 63) >> 3) << 4);
-            auto offr = [&](int r) { return (cbase + r * 128) ^ ((r & 7) << 4); };
-            if (s == 0) {
-                // the belief at the segment start, as the first chunk's start state
-                CAR(0, 0) = make_float2(seg_lambda(i0), seg_lambda(i0 + 1));
-                CAR(1, 0) = make_float2(1.f, 1.f);
-                CAR(2, 0) = make_float2(1.f, 1.f);
-                CAR(3, 0) = i2f(0, 0);
-                CAR(4, 0) = i2f(0, 0);
-            }
-            int rho0 = 0, rho1 = 0;          // references in force (segment-start frame)
-            float2 av[SL], qv[SL];           // a, qn of the sub-block's tokens
-            float bl = 0.f, bln = 0.f;       // beta of token SL*s + lane (lanes < SL): this chunk, next
-            // a, qn of token r of this thread's sub-block in chunk c (identity step
-            // past the segment end); the addresses step by H * DK floats per token
-            const long long tstep = (long long)g.H * (DK / 2);   // in float2
-            auto load_tok = [&](int c, int r, float2 &ra, float2 &rq) {
-                const long long t0s = tb + (long long)c * kC + SL * s;
-                const long long off = ((t0s * g.H + h) * DK + i0) / 2 + r * tstep;
-                if (t0s + r < te) {
-                    ra = __ldg(reinterpret_cast<const float2 *>(g.a) + off);
-                    rq = __ldg(reinterpret_cast<const float2 *>(g.qn) + off);
-                } else {
-                    ra = make_float2(1.f, 1.f);
-                    rq = make_float2(0.f, 0.f);
-                }
-            };
-            auto load_beta = [&](int c) {
-                const long long tok = tb + (long long)c * kC + SL * s + lane;
-                return (lane < SL && tok < te) ? __ldg(g.beta + tok * g.H + h) : 0.f;
-            };
-            if (nchunks > 0) {
+            // ---- diagonal: thread = key i; it walks every token of the segment, so
+            // the precision chain and its exponents stay in registers
+            const int i = warp * 32 + lane;
+            // byte offset of (row r, key i) in a 128B-swizzled tile: sw[r & 7] + 128 r
+            // (the 16-byte chunk index, bits 4-6 of cb, is XORed with r & 7; the row
+            // term leaves those bits alone)
+            const int cb = ((i >> 6) * (kC * 128) + ((i & 7) << 1)) | (((i & 63) >> 3) << 4);
+            int sw[8];
 #pragma unroll
-                for (int r = 0; r < SL; ++r) load_tok(0, r, av[r], qv[r]);
-                bl = load_beta(0);
+            for (int x = 0; x < 8; ++x) sw[x] = cb ^ (x << 4);
+            // beta of tokens lane and 32 + lane of chunk c
+            auto load_beta = [&](int c, int half) {
+                const long long tok = tb + (long long)c * kC + 32 * half + lane;
+                return tok < te ? __ldg(g.beta + tok * g.H + h) : 0.f;
+            };
+            KeyWalk w;
+            w.n = seg_lambda(i);
+            w.d = 1.f;
+            w.p = 1.f;
+            w.E = w.F = 0;
+            w.cl = w.q0 = w.q1 = w.q2 = w.q3 = make_int2(0, 0);
+            int rho = 0;   // reference in force (segment-start frame)
+            float bA = 0.f, bB = 0.f;
+            if (nchunks > 0) {
+                bA = load_beta(0, 0);
+                bB = load_beta(0, 1);
             }
-            float lam_end0 = 0.f, lam_end1 = 0.f, gend0 = 1.f, gend1 = 1.f;
-            int xend0 = 0, xend1 = 0;
             for (int c = 0; c < nchunks; ++c) {
                 const int st = c & 1;
                 const long long tok0 = tb + (long long)c * kC;
-                const int nval = (int)min((long long)SL, max(0LL, te - (tok0 + SL * s)));   // valid tokens of the sub-block
                 uint8_t *qt = sm + L::q0 + st * L::QK;
                 uint8_t *kt = sm + L::k0 + st * L::QK;
                 uint8_t *klo = sm + L::klo0 + st * L::QK;
-                const bool okw = waitw(&stage_full[st], (c >> 1) & 1, abort_flag, g.status);
-                // ---- step 1: the sub-block's Moebius maps for both keys (columns
-                // are the images of (1, 0) and (0, 1); chain d <- a^2 d + qn n,
-                // n <- n + b d with b = beta k^2), and its product of a
-                if (okw) {
-                    float2 n1 = make_float2(1.f, 1.f), d1 = make_float2(0.f, 0.f);
-                    float2 n2 = make_float2(0.f, 0.f), d2 = make_float2(1.f, 1.f), PA = make_float2(1.f, 1.f);
-                    int em0 = 0, em1 = 0, fm0 = 0, fm1 = 0;
-#pragma unroll
-                    for (int b8 = 0; b8 < SL; b8 += 8) {
-                        uint32_t kwb[8];
-#pragma unroll
-                        for (int x = 0; x < 8; ++x) kwb[x] = *reinterpret_cast<const uint32_t *>(kt + offr(b8 + x));
-#pragma unroll
-                        for (int x = 0; x < 8; ++x) {
-                            const int r = b8 + x;
-                            const float2 kf = unpack_bf2(kwb[x]);
-                            const float be = __shfl_sync(0xffffffffu, bl, r);
-                            const float2 a2 = f2mul(av[r], av[r]);
-                            const float2 b = f2mul(f2mul(make_float2(be, be), kf), kf);
-                            d1 = f2fma(a2, d1, f2mul(qv[r], n1));
-                            n1 = f2fma(b, d1, n1);
-                            d2 = f2fma(a2, d2, f2mul(qv[r], n2));
-                            n2 = f2fma(b, d2, n2);
-                            PA = f2mul(PA, av[r]);
-                        }
-                        norm_cols(n1.x, n2.x, d1.x, d2.x, em0);
-                        norm_cols(n1.y, n2.y, d1.y, d2.y, em1);
-                        const int f0 = clampe(expo(PA.x)), f1 = clampe(expo(PA.y));
-                        PA.x *= pow2i(-f0); PA.y *= pow2i(-f1);
-                        fm0 += f0; fm1 += f1;
-                    }
-                    X(0, s) = n1; X(1, s) = n2; X(2, s) = d1; X(3, s) = d2; X(4, s) = PA;
-                    X(5, s) = i2f(em0, em1);
-                    X(6, s) = i2f(fm0, fm1);
+                const float cA = bA, cB = bB;
+                if (c + 1 < nchunks) {
+                    bA = load_beta(c + 1, 0);
+                    bB = load_beta(c + 1, 1);
                 }
-                if (named_bar_or(kGateBar, RL::GT, !okw || *abort_flag)) { ok = false; break; }
-                // ---- step 2: the state at this sub-block's start: the chunk-start
-                // state with the maps of the sub-blocks before it applied
-                float nn[2], dd[2], pa[2];
-                int E[2], F[2];
-                {
-                    const float2 cn = CAR(0, st), cd = CAR(1, st), cp = CAR(2, st), cE = CAR(3, st), cF = CAR(4, st);
-                    nn[0] = cn.x; nn[1] = cn.y; dd[0] = cd.x; dd[1] = cd.y; pa[0] = cp.x; pa[1] = cp.y;
-                    E[0] = __float_as_int(cE.x); E[1] = __float_as_int(cE.y);
-                    F[0] = __float_as_int(cF.x); F[1] = __float_as_int(cF.y);
-                }
-                for (int sj = 0; sj < s; ++sj) {
-                    const float2 m00 = X(0, sj), m01 = X(1, sj), m10 = X(2, sj), m11 = X(3, sj), mp = X(4, sj);
-                    const float2 me = X(5, sj), mf = X(6, sj);
-                    const float n0v = fmaf(m00.x, nn[0], m01.x * dd[0]), d0v = fmaf(m10.x, nn[0], m11.x * dd[0]);
-                    const float n1v = fmaf(m00.y, nn[1], m01.y * dd[1]), d1v = fmaf(m10.y, nn[1], m11.y * dd[1]);
-                    nn[0] = n0v; dd[0] = d0v; nn[1] = n1v; dd[1] = d1v;
-                    pa[0] *= mp.x; pa[1] *= mp.y;
-                    E[0] += __float_as_int(me.x); E[1] += __float_as_int(me.y);
-                    F[0] += __float_as_int(mf.x); F[1] += __float_as_int(mf.y);
-                    norm_state(nn[0], dd[0], pa[0], E[0], F[0]);
-                    norm_state(nn[1], dd[1], pa[1], E[1], F[1]);
-                }
-                // the sub-block's start state, kept for a re-walk
-                const float2 n2s0 = make_float2(nn[0], nn[1]), d2s0 = make_float2(dd[0], dd[1]);
-                const float2 p2s0 = make_float2(pa[0], pa[1]);
-                const int E00 = E[0], E01 = E[1], F00 = F[0], F01 = F[1];
-                bln = (c + 1 < nchunks) ? load_beta(c + 1) : 0.f;
-                // ---- step 3: walk the sub-block and fold every token against the
-                // reference in force (exact while |G - rho| stays within kLost):
-                //   Q' = q/lambda 2^(G - rho) = q pa/n 2^((F-E) - rho)
-                //   K' = beta k 2^(rho - G)   = beta k d/pa 2^(rho - (F-E))
-                // tracking fk = 2^(rho - G) for the chunk's G range; the next chunk's
-                // a, qn go into the freed registers
-                int2 glo, ghi;
-                bool clamped = false;
-                {
-                    float2 n2s = n2s0, d2s = d2s0, p2s = p2s0;
-                    int Ew0 = E00, Ew1 = E01, Fw0 = F00, Fw1 = F01;
-                    // x = (F - E) - rho of the current 8-token group (unclamped): with
-                    // rk = d/pa, G - rho lies in (x - expo(rk) - 1, x - expo(rk)]
-                    int x0 = Fw0 - Ew0 - rho0, x1 = Fw1 - Ew1 - rho1;
-                    clamped = x0 != clampe(x0) || x1 != clampe(x1);
-                    float2 mq = make_float2(pow2i(clampe(x0)), pow2i(clampe(x1)));
-                    float2 mk = make_float2(pow2i(-clampe(x0)), pow2i(-clampe(x1)));
-                    // G just before the sub-block
-                    float2 rkmin = make_float2(__fdividef(d2s.x, p2s.x), __fdividef(d2s.y, p2s.y));
-                    float2 rkmax = rkmin;
-                    // four tokens at a time: their chain steps (the serial part), then
-                    // their folds, which are independent of one another; each token's
-                    // a, qn registers take the next chunk's once it is folded
-                    constexpr int TG = 4;
-#pragma unroll
-                    for (int r0 = 0; r0 < SL; r0 += TG) {
-                        uint32_t kwb[TG], qwb[TG];
-#pragma unroll
-                        for (int x = 0; x < TG; ++x) {
-                            kwb[x] = *reinterpret_cast<const uint32_t *>(kt + offr(r0 + x));
-                            qwb[x] = *reinterpret_cast<const uint32_t *>(qt + offr(r0 + x));
-                        }
-                        float2 nt[TG], dt[TG], pt2[TG], bkt[TG];
-#pragma unroll
-                        for (int x = 0; x < TG; ++x) {
-                            const int r = r0 + x;
-                            const float2 kf = unpack_bf2(kwb[x]);
-                            const float be = __shfl_sync(0xffffffffu, bl, r);
-                            bkt[x] = f2mul(make_float2(be, be), kf);
-                            d2s = f2fma(f2mul(av[r], av[r]), d2s, f2mul(qv[r], n2s));
-                            n2s = f2fma(f2mul(bkt[x], kf), d2s, n2s);
-                            p2s = f2mul(p2s, av[r]);
-                            nt[x] = n2s; dt[x] = d2s; pt2[x] = p2s;
-                        }
-#pragma unroll
-                        for (int x = 0; x < TG; ++x) {
-                            const int r = r0 + x;
-                            // (rows past the segment end are never stored and their K' is
-                            // zero, so their Q' needs no masking)
-                            const float2 qf = unpack_bf2(qwb[x]);
-                            const float2 pn = f2mul(pt2[x], nt[x]);
-                            const float2 rc = make_float2(rcp_approx(pn.x), rcp_approx(pn.y));
-                            const float2 qo = f2mul(f2mul(qf, f2mul(pt2[x], mq)), f2mul(pt2[x], rc));   // q pa/n 2^x
-                            const float2 rk = f2mul(dt[x], f2mul(nt[x], rc));                         // d/pa
-                            const float2 ko = f2mul(bkt[x], f2mul(rk, mk));                            // beta k d/pa 2^-x
-                            rkmin = make_float2(fminf(rkmin.x, rk.x), fminf(rkmin.y, rk.y));
-                            rkmax = make_float2(fmaxf(rkmax.x, rk.x), fmaxf(rkmax.y, rk.y));
-                            const uint32_t kh = pack_bf2(ko.x, ko.y);
-                            const float2 khf = unpack_bf2(kh);
-                            *reinterpret_cast<uint32_t *>(qt + offr(r)) = pack_bf2(qo.x, qo.y);
-                            *reinterpret_cast<uint32_t *>(kt + offr(r)) = kh;
-                            *reinterpret_cast<uint32_t *>(klo + offr(r)) = pack_bf2(ko.x - khf.x, ko.y - khf.y);
-                            if (c + 1 < nchunks) load_tok(c + 1, r, av[r], qv[r]);
-                        }
-                        if (((r0 + TG) & 7) == 0) {
-                            // the 8-token group's G range, renormalisation, next factors
-                            const int r = r0 + TG - 1;
-                            const int lo0 = x0 - expo(rkmax.x) - 1, lo1 = x1 - expo(rkmax.y) - 1;
-                            const int hi0 = x0 - expo(rkmin.x), hi1 = x1 - expo(rkmin.y);
-                            glo = (r == 7) ? make_int2(lo0, lo1) : make_int2(min(glo.x, lo0), min(glo.y, lo1));
-                            ghi = (r == 7) ? make_int2(hi0, hi1) : make_int2(max(ghi.x, hi0), max(ghi.y, hi1));
-                            norm_state(n2s.x, d2s.x, p2s.x, Ew0, Fw0);
-                            norm_state(n2s.y, d2s.y, p2s.y, Ew1, Fw1);
-                            rkmin = make_float2(3.0e38f, 3.0e38f);
-                            rkmax = make_float2(0.f, 0.f);
-                            if (r + 1 < SL) {
-                                x0 = Fw0 - Ew0 - rho0;
-                                x1 = Fw1 - Ew1 - rho1;
-                                clamped |= x0 != clampe(x0) || x1 != clampe(x1);
-                                mq = make_float2(pow2i(clampe(x0)), pow2i(clampe(x1)));
-                                mk = make_float2(pow2i(-clampe(x0)), pow2i(-clampe(x1)));
-                            }
-                        }
-                    }
-                    if (s == NSUB - 1) {
-                        // the chunk-end state starts the next chunk
-                        const int nst = (c + 1) & 1;
-                        CAR(0, nst) = n2s; CAR(1, nst) = d2s; CAR(2, nst) = p2s;
-                        CAR(3, nst) = i2f(Ew0, Ew1);
-                        CAR(4, nst) = i2f(Fw0, Fw1);
-                        if (c == nchunks - 1) {
-                            lam_end0 = n2s.x / d2s.x;
-                            lam_end1 = n2s.y / d2s.y;
-                            gend0 = p2s.x / d2s.x;
-                            gend1 = p2s.y / d2s.y;
-                            xend0 = Fw0 - Ew0;
-                            xend1 = Fw1 - Ew1;
-                        }
-                    }
-                }
-                rng[s * NP + pr] = make_int4(glo.x, ghi.x, glo.y, ghi.y);
-                if (named_bar_or(kGateBar, RL::GT, *abort_flag != 0)) { ok = false; break; }
-                // ---- step 4: references of the pass quarters from the G ranges of
-                // every sub-block (relative to rho): R = 0 keeps the reference
-                int R0[4], R1[4];
-                int lv;
-                bool bad0, bad1;
-                {
-                    int2 qa[4], qb[4];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        constexpr int per = NSUB / 4;
-                        int4 x = rng[(q * per) * NP + pr];
-                        int2 ra = make_int2(x.x, x.y), rb = make_int2(x.z, x.w);
-#pragma unroll
-                        for (int y = 1; y < per; ++y) {
-                            x = rng[(q * per + y) * NP + pr];
-                            ra = runion(ra, make_int2(x.x, x.y));
-                            rb = runion(rb, make_int2(x.z, x.w));
-                        }
-                        qa[q] = ra;
-                        qb[q] = rb;
-                    }
-                    const int l0 = choose_refs(qa, 0, R0, bad0);
-                    const int l1 = choose_refs(qb, 0, R1, bad1);
-                    lv = max(l0, l1);
-                }
-                const int ra = pick4(R0, quarter), rb = pick4(R1, quarter);
-                // the provisional fold of this sub-block is exact while its |G - rho|
-                // stays within kLost and no exponent was clamped; a rescale by more
-                // than 2^100 is not taken in one step either: re-walk instead
-                const bool lost = clamped || glo.x < -kLost || ghi.x > kLost || glo.y < -kLost || ghi.y > kLost ||
-                                  abs(ra) > kLost || abs(rb) > kLost;
-                if (s == 0) {
-                    atomicMax(&lvl[st], (c << 2) | lv);
-                    if (bad0 || bad1) atomicOr(g.status, kStatusRange);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        facd[(st * 4 + q) * DK + i0] = R0[q] - (q ? R0[q - 1] : 0);
-                        facd[(st * 4 + q) * DK + i0 + 1] = R1[q] - (q ? R1[q - 1] : 0);
-                    }
-                    if (LOCAL && p > 0) {
-                        float *rl = g.rlog + ((u * g.NC + chunk_base + c) * 4) * DK + i0;
-#pragma unroll
-                        for (int q = 0; q < 4; ++q)
-                            *reinterpret_cast<float2 *>(rl + q * DK) =
-                                make_float2((float)(rho0 + R0[q]), (float)(rho1 + R1[q]));
-                    }
-                }
-                if (lost) {
-                    // ---- step 5a (strong forgetting): walk the sub-block again from its
-                    // start and fold against the pass reference (a, qn reloaded)
-                    rewalk_fold<DK, SL>(qt, kt, klo, cbase, n2s0, d2s0, p2s0, E00, E01, F00, F01, rho0 + ra, rho1 + rb,
-                                        g.a, g.qn, g.beta, reinterpret_cast<const __nv_bfloat16 *>(g.q),
-                                        reinterpret_cast<const __nv_bfloat16 *>(g.k), tok0 + SL * s, nval, g.H, h, i0);
-                } else if (ra != 0 || rb != 0) {
-                    // ---- step 5b: the reference moved: rescale the folded bf16 words
-                    // exactly by powers of two (Q' by 2^-R, K' by 2^R)
-                    const __nv_bfloat162 sq = __floats2bfloat162_rn(pow2i(-ra), pow2i(-rb));
-                    const __nv_bfloat162 sk = __floats2bfloat162_rn(pow2i(ra), pow2i(rb));
+                if (!waitw(&stage_full[st], (c >> 1) & 1, abort_flag, g.status)) { ok = false; break; }
+                // the chunk-start state, for a re-walk
+                const float nc = w.n, dc = w.d, pc0 = w.p;
+                const int Ec = w.E, Fc = w.F;
+                // d and p are normalised at a slice end, so G - rho lies within 1 of
+                // x = (F - E) - rho; the reference moves to the chunk start once x
+                // has drifted beyond kMove (then the provisional fold needs no rescale
+                // unless G moves by more than kStick - kMove inside the chunk)
+                int x = w.F - w.E - rho;
+                const int pre = abs(x) > kMove ? x : 0;
+                rho += pre;
+                x -= pre;
+                w.x = x;
+                w.clamped = false;
+                w.mq = pow2i(clampe(x));
+                w.mk = pow2i(-clampe(x));
+                // the chunk's ring slots (two slices each), released once read
 #pragma unroll 1
-                    for (int r = 0; r < SL; ++r) {
-                        __nv_bfloat162 *wq = reinterpret_cast<__nv_bfloat162 *>(qt + offr(r));
-                        __nv_bfloat162 *wk = reinterpret_cast<__nv_bfloat162 *>(kt + offr(r));
-                        __nv_bfloat162 *wl = reinterpret_cast<__nv_bfloat162 *>(klo + offr(r));
-                        *wq = __hmul2(*wq, sq);
-                        *wk = __hmul2(*wk, sk);
-                        *wl = __hmul2(*wl, sk);
+                for (int s16 = 0; s16 < kRpc; ++s16) {
+                    const int j = c * kRpc + s16, slot = j % kRs;
+                    if (!waitw(&ring_full[slot], (j / kRs) & 1, abort_flag, g.status)) { ok = false; break; }
+                    float *ra = reinterpret_cast<float *>(sm + L::ring0 + slot * L::RSLOT) + i;
+                    float *rq = ra + kRt * DK;
+                    const long long ts = tok0 + s16 * kRt;
+                    if (ts + kRt > te) {
+                        // past the segment end: identity steps (beta is 0 there); each
+                        // thread rewrites its own key's column only
+                        for (int x = 0; x < kRt; ++x)
+                            if (ts + x >= te) {
+                                ra[x * DK] = 1.f;
+                                rq[x * DK] = 0.f;
+                            }
+                        fence_proxy_async();
+                    }
+                    const float bs = s16 < kRpc / 2 ? cA : cB;
+                    walk_slice<false, DK>(w, qt, kt, klo, sw, 2 * s16, bs, ra, rq, rho);
+                    walk_slice<true, DK>(w, qt, kt, klo, sw, 2 * s16 + 1, bs, ra + kSl * DK, rq + kSl * DK, rho);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&ring_empty[slot]);
+                }
+                if (!ok) break;
+                // ---- references of the pass quarters (relative to rho; R = 0 keeps it)
+                int R[4];
+                bool bad;
+                {
+                    const int2 qr[4] = {w.q0, w.q1, w.q2, w.q3};
+                    const int lv = choose_refs(qr, 0, R, bad);
+                    const int lvw = __reduce_max_sync(0xffffffffu, lv);
+                    if (lane == 0) atomicMax(&lvl[st], (c << 2) | lvw);
+                }
+                if (bad) atomicOr(g.status, kStatusRange);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) facd[(st * 4 + q) * DK + i] = q ? R[q] - R[q - 1] : pre + R[0];
+                if (LOCAL && p > 0) {
+                    float *rl = g.rlog + ((u * g.NC + chunk_base + c) * 4) * DK + i;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) rl[q * DK] = (float)(rho + R[q]);
+                }
+                const int2 wr = runion(runion(w.q0, w.q1), runion(w.q2, w.q3));
+                bool far = false, moved = false;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    far |= abs(R[q]) > kLost;
+                    moved |= R[q] != 0;
+                }
+                // the provisional fold is exact while |G - rho| stayed within kLost and
+                // no exponent clamped; a rescale by more than 2^kLost is not taken in
+                // one step either: re-walk instead
+                if (w.clamped || far || wr.x < -kLost || wr.y > kLost) {
+                    rewalk_key<DK>(qt, kt, klo, cb, nc, dc, pc0, Ec, Fc,
+                                   make_int4(rho + R[0], rho + R[1], rho + R[2], rho + R[3]), g.a, g.qn, g.beta,
+                                   reinterpret_cast<const __nv_bfloat16 *>(g.q),
+                                   reinterpret_cast<const __nv_bfloat16 *>(g.k), tok0,
+                                   (int)min((long long)kC, te - tok0), g.H, h, i);
+                } else if (moved) {
+                    // a quarter's reference moved: rescale its folded bf16 values
+                    // exactly by powers of two (Q' by 2^-R, K' by 2^R)
+#pragma unroll 1
+                    for (int q = 0; q < 4; ++q) {
+                        const int r = pick4(R, q);
+                        if (r == 0) continue;
+                        const float fq = pow2i(-r), fk = pow2i(r);
+#pragma unroll 1
+                        for (int row = kQ * q; row < kQ * (q + 1); ++row) {
+                            const int o = sw[row & 7] + row * 128;
+                            uint16_t *wq = reinterpret_cast<uint16_t *>(qt + o);
+                            uint16_t *wk = reinterpret_cast<uint16_t *>(kt + o);
+                            uint16_t *wl = reinterpret_cast<uint16_t *>(klo + o);
+                            *wq = bf16_bits(bf16_val(*wq) * fq);
+                            *wk = bf16_bits(bf16_val(*wk) * fk);
+                            *wl = bf16_bits(bf16_val(*wl) * fk);
+                        }
                     }
                 }
-                rho0 += R0[3];
-                rho1 += R1[3];
-                if (c == nchunks - 1 && s == NSUB - 1) {
+                rho += R[3];
+                if (c == nchunks - 1) {
                     // final outputs of the segment: 2^(G_end - rho) for the state
                     // export, the precision, and the segment's gate product
-                    facf[i0] = scale2(gend0, xend0 - rho0);
-                    facf[i0 + 1] = scale2(gend1, xend1 - rho1);
-                    if (LOCAL) {
-                        auto prod = [](float gm, int x) {
-                            return x < -250 ? 0.f : (x > 250 ? __int_as_float(0x7f800000) : scale2(gm, x));
-                        };
-                        g.decay[(u * g.P + p) * DK + i0] = prod(gend0, xend0);
-                        g.decay[(u * g.P + p) * DK + i0 + 1] = prod(gend1, xend1);
-                    }
-                    if (last_seg && g.final_lambda) {
-                        g.final_lambda[u * DK + i0] = lam_end0;
-                        g.final_lambda[u * DK + i0 + 1] = lam_end1;
-                    }
+                    const float ge = w.p / w.d;
+                    const int xe = w.F - w.E;
+                    facf[i] = scale2(ge, xe - rho);
+                    if (LOCAL)
+                        g.decay[(u * g.P + p) * DK + i] =
+                            xe < -250 ? 0.f : (xe > 250 ? __int_as_float(0x7f800000) : scale2(ge, xe));
+                    if (last_seg && g.final_lambda) g.final_lambda[u * DK + i] = w.n / w.d;
                 }
-                bl = bln;
                 fence_proxy_async();
                 mbar_arrive(&qk_ready[st]);
             }
-            if (nchunks == 0 && s == 0 && last_seg && g.final_lambda) {
-                const float2 l0 = CAR(0, 0);
-                g.final_lambda[u * DK + i0] = l0.x;
-                g.final_lambda[u * DK + i0 + 1] = l0.y;
-            }
+            if (nchunks == 0 && last_seg && g.final_lambda) g.final_lambda[u * DK + i] = w.n;
         } else {
             // ---- isotropic: one precision per head ---------------------------
             float2 *isof = reinterpret_cast<float2 *>(sm + L::isof0);
@@ -900,11 +805,38 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (warp == 0 && lane == 0 && nchunks == 0 && last_seg && g.final_lambda) g.final_lambda[u] = lam;
         }
         (void)ok;
-    } else {
-        // ================= epilogue warps; thread 0 also issues the TMA loads and
-        // the tcgen05 MMAs at the points where the epilogue synchronises ========
-        const int we = warp - RL::EPIW;        // TMEM lane quarter (warp % 4)
-        const bool issuer = we == 0 && lane == 0;
+    } else if (!ISO && warp == RL::EPIW + 4) {
+        // ================= a / qn producer (diagonal precision): the gate's ring
+        // slots of kRt tokens, and an L2 prefetch of the slot two chunks ahead
+        if (!ISO && lane == 0) {
+            uint8_t *ring = sm + L::ring0;
+            const int nrs = nchunks * kRpc;
+            auto prefetch = [&](int j) {
+                const int tok = (int)(tb + (long long)j * kRt);
+                tma_prefetch_3d(&tm_a, 0, h, tok);
+                tma_prefetch_3d(&tm_qn, 0, h, tok);
+            };
+            for (int j = kRs; j < min(nrs, 2 * kRpc); ++j) prefetch(j);
+            int j = 0;
+            for (; j < nrs; ++j) {
+                const int slot = j % kRs;
+                if (j >= kRs && !wait1(&ring_empty[slot], ((j / kRs) - 1) & 1, abort_flag, g.status)) break;
+                float *dst = reinterpret_cast<float *>(ring + slot * L::RSLOT);
+                const int tok = (int)(tb + (long long)j * kRt);
+                mbar_expect_tx(&ring_full[slot], L::RSLOT);
+                tma_load_3d(dst, &tm_a, &ring_full[slot], 0, h, tok);
+                tma_load_3d(dst + kRt * DK, &tm_qn, &ring_full[slot], 0, h, tok);
+                if (j + 2 * kRpc < nrs) prefetch(j + 2 * kRpc);
+            }
+            // the copies issued land before the CTA exits
+            for (int r = max(0, j - kRs); r < j; ++r)
+                wait_slow(&ring_full[r % kRs], (r / kRs) & 1, abort_flag, g.status, false);
+        }
+    } else if (warp < RL::EPIW + 4) {
+        // ================= epilogue warps: rescale U in TMEM and snapshot it to
+        // bf16 shared memory, mask the score tile into P, store the output rows;
+        // each pass is handed to the MMA warp through mbarriers ==============
+        const int we = warp & 3;               // TMEM lane quarter
         const uint32_t lane_base = (uint32_t)(32 * we) << 16;
         const int row64 = 16 * we + lane;
         const bool v64 = lane < 16;
@@ -914,44 +846,6 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         uint8_t *pt = sm + L::p0;
         const float *eta0 = ((!LOCAL || p == 0) && g.eta0) ? g.eta0 + u * DK * DV : nullptr;
         bool ok = true;
-        // q, k, v tiles of chunk c into stage c & 1, and an L2 prefetch of the
-        // chunk two ahead (its tiles, a and qn: the gate loads those itself)
-        auto load_chunk = [&](int c) {
-            const int tok0 = (int)(tb + (long long)c * kC);
-            const int s = c & 1;
-            mbar_expect_tx(&stage_full[s], 2 * L::QK + L::V);
-#pragma unroll
-            for (int a = 0; a < DK / 64; ++a) {
-                tma_load_3d(sm + L::q0 + s * L::QK + a * kC * 128, &tm_q, &stage_full[s], 64 * a, h, tok0);
-                tma_load_3d(sm + L::k0 + s * L::QK + a * kC * 128, &tm_k, &stage_full[s], 64 * a, h, tok0);
-            }
-#pragma unroll
-            for (int a = 0; a < DV / 64; ++a)
-                tma_load_3d(sm + L::v0 + s * L::V + a * kC * 128, &tm_v, &stage_full[s], 64 * a, h, tok0);
-            if (c + 2 < nchunks) {
-                const int tp = tok0 + 2 * kC;
-#pragma unroll
-                for (int a = 0; a < DK / 64; ++a) {
-                    tma_prefetch_3d(&tm_q, 64 * a, h, tp);
-                    tma_prefetch_3d(&tm_k, 64 * a, h, tp);
-                }
-#pragma unroll
-                for (int a = 0; a < DV / 64; ++a) tma_prefetch_3d(&tm_v, 64 * a, h, tp);
-                if (!ISO) {
-                    tma_prefetch_3d(&tm_a, 0, h, tp);
-                    tma_prefetch_3d(&tm_qn, 0, h, tp);
-                }
-            }
-        };
-        int loaded = 0;                                 // chunks whose loads were issued
-        if (issuer) {
-            // a and qn of chunk 1 (chunk 0 is read at once)
-            if (!ISO && nchunks > 1) {
-                tma_prefetch_3d(&tm_a, 0, h, (int)(tb + kC));
-                tma_prefetch_3d(&tm_qn, 0, h, (int)(tb + kC));
-            }
-            for (; loaded < 2 && loaded < nchunks; ++loaded) load_chunk(loaded);
-        }
         // Belief at the segment start, written into the U columns of TMEM before
         // the first chunk (while the gate works on it): eta0 for whole rows and
         // first segments, zero for the later segments of split rows (their
@@ -971,11 +865,6 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             tmem_wait_st();
         }
-        constexpr uint32_t iS = idesc_bf16(64, 64, false, false);
-        constexpr uint32_t iO = idesc_bf16(64, DV, false, true);
-        constexpr uint32_t iU = idesc_bf16(DK, DV, true, true);
-        const uint32_t tS = tbase + L::colS, tO = tbase + L::colO, tU = tbase + L::colU;
-        const uint32_t uba = smem_u32(sm + L::ub0);
         int pc = 0;                                   // passes so far (barrier phases)
         // The output rows of a pass are read out during the next pass (after its
         // P mask), from the other of two output accumulators, so the epilogue
@@ -1009,50 +898,22 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
             tc_fence_before();
         };
-        // every exit from this loop goes through a reducing barrier, so that the
-        // four warps leave it together
-        for (int c = 0; c < nchunks; ++c) {
+        for (int c = 0; c < nchunks && ok; ++c) {
             const int st = c & 1;
-            if (!waitw(&qk_ready[st], (c >> 1) & 1, abort_flag, g.status)) { ok = false; }
-            if (named_bar_or(kEpiBar, 128, !ok || *abort_flag)) { ok = false; break; }
-            tc_fence_after();
+            if (!waitw(&qk_ready[st], (c >> 1) & 1, abort_flag, g.status)) { ok = false; break; }
             const int lv = lvl[st] & 3;
             const int np = 1 << lv, qper = 4 >> lv;
-            const uint32_t qa = smem_u32(sm + L::q0 + st * L::QK);
-            const uint32_t ka = smem_u32(sm + L::k0 + st * L::QK);
-            const uint32_t va = smem_u32(sm + L::v0 + st * L::V);
-            const uint32_t kloa = smem_u32(sm + L::klo0 + st * L::QK);
-            if (issuer) {
-                if (LOCAL && p > 0) {
-                    // export the folded q tile (the correction pass multiplies it by
-                    // the carried segment-start state)
-                    const int tok0 = (int)(tb + (long long)c * kC);
-#pragma unroll
-                    for (int a = 0; a < DK / 64; ++a)
-                        tma_store_3d(&tm_qs, sm + L::q0 + st * L::QK + a * kC * 128, 64 * a, h, tok0);
-                    tma_store_commit();
-                }
-                // scores of the whole chunk (each pass masks its own block); the
-                // K step moves a descriptor's start address by (bytes >> 4)
-                const uint64_t dq = sdesc_sw128(qa, 16, 1024), dk = sdesc_sw128(ka, 16, 1024);
-#pragma unroll 1
-                for (int kk = 0; kk < DK / 16; ++kk) {
-                    const uint32_t off = ((kk >> 2) * (kC * 128) + (kk & 3) * 32) >> 4;
-                    mma_bf16(tS, dq + off, dk + off, iS, kk > 0);
-                }
-                mma_commit(s_full);
-            }
             for (int k = 0; k < np; ++k) {
                 const int m0 = kQ * qper * k, m1 = m0 + kQ * qper;
-                const int s0 = k * qper, s1 = s0 + qper;      // 16-token slices of this pass
-                const uint32_t tOp = tO + (pc & 1) * DV;      // this pass's output accumulator
-                uint8_t *ptp = pt + (pc & 1) * L::PT;         // and its P buffer
+                uint8_t *ptp = pt + (pc & 1) * L::PT;         // this pass's P buffer
                 // ---- state: U <- 2^d U for this pass's reference, snapshot to bf16
-                if (pc > 0 && !waitw(u_done, (pc - 1) & 1, abort_flag, g.status)) ok = false;
+                // (the previous pass's state update, and its Q' U reading the old
+                // snapshot, have completed)
+                if (pc > 0 && !waitw(u_done, (pc - 1) & 1, abort_flag, g.status)) { ok = false; break; }
                 tc_fence_after();
                 const int d = vU ? facd[(st * 4 + k * qper) * DK + rowU] : 0;
                 const bool rmw = __any_sync(0xffffffffu, d != 0);
-                if (ok) {
+                {
                     if (rmw) tmem_scale_lane<DV>(tbase + lane_base + L::colU, d);
                     uint32_t r2[DV / 32][32];
 #pragma unroll
@@ -1076,20 +937,9 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
                 fence_proxy_async();
                 tc_fence_before();
-                if (named_bar_or(kEpiBar, 128, !ok || *abort_flag)) { ok = false; break; }
-                if (issuer) {
-                    tc_fence_after();
-                    // O = Q' U into this pass's accumulator (its previous contents, two
-                    // passes back, were read out before the barrier)
-                    const uint64_t dq = sdesc_sw128(qa, 16, 1024), du = sdesc_sw128(uba, DK * 128, 1024);
-#pragma unroll 1
-                    for (int kk = 0; kk < DK / 16; ++kk) {
-                        const uint32_t off = ((kk >> 2) * (kC * 128) + (kk & 3) * 32) >> 4;
-                        mma_bf16(tOp, dq + off, du + kk * (2048 >> 4), iO, kk > 0);
-                    }
-                }
+                mbar_arrive(snap_ready);
                 // ---- P = the pass's block of the causal score tile, bf16
-                if (k == 0 && !waitw(s_full, c & 1, abort_flag, g.status)) ok = false;
+                if (k == 0 && !waitw(s_full, c & 1, abort_flag, g.status)) { ok = false; break; }
                 tc_fence_after();
                 if (ok) {
                     uint32_t r2[2][32];
@@ -1117,39 +967,12 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
                 fence_proxy_async();
                 tc_fence_before();
-                if (named_bar_or(kEpiBar, 128, !ok || *abort_flag)) { ok = false; break; }
-                if (issuer) {
-                    tc_fence_after();
-                    // O += P V over this pass's tokens; then the state update, whose
-                    // completion (u_done) the next pass's snapshot waits for
-                    const uint64_t dp = sdesc_sw128(smem_u32(ptp), 16, 1024), dv = sdesc_sw128(va, kC * 128, 1024);
-                    const uint64_t dk = sdesc_sw128(ka, kC * 128, 1024), dl = sdesc_sw128(kloa, kC * 128, 1024);
-#pragma unroll 1
-                    for (int kk = s0; kk < s1; ++kk) mma_bf16(tOp, dp + kk * (32 >> 4), dv + kk * (2048 >> 4), iO, 1);
-                    mma_commit(&o_full[pc & 1]);
-                    // U += K'^T V over this pass's tokens (hi and remainder of K')
-#pragma unroll 1
-                    for (int kk = s0; kk < s1; ++kk) {
-                        mma_bf16(tU, dk + kk * (2048 >> 4), dv + kk * (2048 >> 4), iU, 1);
-                        mma_bf16(tU, dl + kk * (2048 >> 4), dv + kk * (2048 >> 4), iU, 1);
-                    }
-                    mma_commit(u_done);
-                }
+                mbar_arrive(&p_ready[pc & 1]);
                 // ---- output rows of the previous pass (its MMAs have finished
                 // while this pass was prepared)
-                if (ok && pend_c >= 0) emit(pc - 1, pend_c, pend_m0, pend_m1);
+                if (pend_c >= 0) emit(pc - 1, pend_c, pend_m0, pend_m1);
                 pend_c = c; pend_m0 = m0; pend_m1 = m1;
                 ++pc;
-            }
-            if (named_bar_or(kEpiBar, 128, !ok || *abort_flag)) { ok = false; break; }
-            // every MMA of this chunk has completed once its last u_done has (the
-            // state update is the last reader of K' and V): the stage takes the
-            // chunk two ahead once the q' export has read it. Only the issuing
-            // thread waits; the other warps go on to the next chunk.
-            if (issuer) {
-                ok = wait_slow(u_done, (pc - 1) & 1, abort_flag, g.status, true) && ok;
-                if (LOCAL && p > 0) tma_store_wait_read();
-                if (ok && loaded < nchunks) { load_chunk(loaded); ++loaded; }
             }
         }
         if (ok && pend_c >= 0) emit(pc - 1, pend_c, pend_m0, pend_m1);
@@ -1181,23 +1004,134 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 for (int x = 0; x < DV; ++x) dst[rowU * DV + x] = eta0 ? eta0[rowU * DV + x] : 0.f;
             }
         }
-        if (issuer) {
+    } else if (warp == RL::MMAW) {
+        // ================= MMA warp: the q, k, v tile loads, the q' export of
+        // split rows (lane 0), and the tcgen05 MMAs (the converged warp, one
+        // elected lane issuing: see mma_bf16_warp) ===========================
+        bool ok = true;
+        auto load_chunk = [&](int c) {
+            const int tok0 = (int)(tb + (long long)c * kC);
+            const int s = c & 1;
+            mbar_expect_tx(&stage_full[s], 2 * L::QK + L::V);
+    #pragma unroll
+            for (int a = 0; a < DK / 64; ++a) {
+                tma_load_3d(sm + L::q0 + s * L::QK + a * kC * 128, &tm_q, &stage_full[s], 64 * a, h, tok0);
+                tma_load_3d(sm + L::k0 + s * L::QK + a * kC * 128, &tm_k, &stage_full[s], 64 * a, h, tok0);
+            }
+    #pragma unroll
+            for (int a = 0; a < DV / 64; ++a)
+                tma_load_3d(sm + L::v0 + s * L::V + a * kC * 128, &tm_v, &stage_full[s], 64 * a, h, tok0);
+            if (c + 2 < nchunks) {
+                const int tp = tok0 + 2 * kC;
+    #pragma unroll
+                for (int a = 0; a < DK / 64; ++a) {
+                    tma_prefetch_3d(&tm_q, 64 * a, h, tp);
+                    tma_prefetch_3d(&tm_k, 64 * a, h, tp);
+                }
+    #pragma unroll
+                for (int a = 0; a < DV / 64; ++a) tma_prefetch_3d(&tm_v, 64 * a, h, tp);
+            }
+        };
+        int loaded = 0;                                 // chunks whose loads were issued
+        if (lane == 0)
+            for (; loaded < 2 && loaded < nchunks; ++loaded) load_chunk(loaded);
+        loaded = min(2, nchunks);
+        constexpr uint32_t iS = idesc_bf16(64, 64, false, false);
+        constexpr uint32_t iO = idesc_bf16(64, DV, false, true);
+        constexpr uint32_t iU = idesc_bf16(DK, DV, true, true);
+        const uint32_t tS = tbase + L::colS, tO = tbase + L::colO, tU = tbase + L::colU;
+        const uint64_t du = sdesc_sw128(smem_u32(sm + L::ub0), DK * 128, 1024);
+        int pc = 0;
+        for (int c = 0; c < nchunks; ++c) {
+            const int st = c & 1;
+            if (!waitw(&qk_ready[st], (c >> 1) & 1, abort_flag, g.status)) { ok = false; break; }
+            const int lv = lvl[st] & 3;
+            const int np = 1 << lv, qper = 4 >> lv;
+            if (LOCAL && p > 0 && lane == 0) {
+                // export the folded q tile (the correction pass multiplies it by
+                // the carried segment-start state)
+                const int tok0 = (int)(tb + (long long)c * kC);
+#pragma unroll
+                for (int a = 0; a < DK / 64; ++a)
+                    tma_store_3d(&tm_qs, sm + L::q0 + st * L::QK + a * kC * 128, 64 * a, h, tok0);
+                tma_store_commit();
+            }
+            __syncwarp();
+            tc_fence_after();
+            // scores of the whole chunk (each pass masks its own block); a K step
+            // moves a descriptor's start address by (bytes >> 4)
+            const uint32_t qa = smem_u32(sm + L::q0 + st * L::QK), ka = smem_u32(sm + L::k0 + st * L::QK);
+            const uint64_t dq = sdesc_sw128(qa, 16, 1024), dk = sdesc_sw128(ka, 16, 1024);
+#pragma unroll
+            for (int kk = 0; kk < DK / 16; ++kk) {
+                const uint32_t off = ((kk >> 2) * (kC * 128) + (kk & 3) * 32) >> 4;
+                mma_bf16_warp(tS, dq + off, dk + off, iS, kk > 0);
+            }
+            mma_commit_warp(s_full);
+            const uint64_t dv = sdesc_sw128(smem_u32(sm + L::v0 + st * L::V), kC * 128, 1024);
+            const uint64_t dkm = sdesc_sw128(ka, kC * 128, 1024);
+            const uint64_t dl = sdesc_sw128(smem_u32(sm + L::klo0 + st * L::QK), kC * 128, 1024);
+            for (int k = 0; k < np; ++k) {
+                const int s0 = k * qper;                      // first 16-token slice of this pass
+                const uint32_t tOp = tO + (pc & 1) * DV;      // this pass's output accumulator
+                const uint64_t dp = sdesc_sw128(smem_u32(sm + L::p0 + (pc & 1) * L::PT), 16, 1024);
+                // O = Q' U (the snapshot) into this pass's accumulator (its contents
+                // two passes back were read out before the snapshot), then the state
+                // update over the pass's tokens (hi and remainder of K'): it reads
+                // only K' and V, so it runs while P is masked
+                if (!waitw(snap_ready, pc & 1, abort_flag, g.status)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < DK / 16; ++kk) {
+                    const uint32_t off = ((kk >> 2) * (kC * 128) + (kk & 3) * 32) >> 4;
+                    mma_bf16_warp(tOp, dq + off, du + kk * (2048 >> 4), iO, kk > 0);
+                }
+#pragma unroll
+                for (int x = 0; x < 4; ++x)
+                    if (x < qper) {
+                        const uint32_t ko = (s0 + x) * (2048 >> 4);
+                        mma_bf16_warp(tU, dkm + ko, dv + ko, iU, 1);
+                        mma_bf16_warp(tU, dl + ko, dv + ko, iU, 1);
+                    }
+                mma_commit_warp(u_done);
+                // O += P V over the pass's tokens: its last MMA
+                if (!waitw(&p_ready[pc & 1], (pc >> 1) & 1, abort_flag, g.status)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int x = 0; x < 4; ++x)
+                    if (x < qper) mma_bf16_warp(tOp, dp + (s0 + x) * (32 >> 4), dv + (s0 + x) * (2048 >> 4), iO, 1);
+                mma_commit_warp(&o_full[pc & 1]);
+                ++pc;
+            }
+            if (!ok) break;
+            // every MMA of the chunk has completed once its last P V has: the
+            // stage takes the chunk two ahead once the q' export has read it
+            if (!waitw(&o_full[(pc - 1) & 1], ((pc - 1) >> 1) & 1, abort_flag, g.status)) { ok = false; break; }
+            if (lane == 0) {
+                if (LOCAL && p > 0) tma_store_wait_read();
+                if (loaded < nchunks) load_chunk(loaded);
+            }
+            if (loaded < nchunks) ++loaded;
+        }
+        if (lane == 0) {
             if (LOCAL && p > 0) tma_store_wait_all();
             if (!ok || *abort_flag) {
                 // wait (bounded) until every tile load issued has landed
                 for (int c = max(0, loaded - 2); c < loaded; ++c)
                     wait_slow(&stage_full[c & 1], (c >> 1) & 1, abort_flag, g.status, false);
             }
-            // all MMAs issued have completed before TMEM is released
-            mma_commit(td_bar);
-            wait_slow(td_bar, 0, abort_flag, g.status, false);
         }
+        __syncwarp();
+        // all MMAs issued have completed before TMEM is released
+        mma_commit_warp(td_bar);
+        if (lane == 0) wait_slow(td_bar, 0, abort_flag, g.status, false);
+        __syncwarp();
     }
 
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == RL::EPIW) tmem_dealloc(tbase, L::NCOLS);
+    if (warp == RL::MMAW) tmem_dealloc(tbase, L::NCOLS);
 }
 
 // ---- host side ---------------------------------------------------------------
@@ -1253,10 +1187,10 @@ cudaError_t launch_t(const Plan &p, const int *cu, int mode, const void *q, cons
     bool ok = make_tma_map(&mq, q, BF, 2, DK, p.H, p.ntok, 64, kC, true) &&
               make_tma_map(&mk, k, BF, 2, DK, p.H, p.ntok, 64, kC, true) &&
               make_tma_map(&mv, v, BF, 2, DV, p.H, p.ntok, 64, kC, true);
-    // a and qn: L2 prefetch boxes of a whole chunk (the gate loads them itself)
+    // a and qn: ring slots of kRt tokens (their L2 prefetch uses the same boxes)
     if (ok && !p.iso)
-        ok = make_tma_map(&ma, a, F32, 4, DK, p.H, p.ntok, DK, kC, false) &&
-             make_tma_map(&mqn, qn, F32, 4, DK, p.H, p.ntok, DK, kC, false);
+        ok = make_tma_map(&ma, a, F32, 4, DK, p.H, p.ntok, DK, kRt, false) &&
+             make_tma_map(&mqn, qn, F32, 4, DK, p.H, p.ntok, DK, kRt, false);
     else { ma = mq; mqn = mq; }
     if (ok && mode == 2) ok = make_tma_map(&mqs, p.qbuf, BF, 2, DK, p.H, p.ntok, 64, kC, true);
     else mqs = mq;
@@ -1282,7 +1216,8 @@ cudaError_t launch_t(const Plan &p, const int *cu, int mode, const void *q, cons
     g.final_lambda = final_lambda; g.final_eta = final_eta; g.status = status;
     const unsigned grid = (unsigned)((long long)p.N * p.H * p.P);
     if (grid == 0) return cudaSuccess;
-    return launch_pdl(kerns[which], grid, Roles<DK, DV>::THREADS, L::alloc, st, mq, mk, mv, ma, mqn, mqs, g);
+    const int threads = p.iso ? Roles<DK, DV, true>::THREADS : Roles<DK, DV, false>::THREADS;
+    return launch_pdl(kerns[which], grid, threads, L::alloc, st, mq, mk, mv, ma, mqn, mqs, g);
 }
 
 }  // namespace
