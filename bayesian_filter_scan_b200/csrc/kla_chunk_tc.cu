@@ -78,7 +78,6 @@ constexpr int kRt = 16;       // tokens per a / qn ring slot of the diagonal gat
 constexpr int kRpc = kC / kRt;             // ring slots per chunk
 constexpr int kRs = 2;                     // ring slots
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
-constexpr int kGateBar = 1;   // named barrier of the gate warps
 
 // Gate warps first, then the four epilogue warps (TMEM lane quarter = warp % 4),
 // the warp that streams a and qn into the diagonal gate's ring (diagonal only),
@@ -89,6 +88,9 @@ template <int DK, int DV, bool ISO>
 struct Roles {
     static constexpr int NGW = ISO ? 3 : DK / 32;     // gate warps
     static constexpr int GT = NGW * 32;               // gate threads
+    // threads that arrive on qk_ready: every diagonal gate thread; the isotropic
+    // gate's folding warps (warp 0 scans ahead of them)
+    static constexpr int QKA = ISO ? (NGW - 1) * 32 : GT;
     static constexpr int EPIW = NGW;                  // first epilogue warp
     static constexpr int MMAW = NGW + (ISO ? 4 : 5);  // TMEM owner, tile loads, MMA issue
     static constexpr int THREADS = (MMAW + 1) * 32;
@@ -131,7 +133,7 @@ struct Layout {
     static constexpr int isof0 = facf0 + DK * 4;     // [2][kC] float2: iso per-token factors
     static constexpr int lvl0 = isof0 + 2 * kC * 8;  // int[2]: pass level of the chunk, tagged with its index
     static constexpr int bar0 = lvl0 + 16;
-    static constexpr int NBAR = 12 + 2 * kRs;
+    static constexpr int NBAR = 14 + 2 * kRs;
     static constexpr int hold0 = bar0 + NBAR * 8;
     static constexpr int bytes = hold0 + 16;
     static constexpr int alloc = bytes + 1024;
@@ -215,13 +217,17 @@ __device__ __forceinline__ Mob shfl_up_mob(const Mob &m, int d) {
                __shfl_up_sync(0xffffffffu, m.m10, d), __shfl_up_sync(0xffffffffu, m.m11, d)};
 }
 
+// Sum of squares of row `row` of a 128B-swizzled bf16 tile (the order of its
+// 16-byte chunks does not matter). Lane l starts at chunk l, so that a warp
+// reading different rows spreads over the banks (a 4-way conflict, not 32).
 template <int DK>
-__device__ __forceinline__ float row_sumsq(const uint8_t *ktile, int row) {
+__device__ __forceinline__ float row_sumsq(const uint8_t *ktile, int row, int lane) {
     float s = 0.f;
 #pragma unroll
     for (int a = 0; a < DK / 64; ++a) {
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
+        for (int c8 = 0; c8 < 8; ++c8) {
+            const int ch = (c8 + lane) & 7;
             uint4 x = *reinterpret_cast<const uint4 *>(ktile + a * kC * 128 + row * 128 + ch * 16);
             const uint32_t w[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
@@ -431,8 +437,10 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // shared memory; its P tile is (one barrier per P buffer, so that a phase is
     // seen before the barrier can complete again)
     uint64_t *snap_ready = bars + 9, *p_ready = bars + 10;
+    // isotropic gate: the chunk's per-token factors are in shared memory (per stage)
+    uint64_t *scan_done = bars + 12;
     // a / qn ring of the diagonal gate: slot landed, slot read by every gate warp
-    uint64_t *ring_full = bars + 12, *ring_empty = bars + 12 + kRs;
+    uint64_t *ring_full = bars + 14, *ring_empty = bars + 14 + kRs;
     uint32_t *tmem_hold = reinterpret_cast<uint32_t *>(sm + L::hold0);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::hold0 + 4);
     int *lvl = reinterpret_cast<int *>(sm + L::lvl0);
@@ -444,7 +452,7 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(&stage_full[s], 1);
-            mbar_init(&qk_ready[s], RL::GT);
+            mbar_init(&qk_ready[s], RL::QKA);
             lvl[s] = -1;
         }
         mbar_init(s_full, 1);
@@ -453,6 +461,8 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mbar_init(&o_full[1], 1);
         mbar_init(td_bar, 1);
         mbar_init(snap_ready, 128);
+        mbar_init(&scan_done[0], 32);
+        mbar_init(&scan_done[1], 32);
         mbar_init(&p_ready[0], 128);
         mbar_init(&p_ready[1], 128);
         if (!ISO)
@@ -689,6 +699,9 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 lam = seg_lambda(0);
                 if (nchunks > 0) prefetch(0);
             }
+            // warp 0 scans each chunk's precision path and writes its per-token
+            // factors (up to two chunks ahead of the folding); the other gate warps
+            // fold the rows once a chunk's factors are in (scan_done)
             for (int c = 0; c < nchunks; ++c) {
                 const int st = c & 1;
                 const long long tok0 = tb + (long long)c * kC;
@@ -705,8 +718,8 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         const int t0i = 2 * lane, t1i = t0i + 1;
                         const bool va = tok0 + t0i < te, vb = tok0 + t1i < te;
                         const float inv_dk = 1.0f / (float)DK;
-                        const float b0 = va ? cb0 * row_sumsq<DK>(kt, t0i) * inv_dk : 0.f;
-                        const float b1 = vb ? cb1 * row_sumsq<DK>(kt, t1i) * inv_dk : 0.f;
+                        const float b0 = va ? cb0 * row_sumsq<DK>(kt, t0i, lane) * inv_dk : 0.f;
+                        const float b1 = vb ? cb1 * row_sumsq<DK>(kt, t1i, lane) * inv_dk : 0.f;
                         Mob Mp = mob_norm(mob_mul(mob_step(a1, q1, b1), mob_step(a0, q0, b0)));
 #pragma unroll
                         for (int d = 1; d < 32; d <<= 1) {
@@ -715,11 +728,11 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         }
                         Mob Ex = shfl_up_mob(Mp, 1);
                         if (lane == 0) Ex = Mob{1.f, 0.f, 0.f, 1.f};
-                        const float lamA = mob_apply(Ex, lam);
+                        const float lamA = fmaf(Ex.m00, lam, Ex.m01) * rcp_approx(fmaf(Ex.m10, lam, Ex.m11));
                         float g0 = 1.f, lamB = lamA, g1 = 1.f, lamC;
-                        if (va) { float rr = __frcp_rn(fmaf(a0, a0, q0 * lamA)); g0 = a0 * rr; lamB = fmaf(lamA, rr, b0); }
+                        if (va) { float rr = rcp_approx(fmaf(a0, a0, q0 * lamA)); g0 = a0 * rr; lamB = fmaf(lamA, rr, b0); }
                         lamC = lamB;
-                        if (vb) { float rr = __frcp_rn(fmaf(a1, a1, q1 * lamB)); g1 = a1 * rr; lamC = fmaf(lamB, rr, b1); }
+                        if (vb) { float rr = rcp_approx(fmaf(a1, a1, q1 * lamB)); g1 = a1 * rr; lamC = fmaf(lamB, rr, b1); }
                         const float l0 = __log2f(g0), l1 = __log2f(g1);
                         float sum = l0 + l1;
 #pragma unroll
@@ -751,8 +764,10 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         const float Rq = (float)pick4(R, myq);
                         // per-token factors: q / lambda 2^(G - rho_q), beta 2^(rho_q - G)
                         const float e0 = D + G0 - Rq, e1 = D + G1 - Rq;
-                        isof[st * kC + t0i] = va ? make_float2(exp2f(e0) / lamB, cb0 * exp2f(-e0)) : make_float2(0.f, 0.f);
-                        isof[st * kC + t1i] = vb ? make_float2(exp2f(e1) / lamC, cb1 * exp2f(-e1)) : make_float2(0.f, 0.f);
+                        isof[st * kC + t0i] =
+                            va ? make_float2(ex2_approx(e0) * rcp_approx(lamB), cb0 * ex2_approx(-e0)) : make_float2(0.f, 0.f);
+                        isof[st * kC + t1i] =
+                            vb ? make_float2(ex2_approx(e1) * rcp_approx(lamC), cb1 * ex2_approx(-e1)) : make_float2(0.f, 0.f);
                         for (int i = lane; i < DK; i += 32) {
 #pragma unroll
                             for (int q = 0; q < 4; ++q) facd[(st * 4 + q) * DK + i] = R[q] - (q ? R[q - 1] : 0);
@@ -782,22 +797,39 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                         }
                     }
                 }
-                if (named_bar_or(kGateBar, RL::GT, !okw || *abort_flag)) { ok = false; break; }
-                // fold the rows: Q' = q fq, K' = k fk (hi + remainder); thread = (row, key pair)
-                constexpr int NP = DK / 2;
-#pragma unroll 4
-                for (int it = tid; it < kC * NP; it += RL::GT) {
-                    const int row = it / NP, i0 = 2 * (it % NP);
-                    const int off = sw_off(row, i0, kC);
-                    const float2 f = isof[st * kC + row];
-                    const float2 qf = unpack_bf2(*reinterpret_cast<const uint32_t *>(qt + off));
-                    const float2 kf = unpack_bf2(*reinterpret_cast<const uint32_t *>(kt + off));
-                    const float2 ko = make_float2(kf.x * f.y, kf.y * f.y);
-                    const uint32_t kh = pack_bf2(ko.x, ko.y);
-                    const float2 khf = unpack_bf2(kh);
-                    *reinterpret_cast<uint32_t *>(qt + off) = pack_bf2(qf.x * f.x, qf.y * f.x);
-                    *reinterpret_cast<uint32_t *>(kt + off) = kh;
-                    *reinterpret_cast<uint32_t *>(klo + off) = pack_bf2(ko.x - khf.x, ko.y - khf.y);
+                if (warp == 0) {
+                    if (!okw) { ok = false; break; }
+                    mbar_arrive(&scan_done[st]);
+                    continue;
+                }
+                if (!waitw(&scan_done[st], (c >> 1) & 1, abort_flag, g.status)) { ok = false; break; }
+                // fold the rows: Q' = q fq, K' = k fk (hi + remainder). A folding thread
+                // keeps one key pair and a fixed set of rows within every 8-row group
+                // (so that its swizzled offsets are fixed); a warp shares the rows, so
+                // the row factors are broadcast reads
+                {
+                    constexpr int NP = DK / 2, FT = RL::GT - 32;
+                    constexpr int RS = FT / NP, XR = 8 / RS;      // threads per pair, rows per group
+                    const int ft = tid - 32, i0 = 2 * (ft % NP), s = ft / NP;
+                    const int cbp = ((i0 >> 6) * (kC * 128) + ((i0 & 7) << 1)) | (((i0 & 63) >> 3) << 4);
+                    const int x0 = s * XR;
+#pragma unroll 2
+                    for (int r8 = 0; r8 < kC; r8 += 8) {
+#pragma unroll
+                        for (int x = 0; x < XR; ++x) {
+                            const int row = r8 + x0 + x;
+                            const int off = (cbp ^ ((x0 + x) << 4)) + row * 128;
+                            const float2 f = isof[st * kC + row];
+                            const float2 qf = unpack_bf2(*reinterpret_cast<const uint32_t *>(qt + off));
+                            const float2 kf = unpack_bf2(*reinterpret_cast<const uint32_t *>(kt + off));
+                            const float2 ko = make_float2(kf.x * f.y, kf.y * f.y);
+                            const uint32_t kh = pack_bf2(ko.x, ko.y);
+                            const float2 khf = unpack_bf2(kh);
+                            *reinterpret_cast<uint32_t *>(qt + off) = pack_bf2(qf.x * f.x, qf.y * f.x);
+                            *reinterpret_cast<uint32_t *>(kt + off) = kh;
+                            *reinterpret_cast<uint32_t *>(klo + off) = pack_bf2(ko.x - khf.x, ko.y - khf.y);
+                        }
+                    }
                 }
                 fence_proxy_async();
                 mbar_arrive(&qk_ready[st]);
