@@ -120,8 +120,9 @@ static kla_status make_plan(const kla_desc *d, Plan &p, bool precision_only) {
     } else {
         p.NB = (int)((p.T + kBlockTokens - 1) / kBlockTokens);
         if (p.NB < 1) p.NB = 1;
-        // resident walk CTAs per SM (one for every walk kernel)
-        const int per_sm = 1;
+        // resident walk CTAs per SM: two for the tensor-core walk at dk = dv = 64
+        // (its shared memory, TMEM columns and registers fit twice), else one
+        const int per_sm = (chunk_tc_supported(p) && p.dk == 64 && p.dv == 64) ? 2 : 1;
         int P = precision_only ? p.NB : choose_segments((long long)p.N * p.H, p.NB, per_sm);
         p.seg_blocks = (p.NB + P - 1) / P;
         p.P = (p.NB + p.seg_blocks - 1) / p.seg_blocks;

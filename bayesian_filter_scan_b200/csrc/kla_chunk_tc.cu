@@ -94,7 +94,9 @@ struct Roles {
     static constexpr int EPIW = NGW;                  // first epilogue warp
     static constexpr int MMAW = NGW + (ISO ? 4 : 5);  // TMEM owner, tile loads, MMA issue
     static constexpr int THREADS = (MMAW + 1) * 32;
-    static constexpr int MIN_BLOCKS = 1;
+    // two CTAs per SM at dk = dv = 64 (the planner counts on it): 128 registers
+    // per thread, half the shared memory and TMEM each
+    static constexpr int MIN_BLOCKS = (DK == 64 && DV == 64) ? 2 : 1;
 };
 
 struct TcArgs {
@@ -112,6 +114,9 @@ struct TcArgs {
     // mode 2: per chunk, pass quarter and key, the reference rho of the folded
     // q' (segment-start frame): rlog[((u * NC + chunk of the row) * 4 + quarter) * DK + key]
     float *rlog;
+    // test switch (KLA_TEST_WITHHOLD_TILES): the MMA warp issues no tile loads,
+    // so the first wait on them runs out and the bounded-wait path is exercised
+    int withhold_tiles;
 };
 
 template <int DK, int DV>
@@ -138,9 +143,11 @@ struct Layout {
     static constexpr int bytes = hold0 + 16;
     static constexpr int alloc = bytes + 1024;
     static_assert(alloc <= 232448, "shared memory per CTA");
+    static_assert(!(DK == 64 && DV == 64) || 2 * (alloc + 1024) <= 233472, "two CTAs per SM at dk = dv = 64");
     // TMEM columns: the state U, two output accumulators (by pass), the scores
     static constexpr uint32_t NCOLS = (3 * DV + 64 <= 256) ? 256u : 512u;
     static constexpr uint32_t colU = 0, colO = DV, colS = 3 * DV;
+    static_assert(!(DK == 64 && DV == 64) || NCOLS <= 256, "two CTAs' TMEM at dk = dv = 64");
 };
 
 // Byte offset of element (row, col) in a 128B-swizzled bf16 tile stored as
@@ -1065,9 +1072,10 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             }
         };
         int loaded = 0;                                 // chunks whose loads were issued
+        const int nload = g.withhold_tiles ? 0 : nchunks;
         if (lane == 0)
-            for (; loaded < 2 && loaded < nchunks; ++loaded) load_chunk(loaded);
-        loaded = min(2, nchunks);
+            for (; loaded < 2 && loaded < nload; ++loaded) load_chunk(loaded);
+        loaded = min(2, nload);
         constexpr uint32_t iS = idesc_bf16(64, 64, false, false);
         constexpr uint32_t iO = idesc_bf16(64, DV, false, true);
         constexpr uint32_t iU = idesc_bf16(DK, DV, true, true);
@@ -1141,9 +1149,9 @@ kla_chunk_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (!waitw(&o_full[(pc - 1) & 1], ((pc - 1) >> 1) & 1, abort_flag, g.status)) { ok = false; break; }
             if (lane == 0) {
                 if (LOCAL && p > 0) tma_store_wait_read();
-                if (loaded < nchunks) load_chunk(loaded);
+                if (loaded < nload) load_chunk(loaded);
             }
-            if (loaded < nchunks) ++loaded;
+            if (loaded < nload) ++loaded;
         }
         if (lane == 0) {
             if (LOCAL && p > 0) tma_store_wait_all();
@@ -1246,6 +1254,8 @@ cudaError_t launch_t(const Plan &p, const int *cu, int mode, const void *q, cons
     g.rlog = p.rlog;
     g.S_io = S_io; g.decay = decay; g.out = (__nv_bfloat16 *)out;
     g.final_lambda = final_lambda; g.final_eta = final_eta; g.status = status;
+    const char *wt = getenv("KLA_TEST_WITHHOLD_TILES");
+    g.withhold_tiles = (wt && *wt && *wt != '0') ? 1 : 0;
     const unsigned grid = (unsigned)((long long)p.N * p.H * p.P);
     if (grid == 0) return cudaSuccess;
     const int threads = p.iso ? Roles<DK, DV, true>::THREADS : Roles<DK, DV, false>::THREADS;

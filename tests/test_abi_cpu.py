@@ -114,7 +114,7 @@ class _FakePtr:
 
 @pytest.mark.parametrize("shape,expect", [
     # (B, T, H, dk, dv, dtype, mode, packed sequences) -> (segments per row, launches, tensor cores)
-    ((4, 2048, 8, 64, 64, kla.KLA_BF16, kla.KLA_DIAG, 0), (4, 4, True)),      # small layer: 128 CTAs, one per SM
+    ((4, 2048, 8, 64, 64, kla.KLA_BF16, kla.KLA_DIAG, 0), (8, 4, True)),      # small layer: 256 CTAs, two per SM
     ((8, 4096, 16, 128, 128, kla.KLA_BF16, kla.KLA_DIAG, 0), (1, 1, True)),   # 1.3B layer: rows fill the SMs
     ((1, 131072, 16, 128, 128, kla.KLA_BF16, kla.KLA_DIAG, 0), (9, 5, True)),  # long context: separate carry
     ((2, 16384, 32, 64, 128, kla.KLA_BF16, kla.KLA_ISO, 8), (1, 2, True)),   # packed: length ranking + walk

@@ -126,3 +126,24 @@ def test_range_limit_is_reported():
     # the status word is cleared by the check: a valid call afterwards is clean
     w2 = WORKLOADS[2].with_(B=1, H=2, T=256)
     check_against_oracle(w2, make_inputs(w2))
+
+
+def test_bounded_wait_reports_timeout(monkeypatch):
+    # With the tile loads withheld (a test switch of the library), the gate's
+    # first wait on them never completes: after the bounded wait the kernel sets
+    # the abort flag, every role leaves through its teardown, and the status word
+    # reports KLA_ERR_TIMEOUT. No fault, no hang: the context stays usable and a
+    # valid call afterwards is clean.
+    w = WORKLOADS[1].with_(B=1, H=2, T=200)
+    inp = make_inputs(w)
+    d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    # whole rows (one launch: the walk kernel alone meets the withheld tiles)
+    monkeypatch.setenv("KLA_SEGMENTS", "1")
+    monkeypatch.setenv("KLA_TEST_WITHHOLD_TILES", "1")
+    kla.forward(d["q"], d["k"], d["v"], d["a"], d["qn"], d["beta"], B=w.B, T=w.T)
+    with pytest.raises(kla.KlaError) as e:
+        kla.check()
+    assert e.value.status == kla.KLA_ERR_TIMEOUT
+    monkeypatch.delenv("KLA_TEST_WITHHOLD_TILES")
+    monkeypatch.delenv("KLA_SEGMENTS")
+    check_against_oracle(w, inp)
