@@ -58,10 +58,15 @@ typedef enum {
                                  pointer, workspace too small; nothing launched */
     KLA_ERR_UNSUPPORTED = 2,  /* valid request the library does not implement */
     KLA_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed */
-    KLA_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up (kla_check) */
-    KLA_ERR_RANGE = 5         /* the in-chunk log-gate span exceeded the range
-                                 the factorised chunk form represents exactly
-                                 (kla_check); outputs of that call are unreliable */
+    KLA_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up (kla_check);
+                                 the kernel left through its teardown and the
+                                 context stays usable */
+    KLA_ERR_RANGE = 5         /* a 16-token stretch of one key (or of the head, in
+                                 isotropic mode) has a cumulative gate below 2^-160
+                                 (log2 span above 160), beyond what the factorised
+                                 chunk form represents (kla_check); outputs of that
+                                 call are unreliable. Faster forgetting spread over
+                                 longer stretches is computed exactly. */
 } kla_status;
 
 typedef enum { KLA_BF16 = 0, KLA_FP32 = 1 } kla_dtype;   /* dtype of q, k, v, out */
@@ -207,7 +212,10 @@ kla_status kla_forward_noalloc(const kla_desc *desc,
 
 /* Synchronises `stream`, then reads and clears the library's device status
  * word on the current device: KLA_OK, KLA_ERR_RANGE or KLA_ERR_TIMEOUT from any
- * kernel that ran since the last check, or KLA_ERR_CUDA if the stream failed. */
+ * kernel that ran since the last check, or KLA_ERR_CUDA if the stream failed.
+ * (The environment variable KLA_TEST_WITHHOLD_TILES=1, read at each launch of the
+ * tensor-core walk, withholds its tile loads so that its first bounded wait runs
+ * out: a test switch for this status path, off unless set.) */
 kla_status kla_check(cudaStream_t stream);
 
 /* Static description of an error code. */
