@@ -10,6 +10,11 @@ with gcc and marshals numpy / torch CPU arrays through ctypes.
 Parity status: pinned. The tests check the oracle against a textbook
 covariance-form Kalman filter, a full-matrix Kalman filter on one-hot keys,
 closed forms, a hand-worked example and invariants (see tests/test_oracle_pins.py).
+The Kalman Delta Network residual write (``kdn_forward``) is pinned against the
+textbook dense Kalman update for one step from a diagonal prior, the scalar
+Kalman filter for dk = 1, the KLA filter on one-hot keys, and the gated delta
+rule when the predictive covariance is a constant isotropic surrogate (see
+tests/test_kdn_pins.py).
 The isotropic increment beta*|k|^2/dk is pinned for consistency only (it
 reduces to the diagonal filter when dk = 1 and to the closed form when a=1,
 qn=0); the choice of that constant is a reading of the Kalman Delta Networks
@@ -55,6 +60,12 @@ def _load():
             _i32p, ctypes.c_int,
             _f32p, _f32p, _f32p, _f32p, _f32p, _f32p, _f32p, _f32p,
             _f64p, _f64p, _f64p, _f64p, ctypes.c_long, ctypes.c_long, ctypes.c_int]
+        lib.kdn_oracle_forward.restype = ctypes.c_int
+        lib.kdn_oracle_forward.argtypes = [
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            _i32p, ctypes.c_int,
+            _f32p, _f32p, _f32p, _f32p, _f32p, _f32p, _f32p, _f32p,
+            _f64p, _f64p, _f64p, ctypes.c_long, ctypes.c_long, ctypes.c_int]
         lib.kla_oracle_max_threads.restype = ctypes.c_int
         lib.kla_oracle_mobius_element.argtypes = [ctypes.c_double] * 3 + [_f64p]
         lib.kla_oracle_mobius_compose.argtypes = [_f64p, _f64p, _f64p]
@@ -126,6 +137,52 @@ def forward(q, k, v, a, qn, beta, lambda0=None, eta0=None, cu_seqlens=None,
     if want_lambda:
         res["lambda"] = lt
     return res
+
+
+def kdn_forward(q, k, v, a, qn, beta, lambda0=None, M0=None, cu_seqlens=None,
+                B=None, T=None, iso=False, units=None, num_threads=0):
+    """Kalman Delta Network forward with the Kalman-gain residual write (the
+    reading in kla_oracle.c: the exact Kalman mean update from a diagonal /
+    isotropic prior, the posterior precision projected back onto it). Returns
+    ``out`` [Ntok,H,dv], ``final_lambda`` [N,H,dk] (iso [N,H]) and ``final_M``
+    [N,H,dk,dv] (the posterior mean), float64."""
+    lib = _load()
+    q, k, v, a, qn, beta = (_f32(x) for x in (q, k, v, a, qn, beta))
+    lambda0, M0 = _f32(lambda0), _f32(M0)
+    Ntok, H, dk = q.shape
+    dv = v.shape[-1]
+    cu = None
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(
+            cu_seqlens.cpu().numpy() if hasattr(cu_seqlens, "cpu") else cu_seqlens, dtype=np.int32))
+        N = cu.size - 1
+        B_, T_ = 1, Ntok
+    else:
+        B_ = B if B is not None else 1
+        T_ = T if T is not None else Ntok // B_
+        assert B_ * T_ == Ntok
+        N = B_
+    out = np.zeros((Ntok, H, dv))
+    fl = np.zeros((N, H) if iso else (N, H, dk))
+    fm = np.zeros((N, H, dk, dv))
+    ub, ue = (0, -1) if units is None else units
+    err = lib.kdn_oracle_forward(
+        B_, T_, H, dk, dv, int(bool(iso)), _ptr(cu, _i32p), N,
+        _ptr(q, _f32p), _ptr(k, _f32p), _ptr(v, _f32p), _ptr(a, _f32p), _ptr(qn, _f32p),
+        _ptr(beta, _f32p), _ptr(lambda0, _f32p), _ptr(M0, _f32p),
+        _ptr(out, _f64p), _ptr(fl, _f64p), _ptr(fm, _f64p), int(ub), int(ue), int(num_threads))
+    if err:
+        raise RuntimeError("oracle failed (bad shape or out of memory)")
+    return {"out": out, "final_lambda": fl, "final_M": fm}
+
+
+def kdn_forward_inputs(inp: dict, w, **kw):
+    """``kdn_forward`` on a dict produced by the seeded input generator."""
+    return kdn_forward(inp["q"], inp["k"], inp["v"], inp["a"], inp["qn"], inp["beta"],
+                       inp.get("lambda0"), inp.get("M0"), inp.get("cu_seqlens"),
+                       B=None if inp.get("cu_seqlens") is not None else w.B,
+                       T=None if inp.get("cu_seqlens") is not None else w.T,
+                       iso=(w.mode == "iso"), **kw)
 
 
 def forward_inputs(inp: dict, w, **kw):

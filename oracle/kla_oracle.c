@@ -189,3 +189,142 @@ double kla_oracle_mobius_apply(const double *M, double lam)
 {
     return (M[0] * lam + M[1]) / (M[2] * lam + M[3]);
 }
+
+/* ---- Kalman Delta Network: the Kalman-gain residual (delta-style) write ---
+ *
+ * Kalman Delta Networks abstract: the memory is the state of a linear-Gaussian
+ * state-space model; the transition propagates its mean and its uncertainty,
+ * and the Kalman gain weights each residual write; diagonal KDN projects each
+ * one-step posterior onto diagonal Gaussians (online mean-field variational
+ * inference), isotropic KDN keeps one uncertainty scalar per head. The pages
+ * give no equations; this is the plainest reading of that statement:
+ *
+ *   state: mean M[dk][dv] (one column per value dimension, all columns with the
+ *   same key covariance), diagonal covariance diag(1/lambda) (iso: I/lambda).
+ *   predict (the same OU prior as the KLA filter):
+ *       M~[i,:]   = a[t,i] * M[i,:]
+ *       lambda~[i]= lambda[i] / (a[t,i]^2 + qn[t,i] * lambda[i])
+ *   observe v = M^T k + noise of precision beta (per value dimension):
+ *       innovation  r[j] = v[j] - sum_i k[i] M~[i,j]
+ *       gain        G[i] = (k[i]/lambda~[i]) * beta / (1 + beta * sum_i k[i]^2/lambda~[i])
+ *       mean write  M[i,j] = M~[i,j] + G[i] * r[j]      (the exact posterior mean
+ *                   given the diagonal prior: the textbook Kalman update)
+ *       precision   lambda[i] = lambda~[i] + beta * k[i]^2   (the diagonal of the
+ *                   posterior precision lambda~ + beta k k^T: the mean-field
+ *                   projection; iso: + beta * |k|^2 / dk as for the KLA filter)
+ *   readout (posterior mean through the query): o[j] = sum_i q[i] M[i,j]
+ *
+ * So the precision path is the KLA filter's Moebius recursion, and only the mean
+ * write differs: it is coupled across keys through the shared innovation. With
+ * one-hot keys both coincide (per key: M = (lambda~ M~ + beta v)/(lambda~ + beta)).
+ * M0 is the prior mean before the first token (default 0), lambda0 its
+ * precision (default 1); layouts as for kla_oracle_forward, M0 / final_M
+ * [N,H,dk,dv].
+ */
+static int run_kdn_unit(int n, int h, long t0, long t1, int H, int dk, int dv, int iso,
+                        const float *q, const float *k, const float *v,
+                        const float *a, const float *qn, const float *beta,
+                        const float *lambda0, const float *M0,
+                        double *out, double *final_lambda, double *final_M)
+{
+    int nl = iso ? 1 : dk;
+    double *lam = (double *)malloc(sizeof(double) * nl);
+    double *M = (double *)malloc(sizeof(double) * (size_t)dk * dv);
+    double *w = (double *)malloc(sizeof(double) * dk);      /* k / lambda~ */
+    double *r = (double *)malloc(sizeof(double) * dv);      /* innovation */
+    if (!lam || !M || !w || !r) { free(lam); free(M); free(w); free(r); return 1; }
+
+    for (int i = 0; i < nl; ++i)
+        lam[i] = lambda0 ? (double)lambda0[((size_t)n * H + h) * nl + i] : 1.0;
+    for (size_t e = 0; e < (size_t)dk * dv; ++e)
+        M[e] = M0 ? (double)M0[((size_t)n * H + h) * dk * dv + e] : 0.0;
+
+    for (long t = t0; t < t1; ++t) {
+        size_t th = (size_t)t * H + h;
+        const float *qt = q + th * dk, *kt = k + th * dk, *vt = v + th * dv;
+        double bt = (double)beta[th];
+        /* predict: mean decays by a, precision through the OU prior */
+        for (int i = 0; i < dk; ++i) {
+            double ai = iso ? (double)a[th] : (double)a[th * dk + i];
+            double *row = M + (size_t)i * dv;
+            for (int j = 0; j < dv; ++j) row[j] *= ai;
+        }
+        if (iso) {
+            double den = (double)a[th] * (double)a[th] + (double)qn[th] * lam[0];
+            lam[0] = lam[0] / den;
+        } else {
+            for (int i = 0; i < dk; ++i) {
+                double ai = a[th * dk + i];
+                lam[i] = lam[i] / (ai * ai + (double)qn[th * dk + i] * lam[i]);
+            }
+        }
+        /* innovation and gain */
+        double s = 0.0, ksq = 0.0;
+        for (int i = 0; i < dk; ++i) {
+            double ki = kt[i];
+            w[i] = ki / lam[iso ? 0 : i];
+            s += ki * w[i];
+            ksq += ki * ki;
+        }
+        for (int j = 0; j < dv; ++j) {
+            double pred = 0.0;
+            for (int i = 0; i < dk; ++i) pred += (double)kt[i] * M[(size_t)i * dv + j];
+            r[j] = (double)vt[j] - pred;
+        }
+        double gam = bt / (1.0 + bt * s);
+        /* residual write */
+        for (int i = 0; i < dk; ++i) {
+            double gi = gam * w[i];
+            double *row = M + (size_t)i * dv;
+            for (int j = 0; j < dv; ++j) row[j] += gi * r[j];
+        }
+        /* precision: diagonal of the posterior precision */
+        if (iso) lam[0] += bt * ksq / (double)dk;
+        else
+            for (int i = 0; i < dk; ++i) lam[i] += bt * (double)kt[i] * (double)kt[i];
+        if (out) {
+            double *ot = out + th * dv;
+            for (int j = 0; j < dv; ++j) ot[j] = 0.0;
+            for (int i = 0; i < dk; ++i) {
+                double c = qt[i];
+                const double *row = M + (size_t)i * dv;
+                for (int j = 0; j < dv; ++j) ot[j] += c * row[j];
+            }
+        }
+    }
+    if (final_lambda)
+        for (int i = 0; i < nl; ++i) final_lambda[((size_t)n * H + h) * nl + i] = lam[i];
+    if (final_M)
+        memcpy(final_M + ((size_t)n * H + h) * dk * dv, M, sizeof(double) * (size_t)dk * dv);
+    free(lam); free(M); free(w); free(r);
+    return 0;
+}
+
+/* KDN forward; arguments as kla_oracle_forward, M0 / final_M in place of eta. */
+int kdn_oracle_forward(int B, int T, int H, int dk, int dv, int iso,
+                       const int *cu_seqlens, int num_seqs,
+                       const float *q, const float *k, const float *v,
+                       const float *a, const float *qn, const float *beta,
+                       const float *lambda0, const float *M0,
+                       double *out, double *final_lambda, double *final_M,
+                       long units_begin, long units_end, int num_threads)
+{
+    if (B < 0 || T < 0 || H <= 0 || dk <= 0 || dv <= 0) return 1;
+    int N = cu_seqlens ? num_seqs : B;
+    long units = (long)N * H;
+    if (units_end < 0 || units_end > units) units_end = units;
+    if (units_begin < 0) units_begin = 0;
+    int err = 0;
+#ifdef _OPENMP
+    if (num_threads > 0) omp_set_num_threads(num_threads);
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : err)
+#endif
+    for (long u = units_begin; u < units_end; ++u) {
+        int n = (int)(u / H), h = (int)(u % H);
+        long t0 = cu_seqlens ? cu_seqlens[n] : (long)n * T;
+        long t1 = cu_seqlens ? cu_seqlens[n + 1] : (long)(n + 1) * T;
+        err |= run_kdn_unit(n, h, t0, t1, H, dk, dv, iso, q, k, v, a, qn, beta,
+                            lambda0, M0, out, final_lambda, final_M);
+    }
+    return err;
+}
