@@ -40,6 +40,11 @@ cudaError_t launch_state_carry(const Plan &, const float *, const float *, float
 cudaError_t launch_seq_order(const Plan &, const int *, int *, cudaStream_t);
 cudaError_t launch_correct(const Plan &, const float *, const float *, void *, float *, int *, cudaStream_t);
 bool chunk_tc_supported(const Plan &);
+bool kdn_supported(int dk, int dv);
+cudaError_t launch_kdn(int H, long long T, long long units, int dk, int dv, bool iso, bool bf16, const int *cu,
+                       const void *q, const void *k, const void *v, const float *a, const float *qn,
+                       const float *beta, const float *lambda0, const float *M0, void *out, float *final_lambda,
+                       float *final_M, cudaStream_t st);
 cudaError_t launch_chunk_tc(const Plan &, const int *, int, const void *, const void *, const void *,
                             const float *, const float *, const float *, const float *, const float *,
                             const float *, float *, float *, void *, float *, float *, int *,
@@ -300,6 +305,25 @@ kla_status kla_forward_profiled(const kla_desc *d, const void *q, const void *k,
         if (!events[i]) return KLA_ERR_INVALID_ARG;
     return forward_impl(d, q, k, v, a, qn, beta, lambda0, eta0, out, final_lambda, final_eta, ws,
                         ws_bytes, st, events);
+}
+
+kla_status kla_kdn_forward(const kla_desc *d, const void *q, const void *k, const void *v,
+                           const float *a, const float *qn, const float *beta, const float *lambda0,
+                           const float *M0, void *out, float *final_lambda, float *final_M,
+                           cudaStream_t st) {
+    Plan p;
+    kla_status s = make_plan(d, p, false);
+    if (s != KLA_OK) return s;
+    if (!kdn_supported(p.dk, p.dv)) return KLA_ERR_UNSUPPORTED;
+    if (p.ntok == 0 && !p.varlen) return KLA_OK;
+    if (!q || !k || !v || !a || !qn || !beta || !out) return KLA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(a) || !aligned16(qn) ||
+        !aligned4(beta) || !aligned16(out) || !aligned4(lambda0) || !aligned16(M0) ||
+        !aligned4(final_lambda) || !aligned16(final_M))
+        return KLA_ERR_INVALID_ARG;
+    return cuda_status(launch_kdn(p.H, p.T, (long long)p.N * p.H, p.dk, p.dv, p.iso, p.bf16,
+                                  p.varlen ? d->cu_seqlens : nullptr, q, k, v, a, qn, beta, lambda0, M0,
+                                  out, final_lambda, final_M, st));
 }
 
 kla_status kla_plan(const kla_desc *d, int *segments_per_row, int *launches, int *tensor_core) {

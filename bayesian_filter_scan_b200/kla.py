@@ -27,7 +27,7 @@ NOALLOC_SCRATCH_BYTES = 32 << 20
 EXPORTS = ("kla_workspace_bytes", "kla_precision_workspace_bytes", "kla_forward", "kla_forward_profiled",
            "kla_plan", "kla_precision",
            "kla_decode_step", "kla_host_device_bytes", "kla_forward_host", "kla_check",
-           "kla_status_string", "kla_version", "kla_forward_noalloc")
+           "kla_status_string", "kla_version", "kla_forward_noalloc", "kla_kdn_forward")
 
 
 class KlaError(RuntimeError):
@@ -76,6 +76,8 @@ def lib():
         L.kla_forward_host.restype = ctypes.c_int
         L.kla_forward_noalloc.argtypes = [D] + [_P] * 11 + [_P]
         L.kla_forward_noalloc.restype = ctypes.c_int
+        L.kla_kdn_forward.argtypes = [D] + [_P] * 11 + [_P]
+        L.kla_kdn_forward.restype = ctypes.c_int
         L.kla_check.argtypes = [_P]
         L.kla_check.restype = ctypes.c_int
         L.kla_status_string.argtypes = [ctypes.c_int]
@@ -171,6 +173,35 @@ def forward(q, k, v, a, qn, beta, lambda0=None, eta0=None, cu_seqlens=None, B=No
                           nbytes, _stream())
     _check(s, "kla_forward")
     return (out, fl, fe) if final_state else out
+
+
+def kdn_forward(q, k, v, a, qn, beta, lambda0=None, M0=None, cu_seqlens=None, B=None, T=None,
+                mode="diag", final_state=False, out=None):
+    """Kalman Delta Network forward (the Kalman-gain residual write) on CUDA
+    tensors in the layouts of include/kla.h. Returns ``out`` or
+    ``(out, final_lambda, final_M)`` with ``final_state`` (final_M: the
+    posterior mean [N,H,dk,dv])."""
+    m = _mode(mode)
+    desc, N = _desc_from(q, v, B, T, m, cu_seqlens)
+    for name, t in (("q", q), ("k", k), ("v", v), ("a", a), ("qn", qn), ("beta", beta)):
+        if not (t.is_cuda and t.is_contiguous()):
+            raise ValueError("%s must be a contiguous CUDA tensor" % name)
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share a dtype")
+    for name, t in (("a", a), ("qn", qn), ("beta", beta), ("lambda0", lambda0), ("M0", M0)):
+        if t is not None and t.dtype != torch.float32:
+            raise TypeError("%s must be float32" % name)
+    H, dk, dv = q.shape[1], q.shape[2], v.shape[2]
+    if out is None:
+        out = torch.empty(q.shape[0], H, dv, dtype=q.dtype, device=q.device)
+    fl = fm = None
+    if final_state:
+        fl = torch.empty((N, H) if m == KLA_ISO else (N, H, dk), dtype=torch.float32, device=q.device)
+        fm = torch.empty(N, H, dk, dv, dtype=torch.float32, device=q.device)
+    s = lib().kla_kdn_forward(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(qn), _ptr(beta),
+                              _ptr(lambda0), _ptr(M0), _ptr(out), _ptr(fl), _ptr(fm), _stream())
+    _check(s, "kla_kdn_forward")
+    return (out, fl, fm) if final_state else out
 
 
 def precision(k, a, qn, beta, lambda0=None, cu_seqlens=None, B=None, T=None, mode="diag"):

@@ -210,6 +210,28 @@ kla_status kla_forward_noalloc(const kla_desc *desc,
                                void *out, float *final_lambda, float *final_eta,
                                cudaStream_t stream);
 
+/* Kalman Delta Network forward with the Kalman-gain residual (delta-style)
+ * write (Kalman Delta Networks abstract: the memory is the state of a
+ * linear-Gaussian model, the Kalman gain weights each residual write, the
+ * one-step posterior is projected onto diagonal Gaussians (diagonal mode) or
+ * kept isotropic with one uncertainty per head). The state is the posterior
+ * mean M [N,H,dk,dv] and the precision lambda; per token t:
+ *   lambda~ = lambda / (a^2 + qn lambda),  w = k / lambda~,
+ *   gamma = beta / (1 + beta k.w),  r = v - (a M)^T k,
+ *   M = a M + gamma w r^T,  lambda = lambda~ + beta k^2 (iso: + beta |k|^2 / dk),
+ *   o = M^T q.
+ * Arguments as kla_forward, with M0 (prior mean before the first token, or
+ * NULL for 0; 16-byte aligned) and final_M (or NULL) in place of eta0 /
+ * final_eta; no workspace. dk and dv in {16, 32, 64, 128}, else
+ * KLA_ERR_UNSUPPORTED. One CTA per (row or packed sequence, head) walks its
+ * tokens with the mean in registers (CUDA cores). Errors as kla_forward. */
+kla_status kla_kdn_forward(const kla_desc *desc,
+                           const void *q, const void *k, const void *v,
+                           const float *a, const float *qn, const float *beta,
+                           const float *lambda0, const float *M0,
+                           void *out, float *final_lambda, float *final_M,
+                           cudaStream_t stream);
+
 /* Synchronises `stream`, then reads and clears the library's device status
  * word on the current device: KLA_OK, KLA_ERR_RANGE or KLA_ERR_TIMEOUT from any
  * kernel that ran since the last check, or KLA_ERR_CUDA if the stream failed.
