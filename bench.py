@@ -24,6 +24,8 @@ returned). Prints ONE JSON line (rank 0):
                the same workload, on this host's cores.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 3] [--impl reference]
+  python bench.py --variant kdn [--workload 2]   (the Kalman Delta Network residual write:
+               a separate line with the same timing rules, kla_kdn_forward)
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own batch of
 the workload (independent sequences; no collective on the data path), so the
@@ -280,6 +282,116 @@ def arm_config(w, world):
             "parallelism": "dp%d" % world}
 
 
+KDN_METRIC = "KDN residual-write forward tokens/s per layer (B*T/s) on 1 B200; % of HBM"
+
+
+def run_kdn(args, w):
+    """The Kalman Delta Network residual write (kla_kdn_forward) on the
+    workload: one launch per step, device-timed with L2 flushed between steps,
+    against the same algorithmic bytes as the KLA forward (inputs once, output
+    once); end to end with the inputs copied in from pinned host memory and the
+    output copied back inside the timed region; the fp64 oracle on a bounded
+    sample of units as the CPU baseline. One GPU (the path shards like the KLA
+    forward: replicas)."""
+    from bayesian_filter_scan_b200 import kla
+    torch.cuda.set_device(0)
+    kla.lib()
+    inp = make_inputs(w, seed=rank_seed(w, 0))
+    dev = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
+    H, dv = w.H, w.dv
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    sweep = torch.ones(SWEEP_BYTES // 4, dtype=torch.float32, device="cuda")
+    out = torch.empty(w.tokens, H, dv, dtype=dev["q"].dtype, device="cuda")
+
+    def run(d, o):
+        return kla.kdn_forward(d["q"], d["k"], d["v"], d["a"], d["qn"], d["beta"], cu_seqlens=d["cu_seqlens"],
+                               B=w.B, T=w.T, mode=w.mode, out=o)
+
+    def flush_l2():
+        flush.fill_(1)
+        sweep.sum()
+    for _ in range(args.warmup):
+        flush_l2()
+        run(dev, out)
+    torch.cuda.synchronize()
+    kla.check()
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(0)
+    clocks.start()
+    for e0, e1 in ev:
+        flush_l2()
+        e0.record(stream)
+        run(dev, out)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    kla.check()
+    ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev)
+    value = w.tokens / (ms * 1e-3)
+    # end to end: pinned inputs in, output out, inside the timed region
+    pin = {k: (v.pin_memory() if v is not None else None) for k, v in inp.items()}
+    hout = torch.empty(w.tokens, H, dv, dtype=inp["q"].dtype).pin_memory()
+    dbuf = {k: (torch.empty_like(v, device="cuda") if v is not None else None) for k, v in inp.items()}
+    h_in = sum(t.numel() * t.element_size() for k_, t in pin.items()
+               if t is not None and k_ in ("q", "k", "v", "a", "qn", "beta", "cu_seqlens"))
+    e_t, e_steps = 0.0, max(3, min(args.e2e_steps, args.steps))
+    for i in range(e_steps + 2):
+        flush_l2()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for k_, t in pin.items():
+            if t is not None:
+                dbuf[k_].copy_(t, non_blocking=True)
+        run(dbuf, out)
+        hout.copy_(out, non_blocking=True)
+        a1.record(stream)
+        a1.synchronize()
+        if i >= 2:
+            e_t += a0.elapsed_time(a1)
+    e2e_value = w.tokens / (e_t / e_steps * 1e-3)
+    peaks, peak_src = measured_peaks()
+    peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    alg_bytes = bytes_per_token_head(w) * w.tokens * H
+    achieved = alg_bytes / (ms * 1e-3) / 1e9
+    cfg = arm_config(w, 1)
+    cfg["variant"] = "kdn-residual-write"
+    res = {
+        "metric": KDN_METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic", "config": cfg,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": None, "kernel": "kdn_walk_kernel (CUDA cores, one CTA per row x head)",
+                     "alg_bytes_per_launch": alg_bytes, "launch_ms": ms,
+                     "alg_bytes_per_token_head": bytes_per_token_head(w),
+                     "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_src},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h_in,
+                "d2h_bytes_per_step": hout.numel() * hout.element_size()},
+        "gpu_launches": args.steps, "clocks": clk,
+    }
+    if not args.no_cpu_baseline:
+        import oracle
+        t1 = time.perf_counter()
+        oracle.kdn_forward_inputs(inp, w, units=(0, 1))
+        per_unit = max(time.perf_counter() - t1, 1e-4)
+        n_units = int(max(1, min(_units_total(w, inp), 12.0 / per_unit * oracle.max_threads())))
+        t0 = time.perf_counter()
+        ref = oracle.kdn_forward_inputs(inp, w, units=(0, n_units))
+        t = time.perf_counter() - t0
+        res["cpu_baseline"] = {"value": _unit_tokens(w, inp, n_units) / t, "unit": UNIT,
+                               "cores": oracle.max_threads(), "kind": "oracle",
+                               "sample": "%d of %d (row, head) units, fp64 C oracle (residual write), %.3f s" % (
+                                   n_units, _units_total(w, inp), t)}
+        cu = inp["cu_seqlens"].tolist() if inp["cu_seqlens"] is not None else None
+        worst = 0.0
+        for u in range(n_units):
+            n, h = divmod(u, H)
+            s0, s1 = (cu[n], cu[n + 1]) if cu else (n * w.T, (n + 1) * w.T)
+            worst = max(worst, scaled_err(out[s0:s1, h], ref["out"][s0:s1, h]))
+        res["max_err"] = {"out": worst, "units": n_units, "tol": 2e-2 if w.dtype == "bf16" else 1e-4}
+    print(json.dumps(res))
+
+
 def run_reference(args, w):
     """Reference arm: the CPU oracle timed on this host's cores. It loads only
     the oracle, never the CUDA library."""
@@ -320,6 +432,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--variant", default="kla", choices=["kla", "kdn"],
+                    help="kla: the KLA forward (the bench line); kdn: the Kalman Delta Network "
+                         "residual write on the same workload (a separate line)")
     ap.add_argument("--T", type=int, default=None,
                     help="tokens per row instead of the workload's (smaller cases of the same "
                          "workload for profiler captures; not a bench line)")
@@ -331,6 +446,9 @@ def main():
         w = w.with_(T=args.T)
     if args.impl == "reference":
         run_reference(args, w)
+        return
+    if args.variant == "kdn":
+        run_kdn(args, w)
         return
 
     from bayesian_filter_scan_b200 import kla
