@@ -14,7 +14,10 @@ The Kalman Delta Network residual write (``kdn_forward``) is pinned against the
 textbook dense Kalman update for one step from a diagonal prior, the scalar
 Kalman filter for dk = 1, the KLA filter on one-hot keys, and the gated delta
 rule when the predictive covariance is a constant isotropic surrogate (see
-tests/test_kdn_pins.py).
+tests/test_kdn_pins.py). The mixer's input prologue (``prologue``: causal conv,
+SiLU, L2 norm, sigmoid / softplus gates) is plain numpy, pinned against the
+identity kernel, numpy's convolution per channel, closed forms of the gates
+and packed sequences (tests/test_prologue_pins.py).
 The isotropic increment beta*|k|^2/dk is pinned for consistency only (it
 reduces to the diagonal filter when dk = 1 and to the closed form when a=1,
 qn=0); the choice of that constant is a reading of the Kalman Delta Networks
@@ -220,3 +223,66 @@ def time_forward(inp: dict, w, units, num_threads=0) -> tuple:
     t0 = time.perf_counter()
     forward_inputs(inp, w, units=units, want_final=False, num_threads=num_threads)
     return time.perf_counter() - t0
+
+
+# ---- fused prologue of the mixer (1-D causal conv + SiLU, L2 norm, gates) ---
+
+PROLOGUE_EPS = 1e-6
+
+
+def prologue(xq, xk, xv, xa, xqn, xbeta, wq, wk, wv, bq=None, bk=None, bv=None, cu_seqlens=None,
+             B=None, T=None):
+    """The mixer's input prologue (Kalman Linear Attention, technical summary
+    section 4: a Mamba-like block with a 1-D causal convolution and SiLU), in
+    plain numpy fp64, step by step:
+      q = l2norm(silu(conv(xq))), k = l2norm(silu(conv(xk))), v = silu(conv(xv)),
+      a = sigmoid(xa), qn = softplus(xqn), beta = sigmoid(xbeta),
+    conv: per channel c of head h, y[t] = b[h,c] + sum_{w<W} wgt[h,c,w] x[t-(W-1)+w]
+    with x = 0 before the start of t's sequence (each packed sequence starts
+    afresh); l2norm over dk: y / sqrt(sum y^2 + PROLOGUE_EPS). Layouts as the
+    forward's inputs: x* [Ntok,H,d] (xa, xqn [Ntok,H,dk] or [Ntok,H]),
+    weights [H,d,W], biases [H,d]. Returns float64 arrays."""
+    def f64(x):
+        if x is None:
+            return None
+        if hasattr(x, "detach"):
+            x = x.detach().cpu().double().numpy()
+        return np.asarray(x, dtype=np.float64)
+    xq, xk, xv, xa, xqn, xbeta = (f64(x) for x in (xq, xk, xv, xa, xqn, xbeta))
+    wq, wk, wv, bq, bk, bv = (f64(x) for x in (wq, wk, wv, bq, bk, bv))
+    Ntok = xq.shape[0]
+    if cu_seqlens is not None:
+        cu = np.asarray(cu_seqlens.cpu().numpy() if hasattr(cu_seqlens, "cpu") else cu_seqlens, dtype=np.int64)
+    else:
+        B_ = B if B is not None else 1
+        T_ = T if T is not None else Ntok // B_
+        cu = np.arange(B_ + 1, dtype=np.int64) * T_
+
+    def conv(x, wgt, bias):
+        Wd = wgt.shape[-1]
+        y = np.zeros_like(x)
+        for n in range(cu.size - 1):
+            s, e = int(cu[n]), int(cu[n + 1])
+            for t in range(s, e):
+                acc = np.zeros(x.shape[1:]) if bias is None else bias.copy()
+                for w in range(Wd):
+                    src = t - (Wd - 1) + w
+                    if src >= s:
+                        acc = acc + wgt[..., w] * x[src]
+                y[t] = acc
+        return y
+
+    def silu(y):
+        return y / (1.0 + np.exp(-y))
+
+    def l2norm(y):
+        return y / np.sqrt(np.sum(y * y, axis=-1, keepdims=True) + PROLOGUE_EPS)
+
+    def sigmoid(y):
+        return 1.0 / (1.0 + np.exp(-y))
+
+    def softplus(y):
+        return np.log1p(np.exp(-np.abs(y))) + np.maximum(y, 0.0)
+
+    return {"q": l2norm(silu(conv(xq, wq, bq))), "k": l2norm(silu(conv(xk, wk, bk))),
+            "v": silu(conv(xv, wv, bv)), "a": sigmoid(xa), "qn": softplus(xqn), "beta": sigmoid(xbeta)}
