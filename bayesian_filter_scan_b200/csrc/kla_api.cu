@@ -41,6 +41,11 @@ cudaError_t launch_seq_order(const Plan &, const int *, int *, cudaStream_t);
 cudaError_t launch_correct(const Plan &, const float *, const float *, void *, float *, int *, cudaStream_t);
 bool chunk_tc_supported(const Plan &);
 bool kdn_supported(int dk, int dv);
+cudaError_t launch_prologue(int H, long long ntok, long long T, const int *cu, int nseq, int dk, int dv, bool iso,
+                            bool bf16, int W, const void *xq, const void *xk, const void *xv, const float *xa,
+                            const float *xqn, const float *xbeta, const float *wq, const float *wk,
+                            const float *wv, const float *bq, const float *bk, const float *bv, void *q, void *k,
+                            void *v, float *a, float *qn, float *beta, cudaStream_t st);
 cudaError_t launch_kdn(int H, long long T, long long units, int dk, int dv, bool iso, bool bf16, const int *cu,
                        const void *q, const void *k, const void *v, const float *a, const float *qn,
                        const float *beta, const float *lambda0, const float *M0, void *out, float *final_lambda,
@@ -324,6 +329,28 @@ kla_status kla_kdn_forward(const kla_desc *d, const void *q, const void *k, cons
     return cuda_status(launch_kdn(p.H, p.T, (long long)p.N * p.H, p.dk, p.dv, p.iso, p.bf16,
                                   p.varlen ? d->cu_seqlens : nullptr, q, k, v, a, qn, beta, lambda0, M0,
                                   out, final_lambda, final_M, st));
+}
+
+kla_status kla_prologue(const kla_desc *d, int conv_width, const void *xq, const void *xk, const void *xv,
+                        const float *xa, const float *xqn, const float *xbeta, const float *wq,
+                        const float *wk, const float *wv, const float *bq, const float *bk, const float *bv,
+                        void *q, void *k, void *v, float *a, float *qn, float *beta, cudaStream_t st) {
+    Plan p;
+    kla_status s = make_plan(d, p, false);
+    if (s != KLA_OK) return s;
+    if (conv_width < 1 || conv_width > 4) return KLA_ERR_INVALID_ARG;
+    if (!wq || !wk || !wv) return KLA_ERR_INVALID_ARG;
+    if (p.ntok == 0 && !p.varlen) return KLA_OK;
+    if (!xq || !xk || !xv || !xa || !xqn || !xbeta || !q || !k || !v || !a || !qn || !beta)
+        return KLA_ERR_INVALID_ARG;
+    const void *ptrs[] = {xq, xk, xv, xa, xqn, xbeta, wq, wk, wv, bq, bk, bv, q, k, v, a, qn, beta};
+    for (const void *x : ptrs)
+        if (!aligned4(x)) return KLA_ERR_INVALID_ARG;
+    const long long ntok = p.varlen ? -1 : p.ntok;
+    return cuda_status(launch_prologue(p.H, ntok < 0 ? (long long)d->B * d->T : ntok, p.T,
+                                       p.varlen ? d->cu_seqlens : nullptr, p.N, p.dk, p.dv, p.iso, p.bf16,
+                                       conv_width, xq, xk, xv, xa, xqn, xbeta, wq, wk, wv, bq, bk, bv, q, k, v, a,
+                                       qn, beta, st));
 }
 
 kla_status kla_plan(const kla_desc *d, int *segments_per_row, int *launches, int *tensor_core) {

@@ -27,7 +27,8 @@ NOALLOC_SCRATCH_BYTES = 32 << 20
 EXPORTS = ("kla_workspace_bytes", "kla_precision_workspace_bytes", "kla_forward", "kla_forward_profiled",
            "kla_plan", "kla_precision",
            "kla_decode_step", "kla_host_device_bytes", "kla_forward_host", "kla_check",
-           "kla_status_string", "kla_version", "kla_forward_noalloc", "kla_kdn_forward")
+           "kla_status_string", "kla_version", "kla_forward_noalloc", "kla_kdn_forward",
+           "kla_prologue")
 
 
 class KlaError(RuntimeError):
@@ -78,6 +79,8 @@ def lib():
         L.kla_forward_noalloc.restype = ctypes.c_int
         L.kla_kdn_forward.argtypes = [D] + [_P] * 11 + [_P]
         L.kla_kdn_forward.restype = ctypes.c_int
+        L.kla_prologue.argtypes = [D, ctypes.c_int] + [_P] * 18 + [_P]
+        L.kla_prologue.restype = ctypes.c_int
         L.kla_check.argtypes = [_P]
         L.kla_check.restype = ctypes.c_int
         L.kla_status_string.argtypes = [ctypes.c_int]
@@ -202,6 +205,27 @@ def kdn_forward(q, k, v, a, qn, beta, lambda0=None, M0=None, cu_seqlens=None, B=
                               _ptr(lambda0), _ptr(M0), _ptr(out), _ptr(fl), _ptr(fm), _stream())
     _check(s, "kla_kdn_forward")
     return (out, fl, fm) if final_state else out
+
+
+def prologue(xq, xk, xv, xa, xqn, xbeta, wq, wk, wv, bq=None, bk=None, bv=None, cu_seqlens=None,
+             B=None, T=None, mode="diag", out=None):
+    """The mixer's input prologue on CUDA tensors (include/kla.h kla_prologue):
+    returns ``(q, k, v, a, qn, beta)`` in the forward pass's layouts."""
+    m = _mode(mode)
+    desc, N = _desc_from(xq, xv, B, T, m, cu_seqlens)
+    ts = (xq, xk, xv, xa, xqn, xbeta, wq, wk, wv) + tuple(t for t in (bq, bk, bv) if t is not None)
+    for t in ts:
+        if not (t.is_cuda and t.is_contiguous()):
+            raise ValueError("prologue inputs must be contiguous CUDA tensors")
+    W = wq.shape[-1]
+    if out is None:
+        out = (torch.empty_like(xq), torch.empty_like(xk), torch.empty_like(xv), torch.empty_like(xa),
+               torch.empty_like(xqn), torch.empty_like(xbeta))
+    s = lib().kla_prologue(ctypes.byref(desc), W, *[_ptr(t) for t in (xq, xk, xv, xa, xqn, xbeta, wq, wk, wv,
+                                                                        bq, bk, bv)],
+                           *[_ptr(t) for t in out], _stream())
+    _check(s, "kla_prologue")
+    return out
 
 
 def precision(k, a, qn, beta, lambda0=None, cu_seqlens=None, B=None, T=None, mode="diag"):

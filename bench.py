@@ -392,6 +392,82 @@ def run_kdn(args, w):
     print(json.dumps(res))
 
 
+PRO_METRIC = "mixer prologue (conv + SiLU, L2 norm, gates) tokens/s per layer (B*T/s) on 1 B200; % of HBM"
+
+
+def prologue_bytes_per_token_head(w) -> int:
+    """Algorithmic bytes of the prologue per (token, head): every
+    pre-activation read once, every output written once."""
+    es = 2 if w.dtype == "bf16" else 4
+    nl = 1 if w.mode == "iso" else w.dk
+    return 2 * (es * (2 * w.dk + w.dv) + 4 * 2 * nl + 4)
+
+
+def run_prologue(args, w):
+    """kla_prologue on the workload's shape with synthetic pre-activations and
+    conv weights (width 4): device-timed with L2 flushed between steps,
+    against its algorithmic bytes and the measured HBM peak."""
+    from bayesian_filter_scan_b200 import kla
+    torch.cuda.set_device(0)
+    kla.lib()
+    inp = make_inputs(w, seed=rank_seed(w, 0))
+    g = torch.Generator().manual_seed(w.seed)
+    dt = inp["q"].dtype
+    Ntok, H, dk, dv = inp["q"].shape[0], w.H, w.dk, w.dv
+    gate = (Ntok, H) if w.mode == "iso" else (Ntok, H, dk)
+    r = lambda *s_: torch.randn(*s_, generator=g)  # noqa: E731
+    x = {"xq": r(Ntok, H, dk).to(dt), "xk": r(Ntok, H, dk).to(dt), "xv": r(Ntok, H, dv).to(dt),
+         "xa": r(*gate) + 2.0, "xqn": r(*gate) - 2.0, "xbeta": r(Ntok, H),
+         "wq": r(H, dk, 4) / 2, "wk": r(H, dk, 4) / 2, "wv": r(H, dv, 4) / 2,
+         "bq": r(H, dk) * 0.1, "bk": r(H, dk) * 0.1, "bv": r(H, dv) * 0.1}
+    d = {k: v.cuda().contiguous() for k, v in x.items()}
+    cu = inp["cu_seqlens"].cuda() if inp["cu_seqlens"] is not None else None
+    outs = (torch.empty_like(d["xq"]), torch.empty_like(d["xk"]), torch.empty_like(d["xv"]),
+            torch.empty_like(d["xa"]), torch.empty_like(d["xqn"]), torch.empty_like(d["xbeta"]))
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    sweep = torch.ones(SWEEP_BYTES // 4, dtype=torch.float32, device="cuda")
+
+    def step():
+        flush.fill_(1)
+        sweep.sum()
+        kla.prologue(**d, cu_seqlens=cu, B=None if cu is not None else w.B, T=None if cu is not None else w.T,
+                     mode=w.mode, out=outs)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    clocks = ClockSampler(0)
+    clocks.start()
+    ts = []
+    for _ in range(args.steps):
+        flush.fill_(1)
+        sweep.sum()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        kla.prologue(**d, cu_seqlens=cu, B=None if cu is not None else w.B, T=None if cu is not None else w.T,
+                     mode=w.mode, out=outs)
+        e1.record(stream)
+        ts.append((e0, e1))
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms = statistics.mean(a_.elapsed_time(b_) for a_, b_ in ts)
+    peaks, peak_src = measured_peaks()
+    peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    alg = prologue_bytes_per_token_head(w) * w.tokens * H
+    ach = alg / (ms * 1e-3) / 1e9
+    cfg = arm_config(w, 1)
+    cfg["variant"] = "prologue (conv width 4, with bias)"
+    res = {"metric": PRO_METRIC, "value": w.tokens / (ms * 1e-3), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": w.dtype, "data": "synthetic", "config": cfg,
+           "roofline": {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+                        "traffic": None, "kernel": "prologue_kernel", "alg_bytes_per_launch": alg, "launch_ms": ms,
+                        "alg_bytes_per_token_head": prologue_bytes_per_token_head(w),
+                        "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_src},
+           "gpu_launches": args.steps, "clocks": clk}
+    print(json.dumps(res))
+
+
 def run_reference(args, w):
     """Reference arm: the CPU oracle timed on this host's cores. It loads only
     the oracle, never the CUDA library."""
@@ -432,9 +508,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--variant", default="kla", choices=["kla", "kdn"],
+    ap.add_argument("--variant", default="kla", choices=["kla", "kdn", "prologue"],
                     help="kla: the KLA forward (the bench line); kdn: the Kalman Delta Network "
-                         "residual write on the same workload (a separate line)")
+                         "residual write on the same workload; prologue: the mixer's input "
+                         "prologue (separate lines)")
     ap.add_argument("--T", type=int, default=None,
                     help="tokens per row instead of the workload's (smaller cases of the same "
                          "workload for profiler captures; not a bench line)")
@@ -449,6 +526,9 @@ def main():
         return
     if args.variant == "kdn":
         run_kdn(args, w)
+        return
+    if args.variant == "prologue":
+        run_prologue(args, w)
         return
 
     from bayesian_filter_scan_b200 import kla

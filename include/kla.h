@@ -232,6 +232,27 @@ kla_status kla_kdn_forward(const kla_desc *desc,
                            void *out, float *final_lambda, float *final_M,
                            cudaStream_t stream);
 
+/* The mixer's input prologue in one pass (Kalman Linear Attention, technical
+ * summary section 4: a Mamba-like block with a 1-D causal convolution and SiLU
+ * before the mixer): from the pre-activations it writes the forward pass's
+ * inputs,
+ *   q = l2norm(silu(conv(xq))), k = l2norm(silu(conv(xk))), v = silu(conv(xv)),
+ *   a = sigmoid(xa), qn = softplus(xqn), beta = sigmoid(xbeta),
+ * conv: depthwise and causal, y[t,c] = b[c] + sum_{w<W} wgt[c,w] x[t-(W-1)+w,c]
+ * with x = 0 before the start of t's row or packed sequence; l2norm over dk:
+ * y / sqrt(sum y^2 + 1e-6). xq, xk, q, k [Ntok,H,dk] and xv, v [Ntok,H,dv] in
+ * desc->dtype; xa, xqn, a, qn [Ntok,H,dk] (iso [Ntok,H]) and xbeta, beta
+ * [Ntok,H] fp32; weights wq, wk [H,dk,W], wv [H,dv,W] fp32; biases bq, bk
+ * [H,dk], bv [H,dv] fp32 or NULL for none. W = conv_width in 1..4. Device
+ * pointers, 4-byte aligned. Errors as kla_forward. */
+kla_status kla_prologue(const kla_desc *desc, int conv_width,
+                        const void *xq, const void *xk, const void *xv,
+                        const float *xa, const float *xqn, const float *xbeta,
+                        const float *wq, const float *wk, const float *wv,
+                        const float *bq, const float *bk, const float *bv,
+                        void *q, void *k, void *v, float *a, float *qn, float *beta,
+                        cudaStream_t stream);
+
 /* Synchronises `stream`, then reads and clears the library's device status
  * word on the current device: KLA_OK, KLA_ERR_RANGE or KLA_ERR_TIMEOUT from any
  * kernel that ran since the last check, or KLA_ERR_CUDA if the stream failed.
