@@ -343,8 +343,12 @@ kla_status kla_prologue(const kla_desc *d, int conv_width, const void *xq, const
     if (p.ntok == 0 && !p.varlen) return KLA_OK;
     if (!xq || !xk || !xv || !xa || !xqn || !xbeta || !q || !k || !v || !a || !qn || !beta)
         return KLA_ERR_INVALID_ARG;
-    const void *ptrs[] = {xq, xk, xv, xa, xqn, xbeta, wq, wk, wv, bq, bk, bv, q, k, v, a, qn, beta};
-    for (const void *x : ptrs)
+    // rows move as vectors: 16-byte aligned tensors; weights, biases and beta 4-byte
+    const void *vec[] = {xq, xk, xv, xa, xqn, q, k, v, a, qn};
+    for (const void *x : vec)
+        if (!aligned16(x)) return KLA_ERR_INVALID_ARG;
+    const void *sca[] = {xbeta, beta, wq, wk, wv, bq, bk, bv};
+    for (const void *x : sca)
         if (!aligned4(x)) return KLA_ERR_INVALID_ARG;
     const long long ntok = p.varlen ? -1 : p.ntok;
     return cuda_status(launch_prologue(p.H, ntok < 0 ? (long long)d->B * d->T : ntok, p.T,

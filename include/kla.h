@@ -244,7 +244,8 @@ kla_status kla_kdn_forward(const kla_desc *desc,
  * desc->dtype; xa, xqn, a, qn [Ntok,H,dk] (iso [Ntok,H]) and xbeta, beta
  * [Ntok,H] fp32; weights wq, wk [H,dk,W], wv [H,dv,W] fp32; biases bq, bk
  * [H,dk], bv [H,dv] fp32 or NULL for none. W = conv_width in 1..4. Device
- * pointers, 4-byte aligned. Errors as kla_forward. */
+ * pointers: the token tensors 16-byte aligned (rows move as vectors), xbeta,
+ * beta, weights and biases 4-byte aligned. Errors as kla_forward. */
 kla_status kla_prologue(const kla_desc *desc, int conv_width,
                         const void *xq, const void *xk, const void *xv,
                         const float *xa, const float *xqn, const float *xbeta,
