@@ -10,12 +10,13 @@
 // The outputs are the forward pass's inputs in its layouts, so the mixer reads
 // them without another conversion pass.
 //
-// CTA = 128 tokens of one head and one role (q, k, v, or the gates), 8 warps of
-// 16 consecutive tokens; a lane covers dk / 32 (dv / 32) contiguous channels,
-// keeps their conv taps in registers and slides a window of the last W - 1
-// rows along its tokens, so every input row is read once (plus a 3-row halo per
-// warp); a window is cleared where a new row or packed sequence starts. Rows
-// move as one vector per lane and are loaded one token ahead.
+// CTA = 128 tokens of one head and one role (q, k, v, a with beta, or qn). A
+// convolving CTA has 8 warps of 16 consecutive tokens: a warp copies its rows
+// (and the 3 before them) into shared memory, all copies in flight at once; a
+// lane covers dk / 32 (dv / 32) contiguous channels, keeps their conv taps in
+// registers and slides a window of the last W - 1 rows along its tokens; a
+// window is cleared where a new row or packed sequence starts. A gate CTA is
+// elementwise, with 8 vector loads in flight per thread.
 #include "kla_internal.cuh"
 
 namespace kla {
@@ -25,6 +26,7 @@ namespace {
 constexpr int kProWarpTok = 16;  // tokens per warp
 constexpr int kProTok = 8 * kProWarpTok;   // tokens per CTA
 constexpr int kProMaxW = 4;      // widest convolution
+constexpr int kProRoles = 5;     // q, k, v, a and beta, qn
 constexpr float kProEps = 1e-6f;
 
 struct ProArgs {
@@ -39,7 +41,7 @@ struct ProArgs {
     float *a, *qn, *beta;
 };
 
-// N contiguous values (N = 1, 2, 4) as one vector access
+// N contiguous values as one vector access (loads: fp32, N = 1, 4)
 template <int N, typename T>
 __device__ __forceinline__ void ldv(const T *p, float (&x)[N]);
 template <int N, typename T>
@@ -47,45 +49,9 @@ __device__ __forceinline__ void stv(T *p, const float (&x)[N]);
 template <>
 __device__ __forceinline__ void ldv<1, float>(const float *p, float (&x)[1]) { x[0] = __ldg(p); }
 template <>
-__device__ __forceinline__ void ldv<2, float>(const float *p, float (&x)[2]) {
-    const float2 v = __ldg(reinterpret_cast<const float2 *>(p));
-    x[0] = v.x; x[1] = v.y;
-}
-template <>
 __device__ __forceinline__ void ldv<4, float>(const float *p, float (&x)[4]) {
     const float4 v = __ldg(reinterpret_cast<const float4 *>(p));
     x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
-}
-template <>
-__device__ __forceinline__ void ldv<8, float>(const float *p, float (&x)[8]) {
-    const float4 v = __ldg(reinterpret_cast<const float4 *>(p)), w = __ldg(reinterpret_cast<const float4 *>(p) + 1);
-    x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w; x[4] = w.x; x[5] = w.y; x[6] = w.z; x[7] = w.w;
-}
-template <>
-__device__ __forceinline__ void ldv<1, __nv_bfloat16>(const __nv_bfloat16 *p, float (&x)[1]) {
-    x[0] = __bfloat162float(*p);
-}
-template <>
-__device__ __forceinline__ void ldv<2, __nv_bfloat16>(const __nv_bfloat16 *p, float (&x)[2]) {
-    const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p));
-    x[0] = v.x; x[1] = v.y;
-}
-template <>
-__device__ __forceinline__ void ldv<4, __nv_bfloat16>(const __nv_bfloat16 *p, float (&x)[4]) {
-    const uint2 u = __ldg(reinterpret_cast<const uint2 *>(p));
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.x));
-    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&u.y));
-    x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
-}
-template <>
-__device__ __forceinline__ void ldv<8, __nv_bfloat16>(const __nv_bfloat16 *p, float (&x)[8]) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4 *>(p));
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[i]));
-        x[2 * i] = f.x; x[2 * i + 1] = f.y;
-    }
 }
 template <>
 __device__ __forceinline__ void stv<1, float>(float *p, const float (&x)[1]) { *p = x[0]; }
@@ -191,41 +157,75 @@ __device__ __forceinline__ void conv_clear(ConvLane<C> &cl) {
         for (int c = 0; c < C; ++c) cl.hist[r][c] = 0.f;
 }
 
+// Rows held in shared memory per warp: its tokens and the W - 1 before them.
+constexpr int kProRows = kProWarpTok + kProMaxW - 1;
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src)
+                 : "memory");
+}
+
+// C contiguous values of a shared-memory row as floats
+template <int C, typename T>
+__device__ __forceinline__ void lds(const T *p, float (&x)[C]) {
+    if constexpr (std::is_same<T, float>::value) {
+#pragma unroll
+        for (int c = 0; c < C; ++c) x[c] = p[c];
+    } else if constexpr (C == 1) {
+        x[0] = __bfloat162float(p[0]);
+    } else {
+#pragma unroll
+        for (int c = 0; c < C; c += 2) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p + c));
+            x[c] = f.x;
+            if (c + 1 < C) x[c + 1] = f.y;
+        }
+    }
+}
+
 // One convolved tensor (q, k: with the L2 norm over its D channels; v: without)
-// over a warp's tokens [t0, t1): the window slides along them, the rows are
-// loaded one token ahead.
+// over a warp's tokens [t0, t1). The warp first copies its rows (and the W - 1
+// rows before them) into shared memory with asynchronous 16-byte copies, all in
+// flight at once, then slides the window along them.
 template <int D, bool NORM, typename T>
 __device__ __forceinline__ void conv_tensor(const ProArgs &g, const T *x, const float *wgt, const float *bias, T *y,
-                                            int h, int lane, long long t0, long long t1) {
+                                            int h, int lane, long long t0, long long t1, T *rows) {
     constexpr int C = (D + 31) / 32;
+    constexpr int CH = (D * (int)sizeof(T)) / 16;   // 16-byte pieces per row
+    static_assert(CH * 16 == D * (int)sizeof(T), "rows are whole 16-byte pieces");
     const bool act = lane * C < D;
-    ConvLane<C> cl;
-    conv_init<D, C, T>(cl, wgt, bias, g.W, h, lane, act);
     long long s0, s1;
     seq_bounds(g, t0, s0, s1);
+    const long long r0 = max(s0, t0 - (kProMaxW - 1));   // first row the window needs
+    const int nrow = (int)(t1 - r0), off = (int)(r0 - (t0 - (kProMaxW - 1)));
+    for (int e = lane; e < nrow * CH; e += 32) {
+        const int r = e / CH, c = e - r * CH;
+        cp_async16(reinterpret_cast<char *>(rows + (off + r) * D) + 16 * c,
+                   reinterpret_cast<const char *>(x + ((r0 + r) * g.H + h) * D) + 16 * c);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    ConvLane<C> cl;
+    conv_init<D, C, T>(cl, wgt, bias, g.W, h, lane, act);
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncwarp();
     float tmp[C];
     // the window before the warp's first token (rows of the same sequence)
-    for (long long src = max(s0, t0 - (kProMaxW - 1)); src < t0; ++src) {
+    for (int i = off; i < kProMaxW - 1; ++i) {
         float xr[C];
-        if (act) ldv<C, T>(x + (src * g.H + h) * D + lane * C, xr);
+        if (act) lds<C, T>(rows + i * D + lane * C, xr);
         else
 #pragma unroll
             for (int c = 0; c < C; ++c) xr[c] = 0.f;
         conv_step(cl, xr, tmp);
     }
-    float nx[C];
-    auto fetch = [&](long long t) {
-        if (act) ldv<C, T>(x + (t * g.H + h) * D + lane * C, nx);
-        else
-#pragma unroll
-            for (int c = 0; c < C; ++c) nx[c] = 0.f;
-    };
-    fetch(t0);
     for (long long t = t0; t < t1; ++t) {
         float xr[C], yr[C];
+        const int i = (int)(t - t0) + kProMaxW - 1;
+        if (act) lds<C, T>(rows + i * D + lane * C, xr);
+        else
 #pragma unroll
-        for (int c = 0; c < C; ++c) xr[c] = nx[c];
-        if (t + 1 < t1) fetch(t + 1);
+            for (int c = 0; c < C; ++c) xr[c] = 0.f;
         if (t == s1) {
             // a new row or packed sequence: its window starts empty
             long long a0;
@@ -250,56 +250,85 @@ __device__ __forceinline__ void conv_tensor(const ProArgs &g, const T *x, const 
     }
 }
 
-// The gate activations of a warp's tokens.
-template <int DK, bool ISO>
-__device__ __forceinline__ void gate_tokens(const ProArgs &g, int h, int lane, long long t0, long long t1) {
-    constexpr int C = (DK + 31) / 32;
-    for (long long t = t0; t < t1; ++t) {
-        const long long th = t * g.H + h;
-        if (ISO) {
-            if (lane == 0) {
-                g.a[th] = sigm(__ldg(g.xa + th));
-                g.qn[th] = softplus(__ldg(g.xqn + th));
-            }
-        } else if (lane * C < DK) {
-            float xa[C], xn[C];
-            ldv<C, float>(g.xa + th * DK + lane * C, xa);
-            ldv<C, float>(g.xqn + th * DK + lane * C, xn);
+// An elementwise gate over the CTA's tokens [tb, te): out = f(in) on NL values
+// per (token, head); each thread loads a batch of vectors before it computes.
+template <int NL, int F>
+__device__ __forceinline__ void gate_tensor(const ProArgs &g, const float *in, float *out, int h, long long tb,
+                                            long long te) {
+    constexpr int V = NL % 4 == 0 ? 4 : 1;     // floats per access
+    constexpr int PR = NL / V;                  // accesses per row
+    constexpr int B = 8;                        // accesses in flight per thread
+    const int n = (int)(te - tb) * PR;
+    auto f = [](float y) { return F == 0 ? sigm(y) : softplus(y); };
+    for (int e0 = threadIdx.x; e0 < n; e0 += B * blockDim.x) {
+        float xv[B][V];
 #pragma unroll
-            for (int c = 0; c < C; ++c) {
-                xa[c] = sigm(xa[c]);
-                xn[c] = softplus(xn[c]);
+        for (int j = 0; j < B; ++j) {
+            const int e = e0 + j * blockDim.x;
+            if (e < n) {
+                const int r = e / PR, c = e - r * PR;
+                ldv<V, float>(in + ((tb + r) * g.H + h) * NL + c * V, xv[j]);
             }
-            stv<C, float>(g.a + th * DK + lane * C, xa);
-            stv<C, float>(g.qn + th * DK + lane * C, xn);
         }
-        if (lane == 0) g.beta[th] = sigm(__ldg(g.xbeta + th));
+#pragma unroll
+        for (int j = 0; j < B; ++j) {
+            const int e = e0 + j * blockDim.x;
+            if (e < n) {
+                const int r = e / PR, c = e - r * PR;
+#pragma unroll
+                for (int v = 0; v < V; ++v) xv[j][v] = f(xv[j][v]);
+                stv<V, float>(out + ((tb + r) * g.H + h) * NL + c * V, xv[j]);
+            }
+        }
     }
 }
 
-// CTA = (128 tokens, head, role): role 0 q, 1 k, 2 v, 3 the gates; each
-// role holds only its own window and taps in registers.
+// CTA = (role, 128 tokens, head); the roles of one token block are adjacent in
+// the grid so that every SM runs a mix of them: 0 q, 1 k, 2 v (a warp per 16
+// tokens, rows staged in shared memory), 3 a and beta, 4 qn (elementwise).
 template <int DK, int DV, bool ISO, typename T>
 __global__ void __launch_bounds__(256) prologue_kernel(const ProArgs g) {
+    extern __shared__ __align__(16) unsigned char pro_smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int h = blockIdx.y, role = blockIdx.z;
-    const long long t0 = (long long)blockIdx.x * kProTok + warp * kProWarpTok;
+    const int h = blockIdx.y, role = (int)(blockIdx.x % kProRoles);
+    const long long tb = (long long)(blockIdx.x / kProRoles) * kProTok;
+    const long long te = min(tb + kProTok, g.ntok);
+    if (role >= 3) {
+        constexpr int NL = ISO ? 1 : DK;
+        if (role == 3) {
+            gate_tensor<NL, 0>(g, g.xa, g.a, h, tb, te);
+            gate_tensor<1, 0>(g, g.xbeta, g.beta, h, tb, te);
+        } else {
+            gate_tensor<NL, 1>(g, g.xqn, g.qn, h, tb, te);
+        }
+        return;
+    }
+    const long long t0 = tb + warp * kProWarpTok;
     if (t0 >= g.ntok) return;
     const long long t1 = min(t0 + kProWarpTok, g.ntok);
+    constexpr int DM = DK > DV ? DK : DV;
+    T *rows = reinterpret_cast<T *>(pro_smem) + (size_t)warp * kProRows * DM;
     if (role == 0)
-        conv_tensor<DK, true, T>(g, static_cast<const T *>(g.xq), g.wq, g.bq, static_cast<T *>(g.q), h, lane, t0, t1);
+        conv_tensor<DK, true, T>(g, static_cast<const T *>(g.xq), g.wq, g.bq, static_cast<T *>(g.q), h, lane, t0, t1,
+                                 rows);
     else if (role == 1)
-        conv_tensor<DK, true, T>(g, static_cast<const T *>(g.xk), g.wk, g.bk, static_cast<T *>(g.k), h, lane, t0, t1);
-    else if (role == 2)
-        conv_tensor<DV, false, T>(g, static_cast<const T *>(g.xv), g.wv, g.bv, static_cast<T *>(g.v), h, lane, t0, t1);
+        conv_tensor<DK, true, T>(g, static_cast<const T *>(g.xk), g.wk, g.bk, static_cast<T *>(g.k), h, lane, t0, t1,
+                                 rows);
     else
-        gate_tokens<DK, ISO>(g, h, lane, t0, t1);
+        conv_tensor<DV, false, T>(g, static_cast<const T *>(g.xv), g.wv, g.bv, static_cast<T *>(g.v), h, lane, t0, t1,
+                                  rows);
 }
 
 template <int DK, int DV, bool ISO, typename T>
 cudaError_t launch_pro_t(const ProArgs &g, cudaStream_t st) {
-    dim3 grid((unsigned)((g.ntok + kProTok - 1) / kProTok), (unsigned)g.H, 4u);
-    prologue_kernel<DK, DV, ISO, T><<<grid, 256, 0, st>>>(g);
+    static PerDevice<bool> attr;
+    constexpr int DM = DK > DV ? DK : DV;
+    const int smem = 8 * kProRows * DM * (int)sizeof(T);
+    auto kern = prologue_kernel<DK, DV, ISO, T>;
+    cudaError_t e = ensure_smem_attr(attr, kern, smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)((g.ntok + kProTok - 1) / kProTok * kProRoles), (unsigned)g.H);
+    kern<<<grid, 256, smem, st>>>(g);
     return cudaGetLastError();
 }
 
