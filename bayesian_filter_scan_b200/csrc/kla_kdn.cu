@@ -1,6 +1,7 @@
 // kla_kdn.cu -- the Kalman Delta Network forward with the Kalman-gain residual
-// write (sm_100a, CUDA cores). One CTA per (row or packed sequence, head) walks
-// its tokens in order; the mean state lives in registers for the whole walk.
+// write (sm_100a, CUDA cores). One CTA per (row or packed sequence, head, block
+// of value columns) walks its tokens in order; its part of the mean state lives
+// in registers for the whole walk.
 //
 // Kalman Delta Networks abstract: the memory is the state of a linear-Gaussian
 // model whose transition propagates the mean and its uncertainty, the Kalman
@@ -16,8 +17,11 @@
 //   o       = M^T q = (a M)^T q + gamma (q.w) r  readout of the posterior mean
 // (isotropic: a, qn and lambda are scalars per head, lambda += beta |k|^2 / dk).
 //
-// Thread layout: thread t owns value column j = t % dv and rows
-// [rg * dk/RG, (rg + 1) * dk/RG) of M, rg = t / dv, RG = 256 / dv; threads
+// The value columns of M evolve independently given the key-side quantities
+// (a, k, w, gamma), so a (row, head) is split over CTAs by blocks of DVB value
+// columns; each CTA repeats the cheap key-side step. Thread layout inside a
+// CTA: thread t owns column j = cb * DVB + t % DVB and rows
+// [rg * dk/RG, (rg + 1) * dk/RG) of M, rg = t / DVB, RG = 256 / DVB; threads
 // t < dk prepare key t's precision step and gain. Per token: the key threads
 // stage (a, k, q, w) and per-warp partial sums (k.w, q.w, |k|^2) in shared
 // memory; every thread decays its rows and forms its partial dot products with
@@ -71,18 +75,24 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
+// Value columns per CTA: 32, or dv when it is smaller.
+template <int DV>
+constexpr int kdn_dvb() { return DV < 32 ? DV : 32; }
+
 template <int DK, int DV, bool ISO, typename T>
 __global__ void __launch_bounds__(kKdnThreads) kdn_walk_kernel(const KdnArgs g) {
-    constexpr int RG = kKdnThreads / DV;   // row groups
+    constexpr int DVB = kdn_dvb<DV>();     // value columns of this CTA
+    constexpr int RG = kKdnThreads / DVB;  // row groups
     constexpr int RPT = DK / RG;           // rows of M per thread
     constexpr int NWK = (DK + 31) / 32;    // warps holding keys
     static_assert(RPT >= 1 && RPT * RG == DK, "thread layout");
-    __shared__ float s_a[2][DK], s_k[2][DK], s_q[2][DK], s_w[2][DK], s_v[2][DV];
-    __shared__ float s_pk[2][RG][DV], s_pq[2][RG][DV];
+    __shared__ float s_a[2][DK], s_k[2][DK], s_q[2][DK], s_w[2][DK], s_v[2][DVB];
+    __shared__ float s_pk[2][RG][DVB], s_pq[2][RG][DVB];
     __shared__ float s_red[2][NWK][3];
 
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    const int j = tid % DV, rg = tid / DV, i0 = rg * RPT;
+    const int jl = tid % DVB, rg = tid / DVB, i0 = rg * RPT;
+    const int cb = (int)blockIdx.y, j = cb * DVB + jl;   // local and global column
     const long long u = blockIdx.x;
     const int h = (int)(u % g.H);
     const long long n = u / g.H;
@@ -116,7 +126,7 @@ __global__ void __launch_bounds__(kKdnThreads) kdn_walk_kernel(const KdnArgs g) 
             na = __ldg(g.a + th);
             nqn = __ldg(g.qn + th);
         }
-        if (tid < DV) nv = ldx<T>(v, th * DV + tid);
+        if (tid < DVB) nv = ldx<T>(v, th * DV + cb * DVB + tid);
         nb = __ldg(g.beta + th);
     };
     if (te > tb) fetch(tb);
@@ -140,7 +150,7 @@ __global__ void __launch_bounds__(kKdnThreads) kdn_walk_kernel(const KdnArgs g) 
             qw = cq * w;
             kk = ck * ck;
         }
-        if (tid < DV) s_v[buf][tid] = cv;
+        if (tid < DVB) s_v[buf][tid] = cv;
         if (wid < NWK) {
             kw = warp_sum(kw);
             qw = warp_sum(qw);
@@ -170,23 +180,23 @@ __global__ void __launch_bounds__(kKdnThreads) kdn_walk_kernel(const KdnArgs g) 
             ak = fmaf(s_k[buf][i], m[r], ak);
             aq = fmaf(s_q[buf][i], m[r], aq);
         }
-        s_pk[buf][rg][j] = ak;
-        s_pq[buf][rg][j] = aq;
+        s_pk[buf][rg][jl] = ak;
+        s_pq[buf][rg][jl] = aq;
         __syncthreads();
         // ---- the column's innovation, the rank-1 write, the readout
         float mk = 0.f, mq = 0.f;
 #pragma unroll
         for (int x = 0; x < RG; ++x) {
-            mk += s_pk[buf][x][j];
-            mq += s_pq[buf][x][j];
+            mk += s_pk[buf][x][jl];
+            mq += s_pq[buf][x][jl];
         }
-        const float rj = s_v[buf][j] - mk;
+        const float rj = s_v[buf][jl] - mk;
         const float gr = gam * rj;
 #pragma unroll
         for (int r = 0; r < RPT; ++r) m[r] = fmaf(s_w[buf][i0 + r], gr, m[r]);
         if (rg == 0) stx<T>(out, (t * g.H + h) * DV + j, fmaf(gq, gr, mq));
     }
-    if (g.final_lambda) {
+    if (g.final_lambda && cb == 0) {
         if (ISO) { if (tid == 0) g.final_lambda[u] = lam; }
         else if (tid < DK) g.final_lambda[u * DK + tid] = lam;
     }
@@ -198,7 +208,8 @@ __global__ void __launch_bounds__(kKdnThreads) kdn_walk_kernel(const KdnArgs g) 
 
 template <int DK, int DV, bool ISO, typename T>
 cudaError_t launch_kdn_t(long long units, const KdnArgs &g, cudaStream_t st) {
-    kdn_walk_kernel<DK, DV, ISO, T><<<(unsigned)units, kKdnThreads, 0, st>>>(g);
+    const dim3 grid((unsigned)units, (unsigned)(DV / kdn_dvb<DV>()));
+    kdn_walk_kernel<DK, DV, ISO, T><<<grid, kKdnThreads, 0, st>>>(g);
     return cudaGetLastError();
 }
 
