@@ -10,21 +10,28 @@
 // The outputs are the forward pass's inputs in its layouts, so the mixer reads
 // them without another conversion pass.
 //
-// CTA = 128 tokens of one head and one role (q, k, v, a with beta, or qn). A
-// convolving CTA has 8 warps of 16 consecutive tokens: a warp copies its rows
-// (and the 3 before them) into shared memory, all copies in flight at once; a
-// lane covers dk / 32 (dv / 32) contiguous channels, keeps their conv taps in
-// registers and slides a window of the last W - 1 rows along its tokens; a
-// window is cleared where a new row or packed sequence starts. A gate CTA is
-// elementwise, with 8 vector loads in flight per thread.
+// CTA = 8 warps x (tiles of 16 tokens per warp) of one head and one role (q, k,
+// v, a with beta, or qn). A convolving warp walks its consecutive tiles in
+// order: it copies a tile's rows (for the first, also the 3 before them) into
+// shared memory, all copies in flight at once, and the next tile's copies fly
+// while it convolves the current one; a lane covers dk / 32 (dv / 32)
+// contiguous channels, keeps their conv taps in registers and slides a window
+// of the last W - 1 rows along its tokens; a window is cleared where a new row
+// or packed sequence starts. A gate CTA is elementwise, with 8 vector loads in
+// flight per thread.
 #include "kla_internal.cuh"
 
 namespace kla {
 
 namespace {
 
-constexpr int kProWarpTok = 16;  // tokens per warp
-constexpr int kProTok = 8 * kProWarpTok;   // tokens per CTA
+#ifndef KLA_PRO_TILES
+#define KLA_PRO_TILES 1
+#endif
+constexpr int kProTileTok = 16;                        // tokens per tile
+constexpr int kProTiles = KLA_PRO_TILES;               // tiles a warp walks in order
+constexpr int kProWarpTok = kProTiles * kProTileTok;   // tokens per warp
+constexpr int kProTok = 8 * kProWarpTok;               // tokens per CTA
 constexpr int kProMaxW = 4;      // widest convolution
 constexpr int kProRoles = 5;     // q, k, v, a and beta, qn
 constexpr float kProEps = 1e-6f;
@@ -157,8 +164,10 @@ __device__ __forceinline__ void conv_clear(ConvLane<C> &cl) {
         for (int c = 0; c < C; ++c) cl.hist[r][c] = 0.f;
 }
 
-// Rows held in shared memory per warp: its tokens and the W - 1 before them.
-constexpr int kProRows = kProWarpTok + kProMaxW - 1;
+// Rows held in shared memory per warp: two tile buffers, the first with the
+// W - 1 rows before the warp's first token in front of it.
+constexpr int kProBufs = kProTiles > 1 ? 2 : 1;
+constexpr int kProRows = kProMaxW - 1 + kProBufs * kProTileTok;
 
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
@@ -185,69 +194,98 @@ __device__ __forceinline__ void lds(const T *p, float (&x)[C]) {
 }
 
 // One convolved tensor (q, k: with the L2 norm over its D channels; v: without)
-// over a warp's tokens [t0, t1). The warp first copies its rows (and the W - 1
-// rows before them) into shared memory with asynchronous 16-byte copies, all in
-// flight at once, then slides the window along them.
+// over a warp's tokens [tw0, tw1), walked as tiles of 16 tokens. The rows of a
+// tile (for the first, also the W - 1 rows before it) are copied into shared
+// memory with asynchronous 16-byte copies, all in flight at once; the next
+// tile's copies are in flight while the warp convolves the current one (two
+// buffers). The window of the last W - 1 rows slides along the whole span in
+// registers.
 template <int D, bool NORM, typename T>
 __device__ __forceinline__ void conv_tensor(const ProArgs &g, const T *x, const float *wgt, const float *bias, T *y,
-                                            int h, int lane, long long t0, long long t1, T *rows) {
+                                            int h, int lane, long long tw0, long long tw1, T *rows) {
     constexpr int C = (D + 31) / 32;
     constexpr int CH = (D * (int)sizeof(T)) / 16;   // 16-byte pieces per row
     static_assert(CH * 16 == D * (int)sizeof(T), "rows are whole 16-byte pieces");
+    constexpr int H0 = kProMaxW - 1;
     const bool act = lane * C < D;
     long long s0, s1;
-    seq_bounds(g, t0, s0, s1);
-    const long long r0 = max(s0, t0 - (kProMaxW - 1));   // first row the window needs
-    const int nrow = (int)(t1 - r0), off = (int)(r0 - (t0 - (kProMaxW - 1)));
-    for (int e = lane; e < nrow * CH; e += 32) {
-        const int r = e / CH, c = e - r * CH;
-        cp_async16(reinterpret_cast<char *>(rows + (off + r) * D) + 16 * c,
-                   reinterpret_cast<const char *>(x + ((r0 + r) * g.H + h) * D) + 16 * c);
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
+    seq_bounds(g, tw0, s0, s1);
+    const long long r0 = max(s0, tw0 - H0);   // first row the window needs
+    const int off = (int)(r0 - (tw0 - H0));
+    // tile i's first token sits at row slot tile_slot(i) of the warp's rows
+    auto tile_slot = [](int i) { return H0 + (i % kProBufs) * kProTileTok; };
+    // copies of tile i: its rows (and for tile 0 the rows before it), one group
+    auto issue = [&](int i) {
+        const long long a = i == 0 ? r0 : tw0 + (long long)i * kProTileTok;
+        const long long b = min(tw0 + (long long)(i + 1) * kProTileTok, tw1);
+        const int slot0 = i == 0 ? off : tile_slot(i);
+        const int n = a < b ? (int)(b - a) * CH : 0;
+        for (int e = lane; e < n; e += 32) {
+            const int r = e / CH, c = e - r * CH;
+            cp_async16(reinterpret_cast<char *>(rows + (slot0 + r) * D) + 16 * c,
+                       reinterpret_cast<const char *>(x + ((a + r) * g.H + h) * D) + 16 * c);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    issue(0);
+    if (kProTiles > 1) issue(1);
     ConvLane<C> cl;
     conv_init<D, C, T>(cl, wgt, bias, g.W, h, lane, act);
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
-    __syncwarp();
     float tmp[C];
-    // the window before the warp's first token (rows of the same sequence)
-    for (int i = off; i < kProMaxW - 1; ++i) {
-        float xr[C];
-        if (act) lds<C, T>(rows + i * D + lane * C, xr);
-        else
+#pragma unroll 1
+    for (int i = 0; i < kProTiles; ++i) {
+        const long long t0 = tw0 + (long long)i * kProTileTok;
+        // tile i's group is complete once at most the later one is pending
+        if (i + 1 < kProTiles) asm volatile("cp.async.wait_group 1;" ::: "memory");
+        else asm volatile("cp.async.wait_group 0;" ::: "memory");
+        __syncwarp();
+        if (t0 >= tw1) break;
+        if (i == 0) {
+            // the window before the warp's first token (rows of the same sequence)
+            for (int r = off; r < H0; ++r) {
+                float xr[C];
+                if (act) lds<C, T>(rows + r * D + lane * C, xr);
+                else
 #pragma unroll
-            for (int c = 0; c < C; ++c) xr[c] = 0.f;
-        conv_step(cl, xr, tmp);
+                    for (int c = 0; c < C; ++c) xr[c] = 0.f;
+                conv_step(cl, xr, tmp);
+            }
+        }
+        const T *buf = rows + tile_slot(i) * D;
+        const long long t1 = min(t0 + kProTileTok, tw1);
+        for (long long t = t0; t < t1; ++t) {
+            float xr[C], yr[C];
+            if (act) lds<C, T>(buf + (int)(t - t0) * D + lane * C, xr);
+            else
+#pragma unroll
+                for (int c = 0; c < C; ++c) xr[c] = 0.f;
+            if (t == s1) {
+                // a new row or packed sequence: its window starts empty
+                long long a0;
+                seq_bounds(g, t, a0, s1);
+                conv_clear(cl);
+            }
+            conv_step(cl, xr, yr);
+            float ss = 0.f;
+#pragma unroll
+            for (int c = 0; c < C; ++c) {
+                yr[c] = silu(yr[c]);
+                if (act) ss = fmaf(yr[c], yr[c], ss);
+            }
+            if (NORM) {
+#pragma unroll
+                for (int d = 16; d > 0; d >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, d);
+                const float sc = rsqrtf(ss + kProEps);
+#pragma unroll
+                for (int c = 0; c < C; ++c) yr[c] *= sc;
+            }
+            if (act) stv<C, T>(y + (t * g.H + h) * D + lane * C, yr);
+        }
+        // every lane has read this buffer before it is refilled
+        __syncwarp();
+        if (i + 2 < kProTiles) issue(i + 2);
     }
-    for (long long t = t0; t < t1; ++t) {
-        float xr[C], yr[C];
-        const int i = (int)(t - t0) + kProMaxW - 1;
-        if (act) lds<C, T>(rows + i * D + lane * C, xr);
-        else
-#pragma unroll
-            for (int c = 0; c < C; ++c) xr[c] = 0.f;
-        if (t == s1) {
-            // a new row or packed sequence: its window starts empty
-            long long a0;
-            seq_bounds(g, t, a0, s1);
-            conv_clear(cl);
-        }
-        conv_step(cl, xr, yr);
-        float ss = 0.f;
-#pragma unroll
-        for (int c = 0; c < C; ++c) {
-            yr[c] = silu(yr[c]);
-            if (act) ss = fmaf(yr[c], yr[c], ss);
-        }
-        if (NORM) {
-#pragma unroll
-            for (int d = 16; d > 0; d >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, d);
-            const float sc = rsqrtf(ss + kProEps);
-#pragma unroll
-            for (int c = 0; c < C; ++c) yr[c] *= sc;
-        }
-        if (act) stv<C, T>(y + (t * g.H + h) * D + lane * C, yr);
-    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
 // An elementwise gate over the CTA's tokens [tb, te): out = f(in) on NL values
@@ -283,9 +321,10 @@ __device__ __forceinline__ void gate_tensor(const ProArgs &g, const float *in, f
     }
 }
 
-// CTA = (role, 128 tokens, head); the roles of one token block are adjacent in
-// the grid so that every SM runs a mix of them: 0 q, 1 k, 2 v (a warp per 16
-// tokens, rows staged in shared memory), 3 a and beta, 4 qn (elementwise).
+// CTA = (role, token block, head); the roles of one token block are adjacent
+// in the grid so that every SM runs a mix of them: 0 q, 1 k, 2 v (a warp per
+// kProWarpTok tokens, rows staged in shared memory), 3 a and beta, 4 qn
+// (elementwise).
 template <int DK, int DV, bool ISO, typename T>
 __global__ void __launch_bounds__(256) prologue_kernel(const ProArgs g) {
     extern __shared__ __align__(16) unsigned char pro_smem[];
@@ -303,7 +342,7 @@ __global__ void __launch_bounds__(256) prologue_kernel(const ProArgs g) {
         }
         return;
     }
-    const long long t0 = tb + warp * kProWarpTok;
+    const long long t0 = tb + (long long)warp * kProWarpTok;
     if (t0 >= g.ntok) return;
     const long long t1 = min(t0 + kProWarpTok, g.ntok);
     constexpr int DM = DK > DV ? DK : DV;

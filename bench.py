@@ -361,7 +361,7 @@ def run_kdn(args, w):
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic", "config": cfg,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": None, "kernel": "kdn_walk_kernel (CUDA cores, one CTA per row x head)",
+                     "traffic": None, "kernel": "kdn_walk_kernel (CUDA cores, one CTA per row x head x 32 value columns)",
                      "alg_bytes_per_launch": alg_bytes, "launch_ms": ms,
                      "alg_bytes_per_token_head": bytes_per_token_head(w),
                      "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_src},
@@ -403,10 +403,26 @@ def prologue_bytes_per_token_head(w) -> int:
     return 2 * (es * (2 * w.dk + w.dv) + 4 * 2 * nl + 4)
 
 
+def _prologue_sample(x, cu, w, n):
+    """The first n tokens of the flattened token axis as a problem of their
+    own (the rows or packed sequences that start inside it, the last one cut
+    at n): arguments for oracle.prologue."""
+    xs = {k: (v[:n] if k.startswith("x") else v) for k, v in x.items()}
+    if cu is None:
+        T = w.T
+        bounds = list(range(0, n, T)) + [n]
+    else:
+        bounds = [c for c in cu.tolist() if c < n] + [n]
+    return xs, np.asarray(bounds, dtype=np.int64)
+
+
 def run_prologue(args, w):
     """kla_prologue on the workload's shape with synthetic pre-activations and
     conv weights (width 4): device-timed with L2 flushed between steps,
-    against its algorithmic bytes and the measured HBM peak."""
+    against its algorithmic bytes and the measured HBM peak; end to end with
+    the pre-activations copied in from pinned host memory and the six outputs
+    copied back inside the timed region; the numpy fp64 oracle on a bounded
+    prefix of the tokens as the CPU baseline."""
     from bayesian_filter_scan_b200 import kla
     torch.cuda.set_device(0)
     kla.lib()
@@ -451,6 +467,33 @@ def run_prologue(args, w):
     torch.cuda.synchronize()
     clk = clocks.stop()
     ms = statistics.mean(a_.elapsed_time(b_) for a_, b_ in ts)
+    kla.check()
+    # end to end: pinned pre-activations in, the six outputs out, inside the timed region
+    names = ("xq", "xk", "xv", "xa", "xqn", "xbeta")
+    pin = {k: x[k].pin_memory() for k in names}
+    hout = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+    dbuf = dict(d)
+    for k in names:
+        dbuf[k] = torch.empty_like(d[k])
+    e_t, e_steps = 0.0, max(3, min(args.e2e_steps, args.steps))
+    for i in range(e_steps + 2):
+        flush.fill_(1)
+        sweep.sum()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for k in names:
+            dbuf[k].copy_(pin[k], non_blocking=True)
+        kla.prologue(**dbuf, cu_seqlens=cu, B=None if cu is not None else w.B, T=None if cu is not None else w.T,
+                     mode=w.mode, out=outs)
+        for ho, o in zip(hout, outs):
+            ho.copy_(o, non_blocking=True)
+        a1.record(stream)
+        a1.synchronize()
+        if i >= 2:
+            e_t += a0.elapsed_time(a1)
+    e2e = {"value": w.tokens / (e_t / e_steps * 1e-3), "unit": UNIT,
+           "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in pin.values()),
+           "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in hout)}
     peaks, peak_src = measured_peaks()
     peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
     alg = prologue_bytes_per_token_head(w) * w.tokens * H
@@ -464,7 +507,27 @@ def run_prologue(args, w):
                         "traffic": None, "kernel": "prologue_kernel", "alg_bytes_per_launch": alg, "launch_ms": ms,
                         "alg_bytes_per_token_head": prologue_bytes_per_token_head(w),
                         "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_src},
-           "gpu_launches": args.steps, "clocks": clk}
+           "e2e": e2e, "gpu_launches": args.steps, "clocks": clk}
+    if not args.no_cpu_baseline:
+        import oracle
+        cu_h = inp["cu_seqlens"]
+        xs, bounds = _prologue_sample(x, cu_h, w, min(256, Ntok))
+        t1 = time.perf_counter()
+        oracle.prologue(**xs, cu_seqlens=bounds)
+        per_tok = max(time.perf_counter() - t1, 1e-4) / min(256, Ntok)
+        n = int(max(1, min(Ntok, 8192, 12.0 / per_tok)))
+        xs, bounds = _prologue_sample(x, cu_h, w, n)
+        t0 = time.perf_counter()
+        ref = oracle.prologue(**xs, cu_seqlens=bounds)
+        t = time.perf_counter() - t0
+        res["cpu_baseline"] = {"value": n / t, "unit": UNIT, "cores": 1, "kind": "oracle",
+                               "sample": "the first %d of %d tokens (all %d heads), numpy fp64 oracle, %.3f s" % (
+                                   n, Ntok, H, t)}
+        worst = {}
+        for name, o in zip(("q", "k", "v", "a", "qn", "beta"), outs):
+            worst[name] = scaled_err(o[:n], ref[name])
+        res["max_err"] = dict(worst, tokens=n, tol=2e-2 if w.dtype == "bf16" else 1e-4,
+                              definition="max |gpu - oracle| / (1 + |oracle|) over the sampled tokens")
     print(json.dumps(res))
 
 
