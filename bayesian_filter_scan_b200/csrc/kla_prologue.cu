@@ -28,10 +28,7 @@ namespace {
 #ifndef KLA_PRO_TILES
 #define KLA_PRO_TILES 1
 #endif
-constexpr int kProTileTok = 16;                        // tokens per tile
-constexpr int kProTiles = KLA_PRO_TILES;               // tiles a warp walks in order
-constexpr int kProWarpTok = kProTiles * kProTileTok;   // tokens per warp
-constexpr int kProTok = 8 * kProWarpTok;               // tokens per CTA
+constexpr int kProTileTok = 16;  // tokens per tile
 constexpr int kProMaxW = 4;      // widest convolution
 constexpr int kProRoles = 5;     // q, k, v, a and beta, qn
 constexpr float kProEps = 1e-6f;
@@ -164,10 +161,21 @@ __device__ __forceinline__ void conv_clear(ConvLane<C> &cl) {
         for (int c = 0; c < C; ++c) cl.hist[r][c] = 0.f;
 }
 
-// Rows held in shared memory per warp: two tile buffers, the first with the
-// W - 1 rows before the warp's first token in front of it.
-constexpr int kProBufs = kProTiles > 1 ? 2 : 1;
-constexpr int kProRows = kProMaxW - 1 + kProBufs * kProTileTok;
+// The tiling of one instantiation (DM = max(dk, dv) channels of type T): the
+// tiles a warp walks in order (KLA_PRO_TILES, or 1 where two tile buffers per
+// warp would not fit in shared memory), and the rows a warp holds in shared
+// memory: one or two tile buffers, the first with the W - 1 rows before the
+// warp's first token in front of it.
+template <int DM, typename T>
+struct ProShape {
+    static constexpr int two_buf_bytes = 8 * (kProMaxW - 1 + 2 * kProTileTok) * DM * (int)sizeof(T);
+    static constexpr int tiles = (KLA_PRO_TILES > 1 && two_buf_bytes <= 200 * 1024) ? KLA_PRO_TILES : 1;
+    static constexpr int bufs = tiles > 1 ? 2 : 1;
+    static constexpr int rows = kProMaxW - 1 + bufs * kProTileTok;   // rows per warp
+    static constexpr int warp_tok = tiles * kProTileTok;              // tokens per warp
+    static constexpr int cta_tok = 8 * warp_tok;                      // tokens per CTA
+    static constexpr int smem = 8 * rows * DM * (int)sizeof(T);
+};
 
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
@@ -200,9 +208,10 @@ __device__ __forceinline__ void lds(const T *p, float (&x)[C]) {
 // tile's copies are in flight while the warp convolves the current one (two
 // buffers). The window of the last W - 1 rows slides along the whole span in
 // registers.
-template <int D, bool NORM, typename T>
+template <int D, bool NORM, int NT, typename T>
 __device__ __forceinline__ void conv_tensor(const ProArgs &g, const T *x, const float *wgt, const float *bias, T *y,
                                             int h, int lane, long long tw0, long long tw1, T *rows) {
+    constexpr int NB = NT > 1 ? 2 : 1;   // tile buffers
     constexpr int C = (D + 31) / 32;
     constexpr int CH = (D * (int)sizeof(T)) / 16;   // 16-byte pieces per row
     static_assert(CH * 16 == D * (int)sizeof(T), "rows are whole 16-byte pieces");
@@ -213,7 +222,7 @@ __device__ __forceinline__ void conv_tensor(const ProArgs &g, const T *x, const 
     const long long r0 = max(s0, tw0 - H0);   // first row the window needs
     const int off = (int)(r0 - (tw0 - H0));
     // tile i's first token sits at row slot tile_slot(i) of the warp's rows
-    auto tile_slot = [](int i) { return H0 + (i % kProBufs) * kProTileTok; };
+    auto tile_slot = [](int i) { return H0 + (i % NB) * kProTileTok; };
     // copies of tile i: its rows (and for tile 0 the rows before it), one group
     auto issue = [&](int i) {
         const long long a = i == 0 ? r0 : tw0 + (long long)i * kProTileTok;
@@ -228,15 +237,15 @@ __device__ __forceinline__ void conv_tensor(const ProArgs &g, const T *x, const 
         asm volatile("cp.async.commit_group;" ::: "memory");
     };
     issue(0);
-    if (kProTiles > 1) issue(1);
+    if (NT > 1) issue(1);
     ConvLane<C> cl;
     conv_init<D, C, T>(cl, wgt, bias, g.W, h, lane, act);
     float tmp[C];
 #pragma unroll 1
-    for (int i = 0; i < kProTiles; ++i) {
+    for (int i = 0; i < NT; ++i) {
         const long long t0 = tw0 + (long long)i * kProTileTok;
         // tile i's group is complete once at most the later one is pending
-        if (i + 1 < kProTiles) asm volatile("cp.async.wait_group 1;" ::: "memory");
+        if (i + 1 < NT) asm volatile("cp.async.wait_group 1;" ::: "memory");
         else asm volatile("cp.async.wait_group 0;" ::: "memory");
         __syncwarp();
         if (t0 >= tw1) break;
@@ -283,7 +292,7 @@ __device__ __forceinline__ void conv_tensor(const ProArgs &g, const T *x, const 
         }
         // every lane has read this buffer before it is refilled
         __syncwarp();
-        if (i + 2 < kProTiles) issue(i + 2);
+        if (i + 2 < NT) issue(i + 2);
     }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
@@ -323,15 +332,17 @@ __device__ __forceinline__ void gate_tensor(const ProArgs &g, const float *in, f
 
 // CTA = (role, token block, head); the roles of one token block are adjacent
 // in the grid so that every SM runs a mix of them: 0 q, 1 k, 2 v (a warp per
-// kProWarpTok tokens, rows staged in shared memory), 3 a and beta, 4 qn
+// ProShape::warp_tok tokens, rows staged in shared memory), 3 a and beta, 4 qn
 // (elementwise).
 template <int DK, int DV, bool ISO, typename T>
 __global__ void __launch_bounds__(256) prologue_kernel(const ProArgs g) {
     extern __shared__ __align__(16) unsigned char pro_smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int DM = DK > DV ? DK : DV;
+    using S = ProShape<DM, T>;
     const int h = blockIdx.y, role = (int)(blockIdx.x % kProRoles);
-    const long long tb = (long long)(blockIdx.x / kProRoles) * kProTok;
-    const long long te = min(tb + kProTok, g.ntok);
+    const long long tb = (long long)(blockIdx.x / kProRoles) * S::cta_tok;
+    const long long te = min(tb + S::cta_tok, g.ntok);
     if (role >= 3) {
         constexpr int NL = ISO ? 1 : DK;
         if (role == 3) {
@@ -342,31 +353,31 @@ __global__ void __launch_bounds__(256) prologue_kernel(const ProArgs g) {
         }
         return;
     }
-    const long long t0 = tb + (long long)warp * kProWarpTok;
+    const long long t0 = tb + (long long)warp * S::warp_tok;
     if (t0 >= g.ntok) return;
-    const long long t1 = min(t0 + kProWarpTok, g.ntok);
-    constexpr int DM = DK > DV ? DK : DV;
-    T *rows = reinterpret_cast<T *>(pro_smem) + (size_t)warp * kProRows * DM;
+    const long long t1 = min(t0 + S::warp_tok, g.ntok);
+    T *rows = reinterpret_cast<T *>(pro_smem) + (size_t)warp * S::rows * DM;
     if (role == 0)
-        conv_tensor<DK, true, T>(g, static_cast<const T *>(g.xq), g.wq, g.bq, static_cast<T *>(g.q), h, lane, t0, t1,
-                                 rows);
+        conv_tensor<DK, true, S::tiles, T>(g, static_cast<const T *>(g.xq), g.wq, g.bq, static_cast<T *>(g.q), h,
+                                           lane, t0, t1, rows);
     else if (role == 1)
-        conv_tensor<DK, true, T>(g, static_cast<const T *>(g.xk), g.wk, g.bk, static_cast<T *>(g.k), h, lane, t0, t1,
-                                 rows);
+        conv_tensor<DK, true, S::tiles, T>(g, static_cast<const T *>(g.xk), g.wk, g.bk, static_cast<T *>(g.k), h,
+                                           lane, t0, t1, rows);
     else
-        conv_tensor<DV, false, T>(g, static_cast<const T *>(g.xv), g.wv, g.bv, static_cast<T *>(g.v), h, lane, t0, t1,
-                                  rows);
+        conv_tensor<DV, false, S::tiles, T>(g, static_cast<const T *>(g.xv), g.wv, g.bv, static_cast<T *>(g.v), h,
+                                            lane, t0, t1, rows);
 }
 
 template <int DK, int DV, bool ISO, typename T>
 cudaError_t launch_pro_t(const ProArgs &g, cudaStream_t st) {
     static PerDevice<bool> attr;
     constexpr int DM = DK > DV ? DK : DV;
-    const int smem = 8 * kProRows * DM * (int)sizeof(T);
+    using S = ProShape<DM, T>;
+    const int smem = S::smem;
     auto kern = prologue_kernel<DK, DV, ISO, T>;
     cudaError_t e = ensure_smem_attr(attr, kern, smem);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)((g.ntok + kProTok - 1) / kProTok * kProRoles), (unsigned)g.H);
+    dim3 grid((unsigned)((g.ntok + S::cta_tok - 1) / S::cta_tok * kProRoles), (unsigned)g.H);
     kern<<<grid, 256, smem, st>>>(g);
     return cudaGetLastError();
 }
