@@ -17,7 +17,9 @@ rule when the predictive covariance is a constant isotropic surrogate (see
 tests/test_kdn_pins.py). The mixer's input prologue (``prologue``: causal conv,
 SiLU, L2 norm, sigmoid / softplus gates) is plain numpy, pinned against the
 identity kernel, numpy's convolution per channel, closed forms of the gates
-and packed sequences (tests/test_prologue_pins.py).
+and packed sequences (tests/test_prologue_pins.py). The gradients of the filter
+(``backward``, reverse mode over stored states) are pinned against central
+finite differences of the pinned forward (tests/test_backward_pins.py).
 The isotropic increment beta*|k|^2/dk is pinned for consistency only (it
 reduces to the diagonal filter when dk = 1 and to the closed form when a=1,
 qn=0); the choice of that constant is a reading of the Kalman Delta Networks
@@ -69,6 +71,13 @@ def _load():
             _i32p, ctypes.c_int,
             _f32p, _f32p, _f32p, _f32p, _f32p, _f32p, _f32p, _f32p,
             _f64p, _f64p, _f64p, ctypes.c_long, ctypes.c_long, ctypes.c_int]
+        lib.kla_oracle_backward.restype = ctypes.c_int
+        lib.kla_oracle_backward.argtypes = [
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            _i32p, ctypes.c_int,
+            _f32p, _f32p, _f32p, _f32p, _f32p, _f32p, _f32p, _f32p, _f32p, _f32p, _f32p,
+            _f64p, _f64p, _f64p, _f64p, _f64p, _f64p, _f64p, _f64p,
+            ctypes.c_long, ctypes.c_long, ctypes.c_int]
         lib.kla_oracle_max_threads.restype = ctypes.c_int
         lib.kla_oracle_mobius_element.argtypes = [ctypes.c_double] * 3 + [_f64p]
         lib.kla_oracle_mobius_compose.argtypes = [_f64p, _f64p, _f64p]
@@ -140,6 +149,45 @@ def forward(q, k, v, a, qn, beta, lambda0=None, eta0=None, cu_seqlens=None,
     if want_lambda:
         res["lambda"] = lt
     return res
+
+
+def backward(q, k, v, a, qn, beta, dout, lambda0=None, eta0=None, dfinal_lambda=None,
+             dfinal_eta=None, cu_seqlens=None, B=None, T=None, iso=False, units=None, num_threads=0):
+    """Gradients of ``forward`` (reverse mode over the stored per-token states,
+    kla_oracle.c): given dout [Ntok,H,dv] and optionally the gradients of the
+    final state, returns float64 arrays ``dq, dk, dv, da, dqn, dbeta`` (the
+    shapes of the inputs), ``dlambda0`` [N,H,dk] (iso [N,H]) and ``deta0``
+    [N,H,dk,dv]. ``units`` restricts the work as in ``forward``."""
+    lib = _load()
+    q, k, v, a, qn, beta, dout = (_f32(x) for x in (q, k, v, a, qn, beta, dout))
+    lambda0, eta0, dfl, dfe = (_f32(x) for x in (lambda0, eta0, dfinal_lambda, dfinal_eta))
+    Ntok, H, dk = q.shape
+    dv = v.shape[-1]
+    cu = None
+    if cu_seqlens is not None:
+        cu = np.ascontiguousarray(np.asarray(
+            cu_seqlens.cpu().numpy() if hasattr(cu_seqlens, "cpu") else cu_seqlens, dtype=np.int32))
+        N = cu.size - 1
+        B_, T_ = 1, Ntok
+    else:
+        B_ = B if B is not None else 1
+        T_ = T if T is not None else Ntok // B_
+        assert B_ * T_ == Ntok
+        N = B_
+    g = {"dq": np.zeros(q.shape), "dk": np.zeros(k.shape), "dv": np.zeros(v.shape),
+         "da": np.zeros(a.shape), "dqn": np.zeros(qn.shape), "dbeta": np.zeros(beta.shape),
+         "dlambda0": np.zeros((N, H) if iso else (N, H, dk)), "deta0": np.zeros((N, H, dk, dv))}
+    ub, ue = (0, -1) if units is None else units
+    err = lib.kla_oracle_backward(
+        B_, T_, H, dk, dv, int(bool(iso)), _ptr(cu, _i32p), N,
+        _ptr(q, _f32p), _ptr(k, _f32p), _ptr(v, _f32p), _ptr(a, _f32p), _ptr(qn, _f32p),
+        _ptr(beta, _f32p), _ptr(lambda0, _f32p), _ptr(eta0, _f32p), _ptr(dout, _f32p),
+        _ptr(dfl, _f32p), _ptr(dfe, _f32p),
+        *(_ptr(g[n], _f64p) for n in ("dq", "dk", "dv", "da", "dqn", "dbeta", "dlambda0", "deta0")),
+        int(ub), int(ue), int(num_threads))
+    if err:
+        raise RuntimeError("oracle backward failed (bad shape or out of memory)")
+    return g
 
 
 def kdn_forward(q, k, v, a, qn, beta, lambda0=None, M0=None, cu_seqlens=None,

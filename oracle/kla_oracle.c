@@ -328,3 +328,178 @@ int kdn_oracle_forward(int B, int T, int H, int dk, int dv, int iso,
     }
     return err;
 }
+
+/* ---- Gradients of the KLA filter (reverse mode) --------------------------
+ *
+ * Kalman Linear Attention abstract: the layer is meant for efficient parallel
+ * training, so its forward pass has a backward pass. This is the plain reverse
+ * sweep of the recursion above, step by step in reverse order, with every
+ * state kept from the forward sweep (lambda and eta before each token's
+ * predict). Given the loss gradients dout [Ntok,H,dv] and, optionally,
+ * dfinal_lambda / dfinal_eta of the final state, per token (diag, per key i):
+ *   readout  o = sum_i q_i eta'_i / lam'_i:
+ *       dq_i     = sum_j do_j eta'_ij / lam'_i
+ *       deta'_ij+= q_i do_j / lam'_i
+ *       dlam'_i += -q_i (sum_j eta'_ij do_j) / lam'_i^2
+ *   update   eta' = g eta + beta k v^T, lam' = lam~ + beta k^2:
+ *       dg_i     = sum_j deta'_ij eta_ij       (eta: before the predict)
+ *       dv_j    += sum_i deta'_ij beta k_i
+ *       dk_i    += beta sum_j deta'_ij v_j + 2 beta k_i dlam'_i
+ *       dbeta   += sum_i k_i sum_j deta'_ij v_j + sum_i k_i^2 dlam'_i
+ *       dlam~_i  = dlam'_i
+ *   predict  den = a^2 + qn lam, lam~ = lam / den, g = a / den:
+ *       dden     = -(dlam~ lam + dg a) / den^2
+ *       da       = dg / den + 2 a dden,  dqn = lam dden
+ *       dlam_i   = dlam~ / den + qn dden,  deta_ij = g_i deta'_ij
+ * (isotropic: a, qn, g, lam per head; the precision term beta |k|^2 / dk).
+ * The adjoints left after the first token are dlambda0, deta0.
+ */
+static int run_unit_backward(int n, int h, long t0, long t1, int H, int dk, int dv, int iso,
+                             const float *q, const float *k, const float *v,
+                             const float *a, const float *qn, const float *beta,
+                             const float *lambda0, const float *eta0, const float *dout,
+                             const float *dfinal_lambda, const float *dfinal_eta,
+                             double *dq, double *dk_, double *dv_, double *da, double *dqn,
+                             double *dbeta, double *dlambda0, double *deta0)
+{
+    int nl = iso ? 1 : dk;
+    long L = t1 - t0;
+    size_t S = (size_t)dk * dv;
+    /* states before each token's predict: lam_s[t][nl], eta_s[t][dk*dv]; and the final one */
+    double *lam_s = (double *)malloc(sizeof(double) * nl * (size_t)(L + 1));
+    double *eta_s = (double *)malloc(sizeof(double) * S * (size_t)(L + 1));
+    double *dlam = (double *)malloc(sizeof(double) * nl);
+    double *deta = (double *)malloc(sizeof(double) * S);
+    double *dlt = (double *)malloc(sizeof(double) * nl);   /* adjoint of lam~ */
+    double *dg = (double *)malloc(sizeof(double) * nl);
+    double *pk = (double *)malloc(sizeof(double) * dk);    /* sum_j deta'_ij v_j */
+    if (!lam_s || !eta_s || !dlam || !deta || !dlt || !dg || !pk) {
+        free(lam_s); free(eta_s); free(dlam); free(deta); free(dlt); free(dg); free(pk);
+        return 1;
+    }
+    size_t u = (size_t)n * H + h;
+    for (int i = 0; i < nl; ++i) lam_s[i] = lambda0 ? (double)lambda0[u * nl + i] : 1.0;
+    for (size_t e = 0; e < S; ++e) eta_s[e] = eta0 ? (double)eta0[u * S + e] : 0.0;
+
+    /* forward sweep, keeping every state */
+    for (long s = 0; s < L; ++s) {
+        size_t th = (size_t)(t0 + s) * H + h;
+        const float *kt = k + th * dk, *vt = v + th * dv;
+        const double *lp = lam_s + (size_t)s * nl, *ep = eta_s + (size_t)s * S;
+        double *ln = lam_s + (size_t)(s + 1) * nl, *en = eta_s + (size_t)(s + 1) * S;
+        double bt = beta[th], ksq = 0.0;
+        for (int i = 0; i < dk; ++i) ksq += (double)kt[i] * (double)kt[i];
+        for (int i = 0; i < nl; ++i) {
+            double ai = iso ? a[th] : a[th * dk + i], qi = iso ? qn[th] : qn[th * dk + i];
+            double den = ai * ai + qi * lp[i];
+            ln[i] = lp[i] / den + (iso ? bt * ksq / (double)dk : bt * (double)kt[i] * (double)kt[i]);
+        }
+        for (int i = 0; i < dk; ++i) {
+            int c = iso ? 0 : i;
+            double ai = iso ? a[th] : a[th * dk + i], qi = iso ? qn[th] : qn[th * dk + i];
+            double g = ai / (ai * ai + qi * lp[c]);
+            for (int j = 0; j < dv; ++j)
+                en[(size_t)i * dv + j] = g * ep[(size_t)i * dv + j] + bt * (double)kt[i] * (double)vt[j];
+        }
+    }
+
+    /* reverse sweep */
+    for (int i = 0; i < nl; ++i) dlam[i] = dfinal_lambda ? (double)dfinal_lambda[u * nl + i] : 0.0;
+    for (size_t e = 0; e < S; ++e) deta[e] = dfinal_eta ? (double)dfinal_eta[u * S + e] : 0.0;
+    for (long s = L - 1; s >= 0; --s) {
+        size_t th = (size_t)(t0 + s) * H + h;
+        const float *qt = q + th * dk, *kt = k + th * dk, *vt = v + th * dv, *dot = dout + th * dv;
+        const double *lp = lam_s + (size_t)s * nl, *ep = eta_s + (size_t)s * S;
+        const double *ln = lam_s + (size_t)(s + 1) * nl, *en = eta_s + (size_t)(s + 1) * S;
+        double bt = beta[th], db = 0.0;
+        /* readout */
+        for (int i = 0; i < dk; ++i) {
+            int c = iso ? 0 : i;
+            double eo = 0.0;
+            for (int j = 0; j < dv; ++j) eo += en[(size_t)i * dv + j] * (double)dot[j];
+            dq[th * dk + i] = eo / ln[c];
+            dlam[c] += -(double)qt[i] * eo / (ln[c] * ln[c]);
+            for (int j = 0; j < dv; ++j) deta[(size_t)i * dv + j] += (double)qt[i] * (double)dot[j] / ln[c];
+        }
+        /* update */
+        for (int c = 0; c < nl; ++c) dg[c] = 0.0;
+        for (int j = 0; j < dv; ++j) dv_[th * dv + j] = 0.0;
+        for (int i = 0; i < dk; ++i) {
+            int c = iso ? 0 : i;
+            double gi = 0.0, p = 0.0;
+            for (int j = 0; j < dv; ++j) {
+                double d = deta[(size_t)i * dv + j];
+                gi += d * ep[(size_t)i * dv + j];
+                p += d * (double)vt[j];
+                dv_[th * dv + j] += d * bt * (double)kt[i];
+            }
+            dg[c] += gi;
+            pk[i] = p;
+        }
+        for (int i = 0; i < dk; ++i) {
+            int c = iso ? 0 : i;
+            double ki = kt[i];
+            double lamterm = iso ? 2.0 * bt * ki * dlam[0] / (double)dk : 2.0 * bt * ki * dlam[i];
+            dk_[th * dk + i] = bt * pk[i] + lamterm;
+            db += ki * pk[i] + (iso ? ki * ki * dlam[0] / (double)dk : ki * ki * dlam[c]);
+        }
+        dbeta[th] = db;
+        for (int c = 0; c < nl; ++c) dlt[c] = dlam[c];
+        /* predict */
+        for (int c = 0; c < nl; ++c) {
+            double ai = iso ? a[th] : a[th * dk + c], qi = iso ? qn[th] : qn[th * dk + c];
+            double den = ai * ai + qi * lp[c];
+            double dden = -(dlt[c] * lp[c] + dg[c] * ai) / (den * den);
+            double dai = dg[c] / den + 2.0 * ai * dden;
+            double dqi = lp[c] * dden;
+            if (iso) { da[th] = dai; dqn[th] = dqi; }
+            else { da[th * dk + c] = dai; dqn[th * dk + c] = dqi; }
+            dlam[c] = dlt[c] / den + qi * dden;
+        }
+        for (int i = 0; i < dk; ++i) {
+            int c = iso ? 0 : i;
+            double ai = iso ? a[th] : a[th * dk + i], qi = iso ? qn[th] : qn[th * dk + i];
+            double g = ai / (ai * ai + qi * lp[c]);
+            for (int j = 0; j < dv; ++j) deta[(size_t)i * dv + j] *= g;
+        }
+    }
+    if (dlambda0)
+        for (int c = 0; c < nl; ++c) dlambda0[u * nl + c] = dlam[c];
+    if (deta0) memcpy(deta0 + u * S, deta, sizeof(double) * S);
+    free(lam_s); free(eta_s); free(dlam); free(deta); free(dlt); free(dg); free(pk);
+    return 0;
+}
+
+/* Backward of kla_oracle_forward: layouts as there; every gradient output is
+ * [shape of its input] in double; dfinal_lambda / dfinal_eta / dlambda0 /
+ * deta0 may be NULL. Returns 0 on success. */
+int kla_oracle_backward(int B, int T, int H, int dk, int dv, int iso,
+                        const int *cu_seqlens, int num_seqs,
+                        const float *q, const float *k, const float *v,
+                        const float *a, const float *qn, const float *beta,
+                        const float *lambda0, const float *eta0, const float *dout,
+                        const float *dfinal_lambda, const float *dfinal_eta,
+                        double *dq, double *dk_, double *dv_, double *da, double *dqn,
+                        double *dbeta, double *dlambda0, double *deta0,
+                        long units_begin, long units_end, int num_threads)
+{
+    if (B < 0 || T < 0 || H <= 0 || dk <= 0 || dv <= 0 || !dout) return 1;
+    int N = cu_seqlens ? num_seqs : B;
+    long units = (long)N * H;
+    if (units_end < 0 || units_end > units) units_end = units;
+    if (units_begin < 0) units_begin = 0;
+    int err = 0;
+#ifdef _OPENMP
+    if (num_threads > 0) omp_set_num_threads(num_threads);
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : err)
+#endif
+    for (long u = units_begin; u < units_end; ++u) {
+        int n = (int)(u / H), h = (int)(u % H);
+        long t0 = cu_seqlens ? cu_seqlens[n] : (long)n * T;
+        long t1 = cu_seqlens ? cu_seqlens[n + 1] : (long)(n + 1) * T;
+        err |= run_unit_backward(n, h, t0, t1, H, dk, dv, iso, q, k, v, a, qn, beta, lambda0, eta0,
+                                 dout, dfinal_lambda, dfinal_eta, dq, dk_, dv_, da, dqn, dbeta,
+                                 dlambda0, deta0);
+    }
+    return err;
+}
