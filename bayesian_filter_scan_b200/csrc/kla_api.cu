@@ -13,7 +13,8 @@
 //             state carry -> output walk of every segment               (5)
 //     P = 1:  output walk                                                (1)
 // Packed variable-length sequences (cu_seqlens) are walked whole, longest
-// first (one more launch ranks them by length).
+// first (one more launch ranks them by length). kla_kdn_forward and
+// kla_prologue are one launch each; kla_backward is five (seven isotropic).
 // Nothing allocates, nothing synchronises; all work goes on the caller's stream.
 #include <cstdlib>
 #include <cstring>
@@ -46,6 +47,14 @@ cudaError_t launch_prologue(int H, long long ntok, long long T, const int *cu, i
                             const float *xqn, const float *xbeta, const float *wq, const float *wk,
                             const float *wv, const float *bq, const float *bk, const float *bv, void *q, void *k,
                             void *v, float *a, float *qn, float *beta, cudaStream_t st);
+bool backward_supported(int dk, int dv);
+size_t backward_workspace_bytes(long long ntok, int H, long long units, int dk, bool iso);
+cudaError_t launch_backward(int H, long long T, long long ntok, long long units, int dk, int dv, bool iso, bool bf16,
+                            const int *cu, const void *q, const void *k, const void *v, const float *a,
+                            const float *qn, const float *beta, const float *lambda0, const float *eta0,
+                            const void *dout, const float *dfinal_lambda, const float *dfinal_eta, float *dq,
+                            float *dk_, float *dv_, float *da, float *dqn, float *dbeta, float *dlambda0,
+                            float *deta0, void *ws, cudaStream_t st);
 cudaError_t launch_kdn(int H, long long T, long long units, int dk, int dv, bool iso, bool bf16, const int *cu,
                        const void *q, const void *k, const void *v, const float *a, const float *qn,
                        const float *beta, const float *lambda0, const float *M0, void *out, float *final_lambda,
@@ -355,6 +364,40 @@ kla_status kla_prologue(const kla_desc *d, int conv_width, const void *xq, const
                                        p.varlen ? d->cu_seqlens : nullptr, p.N, p.dk, p.dv, p.iso, p.bf16,
                                        conv_width, xq, xk, xv, xa, xqn, xbeta, wq, wk, wv, bq, bk, bv, q, k, v, a,
                                        qn, beta, st));
+}
+
+size_t kla_backward_workspace_bytes(const kla_desc *d) {
+    Plan p;
+    if (make_plan(d, p, false) != KLA_OK || !backward_supported(p.dk, p.dv)) return 0;
+    return backward_workspace_bytes((long long)d->B * d->T, p.H, (long long)p.N * p.H, p.dk, p.iso);
+}
+
+kla_status kla_backward(const kla_desc *d, const void *q, const void *k, const void *v, const float *a,
+                        const float *qn, const float *beta, const float *lambda0, const float *eta0,
+                        const void *dout, const float *dfinal_lambda, const float *dfinal_eta, float *dq,
+                        float *dk, float *dv, float *da, float *dqn, float *dbeta, float *dlambda0, float *deta0,
+                        void *workspace, size_t workspace_bytes, cudaStream_t st) {
+    Plan p;
+    kla_status s = make_plan(d, p, false);
+    if (s != KLA_OK) return s;
+    if (!backward_supported(p.dk, p.dv)) return KLA_ERR_UNSUPPORTED;
+    const long long ntok = (long long)d->B * d->T;
+    if (ntok == 0 && !p.varlen) return KLA_OK;
+    if (!q || !k || !v || !a || !qn || !beta || !dout || !dq || !dk || !dv || !da || !dqn || !dbeta)
+        return KLA_ERR_INVALID_ARG;
+    // rows of q, k, v, dout move as 16-byte vectors; everything else is read per element
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout) || !aligned16(workspace))
+        return KLA_ERR_INVALID_ARG;
+    const void *sca[] = {a, qn, beta, lambda0, eta0, dfinal_lambda, dfinal_eta, dq, dk, dv, da, dqn, dbeta,
+                         dlambda0, deta0};
+    for (const void *x : sca)
+        if (!aligned4(x)) return KLA_ERR_INVALID_ARG;
+    const size_t need = backward_workspace_bytes(ntok, p.H, (long long)p.N * p.H, p.dk, p.iso);
+    if (!workspace || workspace_bytes < need) return KLA_ERR_INVALID_ARG;
+    return cuda_status(launch_backward(p.H, p.T, ntok, (long long)p.N * p.H, p.dk, p.dv, p.iso, p.bf16,
+                                       p.varlen ? d->cu_seqlens : nullptr, q, k, v, a, qn, beta, lambda0, eta0,
+                                       dout, dfinal_lambda, dfinal_eta, dq, dk, dv, da, dqn, dbeta, dlambda0, deta0,
+                                       workspace, st));
 }
 
 kla_status kla_plan(const kla_desc *d, int *segments_per_row, int *launches, int *tensor_core) {

@@ -28,7 +28,7 @@ EXPORTS = ("kla_workspace_bytes", "kla_precision_workspace_bytes", "kla_forward"
            "kla_plan", "kla_precision",
            "kla_decode_step", "kla_host_device_bytes", "kla_forward_host", "kla_check",
            "kla_status_string", "kla_version", "kla_forward_noalloc", "kla_kdn_forward",
-           "kla_prologue")
+           "kla_prologue", "kla_backward_workspace_bytes", "kla_backward")
 
 
 class KlaError(RuntimeError):
@@ -81,6 +81,10 @@ def lib():
         L.kla_kdn_forward.restype = ctypes.c_int
         L.kla_prologue.argtypes = [D, ctypes.c_int] + [_P] * 18 + [_P]
         L.kla_prologue.restype = ctypes.c_int
+        L.kla_backward_workspace_bytes.argtypes = [D]
+        L.kla_backward_workspace_bytes.restype = ctypes.c_size_t
+        L.kla_backward.argtypes = [D] + [_P] * 19 + [_P, ctypes.c_size_t, _P]
+        L.kla_backward.restype = ctypes.c_int
         L.kla_check.argtypes = [_P]
         L.kla_check.restype = ctypes.c_int
         L.kla_status_string.argtypes = [ctypes.c_int]
@@ -205,6 +209,40 @@ def kdn_forward(q, k, v, a, qn, beta, lambda0=None, M0=None, cu_seqlens=None, B=
                               _ptr(lambda0), _ptr(M0), _ptr(out), _ptr(fl), _ptr(fm), _stream())
     _check(s, "kla_kdn_forward")
     return (out, fl, fm) if final_state else out
+
+
+def backward(q, k, v, a, qn, beta, dout, lambda0=None, eta0=None, dfinal_lambda=None, dfinal_eta=None,
+             cu_seqlens=None, B=None, T=None, mode="diag", workspace=None):
+    """Gradients of ``forward`` (include/kla.h kla_backward) on CUDA tensors:
+    returns a dict of fp32 tensors ``dq, dk, dv, da, dqn, dbeta, dlambda0,
+    deta0`` in the layouts of the corresponding inputs."""
+    m = _mode(mode)
+    desc, N = _desc_from(q, v, B, T, m, cu_seqlens)
+    for name, t in (("q", q), ("k", k), ("v", v), ("a", a), ("qn", qn), ("beta", beta), ("dout", dout)):
+        if not (t.is_cuda and t.is_contiguous()):
+            raise ValueError("%s must be a contiguous CUDA tensor" % name)
+    if k.dtype != q.dtype or v.dtype != q.dtype or dout.dtype != q.dtype:
+        raise TypeError("q, k, v, dout must share a dtype")
+    for name, t in (("a", a), ("qn", qn), ("beta", beta), ("lambda0", lambda0), ("eta0", eta0),
+                    ("dfinal_lambda", dfinal_lambda), ("dfinal_eta", dfinal_eta)):
+        if t is not None and t.dtype != torch.float32:
+            raise TypeError("%s must be float32" % name)
+    H, dk, dv = q.shape[1], q.shape[2], v.shape[2]
+    f32 = dict(dtype=torch.float32, device=q.device)
+    g = {"dq": torch.empty(q.shape, **f32), "dk": torch.empty(k.shape, **f32), "dv": torch.empty(v.shape, **f32),
+         "da": torch.empty(a.shape, **f32), "dqn": torch.empty(qn.shape, **f32),
+         "dbeta": torch.empty(beta.shape, **f32),
+         "dlambda0": torch.empty((N, H) if m == KLA_ISO else (N, H, dk), **f32),
+         "deta0": torch.empty(N, H, dk, dv, **f32)}
+    nbytes = lib().kla_backward_workspace_bytes(ctypes.byref(desc))
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=q.device)
+    s = lib().kla_backward(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(qn), _ptr(beta),
+                           _ptr(lambda0), _ptr(eta0), _ptr(dout), _ptr(dfinal_lambda), _ptr(dfinal_eta),
+                           *(_ptr(g[n]) for n in ("dq", "dk", "dv", "da", "dqn", "dbeta", "dlambda0", "deta0")),
+                           _ptr(workspace), workspace.numel(), _stream())
+    _check(s, "kla_backward")
+    return g
 
 
 def prologue(xq, xk, xv, xa, xqn, xbeta, wq, wk, wv, bq=None, bk=None, bv=None, cu_seqlens=None,

@@ -254,6 +254,36 @@ kla_status kla_prologue(const kla_desc *desc, int conv_width,
                         void *q, void *k, void *v, float *a, float *qn, float *beta,
                         cudaStream_t stream);
 
+/* Gradients of kla_forward (Kalman Linear Attention abstract: the layer is
+ * meant for efficient parallel training): given the inputs of a forward call
+ * and dout = dL/dout, plus optionally dL/dfinal_lambda and dL/dfinal_eta (NULL
+ * for zero), writes dL/d of every input in fp32, in the layout of that input:
+ * dq, dk [Ntok,H,dk]; dv [Ntok,H,dv]; da, dqn [Ntok,H,dk] (iso [Ntok,H]);
+ * dbeta [Ntok,H]; dlambda0 [N,H,dk] (iso [N,H]) and deta0 [N,H,dk,dv] (either
+ * may be NULL when not wanted). q, k, v, dout in desc->dtype, 16-byte aligned;
+ * the rest fp32, 4-byte aligned. With q^ = q/lambda, k^ = beta k and the gate
+ * g, the mean recursion is the gated linear one eta_t = g_t eta_{t-1} +
+ * k^_t v_t^T, out_t = eta_t^T q^_t; the library runs a forward sweep (the
+ * mean in registers, dq^ = eta do), two reverse sweeps of the adjoint
+ * d_t = g_{t+1} d_{t+1} + q^_t do_t^T (one over key rows for dk^ and the gate
+ * term g dL/dg = sum over later tokens of q^ dq^ - k^ dk^, one over value
+ * columns for dv), and the scalar precision chain in reverse; no per-token
+ * state is stored (CUDA cores, fp32; one CTA per (row or packed sequence,
+ * head) for each sweep). The workspace (kla_backward_workspace_bytes, caller
+ * owned, 16-byte aligned) holds per-token precisions, gates and partial
+ * gradients. dk and dv in {16, 32, 64, 128}, else KLA_ERR_UNSUPPORTED.
+ * Preconditions as kla_forward (a > 0 in particular: dL/dg is recovered as
+ * (g dL/dg) / g). Errors as kla_forward. */
+size_t kla_backward_workspace_bytes(const kla_desc *desc);
+kla_status kla_backward(const kla_desc *desc,
+                        const void *q, const void *k, const void *v,
+                        const float *a, const float *qn, const float *beta,
+                        const float *lambda0, const float *eta0, const void *dout,
+                        const float *dfinal_lambda, const float *dfinal_eta,
+                        float *dq, float *dk, float *dv, float *da, float *dqn, float *dbeta,
+                        float *dlambda0, float *deta0,
+                        void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* Synchronises `stream`, then reads and clears the library's device status
  * word on the current device: KLA_OK, KLA_ERR_RANGE or KLA_ERR_TIMEOUT from any
  * kernel that ran since the last check, or KLA_ERR_CUDA if the stream failed.

@@ -130,3 +130,26 @@ def test_launch_plan_of_the_workloads(L, shape, expect):
     d = kla.make_desc(B, T, H, dk, dv, dt, mode, _FakePtr() if nseq else None, nseq)
     p = kla.plan(d)
     assert (p["segments"], p["launches"], p["tensor_core"]) == expect
+
+
+def test_backward_host_validation(L):
+    desc = _desc(B=2, T=100, H=4, dk=64, dv=128)
+    n = L.kla_backward_workspace_bytes(ctypes.byref(desc))
+    # per token-head: lambda, gate, dL/dlambda (dk each), dq^, dk^, G (dk each), 3 head scalars;
+    # per unit: the final-state gate term (dk)
+    assert n >= 4 * (2 * 100 * 4 * (6 * 64 + 3) + 8 * 64) and n % 256 == 0
+    p = [ctypes.c_void_p(4096 * (i + 1)) for i in range(19)]
+    ws = ctypes.c_void_p(1 << 24)
+    assert L.kla_backward(ctypes.byref(desc), *p, ws, n - 256, None) == kla.KLA_ERR_INVALID_ARG
+    q = list(p)
+    q[0] = None                     # q
+    assert L.kla_backward(ctypes.byref(desc), *q, ws, n, None) == kla.KLA_ERR_INVALID_ARG
+    q = list(p)
+    q[8] = ctypes.c_void_p(4096 * 9 + 4)   # dout must be 16-byte aligned
+    assert L.kla_backward(ctypes.byref(desc), *q, ws, n, None) == kla.KLA_ERR_INVALID_ARG
+    # dv = 256 is forward-only
+    wide = _desc(dv=256)
+    assert L.kla_backward_workspace_bytes(ctypes.byref(wide)) == 0
+    assert L.kla_backward(ctypes.byref(wide), *p, ws, n, None) == kla.KLA_ERR_UNSUPPORTED
+    # an empty input launches nothing
+    assert L.kla_backward(ctypes.byref(_desc(T=0)), *([None] * 19), None, 0, None) == kla.KLA_OK
