@@ -223,8 +223,9 @@ kla_status kla_forward_noalloc(const kla_desc *desc,
  * Arguments as kla_forward, with M0 (prior mean before the first token, or
  * NULL for 0; 16-byte aligned) and final_M (or NULL) in place of eta0 /
  * final_eta; no workspace. dk and dv in {16, 32, 64, 128}, else
- * KLA_ERR_UNSUPPORTED. One CTA per (row or packed sequence, head) walks its
- * tokens with the mean in registers (CUDA cores). Errors as kla_forward. */
+ * KLA_ERR_UNSUPPORTED. One CTA per (row or packed sequence, head, block of 32
+ * value columns) walks its tokens with its columns of the mean in registers
+ * (CUDA cores). Errors as kla_forward. */
 kla_status kla_kdn_forward(const kla_desc *desc,
                            const void *q, const void *k, const void *v,
                            const float *a, const float *qn, const float *beta,
