@@ -531,6 +531,134 @@ def run_prologue(args, w):
     print(json.dumps(res))
 
 
+BWD_METRIC = "KLA backward (all input gradients) tokens/s per layer (B*T/s) on 1 B200; % of HBM"
+
+
+def backward_bytes_per_token_head(w) -> int:
+    """Algorithmic bytes of the backward per (token, head): the forward's
+    inputs and dL/dout read once, every gradient written once (fp32)."""
+    es = 2 if w.dtype == "bf16" else 4
+    nl = 1 if w.mode == "iso" else w.dk
+    return es * (2 * w.dk + 2 * w.dv) + 4 * 2 * nl + 4 + 4 * (2 * w.dk + w.dv + 2 * nl + 1)
+
+
+def run_backward(args, w):
+    """kla_backward on the workload (gradients of every input given a random
+    dL/dout): device-timed with L2 flushed between steps against its
+    algorithmic bytes; end to end with the inputs and dL/dout copied in from
+    pinned host memory and the gradients copied back inside the timed region;
+    the fp64 oracle's reverse mode on a few units as the CPU baseline."""
+    from bayesian_filter_scan_b200 import kla
+    torch.cuda.set_device(0)
+    kla.lib()
+    inp = make_inputs(w, seed=rank_seed(w, 0))
+    g = torch.Generator().manual_seed(w.seed + 1)
+    inp["dout"] = torch.randn(inp["v"].shape, generator=g).to(inp["v"].dtype)
+    names = ("q", "k", "v", "a", "qn", "beta", "dout")
+    dev = {k: inp[k].cuda() for k in names}
+    cu = inp["cu_seqlens"].cuda() if inp["cu_seqlens"] is not None else None
+    desc, _ = kla._desc_from(dev["q"], dev["v"], w.B, w.T, kla._mode(w.mode), cu)
+    ws = torch.empty(max(16, kla.lib().kla_backward_workspace_bytes(ctypes.byref(desc))), dtype=torch.uint8,
+                     device="cuda")
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    sweep = torch.ones(SWEEP_BYTES // 4, dtype=torch.float32, device="cuda")
+
+    def run(d):
+        return kla.backward(d["q"], d["k"], d["v"], d["a"], d["qn"], d["beta"], d["dout"], cu_seqlens=cu,
+                            B=w.B, T=w.T, mode=w.mode, workspace=ws)
+
+    def flush_l2():
+        flush.fill_(1)
+        sweep.sum()
+    for _ in range(args.warmup):
+        flush_l2()
+        run(dev)
+    torch.cuda.synchronize()
+    kla.check()
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    clocks = ClockSampler(0)
+    clocks.start()
+    for e0, e1 in ev:
+        flush_l2()
+        e0.record(stream)
+        grads = run(dev)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    kla.check()
+    ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev)
+    # end to end: pinned inputs in, the gradients out, inside the timed region
+    pin = {k: inp[k].pin_memory() for k in names}
+    hout = {k: torch.empty(t.shape, dtype=t.dtype).pin_memory() for k, t in grads.items()}
+    dbuf = {k: torch.empty_like(dev[k]) for k in names}
+    e_t, e_steps = 0.0, max(3, min(args.e2e_steps, args.steps))
+    for i in range(e_steps + 2):
+        flush_l2()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for k in names:
+            dbuf[k].copy_(pin[k], non_blocking=True)
+        got = run(dbuf)
+        for k, t in got.items():
+            hout[k].copy_(t, non_blocking=True)
+        a1.record(stream)
+        a1.synchronize()
+        if i >= 2:
+            e_t += a0.elapsed_time(a1)
+    peaks, peak_src = measured_peaks()
+    peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    alg = backward_bytes_per_token_head(w) * w.tokens * w.H
+    ach = alg / (ms * 1e-3) / 1e9
+    cfg = arm_config(w, 1)
+    cfg["variant"] = "backward (all input gradients, random dL/dout)"
+    res = {"metric": BWD_METRIC, "value": w.tokens / (ms * 1e-3), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": w.dtype, "data": "synthetic", "config": cfg,
+           "roofline": {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+                        "traffic": None, "kernel": "kla_backward (five launches, CUDA cores)",
+                        "alg_bytes_per_launch": alg, "launch_ms": ms,
+                        "alg_bytes_per_token_head": backward_bytes_per_token_head(w),
+                        "peak_source": "%s (MEASURED_PEAKS.json hbm_gbs)" % peak_src},
+           "e2e": {"value": w.tokens / (e_t / e_steps * 1e-3), "unit": UNIT,
+                   "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in pin.values()),
+                   "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in hout.values())},
+           "gpu_launches": args.steps * (7 if w.mode == "iso" else 5), "clocks": clk}
+    if not args.no_cpu_baseline:
+        import oracle
+        n_units = min(4, _units_total(w, inp))
+        t0 = time.perf_counter()
+        ref = oracle.backward(inp["q"], inp["k"], inp["v"], inp["a"], inp["qn"], inp["beta"], inp["dout"],
+                              cu_seqlens=inp["cu_seqlens"], B=None if inp["cu_seqlens"] is not None else w.B,
+                              T=None if inp["cu_seqlens"] is not None else w.T, iso=w.mode == "iso",
+                              units=(0, n_units), num_threads=n_units)
+        t = time.perf_counter() - t0
+        res["cpu_baseline"] = {"value": _unit_tokens(w, inp, n_units) / t, "unit": UNIT, "cores": n_units,
+                               "kind": "oracle",
+                               "sample": "%d of %d (row, head) units, fp64 C oracle (reverse mode), %.3f s" % (
+                                   n_units, _units_total(w, inp), t)}
+        cuh = inp["cu_seqlens"].tolist() if inp["cu_seqlens"] is not None else None
+        worst = {}
+        for name, gt in grads.items():
+            gs, ws_ = [], []
+            for u in range(n_units):
+                n, h = divmod(u, w.H)
+                if name in ("dlambda0", "deta0"):
+                    gs.append(gt[n, h].reshape(-1))
+                    ws_.append(ref[name][n, h].reshape(-1))
+                else:
+                    s0, s1 = (cuh[n], cuh[n + 1]) if cuh else (n * w.T, (n + 1) * w.T)
+                    gs.append(gt[s0:s1, h].reshape(-1))
+                    ws_.append(ref[name][s0:s1, h].reshape(-1))
+            gv = torch.cat(gs).double().cpu().numpy()
+            wv = np.concatenate(ws_)
+            scale = float(np.max(np.abs(wv))) if wv.size else 0.0
+            worst[name] = float(np.max(np.abs(gv - wv))) / (scale + 1e-30) if wv.size else 0.0
+        res["max_err"] = dict(worst, units=n_units, tol=2e-3,
+                              definition="max |gpu - oracle| / max |oracle| per gradient over the sampled units")
+    print(json.dumps(res))
+
+
 def run_reference(args, w):
     """Reference arm: the CPU oracle timed on this host's cores. It loads only
     the oracle, never the CUDA library."""
@@ -571,10 +699,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--variant", default="kla", choices=["kla", "kdn", "prologue"],
+    ap.add_argument("--variant", default="kla", choices=["kla", "kdn", "prologue", "backward"],
                     help="kla: the KLA forward (the bench line); kdn: the Kalman Delta Network "
                          "residual write on the same workload; prologue: the mixer's input "
-                         "prologue (separate lines)")
+                         "prologue; backward: the gradients of the KLA forward (separate lines)")
     ap.add_argument("--T", type=int, default=None,
                     help="tokens per row instead of the workload's (smaller cases of the same "
                          "workload for profiler captures; not a bench line)")
@@ -592,6 +720,9 @@ def main():
         return
     if args.variant == "prologue":
         run_prologue(args, w)
+        return
+    if args.variant == "backward":
+        run_backward(args, w)
         return
 
     from bayesian_filter_scan_b200 import kla
